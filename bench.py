@@ -1,0 +1,530 @@
+#!/usr/bin/env python
+"""Benchmark of one speculative-decoding step: target verification + P-EAGLE draft-batch
+construction, through libpspec's C ABI, on the large-batch workload (B=1024 sequences,
+K=7 drafts, vocabulary 201088, hidden 2880, bf16 logits).
+
+A step = one verify call (rejection rule by default, --mode greedy for the greedy rule)
+over the B*(K+1) target rows (and B*K draft rows), whose accepted counts and bonus
+tokens feed one draft-batch construction call.  Inputs are resident in HBM and larger
+than L2 (6.2 GB of logits per step), so every step streams them from DRAM.
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own replica of the
+workload (the sequences are independent; no collective on the data path) and the
+reported time is the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--mode rejection|greedy]
+  python bench.py --impl reference ...   # the CPU oracle on the same workload
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "verify+build step/s and achieved HBM GB/s (% of peak) at B=1024,K=7,V=201088"
+UNIT = "step/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["pspec", "reference"], default="pspec")
+    p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample", type=int, default=192,
+                   help="sequences of the workload the CPU oracle baseline verifies")
+    p.add_argument("--workload", default="b1024", help="b1024 (default), c64 or c1")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str, src_hash: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, or None when there is
+    none or it was taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"traffic_per_launch_bytes:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", txt)
+    if not m or not h or h.group(1) != src_hash:
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def __init__(self, torch_device: int, period_s: float = 0.005):
+        self.samples, self.period, self.ok = [], period_s, False
+        self._stop = threading.Event()
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N = N
+            self.h = self._handle(N, torch_device)
+            self.max_sm = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    @staticmethod
+    def _handle(N, dev):
+        import torch
+        try:
+            uuid = str(torch.cuda.get_device_properties(dev).uuid)
+            return N.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+        except Exception:  # noqa: BLE001
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = dev
+            if vis and vis.split(",")[dev].strip().isdigit():
+                idx = int(vis.split(",")[dev])
+            if N.nvmlDeviceGetCount() == 1:
+                idx = 0
+            return N.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        N = self.N
+        while not self._stop.is_set():
+            try:
+                sm = N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM)
+                pw = N.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                rs = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, pw, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "source": "nvml",
+                    "note": getattr(self, "err", "no samples")}
+        sms = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[2]
+        reasons = sorted(v for k, v in self.REASONS.items() if bits & k and k != 0x1)
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": self.max_sm,
+                "sm_mhz_min": min(sms), "power_w_max": round(max(s[1] for s in self.samples), 1),
+                "reasons": reasons, "samples": len(sms), "source": "nvml"}
+
+
+# ----------------------------------------------------------------------------- workload
+def make_workload(name, device, rank):
+    import torch
+    from speculative_decoding_step_pspec_b200 import inputs as I
+    w = dict(b1024=I.B1024, c64=I.C64, c1=I.C1)[name]
+    w = I.scaled(w, seed=w.seed + 1000 * rank)      # each replica draws its own batch
+    target, draft = I.logits(w, device)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, device)
+    binp = I.build_inputs(w, device, drafts=sampled)
+    if torch.device(device).type == "cuda":
+        torch.cuda.synchronize()
+    return w, dict(target=target, draft=draft, sampled=sampled, greedy=greedy, u=u, build=binp)
+
+
+def algorithmic_bytes(w, mode, accepted):
+    """Bytes the one-pass method must move per step (verify sweep + draft-batch build)."""
+    import numpy as np
+    s = 2 if str(w.dtype).endswith("bfloat16") else 4
+    rows = w.B * ((2 * w.K + 1) if mode == "rejection" else (w.K + 1))
+    verify = rows * w.V * s
+    c = np.asarray(accepted, np.int64) + 1                 # surviving verify rows (L = K+1)
+    H, sh = w.H, s
+    T_in = w.B * (w.K + 1)
+    T_cap = -(-(T_in + w.B * (w.K - 1)) // w.capture_pad) * w.capture_pad
+    hidden = int((c.sum() * H * sh) + ((c + w.K - 1).sum() * H * sh))
+    live_rows = int((c + w.K - 1).sum())
+    meta = T_cap * 21 + T_in * 8 + live_rows * 4 + (w.B + 1) * 8 + w.B * (16 + 4 * w.K)
+    return verify, hidden + meta
+
+
+# ----------------------------------------------------------------------------- pspec arm
+def run_pspec(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import speculative_decoding_step_pspec_b200 as ps
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w, d = make_workload(args.workload, dev, rank)
+    rej = args.mode == "rejection"
+    ws = ps.Workspace(w.B, w.K, w.V, rej, dev)
+    vout = ps.api.verify_outputs(w.B, w.K, dev, False, rej)
+    bi = d["build"]
+    bout = ps.api.build_outputs(w.B, w.K, w.H, bi["T_cap"], bi["verify_hidden"].dtype, dev)
+    drafts = d["sampled"] if rej else d["greedy"]
+
+    def verify(stream=None):
+        if rej:
+            ps.verify_rejection(d["target"], d["draft"], drafts, d["u"], workspace=ws, out=vout)
+        else:
+            ps.verify_greedy(d["target"], drafts, workspace=ws, out=vout)
+
+    def build():
+        ps.build_draft_batch(K=w.K, block_size=w.block_size, mask_id=bi["mask_id"],
+                             pad_id=bi["pad_id"], T_cap=bi["T_cap"], qsl_in=bi["qsl_in"],
+                             verify_tokens=bi["verify_tokens"], verify_pos=bi["verify_pos"],
+                             accepted_len=vout["accepted_len"], bonus=vout["bonus"],
+                             block_table=bi["block_table"], verify_hidden=bi["verify_hidden"],
+                             h_shared=bi["h_shared"], out=bout)
+
+    for _ in range(max(3, args.warmup)):
+        verify()
+        build()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    torch.cuda.synchronize()
+    with sampler:
+        t0.record()
+        for s in range(K):
+            ev[s][0].record()
+            if rej:
+                ps.pspec_set_split_event(ev[s][1])
+            verify()
+            ev[s][2].record()
+            build()
+            ev[s][3].record()
+        t1.record()
+        torch.cuda.synchronize()
+    ps.pspec_set_split_event(None)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+
+    verify_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    build_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    stats_ms = [e[0].elapsed_time(e[1]) for e in ev] if rej else verify_ms
+    draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if rej else None
+    assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
+    acc = vout["accepted_len"].cpu().numpy()
+    vbytes, bbytes = algorithmic_bytes(w, args.mode, acc)
+    hbm, peak_src = peaks()
+    ms_step = elapsed_ms / K
+    step_gbs = (vbytes + bbytes) / (ms_step * 1e-3) / 1e9
+    dom_kernel = "rej_stats_kernel" if rej else "greedy_sweep_kernel"
+    src = ["speculative_decoding_step_pspec_b200/csrc/verify_rejection.cu" if rej else
+           "speculative_decoding_step_pspec_b200/csrc/verify_greedy.cu",
+           "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
+    src_hash = kernel_source_hash(src)
+    dom_ms = statistics.mean(stats_ms)
+    achieved = vbytes / (dom_ms * 1e-3) / 1e9
+    traffic = profiled_traffic(dom_kernel, args.workload, src_hash)
+    launches_per_step = ps.pspec_launches_per_call(2 if rej else 1) + ps.pspec_launches_per_call(0)
+
+    line = {
+        "metric": METRIC, "value": round(world * K / (elapsed_ms * 1e-3), 3), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{args.workload}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
+                        f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
+            "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
+            "l2": "inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9),
+            "parallelism": f"replicas x{world} (independent sequences, no collective)",
+        },
+        "achieved_gbs": round(step_gbs, 1),
+        "pct_of_peak": round(100 * step_gbs / hbm, 2),
+        "algorithmic_bytes_per_step": {"verify": int(vbytes), "build": int(bbytes)},
+        "kernels_ms": {
+            dom_kernel: round(dom_ms, 5),
+            **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if rej else {}),
+            "build_kernel": round(statistics.mean(build_ms), 5),
+        },
+        "build_gbs": round(bbytes / (statistics.mean(build_ms) * 1e-3) / 1e9, 1),
+        "roofline": {
+            "kernel": dom_kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+            "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
+            "algorithmic_bytes_per_launch": int(vbytes),
+        },
+        "gpu_launches": K * launches_per_step,
+        "launches_per_step": launches_per_step,
+        "acceptance": {"mean_accepted": round(float(acc.mean()), 4),
+                       "rate_per_draft": round(float(acc.mean()) / w.K, 4),
+                       "histogram": np.bincount(acc, minlength=w.K + 1).tolist()},
+        "clocks": sampler.summary(),
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, w, d, ps, dev, world)
+    else:
+        line["e2e"] = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args, w, d, acc)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, d, ps, dev, world):
+    """The same step through the public API from pinned HOST buffers: every step copies its
+    inputs host->device, runs verify + build, and reads the results back."""
+    import torch
+    import torch.distributed as dist
+    rej = args.mode == "rejection"
+    bi = d["build"]
+    names = ["target", "draft", "u"] if rej else ["target"]
+    host = {k: torch.empty_like(d[k], device="cpu", pin_memory=True) for k in names}
+    drafts_dev = d["sampled"] if rej else d["greedy"]
+    host["drafts"] = torch.empty_like(drafts_dev, device="cpu", pin_memory=True)
+    bnames = ["qsl_in", "verify_tokens", "verify_pos", "block_table", "verify_hidden", "h_shared"]
+    for k in bnames:
+        host["b_" + k] = torch.empty_like(bi[k], device="cpu", pin_memory=True)
+    for k in names:
+        host[k].copy_(d[k])
+    host["drafts"].copy_(drafts_dev)
+    for k in bnames:
+        host["b_" + k].copy_(bi[k])
+    dv = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    ws = ps.Workspace(w.B, w.K, w.V, rej, dev)
+    vout = ps.api.verify_outputs(w.B, w.K, dev, False, rej)
+    bout = ps.api.build_outputs(w.B, w.K, w.H, bi["T_cap"], bi["verify_hidden"].dtype, dev)
+    res_names = ["out_tokens", "accepted_len", "bonus"]
+    bres_names = ["draft_tokens", "draft_pos", "slot_mapping", "row_kind", "hidden_src",
+                  "qsl_out", "seq_lens_out", "sample_idx"]
+    hres = {k: torch.empty_like(vout[k], device="cpu", pin_memory=True) for k in res_names}
+    hres.update({"b_" + k: torch.empty_like(bout[k], device="cpu", pin_memory=True) for k in bres_names})
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in hres.values())
+
+    def step():
+        for k, t in host.items():
+            dv[k].copy_(t, non_blocking=True)
+        if rej:
+            ps.verify_rejection(dv["target"], dv["draft"], dv["drafts"], dv["u"], workspace=ws, out=vout)
+        else:
+            ps.verify_greedy(dv["target"], dv["drafts"], workspace=ws, out=vout)
+        ps.build_draft_batch(K=w.K, block_size=w.block_size, mask_id=bi["mask_id"],
+                             pad_id=bi["pad_id"], T_cap=bi["T_cap"], qsl_in=dv["b_qsl_in"],
+                             verify_tokens=dv["b_verify_tokens"], verify_pos=dv["b_verify_pos"],
+                             accepted_len=vout["accepted_len"], bonus=vout["bonus"],
+                             block_table=dv["b_block_table"], verify_hidden=dv["b_verify_hidden"],
+                             h_shared=dv["b_h_shared"], out=bout)
+        for k in res_names:
+            hres[k].copy_(vout[k], non_blocking=True)
+        for k in bres_names:
+            hres["b_" + k].copy_(bout[k], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    n = max(1, args.e2e_steps)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    del host, dv
+    return {"value": round(world * n / (ms * 1e-3), 3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": n, "ms_per_step": round(ms / n, 3),
+            "path": "pinned host buffers -> cudaMemcpyAsync -> C-ABI verify + build -> results to host"}
+
+
+def _oracle_inputs(d, seqs):
+    import numpy as np
+    import torch
+
+    def logits(x):
+        x = x[seqs]
+        return x.view(torch.int16).cpu().numpy().view(np.uint16) if x.dtype == torch.bfloat16 else x.float().cpu().numpy()
+    return (logits(d["target"]), logits(d["draft"]), d["sampled"][seqs].cpu().numpy(),
+            d["u"][seqs].cpu().numpy())
+
+
+def _oracle_build_args(w, d, acc, bonus):
+    import torch
+    bi = d["build"]
+    vh = bi["verify_hidden"]
+    vh = vh.view(torch.int16) if vh.dtype == torch.bfloat16 else vh
+    hs = bi["h_shared"]
+    hs = hs.view(torch.int16) if hs.dtype == torch.bfloat16 else hs
+    return dict(K=w.K, block_size=w.block_size, mask_id=bi["mask_id"], pad_id=bi["pad_id"],
+                T_cap=bi["T_cap"], qsl_in=bi["qsl_in"].cpu().numpy(),
+                verify_tokens=bi["verify_tokens"].cpu().numpy(),
+                verify_pos=bi["verify_pos"].cpu().numpy(), accepted_len=acc, bonus=bonus,
+                block_table=bi["block_table"].cpu().numpy(), verify_hidden=vh.cpu().numpy(),
+                h_shared=hs.cpu().numpy())
+
+
+def cpu_baseline(args, w, d, acc):
+    """The oracle as it stands, on the host cores, over a bounded sample of this workload:
+    rejection (or greedy) verify of `cpu_sample` sequences, scaled to the whole batch, plus
+    one full draft-batch construction."""
+    import numpy as np
+    import torch
+
+    import oracle
+    S = min(args.cpu_sample, w.B)
+    seqs = torch.arange(S, device=d["target"].device)
+    t, q, dr, u = _oracle_inputs(d, seqs)
+    threads = max(1, min(os.cpu_count() or 1, S))
+    bargs = _oracle_build_args(w, d, acc.astype(np.int32), np.zeros(w.B, np.int32))
+    t0 = time.perf_counter()
+    if args.mode == "rejection":
+        oracle.verify_rejection(t, q, dr, u, threads=threads)
+    else:
+        oracle.verify_greedy(t, d["greedy"][seqs].cpu().numpy(), threads=threads)
+    t1 = time.perf_counter()
+    oracle.build_draft_batch(**bargs)
+    t2 = time.perf_counter()
+    step_s = (t1 - t0) * (w.B / S) + (t2 - t1)
+    return {"value": round(1.0 / step_s, 5), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{args.mode} verify of {S} of {w.B} sequences (x{w.B / S:.2f}) + one "
+                      f"full draft-batch build; {t1 - t0:.2f} s + {t2 - t1:.2f} s wall, "
+                      f"{threads} threads"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank):
+    """The CPU oracle as the reference arm: each step verifies a rotating bounded sample of
+    the workload's sequences on the host cores and builds the full draft batch; the step
+    time is scaled to the whole batch."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    w, d = make_workload(args.workload, dev, 0)
+    threads = max(1, os.cpu_count() or 1)
+    acc = np.full(w.B, w.K // 2, np.int32)
+    bargs = _oracle_build_args(w, d, acc, np.zeros(w.B, np.int32))
+    # size the per-step sample so that warmup + steps take about two minutes
+    probe = torch.arange(1, device=dev)
+    t, q, dr, u = _oracle_inputs(d, probe)
+    a = time.perf_counter()
+    oracle.verify_rejection(t, q, dr, u) if args.mode == "rejection" else oracle.verify_greedy(t, dr)
+    per_seq = time.perf_counter() - a
+    a = time.perf_counter()
+    oracle.build_draft_batch(**bargs)
+    build_s = time.perf_counter() - a
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    S = int(max(1, min(w.B, threads * max(0.0, budget - build_s) / max(per_seq, 1e-6))))
+    times = []
+    for s in range(args.warmup + args.steps):
+        seqs = (torch.arange(S, device=dev) + s * S) % w.B
+        t, q, dr, u = _oracle_inputs(d, seqs)
+        a = time.perf_counter()
+        if args.mode == "rejection":
+            oracle.verify_rejection(t, q, dr, u, threads=min(threads, S))
+        else:
+            oracle.verify_greedy(t, dr, threads=min(threads, S))
+        b = time.perf_counter()
+        oracle.build_draft_batch(**bargs)
+        c = time.perf_counter()
+        if s >= args.warmup:
+            times.append((b - a) * (w.B / S) + (c - b))
+    step_s = statistics.mean(times)
+    value = round(1.0 / step_s, 5)
+    cores = min(threads, S)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, {args.mode} "
+                               f"verify + P-EAGLE draft-batch build (CPU oracle)",
+                   "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {args.mode} verify of {S} of {w.B} sequences "
+                                   f"(x{w.B / S:.1f}) + one full draft-batch build"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_pspec(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

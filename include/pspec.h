@@ -1,0 +1,251 @@
+/*
+ * pspec.h -- C ABI of libpspec: the per-step hot path of speculative decoding with
+ * P-EAGLE parallel drafting, on one NVIDIA B200 (sm_100a).
+ *
+ * Three operations, each one or two hand-written CUDA kernels:
+ *
+ *   pspec_verify_greedy       target verification, greedy rule
+ *   pspec_verify_rejection    target verification, rejection rule
+ *   pspec_build_draft_batch   parallel-draft batch construction
+ *
+ * Sources (page title, section):
+ *   "Capstone 14: speculative decoding inference server", section "Concept": the target
+ *     checks the k drafts in one forward pass and an accepted prefix replaces the greedy
+ *     path; section "Architecture": accept the prefix, resample for the rejected suffix.
+ *   rskf.cn speculative-decoding article, section 2.2 (table row "target model"): the
+ *     output must be identical to plain autoregressive decoding.  Section 2.1 names the
+ *     vocabulary-wide softmax and the memory-bandwidth bound of decode.
+ *   "Eagle parallel speculative decoding, vLLM, TorchSpec", section "Parallel
+ *     architecture": drafter inputs pair context tokens with their hidden states, the
+ *     next-token slot with h_context and prediction slots 2..K with a mask token and the
+ *     shared hidden state h_shared; section "TorchSpec integration": the draft batch
+ *     metadata (copy, scatter, insert, pad, mask, remap) is rebuilt on the GPU, h_shared
+ *     is broadcast into the mask slots by a separate copy, and rejected tokens take
+ *     PADDING_SLOT_ID = -1 in the KV slot mapping.
+ *
+ * Conventions shared by every entry point:
+ *   - Every array pointer is caller-owned DEVICE memory (cudaMalloc / torch tensors).  The
+ *     argument structs themselves are host memory and are read before the call returns.
+ *   - Calls are asynchronous on the caller's stream: the library never synchronises the
+ *     host, never allocates, and launches nothing outside the given stream.
+ *   - Host-side checks (null pointers, sizes, alignment, capacity) return an error status
+ *     and launch nothing.  Invalid VALUES found on the device (a token outside [0, V), an
+ *     accepted count outside [0, K], a block lookup outside the table, a malformed query
+ *     offset array) never trap: the kernel ORs a PSPEC_DEVERR_* bit into *err and writes a
+ *     documented safe output instead.  *err is only ever OR-ed, so zero it before a call
+ *     whose bits you want to read alone.
+ *   - Results are deterministic: repeated calls on the same inputs give bit-identical
+ *     outputs (segment partials are merged in a fixed order; no floating-point atomics).
+ */
+#ifndef PSPEC_H
+#define PSPEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define PSPEC_API __attribute__((visibility("default")))
+#else
+#define PSPEC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PSPEC_OK = 0,
+  PSPEC_ERR_INVALID_ARG = 1,  /* a host-side check failed; nothing was launched */
+  PSPEC_ERR_UNSUPPORTED = 2,  /* a valid but unsupported request (e.g. K > 31) */
+  PSPEC_ERR_CUDA = 3,         /* a launch failed; cudaGetLastError() has the cause */
+  PSPEC_ERR_WORKSPACE = 4     /* workspace pointer NULL, misaligned or too small */
+} pspec_status;
+
+typedef enum { PSPEC_F32 = 0, PSPEC_BF16 = 1 } pspec_dtype;
+
+/* Bits OR-ed into the device error word. */
+#define PSPEC_DEVERR_TOKEN_RANGE 0x1   /* draft token outside [0, V): never accepted */
+#define PSPEC_DEVERR_ACCEPT_RANGE 0x2  /* accepted_len outside [0, K]: clamped into it */
+#define PSPEC_DEVERR_BLOCK_RANGE 0x4   /* position < 0, pos/block_size >= max_blocks or a
+                                          negative block id: that row's slot is -1 */
+#define PSPEC_DEVERR_LAYOUT 0x8        /* qsl_in not an offset array, or a sequence with
+                                          fewer than K+1 verify rows */
+
+/* Row kinds written to pspec_build_args.row_kind. */
+#define PSPEC_ROW_CTX 0   /* context row: accepted token paired with its target hidden */
+#define PSPEC_ROW_NTP 1   /* next-token row: bonus token paired with h_context */
+#define PSPEC_ROW_MASK 2  /* prediction slot 2..K: mask token paired with h_shared */
+#define PSPEC_ROW_REJ 3   /* rejected verify row: pad token, slot -1, hidden unwritten */
+#define PSPEC_ROW_PAD 4   /* capacity padding: pad token, position 0, slot -1 */
+
+#define PSPEC_PADDING_SLOT_ID (-1)
+#define PSPEC_MAX_K 31    /* the accept decisions of one sequence live in one 32-bit mask */
+
+/*
+ * Verification arguments.
+ *
+ * Layout: logits rows are row-major with a row stride of `ld` elements (ld >= V); row k of
+ * sequence i is at base + (i*(K+1) + k)*ld for the target and base + (i*K + k)*ld for the
+ * draft.  Bases need only element alignment; V and ld may be anything.  Rows are streamed
+ * with 16-byte loads from their first 16-byte boundary on; an unaligned head and a ragged
+ * tail (fewer than 8 bf16 / 4 fp32 elements each) are read with scalar loads, so rows
+ * that start on a 16-byte boundary (base 16-byte aligned, ld*sizeof(elem) a multiple of
+ * 16) are read fastest.
+ */
+typedef struct {
+  int B;                       /* sequences; B = 0 is a no-op */
+  int K;                       /* drafts per sequence, 1 <= K <= PSPEC_MAX_K */
+  int V;                       /* vocabulary size, >= 1 */
+  long long ld;                /* row stride of the logits in elements, >= V */
+  pspec_dtype dtype;           /* logits dtype (both sides) */
+  const void *target_logits;   /* [B, K+1, ld] target rows; row k scores position k */
+  const void *draft_logits;    /* [B, K, ld] draft rows (rejection only; else NULL) */
+  const int32_t *draft_tokens; /* [B, K] drafted token ids */
+  const float *uniforms;       /* [B, K+1] in [0,1) (rejection only): column k < K is the
+                                  accept test of draft k, column K drives the resample or
+                                  bonus draw.  The caller owns the random numbers, so
+                                  results do not depend on any generator in the library. */
+  int32_t *out_tokens;         /* [B, K+1] out: accepted drafts, then the bonus token, then
+                                  -1 up to K+1 entries */
+  int32_t *accepted_len;       /* [B] out: a_i in [0, K] */
+  int32_t *bonus;              /* [B] out: the token emitted after the accepted prefix */
+  /* Optional fp32 diagnostics (NULL skips each): */
+  float *target_lse;           /* [B, K+1] log-sum-exp of each target row */
+  float *draft_lse;            /* [B, K]   log-sum-exp of each draft row (rejection) */
+  float *p_at_draft;           /* [B, K]   target softmax probability of draft k (rejection) */
+  float *q_at_draft;           /* [B, K]   draft softmax probability of draft k (rejection) */
+  float *residual_mass;        /* [B]      Z = sum max(0, p - q) of the resampled row, or
+                                           sum p of the bonus row (rejection) */
+  int32_t *err;                /* device error word (required); bits are OR-ed in */
+} pspec_verify_args;
+
+/*
+ * Workspace for the verify calls: scratch device memory owned by the caller, at least
+ * pspec_verify_workspace_bytes(B, K, V, rejection) bytes, 256-byte aligned.  It must be
+ * zero-filled once (cudaMemsetAsync) before its first use; every call leaves its
+ * per-sequence counters back at zero, so later calls need no re-initialisation.  Calls
+ * that share one workspace must not overlap on the GPU (use one workspace per stream).
+ */
+PSPEC_API size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection);
+
+/*
+ * Greedy verification ("any accepted prefix replaces the greedy path").
+ * For each sequence i: g_k = argmax over the vocabulary of target row k (the lowest id
+ * wins ties); a_i = the number of leading drafts with d_k == g_k; bonus = g_{a_i};
+ * out_tokens = [d_0 .. d_{a_i-1}, bonus, -1 ...].  target_lse is written when non-NULL.
+ * One kernel launch: a vocabulary sweep over all B*(K+1) target rows; the last CTA of
+ * each sequence combines its row partials.  Errors: PSPEC_ERR_INVALID_ARG for bad
+ * arguments; a draft token outside [0, V) is treated as a mismatch and sets
+ * PSPEC_DEVERR_TOKEN_RANGE.
+ */
+PSPEC_API pspec_status pspec_verify_greedy(const pspec_verify_args *args, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Rejection-rule verification ("accept prefix; resample for rejected suffix", lossless).
+ * p_k = softmax(target row k), q_k = softmax(draft row k).  Draft k is accepted iff
+ * u_k * q_k(d_k) < p_k(d_k) (that is, with probability min(1, p/q)); a_i is the first
+ * rejected position, K if none.  The emitted token after the prefix is drawn by inverse
+ * CDF in token-id order with u_K: from r = max(0, p_{a_i} - q_{a_i}) after a rejection,
+ * from r = p_K when every draft passed; token = the smallest t with
+ * sum_{v<=t} r_v > u_K * sum r (if rounding leaves none, the last t with r_t > 0; if the
+ * residual sums to zero, the draw uses p_{a_i} itself).  Two launches: a vocabulary
+ * sweep over the 2K+1 rows of every sequence (softmax statistics and the accept mask),
+ * then a chunked inverse-CDF draw over each sequence's row a_i.  A draft token outside
+ * [0, V) has p = q = 0, is rejected, and sets PSPEC_DEVERR_TOKEN_RANGE.
+ */
+PSPEC_API pspec_status pspec_verify_rejection(const pspec_verify_args *args, void *workspace,
+                                    size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Draft-batch construction arguments.
+ *
+ * Verify batch: sequence i owns rows [qsl_in[i], qsl_in[i+1]) of the verify arrays, with
+ * L_i = qsl_in[i+1] - qsl_in[i] >= K+1 rows whose last K are its drafts.  After
+ * verification a_i drafts were accepted, so c_i = L_i - K + a_i verify rows survive and
+ * the last survivor's target hidden state is h_context.  Output span of sequence i, at
+ * qsl_out[i] = qsl_in[i] + i*(K-1), length L_i + K - 1, in this order:
+ *   rows 0 .. c_i-2     CTX  token verify_tokens[s+j+1], hidden verify row s+j,
+ *                            position verify_pos[s+j]                    (s = qsl_in[i])
+ *   row  c_i-1          NTP  token bonus[i], hidden verify row s+c_i-1 (h_context),
+ *                            position P = verify_pos[s+c_i-1]
+ *   rows c_i .. c_i+K-2 MASK token mask_id, hidden h_shared, position P + m (m = 1..K-1)
+ *   last K - a_i rows   REJ  token pad_id, position of the rejected verify row, slot -1
+ * Rows [qsl_out[B], T_cap) are PAD rows (pad_id, position 0, slot -1).
+ * Slots of CTX/NTP/MASK rows: block_table[i][pos / block_size] * block_size
+ * + pos % block_size.  seq_lens_out[i] = P + K (last mask position + 1).
+ * sample_idx[i*K + k] = qsl_out[i] + c_i - 1 + k (the NTP row and the mask rows).
+ * hidden_src[row] = the verify row copied into draft_hidden[row] (CTX/NTP), else -1.
+ * draft_hidden rows of kind REJ and PAD are not written.
+ */
+typedef struct {
+  int B;                          /* sequences; B = 0 writes only the PAD rows */
+  int K;                          /* drafts per sequence, 1 <= K <= PSPEC_MAX_K */
+  int H;                          /* hidden size (elements) */
+  pspec_dtype hidden_dtype;       /* element type of verify_hidden / h_shared / draft_hidden */
+  int block_size;                 /* KV block size in tokens, >= 1 */
+  int max_blocks;                 /* columns of block_table, >= 1 */
+  int mask_id;                    /* token id of the mask placeholder */
+  int pad_id;                     /* token id written to REJ and PAD rows */
+  int T_in;                       /* verify rows */
+  int T_cap;                      /* output rows, >= T_in + B*(K-1) */
+  const int32_t *qsl_in;          /* [B+1] verify query offsets, qsl_in[0] = 0 */
+  const int32_t *verify_tokens;   /* [T_in] */
+  const int32_t *verify_pos;      /* [T_in] */
+  const int32_t *accepted_len;    /* [B] a_i from the verify step */
+  const int32_t *bonus;           /* [B] bonus token from the verify step */
+  const int32_t *block_table;     /* [B, max_blocks] KV block ids */
+  const void *verify_hidden;      /* [T_in, H] target hidden states (16-byte aligned rows) */
+  const void *h_shared;           /* [H] learned shared hidden state (16-byte aligned) */
+  int32_t *draft_tokens;          /* [T_cap] out */
+  int32_t *draft_pos;             /* [T_cap] out */
+  int64_t *slot_mapping;          /* [T_cap] out, PSPEC_PADDING_SLOT_ID for REJ/PAD rows */
+  uint8_t *row_kind;              /* [T_cap] out, PSPEC_ROW_* */
+  int32_t *hidden_src;            /* [T_cap] out */
+  int32_t *qsl_out;               /* [B+1] out */
+  int32_t *seq_lens_out;          /* [B] out */
+  int32_t *sample_idx;            /* [B, K] out */
+  void *draft_hidden;             /* [T_cap, H] out (16-byte aligned rows) */
+  int32_t *err;                   /* device error word (required) */
+} pspec_build_args;
+
+/*
+ * Parallel-draft batch construction: one launch.  Its CTAs take one of two roles: the
+ * metadata role writes every per-row and per-sequence output, the hidden role copies the
+ * CTX/NTP hidden rows and broadcasts h_shared into the MASK rows with 16-byte stores.
+ * H * sizeof(elem) must be a multiple of 16 and the hidden bases 16-byte aligned
+ * (PSPEC_ERR_INVALID_ARG otherwise).  Invalid values on the device: accepted_len outside
+ * [0, K] is clamped (PSPEC_DEVERR_ACCEPT_RANGE); an out-of-table lookup gives slot -1
+ * (PSPEC_DEVERR_BLOCK_RANGE); a sequence with L_i < K+1 keeps its span as PAD rows with
+ * seq_lens_out 0 and sample_idx -1 (PSPEC_DEVERR_LAYOUT); a qsl_in that is not an offset
+ * array (qsl_in[0] != 0, decreasing, or qsl_in[B] > T_in) sets PSPEC_DEVERR_LAYOUT and
+ * leaves the outputs unspecified but every access in bounds.
+ */
+PSPEC_API pspec_status pspec_build_draft_batch(const pspec_build_args *args, cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+PSPEC_API const char *pspec_status_string(pspec_status status);
+
+/* Number of kernel launches one successful call of each kind issues on its stream:
+   0 = pspec_build_draft_batch, 1 = pspec_verify_greedy, 2 = pspec_verify_rejection;
+   -1 for any other value.  Used to count launches per decode step. */
+PSPEC_API int pspec_launches_per_call(int which);
+
+/* Tuning: force the verify sweeps' segment length (elements of one row handled by one
+   CTA; rounded up to a multiple of 8).  0 restores the automatic choice, which aims at
+   about 32 CTAs per SM and at most 65536 elements per CTA.  The segment length changes
+   pspec_verify_workspace_bytes, so size workspaces after setting it.  Process-wide; not
+   synchronised with calls running on other host threads. */
+PSPEC_API void pspec_set_segment_elems(long long elems);
+
+/* Profiling hook: while `event` is non-NULL, every pspec_verify_rejection call records it
+   on the call's stream between its two launches (after the statistics sweep, before the
+   draw), so that a caller can time each launch with CUDA events.  NULL turns it off.
+   Process-wide; the event is owned by the caller. */
+PSPEC_API void pspec_set_split_event(cudaEvent_t event);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PSPEC_H */

@@ -1,0 +1,15 @@
+"""speculative_decoding_step_pspec_b200 -- the per-step hot path of speculative decoding
+with P-EAGLE parallel drafting on one B200 (sm_100a).
+
+libpspec.so (hand-written CUDA, C ABI in ``include/pspec.h``) does all the work; this
+package is its thin ctypes binding (``_binding``, the C names), allocation helpers
+(``api``) and the seeded synthetic input generators (``inputs``).  Importing it fails if
+the library has not been built: there is no CPU fallback.
+"""
+from ._binding import (  # noqa: F401
+    EXPORTED, LIB, PspecError, library_path, pspec_build_draft_batch,
+    pspec_launches_per_call, pspec_set_segment_elems, pspec_set_split_event,
+    pspec_status_string,
+    pspec_verify_greedy, pspec_verify_rejection, pspec_verify_workspace_bytes,
+)
+from .api import Workspace, build_draft_batch, verify_greedy, verify_rejection  # noqa: F401

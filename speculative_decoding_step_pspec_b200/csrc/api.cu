@@ -1,0 +1,176 @@
+// api.cu -- the C entry points of libpspec: host-side validation, workspace planning and
+// kernel launches.  Every check here runs before any launch; a failed check returns a
+// status and touches no device memory.
+#include <stdint.h>
+#include <stdlib.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+#include "pspec.h"
+
+namespace {
+
+using namespace pspec;
+
+long long g_seg_override = 0;   // 0 = automatic segment length
+cudaEvent_t g_split_event = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t elem_bytes(pspec_dtype d) { return d == PSPEC_BF16 ? 2 : 4; }
+
+bool dtype_ok(pspec_dtype d) { return d == PSPEC_F32 || d == PSPEC_BF16; }
+
+pspec_status check_verify(const pspec_verify_args* a, bool rejection) {
+  if (!a) return PSPEC_ERR_INVALID_ARG;
+  if (a->B < 0 || a->K < 1 || a->V < 1 || a->ld < a->V) return PSPEC_ERR_INVALID_ARG;
+  if (a->K > PSPEC_MAX_K) return PSPEC_ERR_UNSUPPORTED;
+  if (!dtype_ok(a->dtype)) return PSPEC_ERR_INVALID_ARG;
+  if (!a->err) return PSPEC_ERR_INVALID_ARG;
+  if (a->B == 0) return PSPEC_OK;
+  if (!a->target_logits || !a->draft_tokens || !a->out_tokens || !a->accepted_len || !a->bonus)
+    return PSPEC_ERR_INVALID_ARG;
+  if (rejection && (!a->draft_logits || !a->uniforms)) return PSPEC_ERR_INVALID_ARG;
+  const size_t eb = elem_bytes(a->dtype);
+  if (!aligned_to(a->target_logits, eb)) return PSPEC_ERR_INVALID_ARG;
+  if (rejection && !aligned_to(a->draft_logits, eb)) return PSPEC_ERR_INVALID_ARG;
+  // grid size: rows x segments must fit one launch
+  const long long rows = (long long)a->B * (rejection ? 2 * a->K + 1 : a->K + 1);
+  if (rows * ((a->V + kSegMin - 1) / kSegMin) >= 0x7fffffffLL) return PSPEC_ERR_UNSUPPORTED;
+  return PSPEC_OK;
+}
+
+pspec_status check_workspace(void* ws, size_t bytes, const VerifyPlan& p) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < p.bytes)
+    return PSPEC_ERR_WORKSPACE;
+  return PSPEC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection) {
+  if (B < 0 || K < 1 || K > PSPEC_MAX_K || V < 1) return 0;
+  return make_verify_plan(B, K, V, rejection, g_seg_override).bytes;
+}
+
+pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  pspec_status st = check_verify(a, false);
+  if (st != PSPEC_OK || a->B == 0) return st;
+  const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 0, g_seg_override);
+  st = check_workspace(workspace, workspace_bytes, p);
+  if (st != PSPEC_OK) return st;
+  GreedyLaunch L{};
+  L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
+  L.S = p.S; L.seg = p.seg;
+  L.target = a->target_logits;
+  L.draft_tokens = a->draft_tokens;
+  L.out_tokens = a->out_tokens;
+  L.accepted_len = a->accepted_len;
+  L.bonus = a->bonus;
+  L.target_lse = a->target_lse;
+  L.err = a->err;
+  char* ws = static_cast<char*>(workspace);
+  L.cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+  L.part = ws + p.off_part;
+  return launch_greedy(L, stream) == cudaSuccess ? PSPEC_OK : PSPEC_ERR_CUDA;
+}
+
+pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+  pspec_status st = check_verify(a, true);
+  if (st != PSPEC_OK || a->B == 0) return st;
+  const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 1, g_seg_override);
+  st = check_workspace(workspace, workspace_bytes, p);
+  if (st != PSPEC_OK) return st;
+  RejectionLaunch L{};
+  L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
+  L.S = p.S; L.seg = p.seg;
+  L.tiles = p.tiles; L.tiles_per_chunk = p.tiles_per_chunk; L.C = p.C;
+  L.target = a->target_logits;
+  L.draft = a->draft_logits;
+  L.draft_tokens = a->draft_tokens;
+  L.uniforms = a->uniforms;
+  L.out_tokens = a->out_tokens;
+  L.accepted_len = a->accepted_len;
+  L.bonus = a->bonus;
+  L.target_lse = a->target_lse;
+  L.draft_lse = a->draft_lse;
+  L.p_at_draft = a->p_at_draft;
+  L.q_at_draft = a->q_at_draft;
+  L.residual_mass = a->residual_mass;
+  L.err = a->err;
+  char* ws = static_cast<char*>(workspace);
+  L.cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+  L.cnt2 = reinterpret_cast<int*>(ws + p.off_cnt2);
+  L.part = ws + p.off_part;
+  L.seq = ws + p.off_seq;
+  L.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
+  return launch_rejection(L, stream, g_split_event) == cudaSuccess ? PSPEC_OK : PSPEC_ERR_CUDA;
+}
+
+pspec_status pspec_build_draft_batch(const pspec_build_args* a, cudaStream_t stream) {
+  if (!a) return PSPEC_ERR_INVALID_ARG;
+  if (a->B < 0 || a->K < 1 || a->H < 1 || a->block_size < 1 || a->max_blocks < 1 ||
+      a->T_in < 0 || a->T_cap < 0)
+    return PSPEC_ERR_INVALID_ARG;
+  if (a->K > PSPEC_MAX_K) return PSPEC_ERR_UNSUPPORTED;
+  if (!dtype_ok(a->hidden_dtype)) return PSPEC_ERR_INVALID_ARG;
+  if ((long long)a->T_cap < (long long)a->T_in + (long long)a->B * (a->K - 1))
+    return PSPEC_ERR_INVALID_ARG;
+  if (!a->qsl_in || !a->err || !a->draft_tokens || !a->draft_pos || !a->slot_mapping ||
+      !a->row_kind || !a->hidden_src || !a->qsl_out)
+    return PSPEC_ERR_INVALID_ARG;
+  if (a->B > 0 && (!a->verify_tokens || !a->verify_pos || !a->accepted_len || !a->bonus ||
+                   !a->block_table || !a->seq_lens_out || !a->sample_idx))
+    return PSPEC_ERR_INVALID_ARG;
+  const bool hidden = a->draft_hidden != nullptr;
+  if (hidden) {
+    if (!a->h_shared || (a->T_in > 0 && !a->verify_hidden)) return PSPEC_ERR_INVALID_ARG;
+    if (((long long)a->H * (long long)elem_bytes(a->hidden_dtype)) % 16 != 0)
+      return PSPEC_ERR_INVALID_ARG;
+    if (!aligned16(a->draft_hidden) || !aligned16(a->h_shared) ||
+        (a->verify_hidden && !aligned16(a->verify_hidden)))
+      return PSPEC_ERR_INVALID_ARG;
+  }
+  const long long meta_threads = (long long)a->T_cap + a->B + 1;
+  const long long hid_rows = (long long)a->T_in + (long long)a->B * (a->K - 1);
+  if ((meta_threads + kThreads - 1) / kThreads + (hid_rows + kWarps - 1) / kWarps >= 0x7fffffffLL)
+    return PSPEC_ERR_UNSUPPORTED;
+  BuildLaunch L{};
+  L.a = *a;
+  L.row_vecs = (long long)a->H * (long long)elem_bytes(a->hidden_dtype) / 16;
+  L.meta_blocks = (int)((meta_threads + kThreads - 1) / kThreads);
+  L.hid_rows = (int)hid_rows;
+  return launch_build(L, stream) == cudaSuccess ? PSPEC_OK : PSPEC_ERR_CUDA;
+}
+
+const char* pspec_status_string(pspec_status s) {
+  switch (s) {
+    case PSPEC_OK: return "PSPEC_OK";
+    case PSPEC_ERR_INVALID_ARG: return "PSPEC_ERR_INVALID_ARG";
+    case PSPEC_ERR_UNSUPPORTED: return "PSPEC_ERR_UNSUPPORTED";
+    case PSPEC_ERR_CUDA: return "PSPEC_ERR_CUDA";
+    case PSPEC_ERR_WORKSPACE: return "PSPEC_ERR_WORKSPACE";
+  }
+  return "PSPEC_ERR_UNKNOWN";
+}
+
+int pspec_launches_per_call(int which) {
+  switch (which) {
+    case 0: return 1;   // build: one launch, two CTA roles
+    case 1: return 1;   // greedy: one sweep launch
+    case 2: return 2;   // rejection: stats sweep + draw
+  }
+  return -1;
+}
+
+void pspec_set_segment_elems(long long elems) { g_seg_override = elems > 0 ? elems : 0; }
+
+void pspec_set_split_event(cudaEvent_t event) { g_split_event = event; }
+
+}  // extern "C"

@@ -1,0 +1,70 @@
+// kernels.h -- launch descriptors passed by value to the libpspec kernels.
+//
+// The C entry points (api.cu) validate the caller's arguments, build one of these from the
+// argument struct and the workspace plan, and call the matching launcher.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pspec.h"
+
+namespace pspec {
+
+struct GreedyLaunch {
+  int B, K, V;
+  long long ld;
+  pspec_dtype dtype;
+  int S;                 // segments per row
+  long long seg;         // elements per segment
+  const void* target;
+  const int32_t* draft_tokens;
+  int32_t* out_tokens;
+  int32_t* accepted_len;
+  int32_t* bonus;
+  float* target_lse;     // optional
+  int32_t* err;
+  int* cnt;              // workspace: tickets [B]
+  void* part;            // workspace: GreedyPart [B*(K+1)*S]
+};
+
+struct RejectionLaunch {
+  int B, K, V;
+  long long ld;
+  pspec_dtype dtype;
+  int S;
+  long long seg;
+  int tiles, tiles_per_chunk, C;
+  const void* target;
+  const void* draft;
+  const int32_t* draft_tokens;
+  const float* uniforms;
+  int32_t* out_tokens;
+  int32_t* accepted_len;
+  int32_t* bonus;
+  float* target_lse;     // optional
+  float* draft_lse;      // optional
+  float* p_at_draft;     // optional
+  float* q_at_draft;     // optional
+  float* residual_mass;  // optional
+  int32_t* err;
+  int* cnt;              // workspace: sweep tickets [B]
+  int* cnt2;             // workspace: resample tickets [B]
+  void* part;            // workspace: RejPart [B*(2K+1)*S]
+  void* seq;             // workspace: SeqInfo [B]
+  double* tile_sums;     // workspace: [B*tiles]
+};
+
+struct BuildLaunch {
+  pspec_build_args a;
+  long long row_vecs;    // 16-byte vectors per hidden row
+  int meta_blocks;       // CTAs of the metadata role (the rest copy hidden rows)
+  int hid_rows;          // rows the hidden role inspects: T_in + B*(K-1)
+};
+
+cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream);
+// split_event (may be null) is recorded between the statistics sweep and the draw.
+cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream, cudaEvent_t split_event);
+cudaError_t launch_build(const BuildLaunch& L, cudaStream_t stream);
+
+}  // namespace pspec

@@ -1,0 +1,102 @@
+// plan.h -- launch plans and workspace layout of the verify kernels (host + device).
+//
+// A verify call sweeps rows x segments CTAs.  The plan fixes the segment length (a
+// multiple of 8 elements, so every segment starts on a 16-byte boundary for both dtypes),
+// the resample tiling, and the byte offsets of each region of the caller's workspace.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pspec {
+
+constexpr int kNumSMs = 148;             // B200
+constexpr int kTile = 2048;              // resample tile: 256 threads x 8 elements
+constexpr long long kSegMin = 2048;      // one 16-byte vector per thread (bf16)
+constexpr long long kSegMax = 65536;     // bounds the tail of the last wave
+constexpr int kTargetCtas = kNumSMs * 32;
+constexpr int kResampleTargetCtas = kNumSMs * 8;
+constexpr int kTilesPerChunkMax = 8;
+
+// Per-(row, segment) partial of the greedy sweep.
+struct GreedyPart {
+  float v;   // best value
+  int i;     // its token id (kNoIndex when the segment is empty)
+  float m;   // running max of the segment (lse)
+  float s;   // sum of exp(x - m) over the segment (lse)
+};
+
+// Per-(row, segment) partial of the rejection sweep.
+struct RejPart {
+  float m;
+  float s;
+};
+
+// Per-sequence result of the rejection sweep, read by the resample kernel.
+struct SeqInfo {
+  double mt, st;   // max and sum-exp of target row a_i
+  double mq, sq;   // the same for draft row a_i (unused when a_i = K)
+  int a;           // accepted drafts a_i
+  int pad[3];
+};
+
+struct VerifyPlan {
+  int rows;               // rows swept per sequence: K+1 (greedy) or 2K+1 (rejection)
+  int S;                  // segments per row
+  long long seg;          // elements per segment
+  int tiles;              // resample tiles per row
+  int tiles_per_chunk;    // resample tiles per CTA
+  int C;                  // resample CTAs per sequence
+  size_t off_cnt;         // int32[B]  sweep tickets
+  size_t off_cnt2;        // int32[B]  resample tickets
+  size_t off_part;        // partials [B*rows*S]
+  size_t off_seq;         // SeqInfo[B]
+  size_t off_tiles;       // double[B*tiles]
+  size_t bytes;           // total
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// seg_override > 0 forces the segment length (rounded up to a multiple of 8).
+inline VerifyPlan make_verify_plan(int B, int K, int V, int rejection, long long seg_override) {
+  VerifyPlan p{};
+  p.rows = rejection ? 2 * K + 1 : K + 1;
+  long long rows_total = (long long)B * p.rows;
+  long long s_lo = (V + kSegMax - 1) / kSegMax;
+  long long s_hi = (V + kSegMin - 1) / kSegMin;
+  if (s_hi < 1) s_hi = 1;
+  long long S = rows_total > 0 ? (kTargetCtas + rows_total - 1) / rows_total : 1;
+  if (S < s_lo) S = s_lo;
+  if (S > s_hi) S = s_hi;
+  if (S < 1) S = 1;
+  long long seg = (V + S - 1) / S;
+  if (seg_override > 0) seg = seg_override;
+  seg = (seg + 7) / 8 * 8;
+  p.seg = seg;
+  p.S = (int)((V + seg - 1) / seg);
+  p.tiles = (V + kTile - 1) / kTile;
+  int C = B > 0 ? (kResampleTargetCtas + B - 1) / B : 1;
+  int c_lo = (p.tiles + kTilesPerChunkMax - 1) / kTilesPerChunkMax;
+  if (C < c_lo) C = c_lo;
+  if (C > p.tiles) C = p.tiles;
+  if (C < 1) C = 1;
+  p.tiles_per_chunk = (p.tiles + C - 1) / C;
+  p.C = (p.tiles + p.tiles_per_chunk - 1) / p.tiles_per_chunk;
+
+  size_t off = 0;
+  p.off_cnt = off;
+  off = align256(off + sizeof(int32_t) * (size_t)B);
+  p.off_cnt2 = off;
+  off = align256(off + (rejection ? sizeof(int32_t) * (size_t)B : 0));
+  p.off_part = off;
+  size_t part_sz = rejection ? sizeof(RejPart) : sizeof(GreedyPart);
+  off = align256(off + part_sz * (size_t)B * p.rows * p.S);
+  p.off_seq = off;
+  off = align256(off + (rejection ? sizeof(SeqInfo) * (size_t)B : 0));
+  p.off_tiles = off;
+  off = align256(off + (rejection ? sizeof(double) * (size_t)B * p.tiles : 0));
+  p.bytes = off;
+  return p;
+}
+
+}  // namespace pspec

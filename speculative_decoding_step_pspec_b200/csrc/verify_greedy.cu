@@ -1,0 +1,178 @@
+// verify_greedy.cu -- greedy target verification (one launch).
+//
+// "Any accepted prefix replaces the greedy path" ("Capstone 14: speculative decoding
+// inference server", section "Concept"): for each sequence the target's argmax over the
+// vocabulary is taken on each of its K+1 rows, the accepted prefix is the run of leading
+// drafts equal to it, and the token after the prefix is the argmax of the next row.
+//
+// Design: the grid is B*(K+1) rows x S segments, one CTA per segment, 16-byte streaming
+// loads with four vectors in flight per thread.  The bf16 max of each vector is taken
+// on packed pairs (max.bf16x2), and only a vector that beats the running best is
+// unpacked to find the first position of its maximum.  Each CTA writes one partial;
+// an atomic ticket per sequence elects the CTA that finishes the sequence last, and that
+// CTA merges the partials in segment order (deterministic, lowest id wins ties) and
+// writes the accepted length, the bonus token and the output tokens.  No CTA waits.
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+
+namespace pspec {
+
+namespace {
+
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ float vec_max(const uint4& v, BF16Tag) {
+  uint32_t m = bmax2(bmax2(v.x, v.y), bmax2(v.z, v.w));
+  return fmaxf(bf16_lo(m), bf16_hi(m));
+}
+__device__ __forceinline__ float vec_max(const uint4& v, F32Tag) {
+  return fmaxf(fmaxf(__uint_as_float(v.x), __uint_as_float(v.y)),
+               fmaxf(__uint_as_float(v.z), __uint_as_float(v.w)));
+}
+
+template <typename Tag, bool kLse>
+__device__ __forceinline__ void consume(const uint4& v, long long idx0, VI& best, MS& ms) {
+  constexpr int W = Tag::kVec;
+  float vmax = vec_max(v, Tag{});
+  if (kLse || vmax > best.v) {
+    float x[W];
+    unpack(v, x, Tag{});
+    if (vmax > best.v) {
+      int j = 0;
+#pragma unroll
+      for (int t = W - 1; t >= 0; --t)
+        if (x[t] == vmax) j = t;
+      best.v = vmax;
+      best.i = (int)(idx0 + j);
+    }
+    if (kLse && vmax != -INFINITY) {
+      if (vmax > ms.m) {
+        ms.s = ms.m == -INFINITY ? 0.f : ms.s * ex2((ms.m - vmax) * kLog2e);
+        ms.m = vmax;
+      }
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < W; ++t) acc += ex2((x[t] - ms.m) * kLog2e);
+      ms.s += acc;
+    }
+  }
+}
+
+template <typename Tag, bool kLse>
+__global__ void __launch_bounds__(kThreads)
+greedy_sweep_kernel(const GreedyLaunch L) {
+  using elem = typename Tag::elem;
+  const long long item = blockIdx.x;
+  const int s = (int)(item % L.S);
+  const long long rowg = item / L.S;                 // i*(K+1) + k
+  const int i = (int)(rowg / (L.K + 1));
+  const elem* row = static_cast<const elem*>(L.target) + rowg * L.ld;
+  const long long lo = (long long)s * L.seg;
+  const long long hi = min((long long)L.V, lo + L.seg);
+
+  VI best{-INFINITY, kNoIndex};
+  MS ms{-INFINITY, 0.f};
+  sweep_segment<Tag, 4>(
+      row, lo, hi,
+      [&](const uint4& v, long long idx0) { consume<Tag, kLse>(v, idx0, best, ms); },
+      [&](float x, long long t) {
+        if (x > best.v) { best.v = x; best.i = (int)t; }
+        if (kLse && x != -INFINITY) ms = ms_merge(ms, MS{x, 1.f});
+      });
+
+  // CTA reduction
+  __shared__ VI s_vi[kWarps];
+  __shared__ MS s_ms[kWarps];
+  __shared__ int s_last;
+  best = warp_argmax(best);
+  if (kLse) ms = warp_merge_ms(ms);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) { s_vi[warp] = best; s_ms[warp] = ms; }
+  __syncthreads();
+  if (warp == 0) {
+    best = lane < kWarps ? s_vi[lane] : VI{-INFINITY, kNoIndex};
+    ms = lane < kWarps ? s_ms[lane] : MS{-INFINITY, 0.f};
+    best = warp_argmax(best);
+    if (kLse) ms = warp_merge_ms(ms);
+    if (lane == 0) {
+      GreedyPart* part = reinterpret_cast<GreedyPart*>(L.part);
+      part[item] = GreedyPart{best.v, best.i, ms.m, ms.s};
+      __threadfence();
+      int t = atomicAdd(L.cnt + i, 1);
+      s_last = (t == L.S * (L.K + 1) - 1);
+    }
+  }
+  __syncthreads();
+  if (!s_last) return;
+
+  // This CTA finished sequence i last: merge its (K+1) x S partials in segment order.
+  __threadfence();
+  if (warp != 0) return;
+  const int K = L.K;
+  const GreedyPart* part =
+      reinterpret_cast<const GreedyPart*>(L.part) + (long long)i * (K + 1) * L.S;
+  int g = 0;          // argmax of row `lane`
+  double lse = 0.0;
+  if (lane <= K) {
+    VI b{-INFINITY, kNoIndex};
+    float M = -INFINITY;
+    for (int t = 0; t < L.S; ++t) {
+      GreedyPart q = ld_cg(part + (long long)lane * L.S + t);
+      if (q.v > b.v) b = VI{q.v, q.i};
+      M = fmaxf(M, q.m);
+    }
+    g = b.i == kNoIndex ? 0 : b.i;       // a row of -inf / NaN only: token 0
+    if (kLse) {
+      double S = 0.0;
+      if (M != -INFINITY)
+        for (int t = 0; t < L.S; ++t) {
+          GreedyPart q = ld_cg(part + (long long)lane * L.S + t);
+          if (q.m != -INFINITY) S += (double)q.s * exp((double)q.m - (double)M);
+        }
+      lse = M == -INFINITY ? -INFINITY : (double)M + log(S);
+    }
+  }
+  int d = -1;
+  bool bad = false;
+  if (lane < K) {
+    d = L.draft_tokens[(long long)i * K + lane];
+    bad = d < 0 || d >= L.V;
+  }
+  unsigned match = __ballot_sync(0xffffffffu, lane < K && !bad && d == g);
+  unsigned anybad = __ballot_sync(0xffffffffu, bad);
+  int a = __ffs(~match) - 1;             // first mismatch
+  if (a > K) a = K;
+  int bonus = __shfl_sync(0xffffffffu, g, a);
+  if (lane <= K) {
+    L.out_tokens[(long long)i * (K + 1) + lane] = lane < a ? d : (lane == a ? bonus : -1);
+    if (kLse) L.target_lse[(long long)i * (K + 1) + lane] = (float)lse;
+  }
+  if (lane == 0) {
+    L.accepted_len[i] = a;
+    L.bonus[i] = bonus;
+    if (anybad) set_err(L.err, PSPEC_DEVERR_TOKEN_RANGE);
+    L.cnt[i] = 0;                        // ticket back to zero for the next call
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream) {
+  const long long grid = (long long)L.B * (L.K + 1) * L.S;
+  const bool lse = L.target_lse != nullptr;
+  if (L.dtype == PSPEC_BF16) {
+    if (lse) greedy_sweep_kernel<BF16Tag, true><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+    else greedy_sweep_kernel<BF16Tag, false><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+  } else {
+    if (lse) greedy_sweep_kernel<F32Tag, true><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+    else greedy_sweep_kernel<F32Tag, false><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pspec

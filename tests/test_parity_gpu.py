@@ -1,0 +1,372 @@
+"""GPU parity: libpspec's kernels (through the C ABI) against the CPU oracle.
+
+Every workload runs at its full size in the launch configuration the benchmark uses; the
+oracle checks all sequences where it finishes in seconds and a seeded sample otherwise,
+and invariants that hold at any size are checked on every sequence.  Smaller cases cover
+several segments and tiles with ragged tails, padded row strides, the edge cases (K = 1,
+K = 31, V < one vector, -inf rows, out-of-range tokens, empty batches) and determinism.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import speculative_decoding_step_pspec_b200 as ps
+from speculative_decoding_step_pspec_b200 import inputs as I
+from tests import parity_util as U
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _sample(B, n, seed):
+    if B <= n:
+        return np.arange(B)
+    return np.sort(np.random.default_rng(seed).choice(B, size=n, replace=False))
+
+
+def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True):
+    V = target.shape[2]
+    gr = ps.verify_greedy(target, greedy_drafts, want_lse=diag)
+    rj = ps.verify_rejection(target, draft, sampled, u, diagnostics=diag)
+    torch.cuda.synchronize()
+    U.check_verify_invariants(gr, greedy_drafts, V)
+    U.check_verify_invariants(rj, sampled, V)
+    og = U.oracle_greedy(target, greedy_drafts, seqs)
+    U.compare_greedy(gr, og, seqs)
+    orj = U.oracle_rejection(target, draft, sampled, u, seqs)
+    flagged = U.compare_rejection(rj, orj, seqs)
+    n = len(orj["flags"])
+    assert flagged <= max(1, n // 100), f"{flagged} of {n} sequences flagged as near-ties"
+    return gr, rj, orj
+
+
+# --------------------------------------------------------------------------- workloads
+def test_tiny_workload():
+    t = I.tiny_verify_numpy()
+    target = torch.from_numpy(t["target"]).to(DEV)
+    draft = torch.from_numpy(t["draft"]).to(DEV)
+    d = torch.from_numpy(t["draft_tokens"]).to(DEV)
+    u = torch.from_numpy(t["uniforms"]).to(DEV)
+    _verify_both(target, draft, d, d, u)
+    inp = I.build_inputs(I.TINY, DEV, ctx=t["ctx"], a_prev=t["a_prev"])
+    _build_and_compare(inp)
+
+
+@pytest.mark.parametrize("name", ["c1", "c64"])
+def test_workload_all_sequences(name):
+    w = I.WORKLOADS[name]
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    _verify_both(target, draft, sampled, greedy, u)
+    if name == "c64":   # the stated drafts are sampled for both modes at c=64
+        gr = ps.verify_greedy(target, sampled)
+        U.compare_greedy(gr, U.oracle_greedy(target, sampled, want_lse=False))
+    inp = I.build_inputs(w, DEV, drafts=sampled)
+    _build_and_compare(inp)
+
+
+def test_b1024_sampled():
+    w = I.B1024
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    seqs = _sample(w.B, 48, 7)
+    _, rj, _ = _verify_both(target, draft, sampled, greedy, u, seqs=seqs)
+    # the step chains: this verify's accepted counts and bonus tokens feed the build
+    inp = I.build_inputs(w, DEV, drafts=sampled)
+    inp["accepted_len"] = rj["accepted_len"].clone()
+    inp["bonus"] = rj["bonus"].clone()
+    _build_and_compare(inp)
+
+
+@pytest.mark.parametrize("K", I.DEPTH_K)
+@pytest.mark.parametrize("sigma", I.DEPTH_SIGMA)
+def test_depth_sweep_sampled(K, sigma):
+    w = I.depth(K, sigma)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    _verify_both(target, draft, sampled, greedy, u, seqs=_sample(w.B, 12, K))
+    _build_and_compare(I.build_inputs(w, DEV, drafts=sampled))
+
+
+# --------------------------------------------------------------------------- shapes
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("V,seg", [(1, 0), (7, 0), (8, 0), (2047, 0), (5003, 1024), (70001, 4096),
+                                   (70001, 0)])
+@pytest.mark.parametrize("K", [1, 4])
+def test_ragged_multi_segment(dtype, V, seg, K):
+    B = 5
+    w = I.Workload("t", B, K, V, 16, 4, dtype, seed=V + K, sigma_t=2.0, sigma_d=0.6)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    ps.pspec_set_segment_elems(seg)
+    try:
+        _verify_both(target, draft, sampled, greedy, u)
+    finally:
+        ps.pspec_set_segment_elems(0)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_padded_row_stride(dtype):
+    B, K, V = 6, 3, 3001
+    ld = 3008 if dtype == torch.bfloat16 else 3004
+    w = I.Workload("t", B, K, V, 16, 4, dtype, seed=3, sigma_t=2.0, sigma_d=0.6)
+    t0, q0 = I.logits(w, DEV)
+    tb = torch.full((B, K + 1, ld), 99.0, dtype=dtype, device=DEV)
+    qb = torch.full((B, K, ld), -99.0, dtype=dtype, device=DEV)
+    tb[:, :, :V] = t0
+    qb[:, :, :V] = q0
+    target, draft = tb[:, :, :V], qb[:, :, :V]            # views: row stride ld > V
+    sampled, greedy = I.draft_tokens(w, q0)
+    u = I.uniforms(w, DEV)
+    gr = ps.verify_greedy(target, greedy, want_lse=True)
+    rj = ps.verify_rejection(target, draft, sampled, u, diagnostics=True)
+    U.compare_greedy(gr, U.oracle_greedy(t0, greedy))
+    U.compare_rejection(rj, U.oracle_rejection(t0, q0, sampled, u))
+
+
+def test_max_K():
+    w = I.Workload("t", 3, 31, 300, 16, 4, torch.bfloat16, seed=31, sigma_t=1.0, sigma_d=0.05)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    _verify_both(target, draft, sampled, greedy, u)
+    # identical drafts pass all 31 positions
+    rj = ps.verify_rejection(target, target[:, :31].contiguous(), sampled, u)
+    assert (rj["accepted_len"].cpu() == 31).all()
+    gr = ps.verify_greedy(target, target[:, :31].float().argmax(-1).int())
+    assert (gr["accepted_len"].cpu() == 31).all()
+
+
+def test_neg_inf_rows_and_entries():
+    B, K, V = 6, 2, 4000
+    g = torch.Generator(device=DEV).manual_seed(9)
+    target = torch.randn((B, K + 1, V), generator=g, device=DEV) * 2
+    draft = target[:, :K] + torch.randn((B, K, V), generator=g, device=DEV)
+    target[0, 0, :] = -float("inf")                       # a row with no mass at all
+    target[1, :, ::3] = -float("inf")                     # masked vocabulary entries
+    draft[1, :, 1::3] = -float("inf")
+    draft[2, 1, :] = -float("inf")
+    target[3, 0, 17] = -float("inf")
+    d = torch.randint(0, V, (B, K), generator=g, device=DEV, dtype=torch.int32)
+    d[3, 0] = 17                                          # p(d) = 0: always rejected
+    u = torch.rand((B, K + 1), generator=g, device=DEV)
+    gr = ps.verify_greedy(target, d, want_lse=True)
+    rj = ps.verify_rejection(target, draft, d, u, diagnostics=True)
+    U.compare_greedy(gr, U.oracle_greedy(target, d))
+    U.compare_rejection(rj, U.oracle_rejection(target, draft, d, u))
+    assert rj["accepted_len"][3].item() == 0
+
+
+def test_out_of_range_draft_tokens():
+    w = I.Workload("t", 4, 3, 1000, 16, 4, torch.bfloat16, seed=4, sigma_t=2.0, sigma_d=0.1)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    bad = greedy.clone()
+    bad[0, 0] = -1
+    bad[2, 1] = w.V
+    gr = ps.verify_greedy(target, bad)
+    rj = ps.verify_rejection(target, draft, bad, u, diagnostics=True)
+    assert gr["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
+    assert rj["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
+    U.compare_greedy(gr, U.oracle_greedy(target, bad, want_lse=False))
+    U.compare_rejection(rj, U.oracle_rejection(target, draft, bad, u))
+    assert gr["accepted_len"][0].item() == 0 and rj["accepted_len"][0].item() == 0
+
+
+def test_determinism_and_workspace_reuse():
+    w = I.scaled(I.C64, B=16, V=50000)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    ws = ps.Workspace(w.B, w.K, w.V, True)
+    outs = [ps.verify_rejection(target, draft, sampled, u, diagnostics=True, workspace=ws)
+            for _ in range(3)]
+    for o in outs[1:]:
+        for k in o:
+            assert torch.equal(o[k], outs[0][k]), k
+    # the counters left at zero serve a smaller batch next
+    r = ps.verify_rejection(target[:5], draft[:5], sampled[:5], u[:5], workspace=ws)
+    for k in ("out_tokens", "accepted_len", "bonus"):
+        assert torch.equal(r[k], outs[0][k][:5]), k
+    wsg = ps.Workspace(w.B, w.K, w.V, False)
+    g1 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
+    g2 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_empty_batch():
+    t = torch.empty((0, 4, 100), dtype=torch.bfloat16, device=DEV)
+    q = torch.empty((0, 3, 100), dtype=torch.bfloat16, device=DEV)
+    d = torch.empty((0, 3), dtype=torch.int32, device=DEV)
+    u = torch.empty((0, 4), dtype=torch.float32, device=DEV)
+    ps.verify_greedy(t, d)
+    ps.verify_rejection(t, q, d, u)
+    torch.cuda.synchronize()
+
+
+# --------------------------------------------------------------------------- exactness
+def test_threshold_probing_exact_rule():
+    """The kernel's accept decisions flip exactly at tau = min(1, p/q) and its draws follow
+    the residual's CDF: u = tau - 2e-6 accepts, tau + 2e-6 rejects, and u at the middle of
+    each CDF interval returns that interval's token (V = 8, K = 2, all 64 draft tuples)."""
+    from tests.oracle_pins import _prefix_logits
+    import itertools
+    import scipy.special as sps
+    V, K = 8, 2
+    tuples = list(itertools.product(range(V), repeat=K))
+    t = np.stack([np.stack([_prefix_logits(tp[:k], V, 1) for k in range(K + 1)]) for tp in tuples])
+    q = np.stack([np.stack([_prefix_logits(tp[:k], V, 2) for k in range(K)]) for tp in tuples])
+    d = np.array(tuples, np.int32)
+    P = sps.softmax(t.astype(np.float64), axis=2)
+    Q = sps.softmax(q.astype(np.float64), axis=2)
+    rows_t, rows_q, rows_d, rows_u, expect_a, expect_tok = [], [], [], [], [], []
+    for n in range(len(tuples)):
+        for k in range(K):
+            tau = min(1.0, P[n, k, d[n, k]] / Q[n, k, d[n, k]])
+            for du, acc in ((-2e-6, True), (2e-6, False)):
+                uu = tau + du
+                if not (0.0 <= uu < 1.0):
+                    continue
+                u = np.zeros(K + 1, np.float32)
+                u[k] = uu
+                rows_t.append(t[n]); rows_q.append(q[n]); rows_d.append(d[n]); rows_u.append(u)
+                expect_a.append((k, acc)); expect_tok.append(-1)
+            # draws after a rejection at k
+            if tau < 1.0 - 1e-5:
+                r = np.maximum(P[n, k] - Q[n, k], 0.0)
+                F = np.concatenate([[0.0], np.cumsum(r) / r.sum()])
+                for tok in range(V):
+                    if F[tok + 1] - F[tok] < 1e-5:
+                        continue
+                    u = np.zeros(K + 1, np.float32)
+                    u[k] = np.nextafter(np.float32(1), np.float32(0))
+                    u[K] = (F[tok] + F[tok + 1]) / 2
+                    rows_t.append(t[n]); rows_q.append(q[n]); rows_d.append(d[n]); rows_u.append(u)
+                    expect_a.append((k, False)); expect_tok.append(tok)
+        # the bonus draw after K acceptances follows p_K
+        F = np.concatenate([[0.0], np.cumsum(P[n, K])])
+        for tok in range(V):
+            if F[tok + 1] - F[tok] < 1e-5:
+                continue
+            u = np.zeros(K + 1, np.float32)
+            u[K] = (F[tok] + F[tok + 1]) / 2
+            rows_t.append(t[n]); rows_q.append(q[n]); rows_d.append(d[n]); rows_u.append(u)
+            expect_a.append((K, None)); expect_tok.append(tok)
+    T = torch.from_numpy(np.stack(rows_t)).to(DEV)
+    Qd = torch.from_numpy(np.stack(rows_q)).to(DEV)
+    D = torch.from_numpy(np.stack(rows_d)).to(DEV)
+    Uu = torch.from_numpy(np.stack(rows_u)).to(DEV)
+    r = ps.verify_rejection(T, Qd, D, Uu)
+    a = r["accepted_len"].cpu().numpy()
+    bonus = r["bonus"].cpu().numpy()
+    o = oracle.verify_rejection(np.stack(rows_t), np.stack(rows_q), np.stack(rows_d), np.stack(rows_u))
+    for n, ((k, acc), tok) in enumerate(zip(expect_a, expect_tok)):
+        if acc is True:
+            assert a[n] > k, n
+        elif acc is False:
+            assert a[n] == k, n
+        else:
+            assert a[n] == K, n
+        if tok >= 0:
+            assert bonus[n] == tok, (n, bonus[n], tok)
+            assert o["bonus"][n] == tok
+    assert np.array_equal(a, o["accepted_len"])
+
+
+# --------------------------------------------------------------------------- build
+def _build_and_compare(inp, check_hidden=True):
+    dh = U.hidden_sentinel(inp["T_cap"], inp["H"], inp["verify_hidden"].dtype, DEV)
+    init = dh.view(torch.int16).cpu().numpy() if dh.dtype == torch.bfloat16 else dh.cpu().numpy()
+    out = ps.api.build_outputs(inp["B"], inp["K"], inp["H"], inp["T_cap"], dh.dtype, DEV)
+    out["draft_hidden"] = dh
+    g = ps.build_draft_batch(
+        K=inp["K"], block_size=inp["block_size"], mask_id=inp["mask_id"], pad_id=inp["pad_id"],
+        T_cap=inp["T_cap"], qsl_in=inp["qsl_in"], verify_tokens=inp["verify_tokens"],
+        verify_pos=inp["verify_pos"], accepted_len=inp["accepted_len"], bonus=inp["bonus"],
+        block_table=inp["block_table"], verify_hidden=inp["verify_hidden"],
+        h_shared=inp["h_shared"], out=out)
+    torch.cuda.synchronize()
+    o = U.oracle_build(inp, init)
+    U.compare_build(g, o, check_hidden)
+    return g, o
+
+
+def _torchify(case, dtype=torch.bfloat16):
+    def i32(x):
+        return torch.as_tensor(np.asarray(x, np.int32), device=DEV)
+    B = len(case["qsl_in"]) - 1
+    return dict(B=B, K=case["K"], H=case["verify_hidden"].shape[1], block_size=case["block_size"],
+                mask_id=case["mask_id"], pad_id=case["pad_id"], T_cap=case["T_cap"],
+                qsl_in=i32(case["qsl_in"]), verify_tokens=i32(case["verify_tokens"]),
+                verify_pos=i32(case["verify_pos"]), accepted_len=i32(case["accepted_len"]),
+                bonus=i32(case["bonus"]), block_table=i32(case["block_table"]),
+                verify_hidden=torch.from_numpy(case["verify_hidden"]).to(DEV).to(dtype),
+                h_shared=torch.from_numpy(case["h_shared"]).to(DEV).to(dtype))
+
+
+@pytest.mark.parametrize("K,L_extra,bs,H", [(1, 0, 4, 8), (3, 0, 4, 16), (7, 0, 16, 64),
+                                            (4, 5, 8, 24), (31, 2, 16, 8), (7, 40, 16, 2880)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_build_random_layouts(K, L_extra, bs, H, dtype):
+    from tests.oracle_pins import random_build_case
+    rng = np.random.default_rng(K * 100 + L_extra)
+    case = random_build_case(rng, B=37, K=K, H=H, bs=bs, L_extra=L_extra)
+    _build_and_compare(_torchify(case, dtype))
+
+
+def test_build_worked_example_on_gpu():
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "build_worked_example.json")))
+    case = dict(g, verify_hidden=np.arange(8 * 8, dtype=np.float32).reshape(8, 8),
+                h_shared=np.full(8, -1.0, np.float32))
+    out, _ = _build_and_compare(_torchify(case, torch.float32))
+    for k, v in g["expect"].items():
+        assert out[k].cpu().numpy().tolist() == v, k
+
+
+def test_build_invalid_values():
+    from tests.oracle_pins import random_build_case
+    rng = np.random.default_rng(22)
+    case = random_build_case(rng, B=6, K=3, H=8, bs=4)
+    _build_and_compare(_torchify(dict(case, accepted_len=np.array([-2, 0, 1, 9, 3, 2]))))
+    t = case["block_table"].copy()
+    t[2, :] = -1
+    _build_and_compare(_torchify(dict(case, block_table=t)))
+    p = case["verify_pos"].copy()
+    p[5] = -4
+    p[9] = 10 ** 6
+    _build_and_compare(_torchify(dict(case, verify_pos=p)))
+    q = np.array(case["qsl_in"]).copy()
+    q[2] = q[1] + 2                  # a sequence with fewer than K+1 rows
+    _build_and_compare(_torchify(dict(case, qsl_in=q)))
+    q = np.array(case["qsl_in"]).copy()
+    q[3] = q[2] - 1                  # not an offset array: only the error bit is defined
+    inp = _torchify(dict(case, qsl_in=q))
+    out = ps.build_draft_batch(K=3, block_size=4, mask_id=inp["mask_id"], pad_id=inp["pad_id"],
+                               T_cap=inp["T_cap"], qsl_in=inp["qsl_in"],
+                               verify_tokens=inp["verify_tokens"], verify_pos=inp["verify_pos"],
+                               accepted_len=inp["accepted_len"], bonus=inp["bonus"],
+                               block_table=inp["block_table"], verify_hidden=inp["verify_hidden"],
+                               h_shared=inp["h_shared"])
+    assert out["err"].item() & ps._binding.PSPEC_DEVERR_LAYOUT
+
+
+def test_build_empty_batch_pads():
+    inp = dict(B=0, K=3, H=8, block_size=4, mask_id=5, pad_id=6, T_cap=10,
+               qsl_in=torch.zeros(1, dtype=torch.int32, device=DEV),
+               verify_tokens=torch.zeros(0, dtype=torch.int32, device=DEV),
+               verify_pos=torch.zeros(0, dtype=torch.int32, device=DEV),
+               accepted_len=torch.zeros(0, dtype=torch.int32, device=DEV),
+               bonus=torch.zeros(0, dtype=torch.int32, device=DEV),
+               block_table=torch.zeros((1, 1), dtype=torch.int32, device=DEV),
+               verify_hidden=torch.zeros((0, 8), dtype=torch.float32, device=DEV),
+               h_shared=torch.zeros(8, dtype=torch.float32, device=DEV))
+    _build_and_compare(inp)
