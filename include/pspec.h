@@ -211,6 +211,32 @@ typedef struct {
 } pspec_build_args;
 
 /*
+ * Greedy verification with no allocation by anyone (the pages have no counterpart: this
+ * serves callers that cannot provide device memory).  Some callers cannot hand this
+ * library a workspace: a serving engine that reserves nearly all HBM for its KV cache at
+ * start-up and gives memory out only through its own pool, a program that links only this
+ * C library and has no device allocator, or a latency-critical path that cannot afford
+ * cudaMalloc's implicit device synchronisation.  This entry point computes exactly what
+ * pspec_verify_greedy computes (same kernel, same outputs) but keeps its scratch in a
+ * fixed array of PSPEC_NOALLOC_SCRATCH_BYTES inside the library's device image, so neither
+ * side calls cudaMalloc, cudaFree or any allocating routine.
+ *   - Every GPU that loads the library holds that array until the process exits.
+ *   - The first call on a device (with that device current) looks up the array's device
+ *     address, once per device; make that first call before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's contents: each
+ *     call clears its tickets first (an asynchronous memset on `stream`), and calls whose
+ *     executions overlap on the GPU race on it, so order them (one stream, or events).
+ *   - It always uses the automatic segment length (pspec_set_segment_elems does not apply).
+ *     A call needs pspec_verify_workspace_bytes(B, K, V, 0) bytes with the automatic
+ *     segment length; above PSPEC_NOALLOC_SCRATCH_BYTES it returns PSPEC_ERR_UNSUPPORTED
+ *     and launches nothing (B = 1024, K = 7, V = 201088 needs about 0.5 MiB).
+ * Arguments, layout, outputs and device error bits are those of pspec_verify_greedy.
+ */
+#define PSPEC_NOALLOC_SCRATCH_BYTES (4u << 20)
+PSPEC_API pspec_status pspec_verify_greedy_noalloc(const pspec_verify_args *args,
+                                                   cudaStream_t stream);
+
+/*
  * Parallel-draft batch construction: one launch.  Its CTAs take one of two roles: the
  * metadata role writes every per-row and per-sequence output, the hidden role copies the
  * CTX/NTP hidden rows and broadcasts h_shared into the MASK rows with 16-byte stores.

@@ -26,7 +26,7 @@ PSPEC_MAX_K = 31
 EXPORTED = (
     "pspec_verify_workspace_bytes", "pspec_verify_greedy", "pspec_verify_rejection",
     "pspec_build_draft_batch", "pspec_status_string", "pspec_launches_per_call",
-    "pspec_set_segment_elems", "pspec_set_split_event",
+    "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
 )
 
 
@@ -248,3 +248,26 @@ def pspec_build_draft_batch(*, K, block_size, mask_id, pad_id, T_cap, qsl_in, ve
     st = LIB.pspec_build_draft_batch(ctypes.byref(a), _stream(stream))
     if st != PSPEC_OK:
         raise PspecError("pspec_build_draft_batch", st)
+
+
+_NOALLOC_SIGNATURE_SET = False
+
+
+def pspec_verify_greedy_noalloc(*, target_logits, draft_tokens, out_tokens, accepted_len, bonus,
+                                err, target_lse=None, stream=None) -> None:
+    """Greedy verify with the library's own fixed scratch: for callers that cannot hand the
+    library a workspace (their device memory is all reserved up front, or they have no
+    device allocator).  Same arguments and outputs as pspec_verify_greedy minus the
+    workspace; raises PspecError (PSPEC_ERR_UNSUPPORTED) when the call needs more than the
+    fixed scratch."""
+    global _NOALLOC_SIGNATURE_SET
+    if not _NOALLOC_SIGNATURE_SET:
+        LIB.pspec_verify_greedy_noalloc.argtypes = [ctypes.POINTER(pspec_verify_args), _P]
+        LIB.pspec_verify_greedy_noalloc.restype = _I
+        _NOALLOC_SIGNATURE_SET = True
+    K = int(target_logits.shape[1]) - 1
+    a = _verify_args(target_logits, None, draft_tokens, None, out_tokens, accepted_len, bonus,
+                     err, target_lse, None, None, None, None, K)
+    st = LIB.pspec_verify_greedy_noalloc(ctypes.byref(a), _stream(stream))
+    if st != PSPEC_OK:
+        raise PspecError("pspec_verify_greedy_noalloc", st)
