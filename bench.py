@@ -48,6 +48,8 @@ def parse_args():
     p.add_argument("--cpu-sample", type=int, default=192,
                    help="sequences of the workload the CPU oracle baseline verifies")
     p.add_argument("--workload", default="b1024", help="b1024 (default), c64 or c1")
+    p.add_argument("--build-only", action="store_true",
+                   help="time the draft-batch construction alone (profiling aid: no logits)")
     return p.parse_args()
 
 
@@ -450,6 +452,50 @@ def cpu_baseline(args, w, d, acc):
                       f"{threads} threads"}
 
 
+def run_build_only(args, local_rank):
+    """The draft-batch construction alone on the workload's shapes (accepted counts drawn
+    by the input generator): a profiling aid that holds only the build's buffers."""
+    import torch
+
+    import speculative_decoding_step_pspec_b200 as ps
+    from speculative_decoding_step_pspec_b200 import inputs as I
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = dict(b1024=I.B1024, c64=I.C64, c1=I.C1)[args.workload]
+    bi = I.build_inputs(w, dev)
+    out = ps.api.build_outputs(w.B, w.K, w.H, bi["T_cap"], bi["verify_hidden"].dtype, dev)
+
+    def build():
+        ps.build_draft_batch(K=w.K, block_size=w.block_size, mask_id=bi["mask_id"],
+                             pad_id=bi["pad_id"], T_cap=bi["T_cap"], qsl_in=bi["qsl_in"],
+                             verify_tokens=bi["verify_tokens"], verify_pos=bi["verify_pos"],
+                             accepted_len=bi["accepted_len"], bonus=bi["bonus"],
+                             block_table=bi["block_table"], verify_hidden=bi["verify_hidden"],
+                             h_shared=bi["h_shared"], out=out)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2: evict between steps
+    for _ in range(max(3, args.warmup)):
+        build()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        build()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    _, bbytes = algorithmic_bytes(w, "greedy", bi["accepted_len"].cpu().numpy())
+    ms = statistics.median(times)
+    hbm, _ = peaks()
+    print(json.dumps({"metric": "draft-batch build alone (L2 flushed between launches)",
+                      "workload": args.workload, "ms_median": round(ms, 5),
+                      "ms_p10": round(sorted(times)[len(times) // 10], 5),
+                      "algorithmic_bytes": int(bbytes), "gbs": round(bbytes / (ms * 1e-3) / 1e9, 1),
+                      "frac_of_peak": round(bbytes / (ms * 1e-3) / 1e9 / hbm, 4),
+                      "err": int(out["err"].item())}), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, rank):
     """The CPU oracle as the reference arm: each step verifies a rotating bounded sample of
@@ -527,7 +573,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_pspec(args, rank, world, local_rank)
+        if args.build_only:
+            run_build_only(args, local_rank)
+        else:
+            run_pspec(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()

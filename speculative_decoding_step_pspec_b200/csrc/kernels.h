@@ -52,7 +52,7 @@ struct RejectionLaunch {
   int* cnt2;             // workspace: resample tickets [B]
   void* part;            // workspace: RejPart [B*(2K+1)*S]
   void* seq;             // workspace: SeqInfo [B]
-  double* tile_sums;     // workspace: [B*tiles]
+  double* tile_sums;     // workspace: [B*tiles] sums of r over 256-element tiles
 };
 
 struct BuildLaunch {

@@ -11,12 +11,12 @@
 namespace pspec {
 
 constexpr int kNumSMs = 148;             // B200
-constexpr int kTile = 2048;              // resample tile: 256 threads x 8 elements
+constexpr int kDrawTile = 256;           // draw tile: one warp, 32 lanes x 8 elements
 constexpr long long kSegMin = 2048;      // one 16-byte vector per thread (bf16)
 constexpr long long kSegMax = 65536;     // bounds the tail of the last wave
 constexpr int kTargetCtas = kNumSMs * 32;
 constexpr int kResampleTargetCtas = kNumSMs * 8;
-constexpr int kTilesPerChunkMax = 8;
+constexpr int kDrawTilesPerCta = 64;     // separate draw launch: at most 8 tiles per warp
 
 // Per-(row, segment) partial of the greedy sweep.
 struct GreedyPart {
@@ -44,9 +44,9 @@ struct VerifyPlan {
   int rows;               // rows swept per sequence: K+1 (greedy) or 2K+1 (rejection)
   int S;                  // segments per row
   long long seg;          // elements per segment
-  int tiles;              // resample tiles per row
-  int tiles_per_chunk;    // resample tiles per CTA
-  int C;                  // resample CTAs per sequence
+  int tiles;              // draw tiles per row
+  int tiles_per_chunk;    // draw tiles per CTA of the separate draw launch
+  int C;                  // CTAs per sequence of the separate draw launch
   size_t off_cnt;         // int32[B]  sweep tickets
   size_t off_cnt2;        // int32[B]  resample tickets
   size_t off_part;        // partials [B*rows*S]
@@ -74,9 +74,9 @@ inline VerifyPlan make_verify_plan(int B, int K, int V, int rejection, long long
   seg = (seg + 7) / 8 * 8;
   p.seg = seg;
   p.S = (int)((V + seg - 1) / seg);
-  p.tiles = (V + kTile - 1) / kTile;
+  p.tiles = (V + kDrawTile - 1) / kDrawTile;
   int C = B > 0 ? (kResampleTargetCtas + B - 1) / B : 1;
-  int c_lo = (p.tiles + kTilesPerChunkMax - 1) / kTilesPerChunkMax;
+  int c_lo = (p.tiles + kDrawTilesPerCta - 1) / kDrawTilesPerCta;
   if (C < c_lo) C = c_lo;
   if (C > p.tiles) C = p.tiles;
   if (C < 1) C = 1;

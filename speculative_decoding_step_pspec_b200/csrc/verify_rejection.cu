@@ -7,17 +7,16 @@
 // drawn from norm(max(0, p_{a_i} - q_{a_i})), and when every draft passes it is drawn from
 // the target's row K.
 //
-// Launch 1 (stats sweep): grid B*(2K+1) rows x S segments.  Each CTA streams one segment
+// Stats sweep: grid B*(2K+1) rows x S segments.  Each CTA streams one segment
 // of one target or draft row with 16-byte loads and keeps an online (max, sum exp) pair.
 // The CTA that finishes a sequence last (atomic ticket, no waiting) merges the partials
-// in segment order in double, evaluates p(d_k) and q(d_k), builds the accept bitmask
-// (one bit per draft, so the first rejection is one find-first-set), and stores the
-// statistics of row a_i for the draw.
+// in segment order in double, evaluates p(d_k) and q(d_k), and builds the accept bitmask
+// (one bit per draft, so the first rejection is one find-first-set).
 //
-// Launch 2 (draw): grid B x C chunks over row a_i of every sequence.  Each CTA sums
-// r = max(0, p - q) (or p) over its 2048-element tiles and stores one double per tile.
-// The last CTA of the sequence prefix-sums the tile sums, picks the tile that holds
-// u_K * Z, and rescans only that tile with a block-wide scan to find the token.
+// Draw launch: grid B x C CTAs over 256-element warp tiles of each sequence's row a_i.
+// Each warp sums r = max(0, p - q) (or p) over its own tiles, with no block barrier per
+// tile, and stores one double per tile; the CTA that finishes a sequence last prefix-sums
+// the tile sums, picks the tile holding u_K * Z and rescans that tile with one warp.
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
@@ -51,6 +50,269 @@ __device__ __forceinline__ const elem* sweep_row(const RejectionLaunch& L, int i
   if (r <= L.K)
     return static_cast<const elem*>(L.target) + ((long long)i * (L.K + 1) + r) * L.ld;
   return static_cast<const elem*>(L.draft) + ((long long)i * L.K + (r - L.K - 1)) * L.ld;
+}
+
+// ---------------------------------------------------------------------------------------
+// The draw.  r(t) for t in [0, V): max(0, p(t) - q(t)) (resid) or p(t) (target only),
+// each probability computed in fp32 as 2^((x - M) log2 e) / S.  The tile sums and the
+// rescan compute r through the same code, so both see bit-identical values.
+constexpr int kWTile = 256;   // one warp tile: 32 lanes x 8 consecutive elements
+
+struct DrawRow {
+  const void* trow;
+  const void* qrow;
+  float mt, inv_st, mq, inv_sq;
+  bool resid;
+};
+
+__device__ __forceinline__ DrawRow make_draw_row(const RejectionLaunch& L, int elem_bytes, int i,
+                                                 int a, double mt, double st, double mq,
+                                                 double sq) {
+  DrawRow D;
+  const char* t = static_cast<const char*>(L.target);
+  const char* q = static_cast<const char*>(L.draft);
+  D.trow = t + ((long long)i * (L.K + 1) + a) * L.ld * elem_bytes;
+  D.resid = a < L.K;
+  D.qrow = D.resid ? q + ((long long)i * L.K + a) * L.ld * elem_bytes : D.trow;
+  D.mt = (float)mt;
+  D.inv_st = st > 0.0 ? (float)(1.0 / st) : 0.f;
+  D.mq = (float)mq;
+  D.inv_sq = sq > 0.0 ? (float)(1.0 / sq) : 0.f;
+  return D;
+}
+
+// Eight consecutive elements [t0, t0+8) of a row: 16-byte loads when the group lies inside
+// the row on a 16-byte boundary, else scalar loads (-inf past V) when the values are read.
+template <typename Tag>
+struct Raw8 {
+  uint4 v[8 / Tag::kVec];
+  bool fast;
+};
+
+template <typename Tag>
+__device__ __forceinline__ void raw8_load(const void* rowp, int V, long long t0, Raw8<Tag>& R) {
+  const typename Tag::elem* row = static_cast<const typename Tag::elem*>(rowp);
+  R.fast = t0 + 8 <= V && (reinterpret_cast<uintptr_t>(row + t0) & 15u) == 0;
+  if (R.fast) {
+#pragma unroll
+    for (int k = 0; k < 8 / Tag::kVec; ++k) R.v[k] = ld_stream(row + t0 + k * Tag::kVec);
+  }
+}
+
+template <typename Tag>
+__device__ __forceinline__ void raw8_values(const void* rowp, int V, long long t0,
+                                            const Raw8<Tag>& R, float (&x)[8]) {
+  const typename Tag::elem* row = static_cast<const typename Tag::elem*>(rowp);
+  if (R.fast) {
+    if constexpr (Tag::kVec == 8) {
+      unpack(R.v[0], x, BF16Tag{});
+    } else {
+      float lo[4], hi[4];
+      unpack(R.v[0], lo, F32Tag{});
+      unpack(R.v[1], hi, F32Tag{});
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { x[j] = lo[j]; x[4 + j] = hi[j]; }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = t0 + j < V ? load_scalar(row, t0 + j) : -INFINITY;
+  }
+}
+
+__device__ __forceinline__ float draw_r(const DrawRow& D, float xt, float xq) {
+  const float pt = (D.mt == -INFINITY || xt == -INFINITY) ? 0.f : ex2((xt - D.mt) * kLog2e) * D.inv_st;
+  if (!D.resid) return pt;
+  const float pq = (D.mq == -INFINITY || xq == -INFINITY) ? 0.f : ex2((xq - D.mq) * kLog2e) * D.inv_sq;
+  return fmaxf(pt - pq, 0.f);
+}
+
+template <typename Tag>
+__device__ __forceinline__ void r8(const DrawRow& D, int V, long long t0, float (&r)[8]) {
+  Raw8<Tag> T, Q;
+  raw8_load<Tag>(D.trow, V, t0, T);
+  if (D.resid) raw8_load<Tag>(D.qrow, V, t0, Q);
+  float xt[8], xq[8];
+  raw8_values<Tag>(D.trow, V, t0, T, xt);
+  if (D.resid) raw8_values<Tag>(D.qrow, V, t0, Q, xq);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) r[j] = draw_r(D, xt[j], D.resid ? xq[j] : 0.f);
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// This warp's share of the tile sums: tiles t_begin, t_begin + stride, ... below t_end,
+// two tiles per iteration with all their loads issued before any arithmetic.
+template <typename Tag>
+__device__ void warp_tile_sums(const DrawRow& D, int V, long long t_begin, long long t_end,
+                               long long stride, double* ts) {
+  const int lane = threadIdx.x & 31;
+  for (long long t = t_begin; t < t_end; t += 2 * stride) {
+    const long long t2 = t + stride;
+    const bool two = t2 < t_end;
+    const long long e1 = t * kWTile + lane * 8, e2 = t2 * kWTile + lane * 8;
+    Raw8<Tag> T1, Q1, T2, Q2;
+    raw8_load<Tag>(D.trow, V, e1, T1);
+    if (D.resid) raw8_load<Tag>(D.qrow, V, e1, Q1);
+    if (two) {
+      raw8_load<Tag>(D.trow, V, e2, T2);
+      if (D.resid) raw8_load<Tag>(D.qrow, V, e2, Q2);
+    }
+    float x[8], y[8];
+    float s1 = 0.f, s2 = 0.f;
+    raw8_values<Tag>(D.trow, V, e1, T1, x);
+    if (D.resid) raw8_values<Tag>(D.qrow, V, e1, Q1, y);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s1 += draw_r(D, x[j], D.resid ? y[j] : 0.f);
+    if (two) {
+      raw8_values<Tag>(D.trow, V, e2, T2, x);
+      if (D.resid) raw8_values<Tag>(D.qrow, V, e2, Q2, y);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s2 += draw_r(D, x[j], D.resid ? y[j] : 0.f);
+    }
+    const double d1 = warp_sum((double)s1);
+    const double d2 = warp_sum((double)s2);
+    if (lane == 0) {
+      ts[t] = d1;
+      if (two) ts[t2] = d2;
+    }
+  }
+}
+
+__device__ __forceinline__ double block_sum(double v, double* s_red) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  double t = 0.0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t += s_red[w];
+  return t;
+}
+
+// Exclusive prefix over the CTA of one double per thread; returns the prefix and sets *total.
+__device__ __forceinline__ double block_exclusive_scan(double v, double* s_red, double* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    double n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  __syncthreads();
+  if (lane == 31) s_red[warp] = incl;
+  __syncthreads();
+  double base = 0.0, all = 0.0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) base += s_red[w];
+    all += s_red[w];
+  }
+  *total = all;
+  return base + incl - v;
+}
+
+struct DrawShared {
+  double red[kWarps + 1];
+  int found;
+  int token;
+};
+
+// One CTA, all threads, once the tile sums ts[0..tiles) of row a_i are in place: Z, the
+// first tile whose inclusive prefix exceeds u*Z, and the first token of that tile whose
+// running sum does (the last positive r of the tile if rounding leaves none; token 0 if
+// the row holds no mass at all).  A residual that sums to zero is redrawn from p itself.
+template <typename Tag>
+__device__ int draw_finish(DrawRow& D, int V, int tiles, double u, double* ts, DrawShared& sh,
+                           double* Zout) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  double Z = 0.0;
+  for (int t0 = 0; t0 < tiles; t0 += kThreads)
+    Z += block_sum(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
+  if (Z == 0.0 && D.resid) {
+    D.resid = false;                       // max(0, p - q) vanished: draw from p
+    D.qrow = D.trow;
+    __syncthreads();
+    warp_tile_sums<Tag>(D, V, warp, tiles, kWarps, ts);
+    __syncthreads();
+    Z = 0.0;
+    for (int t0 = 0; t0 < tiles; t0 += kThreads)
+      Z += block_sum(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
+  }
+  const double thr = u * Z;
+
+  int tile = -1;
+  double tile_base = 0.0;
+  double base = 0.0;
+  for (int t0 = 0; t0 < tiles; t0 += kThreads) {
+    const int t = t0 + tid;
+    const double v = t < tiles ? ld_cg(ts + t) : 0.0;
+    double tot;
+    const double ex = block_exclusive_scan(v, sh.red, &tot);
+    if (tid == 0) sh.found = 0x7fffffff;
+    __syncthreads();
+    if (t < tiles && v > 0.0 && base + ex + v > thr) atomicMin(&sh.found, t);
+    __syncthreads();
+    const int f = sh.found;
+    if (f != 0x7fffffff) {
+      if (t == f) sh.red[kWarps] = base + ex;
+      __syncthreads();
+      tile = f;
+      tile_base = sh.red[kWarps];
+      break;                               // f is the same on every thread
+    }
+    base += tot;
+  }
+  if (tile < 0 && Z > 0.0) {
+    // rounding kept every prefix at or below u*Z: the last tile holding any mass
+    if (tid == 0) sh.found = -1;
+    __syncthreads();
+    for (int t = tid; t < tiles; t += kThreads)
+      if (ld_cg(ts + t) > 0.0) atomicMax(&sh.found, t);
+    __syncthreads();
+    tile = sh.found;
+    if (tile >= 0) {
+      tile_base = thr;                     // no crossing inside: take its last positive r
+    }
+  }
+  if (warp == 0) {
+    int token = 0;
+    if (tile >= 0) {
+      const long long e0 = (long long)tile * kWTile + lane * 8;
+      float r[8];
+      r8<Tag>(D, V, e0, r);
+      float incl[8], run = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { run += r[j]; incl[j] = run; }
+      double inc = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+      }
+      const double ex = inc - (double)run;
+      int cand = 0x7fffffff, lastpos = -1;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (r[j] > 0.f) lastpos = (int)(e0 + j);
+        if (cand == 0x7fffffff && tile_base + ex + (double)incl[j] > thr) cand = (int)(e0 + j);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
+        lastpos = max(lastpos, __shfl_xor_sync(0xffffffffu, lastpos, o));
+      }
+      token = cand != 0x7fffffff ? cand : (lastpos >= 0 ? lastpos : 0);
+    }
+    if (lane == 0) sh.token = token;
+  }
+  __syncthreads();
+  *Zout = Z;
+  return sh.token;
 }
 
 template <typename Tag>
@@ -115,6 +377,7 @@ rej_stats_kernel(const RejectionLaunch L) {
   __syncthreads();
   if (warp != 0) return;
 
+  {
   int d = -1;
   bool bad = false, accept = false;
   double p = 0.0, q = 0.0;
@@ -164,225 +427,41 @@ rej_stats_kernel(const RejectionLaunch L) {
     if (anybad) set_err(L.err, PSPEC_DEVERR_TOKEN_RANGE);
     L.cnt[i] = 0;
   }
+  }  // warp 0
 }
 
-// ---------------------------------------------------------------------------------------
-// The draw.  r(t) for t in [0, V): max(0, p(t) - q(t)) (kResid) or p(t) (target only),
-// each probability computed in fp32 as 2^((x - M) log2 e) / S.  The chunk pass and the
-// rescan call the same function, so both see bit-identical r values.
-struct DrawRow {
-  const void* trow;
-  const void* qrow;
-  float mt, inv_st, mq, inv_sq;
-  bool resid;
-};
-
-template <typename Tag>
-__device__ __forceinline__ void load8(const typename Tag::elem* row, int V, long long t0,
-                                      float (&x)[8]) {
-  if (t0 + 8 <= V && (reinterpret_cast<uintptr_t>(row + t0) & 15u) == 0) {
-    if constexpr (Tag::kVec == 8) {
-      unpack(ld_stream(row + t0), x, BF16Tag{});
-    } else {
-      float lo[4], hi[4];
-      unpack(ld_stream(row + t0), lo, F32Tag{});
-      unpack(ld_stream(row + t0 + 4), hi, F32Tag{});  // 32 bytes: both halves aligned
-#pragma unroll
-      for (int j = 0; j < 4; ++j) { x[j] = lo[j]; x[4 + j] = hi[j]; }
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) x[j] = t0 + j < V ? load_scalar(row, t0 + j) : -INFINITY;
-  }
-}
-
-template <typename Tag>
-__device__ __forceinline__ void tile_values(const DrawRow& D, int V, long long t0, float (&r)[8]) {
-  using elem = typename Tag::elem;
-  float xt[8], xq[8];
-  load8<Tag>(static_cast<const elem*>(D.trow), V, t0, xt);
-  if (D.resid) load8<Tag>(static_cast<const elem*>(D.qrow), V, t0, xq);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    float pt = (D.mt == -INFINITY || xt[j] == -INFINITY) ? 0.f
-                                                         : ex2((xt[j] - D.mt) * kLog2e) * D.inv_st;
-    if (D.resid) {
-      float pq = (D.mq == -INFINITY || xq[j] == -INFINITY)
-                     ? 0.f
-                     : ex2((xq[j] - D.mq) * kLog2e) * D.inv_sq;
-      r[j] = fmaxf(pt - pq, 0.f);
-    } else {
-      r[j] = pt;
-    }
-  }
-}
-
-__device__ __forceinline__ double block_sum(double v, double* s_red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) s_red[warp] = v;
-  __syncthreads();
-  double t = 0.0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) t += s_red[w];
-  return t;
-}
-
-// Exclusive prefix over the CTA of one double per thread; returns the prefix and sets *total.
-__device__ __forceinline__ double block_exclusive_scan(double v, double* s_red, double* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    double n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  __syncthreads();
-  if (lane == 31) s_red[warp] = incl;
-  __syncthreads();
-  double base = 0.0, all = 0.0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    if (w < warp) base += s_red[w];
-    all += s_red[w];
-  }
-  *total = all;
-  return base + incl - v;
-}
-
-template <typename Tag>
-__device__ double tile_sum(const DrawRow& D, int V, int tile, double* s_red) {
-  float r[8];
-  tile_values<Tag>(D, V, (long long)tile * kTile + threadIdx.x * 8, r);
-  float th = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) th += r[j];
-  return block_sum((double)th, s_red);
-}
-
+// The draw launch: B x C CTAs over the warp tiles of each sequence's row a_i.
 template <typename Tag>
 __global__ void __launch_bounds__(kThreads)
 rej_draw_kernel(const RejectionLaunch L) {
+  using elem = typename Tag::elem;
   const int K = L.K;
   const int i = blockIdx.x / L.C;
   const int c = blockIdx.x % L.C;
-  __shared__ double s_red[kWarps];
+  const int warp = threadIdx.x >> 5;
   __shared__ int s_last;
-  __shared__ int s_tok;
+  __shared__ DrawShared sh;
 
   const SeqInfo si = reinterpret_cast<const SeqInfo*>(L.seq)[i];  // previous launch
-  const int a = si.a;
-  DrawRow D;
-  D.trow = static_cast<const typename Tag::elem*>(L.target) + ((long long)i * (K + 1) + a) * L.ld;
-  D.resid = a < K;
-  D.qrow = D.resid ? static_cast<const typename Tag::elem*>(L.draft) + ((long long)i * K + a) * L.ld
-                   : D.trow;
-  D.mt = (float)si.mt;
-  D.inv_st = si.st > 0.0 ? (float)(1.0 / si.st) : 0.f;
-  D.mq = (float)si.mq;
-  D.inv_sq = si.sq > 0.0 ? (float)(1.0 / si.sq) : 0.f;
-
+  DrawRow D = make_draw_row(L, sizeof(elem), i, si.a, si.mt, si.st, si.mq, si.sq);
   double* ts = L.tile_sums + (long long)i * L.tiles;
-  const int t_lo = c * L.tiles_per_chunk;
-  const int t_hi = min(L.tiles, t_lo + L.tiles_per_chunk);
-  for (int t = t_lo; t < t_hi; ++t) {
-    double v = tile_sum<Tag>(D, L.V, t, s_red);
-    if (threadIdx.x == 0) ts[t] = v;
-  }
+  const long long t_lo = (long long)c * L.tiles_per_chunk;
+  const long long t_hi = min((long long)L.tiles, t_lo + L.tiles_per_chunk);
+  warp_tile_sums<Tag>(D, L.V, t_lo + warp, t_hi, kWarps, ts);
+  __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    int t = atomicAdd(L.cnt2 + i, 1);
+    const int t = atomicAdd(L.cnt2 + i, 1);
     s_last = (t == L.C - 1);
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-
-  // ---- last CTA: Z, the tile holding u*Z, and the token inside it
-  const double u = (double)L.uniforms[(long long)i * (K + 1) + K];
-  double Z = 0.0;
-  for (int t0 = 0; t0 < L.tiles; t0 += kThreads) {
-    double v = t0 + (int)threadIdx.x < L.tiles ? ld_cg(ts + t0 + threadIdx.x) : 0.0;
-    Z += block_sum(v, s_red);
-  }
-  if (Z == 0.0 && D.resid) {
-    // max(0, p - q) vanished everywhere: draw from p itself
-    D.resid = false;
-    D.qrow = D.trow;
-    Z = 0.0;
-    for (int t = 0; t < L.tiles; ++t) {
-      double v = tile_sum<Tag>(D, L.V, t, s_red);
-      if (threadIdx.x == 0) ts[t] = v;
-      Z += v;
-    }
-    __syncthreads();
-    __threadfence_block();
-  }
-  const double thr = u * Z;
-
-  // first tile whose inclusive prefix exceeds thr
-  int tile = -1;
-  double tile_base = 0.0;
-  {
-    double base = 0.0;
-    if (threadIdx.x == 0) s_tok = 0x7fffffff;
-    for (int t0 = 0; t0 < L.tiles && tile < 0; t0 += kThreads) {
-      const int t = t0 + threadIdx.x;
-      double v = t < L.tiles ? ld_cg(ts + t) : 0.0;
-      double tot;
-      double ex = block_exclusive_scan(v, s_red, &tot);
-      if (t < L.tiles && base + ex + v > thr) atomicMin(&s_tok, t);
-      __syncthreads();
-      int found = s_tok;
-      if (found != 0x7fffffff) {
-        tile = found;
-        // base of the found tile: re-read the prefix from the owning thread
-        if (t == found) s_red[0] = base + ex;
-        __syncthreads();
-        tile_base = s_red[0];
-      }
-      base += tot;
-      __syncthreads();
-    }
-  }
-
-  int token = 0;
-  if (tile >= 0) {
-    float r[8];
-    const long long t0 = (long long)tile * kTile + threadIdx.x * 8;
-    tile_values<Tag>(D, L.V, t0, r);
-    float incl[8];
-    float run = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) { run += r[j]; incl[j] = run; }
-    double tot;
-    double ex = block_exclusive_scan((double)run, s_red, &tot);
-    int cand = 0x7fffffff, lastpos = -1;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (r[j] > 0.f) lastpos = (int)(t0 + j);
-      if (cand == 0x7fffffff && tile_base + ex + (double)incl[j] > thr) cand = (int)(t0 + j);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) { s_tok = 0x7fffffff; }
-    __syncthreads();
-    if (cand != 0x7fffffff) atomicMin(&s_tok, cand);
-    __syncthreads();
-    token = s_tok;
-    if (token == 0x7fffffff) {
-      // rounding left the crossing outside the rescan: the last positive r of the tile
-      __syncthreads();
-      if (threadIdx.x == 0) s_tok = -1;
-      __syncthreads();
-      if (lastpos >= 0) atomicMax(&s_tok, lastpos);
-      __syncthreads();
-      token = s_tok < 0 ? 0 : s_tok;
-    }
-  }
+  double Z;
+  const int token = draw_finish<Tag>(D, L.V, L.tiles, (double)L.uniforms[(long long)i * (K + 1) + K],
+                                     ts, sh, &Z);
   if (threadIdx.x == 0) {
-    L.out_tokens[(long long)i * (K + 1) + a] = token;
+    L.out_tokens[(long long)i * (K + 1) + si.a] = token;
     L.bonus[i] = token;
     if (L.residual_mass) L.residual_mass[i] = (float)Z;
     L.cnt2[i] = 0;
