@@ -42,6 +42,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["pspec", "reference"], default="pspec")
     p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
+    p.add_argument("--path", choices=["auto", "sweep", "early"], default="auto",
+                   help="verify path: automatic selection, full sweep, or early exit")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -177,12 +179,24 @@ def make_workload(name, device, rank):
     return w, dict(target=target, draft=draft, sampled=sampled, greedy=greedy, u=u, build=binp)
 
 
-def algorithmic_bytes(w, mode, accepted):
-    """Bytes the one-pass method must move per step (verify sweep + draft-batch build)."""
+def verify_rows(w, mode, accepted, early_exit):
+    """Logit rows a verify pass must read: every row (full sweep), or with early exit only
+    the rows of positions 0..a_i (target and draft rows for the rejection rule; the
+    target's row K as well when all K drafts pass)."""
+    import numpy as np
+    if not early_exit:
+        return w.B * ((2 * w.K + 1) if mode == "rejection" else (w.K + 1))
+    a = np.asarray(accepted, np.int64)
+    if mode == "rejection":
+        return int(np.where(a < w.K, 2 * (a + 1), 2 * w.K + 1).sum())
+    return int((a + 1).sum())
+
+
+def algorithmic_bytes(w, mode, accepted, early_exit=False):
+    """Bytes the method must move per step (verify + draft-batch build)."""
     import numpy as np
     s = 2 if str(w.dtype).endswith("bfloat16") else 4
-    rows = w.B * ((2 * w.K + 1) if mode == "rejection" else (w.K + 1))
-    verify = rows * w.V * s
+    verify = verify_rows(w, mode, accepted, early_exit) * w.V * s
     c = np.asarray(accepted, np.int64) + 1                 # surviving verify rows (L = K+1)
     H, sh = w.H, s
     T_in = w.B * (w.K + 1)
@@ -203,6 +217,7 @@ def run_pspec(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2}[args.path])
     w, d = make_workload(args.workload, dev, rank)
     rej = args.mode == "rejection"
     ws = ps.Workspace(w.B, w.K, w.V, rej, dev)
@@ -227,7 +242,11 @@ def run_pspec(args, rank, world, local_rank):
 
     for _ in range(max(3, args.warmup)):
         verify()
+        lv = ps.pspec_last_launches()
+        path = ps.pspec_last_verify_path()
         build()
+        lb = ps.pspec_last_launches()
+    launches_per_step = lv + lb
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -266,19 +285,27 @@ def run_pspec(args, rank, world, local_rank):
     draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if rej else None
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
     acc = vout["accepted_len"].cpu().numpy()
-    vbytes, bbytes = algorithmic_bytes(w, args.mode, acc)
+    early = path == 2
+    vbytes, bbytes = algorithmic_bytes(w, args.mode, acc, early)
+    full_vbytes, _ = algorithmic_bytes(w, args.mode, acc, False)
     hbm, peak_src = peaks()
     ms_step = elapsed_ms / K
     step_gbs = (vbytes + bbytes) / (ms_step * 1e-3) / 1e9
-    dom_kernel = "rej_stats_kernel" if rej else "greedy_sweep_kernel"
-    src = ["speculative_decoding_step_pspec_b200/csrc/verify_rejection.cu" if rej else
-           "speculative_decoding_step_pspec_b200/csrc/verify_greedy.cu",
-           "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
+    if early:
+        dom_kernel = "ee_kernel"
+        src = ["speculative_decoding_step_pspec_b200/csrc/verify_early_exit.cu",
+               "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
+               "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
+    else:
+        dom_kernel = "rej_stats_kernel" if rej else "greedy_sweep_kernel"
+        src = ["speculative_decoding_step_pspec_b200/csrc/verify_rejection.cu" if rej else
+               "speculative_decoding_step_pspec_b200/csrc/verify_greedy.cu",
+               "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
+               "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
     src_hash = kernel_source_hash(src)
     dom_ms = statistics.mean(stats_ms)
     achieved = vbytes / (dom_ms * 1e-3) / 1e9
     traffic = profiled_traffic(dom_kernel, args.workload, src_hash)
-    launches_per_step = ps.pspec_launches_per_call(2 if rej else 1) + ps.pspec_launches_per_call(0)
 
     line = {
         "metric": METRIC, "value": round(world * K / (elapsed_ms * 1e-3), 3), "unit": UNIT,
@@ -289,15 +316,17 @@ def run_pspec(args, rank, world, local_rank):
             "workload": f"{args.workload}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
                         f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
+            "verify_path": "early exit (cluster per sequence)" if early else "full sweep",
             "l2": "inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9),
             "parallelism": f"replicas x{world} (independent sequences, no collective)",
         },
         "achieved_gbs": round(step_gbs, 1),
         "pct_of_peak": round(100 * step_gbs / hbm, 2),
-        "algorithmic_bytes_per_step": {"verify": int(vbytes), "build": int(bbytes)},
+        "algorithmic_bytes_per_step": {"verify": int(vbytes), "build": int(bbytes),
+                                       "verify_full_sweep": int(full_vbytes)},
         "kernels_ms": {
             dom_kernel: round(dom_ms, 5),
-            **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if rej else {}),
+            **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if rej and not early else {}),
             "build_kernel": round(statistics.mean(build_ms), 5),
         },
         "build_gbs": round(bbytes / (statistics.mean(build_ms) * 1e-3) / 1e9, 1),

@@ -71,6 +71,8 @@ typedef enum { PSPEC_F32 = 0, PSPEC_BF16 = 1 } pspec_dtype;
                                           negative block id: that row's slot is -1 */
 #define PSPEC_DEVERR_LAYOUT 0x8        /* qsl_in not an offset array, or a sequence with
                                           fewer than K+1 verify rows */
+#define PSPEC_DEVERR_TIMEOUT 0x10      /* a bounded wait for an asynchronous copy ran out
+                                          (outputs of that call are not valid) */
 
 /* Row kinds written to pspec_build_args.row_kind. */
 #define PSPEC_ROW_CTX 0   /* context row: accepted token paired with its target hidden */
@@ -134,8 +136,9 @@ PSPEC_API size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection
  * For each sequence i: g_k = argmax over the vocabulary of target row k (the lowest id
  * wins ties); a_i = the number of leading drafts with d_k == g_k; bonus = g_{a_i};
  * out_tokens = [d_0 .. d_{a_i-1}, bonus, -1 ...].  target_lse is written when non-NULL.
- * One kernel launch: a vocabulary sweep over all B*(K+1) target rows; the last CTA of
- * each sequence combines its row partials.  Errors: PSPEC_ERR_INVALID_ARG for bad
+ * One kernel launch.  Full sweep: all B*(K+1) target rows, the last CTA of each sequence
+ * combining its row partials.  Early exit (see pspec_set_verify_path): one cluster of
+ * CTAs per sequence reads rows 0, 1, ... in order and stops at the first mismatch.  Errors: PSPEC_ERR_INVALID_ARG for bad
  * arguments; a draft token outside [0, V) is treated as a mismatch and sets
  * PSPEC_DEVERR_TOKEN_RANGE.
  */
@@ -150,9 +153,12 @@ PSPEC_API pspec_status pspec_verify_greedy(const pspec_verify_args *args, void *
  * CDF in token-id order with u_K: from r = max(0, p_{a_i} - q_{a_i}) after a rejection,
  * from r = p_K when every draft passed; token = the smallest t with
  * sum_{v<=t} r_v > u_K * sum r (if rounding leaves none, the last t with r_t > 0; if the
- * residual sums to zero, the draw uses p_{a_i} itself).  Two launches: a vocabulary
- * sweep over the 2K+1 rows of every sequence (softmax statistics and the accept mask),
- * then a chunked inverse-CDF draw over each sequence's row a_i.  A draft token outside
+ * residual sums to zero, the draw uses p_{a_i} itself).  Full sweep: two launches, a
+ * vocabulary sweep over the 2K+1 rows of every sequence (softmax statistics and the
+ * accept mask), then a chunked inverse-CDF draw over each sequence's row a_i.  Early exit
+ * (see pspec_set_verify_path): one launch, one cluster of CTAs per sequence reading the
+ * target and draft rows of positions 0, 1, ... into shared memory and stopping at the
+ * first rejection, where it draws from the rows it holds.  A draft token outside
  * [0, V) has p = q = 0, is rejected, and sets PSPEC_DEVERR_TOKEN_RANGE.
  */
 PSPEC_API pspec_status pspec_verify_rejection(const pspec_verify_args *args, void *workspace,
@@ -253,10 +259,22 @@ PSPEC_API pspec_status pspec_build_draft_batch(const pspec_build_args *args, cud
 /* Human-readable name of a status code (static storage). */
 PSPEC_API const char *pspec_status_string(pspec_status status);
 
-/* Number of kernel launches one successful call of each kind issues on its stream:
-   0 = pspec_build_draft_batch, 1 = pspec_verify_greedy, 2 = pspec_verify_rejection;
-   -1 for any other value.  Used to count launches per decode step. */
-PSPEC_API int pspec_launches_per_call(int which);
+/* Number of kernel launches the most recent successful call made on this host thread
+   issued (0 for an empty batch).  Used to count launches per decode step. */
+PSPEC_API int pspec_last_launches(void);
+
+/* Verify path selection (process-wide; not synchronised with calls on other threads):
+   0 (default) automatic -- the early-exit path when B >= 64, no per-row diagnostic is
+     requested (target_lse, draft_lse, p_at_draft, q_at_draft all NULL), V is a multiple
+     of 8 and the logits rows start on 16-byte boundaries; otherwise the full sweep;
+   1 always the full sweep;
+   2 always the early-exit path (PSPEC_ERR_UNSUPPORTED when the arguments do not allow it).
+   Both paths give the same outputs; they differ in which rows they read. */
+PSPEC_API void pspec_set_verify_path(int path);
+
+/* The path the most recent successful verify call on this host thread took: 1 full sweep,
+   2 early exit, 0 none yet. */
+PSPEC_API int pspec_last_verify_path(void);
 
 /* Tuning: force the verify sweeps' segment length (elements of one row handled by one
    CTA; rounded up to a multiple of 8).  0 restores the automatic choice, which aims at
@@ -267,8 +285,8 @@ PSPEC_API void pspec_set_segment_elems(long long elems);
 
 /* Profiling hook: while `event` is non-NULL, every pspec_verify_rejection call records it
    on the call's stream between its two launches (after the statistics sweep, before the
-   draw), so that a caller can time each launch with CUDA events.  NULL turns it off.
-   Process-wide; the event is owned by the caller. */
+   draw; after the single launch of the early-exit path), so that a caller can time each
+   launch with CUDA events.  NULL turns it off.  Process-wide; the caller owns the event. */
 PSPEC_API void pspec_set_split_event(cudaEvent_t event);
 
 #ifdef __cplusplus

@@ -18,14 +18,15 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpspec.s
 PSPEC_OK, PSPEC_ERR_INVALID_ARG, PSPEC_ERR_UNSUPPORTED, PSPEC_ERR_CUDA, PSPEC_ERR_WORKSPACE = range(5)
 PSPEC_F32, PSPEC_BF16 = 0, 1
 PSPEC_DEVERR_TOKEN_RANGE, PSPEC_DEVERR_ACCEPT_RANGE = 0x1, 0x2
-PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT = 0x4, 0x8
+PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT, PSPEC_DEVERR_TIMEOUT = 0x4, 0x8, 0x10
 PSPEC_ROW_CTX, PSPEC_ROW_NTP, PSPEC_ROW_MASK, PSPEC_ROW_REJ, PSPEC_ROW_PAD = range(5)
 PSPEC_PADDING_SLOT_ID = -1
 PSPEC_MAX_K = 31
 
 EXPORTED = (
     "pspec_verify_workspace_bytes", "pspec_verify_greedy", "pspec_verify_rejection",
-    "pspec_build_draft_batch", "pspec_status_string", "pspec_launches_per_call",
+    "pspec_build_draft_batch", "pspec_status_string", "pspec_last_launches",
+    "pspec_set_verify_path", "pspec_last_verify_path",
     "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
 )
 
@@ -77,8 +78,12 @@ def _load():
     lib.pspec_build_draft_batch.restype = _I
     lib.pspec_status_string.argtypes = [_I]
     lib.pspec_status_string.restype = ctypes.c_char_p
-    lib.pspec_launches_per_call.argtypes = [_I]
-    lib.pspec_launches_per_call.restype = _I
+    lib.pspec_last_launches.argtypes = []
+    lib.pspec_last_launches.restype = _I
+    lib.pspec_set_verify_path.argtypes = [_I]
+    lib.pspec_set_verify_path.restype = None
+    lib.pspec_last_verify_path.argtypes = []
+    lib.pspec_last_verify_path.restype = _I
     lib.pspec_set_segment_elems.argtypes = [ctypes.c_longlong]
     lib.pspec_set_segment_elems.restype = None
     lib.pspec_set_split_event.argtypes = [_P]
@@ -135,8 +140,19 @@ def pspec_status_string(status: int) -> str:
     return LIB.pspec_status_string(int(status)).decode()
 
 
-def pspec_launches_per_call(which: int) -> int:
-    return LIB.pspec_launches_per_call(int(which))
+def pspec_last_launches() -> int:
+    """Kernel launches the most recent successful call on this thread issued."""
+    return LIB.pspec_last_launches()
+
+
+def pspec_last_verify_path() -> int:
+    """1 full sweep, 2 early exit: the path of the most recent verify call on this thread."""
+    return LIB.pspec_last_verify_path()
+
+
+def pspec_set_verify_path(path: int) -> None:
+    """0 automatic, 1 full sweep, 2 early exit (see include/pspec.h)."""
+    LIB.pspec_set_verify_path(int(path))
 
 
 def pspec_set_segment_elems(elems: int) -> None:

@@ -22,7 +22,8 @@ class Workspace:
         return self.tensor.numel() >= _b.pspec_verify_workspace_bytes(B, K, V, rejection)
 
 
-def verify_outputs(Bn: int, K: int, device, diagnostics: bool, rejection: bool) -> dict:
+def verify_outputs(Bn: int, K: int, device, diagnostics: bool, rejection: bool,
+                   residual_mass: bool = False) -> dict:
     i32 = dict(dtype=torch.int32, device=device)
     f32 = dict(dtype=torch.float32, device=device)
     out = {
@@ -38,6 +39,8 @@ def verify_outputs(Bn: int, K: int, device, diagnostics: bool, rejection: bool) 
             out["p_at_draft"] = torch.empty((Bn, K), **f32)
             out["q_at_draft"] = torch.empty((Bn, K), **f32)
             out["residual_mass"] = torch.empty((Bn,), **f32)
+    elif residual_mass and rejection:
+        out["residual_mass"] = torch.empty((Bn,), **f32)
     return out
 
 
@@ -58,13 +61,15 @@ def verify_greedy(target_logits: torch.Tensor, draft_tokens: torch.Tensor, *,
 
 def verify_rejection(target_logits: torch.Tensor, draft_logits: torch.Tensor,
                      draft_tokens: torch.Tensor, uniforms: torch.Tensor, *,
-                     diagnostics: bool = False, workspace: Workspace | None = None, out=None,
-                     stream=None) -> dict:
+                     diagnostics: bool = False, residual_mass: bool = False,
+                     workspace: Workspace | None = None, out=None, stream=None) -> dict:
     """Rejection-rule verify.  Returns out_tokens, accepted_len, bonus, err (+ fp32
-    diagnostics target_lse, draft_lse, p_at_draft, q_at_draft, residual_mass)."""
+    diagnostics target_lse, draft_lse, p_at_draft, q_at_draft, residual_mass; or only
+    residual_mass)."""
     Bn, K1, V = target_logits.shape
     K = K1 - 1
-    o = out if out is not None else verify_outputs(Bn, K, target_logits.device, diagnostics, True)
+    o = out if out is not None else verify_outputs(Bn, K, target_logits.device, diagnostics, True,
+                                                   residual_mass)
     ws = workspace if workspace is not None else Workspace(Bn, K, V, True, target_logits.device)
     _b.pspec_verify_rejection(target_logits=target_logits, draft_logits=draft_logits,
                              draft_tokens=draft_tokens, uniforms=uniforms,

@@ -15,6 +15,9 @@ using namespace pspec;
 
 long long g_seg_override = 0;   // 0 = automatic segment length
 cudaEvent_t g_split_event = nullptr;
+int g_verify_path = 0;          // 0 automatic, 1 full sweep, 2 early exit
+thread_local int t_last_launches = 0;
+thread_local int t_last_path = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -42,6 +45,47 @@ pspec_status check_verify(const pspec_verify_args* a, bool rejection) {
   return PSPEC_OK;
 }
 
+// The early-exit cluster path, when the arguments allow it and the selection asks for it:
+// returns true and sets *st when it handled the call.
+bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t stream,
+                    pspec_status* st) {
+  const bool diagnostics = a->target_lse || a->draft_lse || a->p_at_draft || a->q_at_draft;
+  if (g_verify_path == 1) return false;
+  if (g_verify_path == 0 && (a->B < kEarlyExitMinB || diagnostics)) return false;
+  const int eb = (int)elem_bytes(a->dtype);
+  EarlyExitPlan ep = make_early_exit_plan(a->V, kEarlyExitCluster);
+  if (!ep.ok) ep = make_early_exit_plan(a->V, 16);
+  const bool aligned = aligned16(a->target_logits) && (!rejection || aligned16(a->draft_logits)) &&
+                       (a->ld * eb) % 16 == 0;
+  if (!ep.ok || !aligned || diagnostics) {
+    if (g_verify_path == 0) return false;
+    *st = PSPEC_ERR_UNSUPPORTED;            // early exit forced on arguments it cannot take
+    return true;
+  }
+  EarlyExitLaunch L{};
+  L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
+  L.rejection = rejection;
+  L.G = ep.G; L.vs = ep.vs;
+  L.target = a->target_logits;
+  L.draft = a->draft_logits;
+  L.draft_tokens = a->draft_tokens;
+  L.uniforms = a->uniforms;
+  L.out_tokens = a->out_tokens;
+  L.accepted_len = a->accepted_len;
+  L.bonus = a->bonus;
+  L.residual_mass = rejection ? a->residual_mass : nullptr;
+  L.err = a->err;
+  if (launch_early_exit(L, stream) != cudaSuccess) {
+    *st = PSPEC_ERR_CUDA;
+    return true;
+  }
+  if (rejection && g_split_event) cudaEventRecord(g_split_event, stream);
+  t_last_launches = 1;
+  t_last_path = 2;
+  *st = PSPEC_OK;
+  return true;
+}
+
 pspec_status check_workspace(void* ws, size_t bytes, const VerifyPlan& p) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < p.bytes)
     return PSPEC_ERR_WORKSPACE;
@@ -60,10 +104,12 @@ size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection) {
 pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
                                  size_t workspace_bytes, cudaStream_t stream) {
   pspec_status st = check_verify(a, false);
-  if (st != PSPEC_OK || a->B == 0) return st;
+  if (st != PSPEC_OK) return st;
+  if (a->B == 0) { t_last_launches = 0; return st; }
   const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 0, g_seg_override);
   st = check_workspace(workspace, workspace_bytes, p);
   if (st != PSPEC_OK) return st;
+  if (try_early_exit(a, false, stream, &st)) return st;
   GreedyLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.S = p.S; L.seg = p.seg;
@@ -77,16 +123,21 @@ pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
   char* ws = static_cast<char*>(workspace);
   L.cnt = reinterpret_cast<int*>(ws + p.off_cnt);
   L.part = ws + p.off_part;
-  return launch_greedy(L, stream) == cudaSuccess ? PSPEC_OK : PSPEC_ERR_CUDA;
+  if (launch_greedy(L, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
+  t_last_launches = 1;
+  t_last_path = 1;
+  return PSPEC_OK;
 }
 
 pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
                                     size_t workspace_bytes, cudaStream_t stream) {
   pspec_status st = check_verify(a, true);
-  if (st != PSPEC_OK || a->B == 0) return st;
+  if (st != PSPEC_OK) return st;
+  if (a->B == 0) { t_last_launches = 0; return st; }
   const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 1, g_seg_override);
   st = check_workspace(workspace, workspace_bytes, p);
   if (st != PSPEC_OK) return st;
+  if (try_early_exit(a, true, stream, &st)) return st;
   RejectionLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.S = p.S; L.seg = p.seg;
@@ -110,7 +161,10 @@ pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
   L.part = ws + p.off_part;
   L.seq = ws + p.off_seq;
   L.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
-  return launch_rejection(L, stream, g_split_event) == cudaSuccess ? PSPEC_OK : PSPEC_ERR_CUDA;
+  if (launch_rejection(L, stream, g_split_event) != cudaSuccess) return PSPEC_ERR_CUDA;
+  t_last_launches = 2;
+  t_last_path = 1;
+  return PSPEC_OK;
 }
 
 pspec_status pspec_build_draft_batch(const pspec_build_args* a, cudaStream_t stream) {
@@ -146,7 +200,9 @@ pspec_status pspec_build_draft_batch(const pspec_build_args* a, cudaStream_t str
   L.row_vecs = (long long)a->H * (long long)elem_bytes(a->hidden_dtype) / 16;
   L.meta_blocks = (int)((meta_threads + kThreads - 1) / kThreads);
   L.hid_rows = (int)hid_rows;
-  return launch_build(L, stream) == cudaSuccess ? PSPEC_OK : PSPEC_ERR_CUDA;
+  if (launch_build(L, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
+  t_last_launches = 1;
+  return PSPEC_OK;
 }
 
 const char* pspec_status_string(pspec_status s) {
@@ -160,14 +216,11 @@ const char* pspec_status_string(pspec_status s) {
   return "PSPEC_ERR_UNKNOWN";
 }
 
-int pspec_launches_per_call(int which) {
-  switch (which) {
-    case 0: return 1;   // build: one launch, two CTA roles
-    case 1: return 1;   // greedy: one sweep launch
-    case 2: return 2;   // rejection: stats sweep + draw
-  }
-  return -1;
-}
+int pspec_last_launches(void) { return t_last_launches; }
+
+int pspec_last_verify_path(void) { return t_last_path; }
+
+void pspec_set_verify_path(int path) { g_verify_path = (path == 1 || path == 2) ? path : 0; }
 
 void pspec_set_segment_elems(long long elems) { g_seg_override = elems > 0 ? elems : 0; }
 

@@ -82,7 +82,37 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ---------------------------------------------------------------------------------------
-// (max, sum of exp(x - max)) pairs.  A pair with m = -inf holds no mass.
+// Packed fp32 pairs (sm_100): (d0, d1) = (a0, a1) * b + c and (d0, d1) += (a0, a1), one
+// instruction each.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(d0), "f"(d1), "f"(a0), "f"(a1));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// ---------------------------------------------------------------------------------------
+// Softmax normaliser partials in base-2 units: (m, s) stands for s * 2^m with
+// s = sum over its elements of 2^(x * kLog2e - m).  Forming every exponent as one fused
+// multiply-add x * kLog2e - m (instead of (x - m) * log2 e) halves the arithmetic per
+// logit; the double-precision merges convert back with the same constant, so the result
+// is the softmax of x * (kLog2e ln 2), within 1.4e-8 of the softmax of x.  A pair with
+// m = -inf holds no mass.
 struct MS {
   float m;
   float s;
@@ -91,8 +121,8 @@ struct MS {
 __device__ __forceinline__ MS ms_merge(MS a, MS b) {
   float M = fmaxf(a.m, b.m);
   if (M == -INFINITY) return MS{-INFINITY, 0.f};
-  float sa = a.m == -INFINITY ? 0.f : a.s * ex2((a.m - M) * kLog2e);
-  float sb = b.m == -INFINITY ? 0.f : b.s * ex2((b.m - M) * kLog2e);
+  float sa = a.m == -INFINITY ? 0.f : a.s * ex2(a.m - M);
+  float sb = b.m == -INFINITY ? 0.f : b.s * ex2(b.m - M);
   return MS{M, sa + sb};
 }
 
@@ -158,6 +188,32 @@ __device__ __forceinline__ void sweep_segment(const typename Tag::elem* row, lon
       if (v < nvec) vec(buf[u], a0 + v * W);
     }
   }
+  const long long t = a0 + nvec * W + threadIdx.x;
+  if (t < hi) one(load_scalar(row, t), t);
+}
+
+// The same walk with the vectors handed over in batches of U (one batch = the U vectors a
+// thread has in flight together); a last incomplete batch goes vector by vector.
+template <typename Tag, int U, typename FBatch, typename FVec, typename FOne>
+__device__ __forceinline__ void sweep_segment_batched(const typename Tag::elem* row, long long lo,
+                                                      long long hi, FBatch batch, FVec vec,
+                                                      FOne one) {
+  using elem = typename Tag::elem;
+  constexpr int W = Tag::kVec;
+  const int mis = (int)((reinterpret_cast<uintptr_t>(row + lo) & 15u) / sizeof(elem));
+  const long long head = mis == 0 ? 0 : min((long long)(W - mis), hi - lo);
+  if ((long long)threadIdx.x < head) one(load_scalar(row, lo + threadIdx.x), lo + threadIdx.x);
+  const long long a0 = lo + head;
+  const long long nvec = (hi - a0) / W;
+  const uint4* vp = reinterpret_cast<const uint4*>(row + a0);
+  long long v0 = threadIdx.x;
+  for (; v0 + (long long)(U - 1) * kThreads < nvec; v0 += (long long)U * kThreads) {
+    uint4 buf[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) buf[u] = ld_stream(vp + v0 + (long long)u * kThreads);
+    batch(buf);
+  }
+  for (; v0 < nvec; v0 += kThreads) vec(ld_stream(vp + v0), a0 + v0 * W);
   const long long t = a0 + nvec * W + threadIdx.x;
   if (t < hi) one(load_scalar(row, t), t);
 }

@@ -55,6 +55,24 @@ struct RejectionLaunch {
   double* tile_sums;     // workspace: [B*tiles] sums of r over 256-element tiles
 };
 
+struct EarlyExitLaunch {
+  int B, K, V;
+  long long ld;
+  pspec_dtype dtype;
+  int rejection;         // 1: rejection rule, 0: greedy
+  int G;                 // CTAs per cluster (one cluster per sequence): 8 or 16
+  long long vs;          // slice of each row per CTA (elements, multiple of 8)
+  const void* target;
+  const void* draft;
+  const int32_t* draft_tokens;
+  const float* uniforms;
+  int32_t* out_tokens;
+  int32_t* accepted_len;
+  int32_t* bonus;
+  float* residual_mass;  // optional
+  int32_t* err;
+};
+
 struct BuildLaunch {
   pspec_build_args a;
   long long row_vecs;    // 16-byte vectors per hidden row
@@ -66,5 +84,6 @@ cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream);
 // split_event (may be null) is recorded between the statistics sweep and the draw.
 cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream, cudaEvent_t split_event);
 cudaError_t launch_build(const BuildLaunch& L, cudaStream_t stream);
+cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream);
 
 }  // namespace pspec

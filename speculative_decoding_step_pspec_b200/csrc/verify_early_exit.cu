@@ -1,0 +1,396 @@
+// verify_early_exit.cu -- target verification that stops at the first rejection.
+//
+// The accept rule is sequential ("Capstone 14: speculative decoding inference server",
+// section "Architecture": accept the prefix, resample for the rejected suffix): once
+// draft k is rejected, rows k+1..K of that sequence do not influence the result.  This
+// path reads only rows 0..a_i (and row K when every draft passes), which at the pages'
+// 60-80 % acceptance is well under half of the full sweep's bytes, and its outputs are
+// the full sweep's outputs.
+//
+// Design (one thread-block cluster of G CTAs per sequence, G = 8 or 16):
+//   * position k = 0, 1, ...: each CTA streams its 1/G slice of target row k (and of draft
+//     row k for the rejection rule) with 16-byte loads, four vectors per row in flight per
+//     thread, and reduces it to (max, sum exp) or to its argmax;
+//   * one cluster barrier; then every CTA reads the G slice partials through distributed
+//     shared memory in rank order and takes the same decision (u q < p, or draft ==
+//     argmax), so no second barrier or broadcast is needed (partials are double-buffered
+//     by position parity, so the next position cannot overwrite what a slower CTA reads);
+//   * rejection rule: at the stop position each CTA sums r = max(0, p - q) (or p) over
+//     256-element warp tiles of its slice, re-read right after the statistics pass
+//     (usually from L2); the slice totals are prefix-summed in rank order on every CTA, and
+//     the CTA whose slice holds u_K * Z rescans one tile.
+// Rows are held in registers, not shared memory, so that six CTAs fit per SM and about a
+// hundred sequences are in flight: measured on B200, caching each 100 KB slice pair in
+// shared memory (two CTAs per SM) left HBM idle between positions.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+#include "verify_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace pspec {
+
+namespace {
+
+#ifndef PSPEC_EE_REJ_UNROLL
+#define PSPEC_EE_REJ_UNROLL 2
+#endif
+#ifndef PSPEC_EE_MIN_BLOCKS
+#define PSPEC_EE_MIN_BLOCKS 6
+#endif
+constexpr int kEERejUnroll = PSPEC_EE_REJ_UNROLL;   // vectors per row in flight (rejection)
+constexpr int kEEMinBlocks = PSPEC_EE_MIN_BLOCKS;   // CTAs per SM the register budget targets
+
+// A CTA's contribution to one position.
+struct EEPart {
+  float mt, st;      // (max, sum exp) of its slice of the target row
+  float mq, sq;      // the same for the draft row
+  float bv;          // argmax value of its target slice (greedy)
+  int bi;            // argmax index (global token id; kNoIndex when empty)
+};
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// r over eight consecutive row elements [t0, t0+8) of this CTA's slice (global memory,
+// usually still in L2 from the statistics pass), 0 at or past the slice end n.
+template <typename Tag>
+__device__ __forceinline__ void slice_r8(const DrawRow& D, long long lo, int n, int e0, float (&r)[8]) {
+  if (e0 >= n) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) r[j] = 0.f;
+    return;
+  }
+  using elem = typename Tag::elem;
+  const elem* tp = static_cast<const elem*>(D.trow) + lo + e0;
+  const elem* qp = static_cast<const elem*>(D.qrow) + lo + e0;
+  float xt[8], xq[8];
+  if constexpr (Tag::kVec == 8) {
+    unpack(ld_stream(tp), xt, BF16Tag{});
+    if (D.resid) unpack(ld_stream(qp), xq, BF16Tag{});
+  } else {
+    float a[4], b[4];
+    unpack(ld_stream(tp), a, F32Tag{});
+    unpack(ld_stream(tp + 4), b, F32Tag{});
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { xt[j] = a[j]; xt[4 + j] = b[j]; }
+    if (D.resid) {
+      unpack(ld_stream(qp), a, F32Tag{});
+      unpack(ld_stream(qp + 4), b, F32Tag{});
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { xq[j] = a[j]; xq[4 + j] = b[j]; }
+    }
+  }
+  draw_r8(D, xt, xq, r);
+}
+
+template <typename Tag, int G, bool kRej>
+__global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyExitLaunch L) {
+  using elem = typename Tag::elem;
+  constexpr int W = Tag::kVec;
+  constexpr int U = kRej ? kEERejUnroll : 4;                 // vectors in flight per row
+  cg::cluster_group cluster = cg::this_cluster();
+  const int g = (int)cluster.block_rank();
+  const int i = (int)(blockIdx.x / G);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int K = L.K;
+
+  __shared__ EEPart part[2];                                 // by position parity
+  __shared__ double tot_slice;                               // draw: sum of r over the slice
+  __shared__ double tsum[kMaxSliceTiles];
+  __shared__ MS s_ms[2][kWarps];
+  __shared__ VI s_vi[kWarps];
+  __shared__ int s_stop;
+  __shared__ float s_dec[4];
+  __shared__ int s_tile;
+  __shared__ double s_base;
+
+  const long long lo = (long long)g * L.vs;                 // this CTA's slice [lo, lo + n)
+  const int n = (int)max(0LL, min((long long)L.V, lo + L.vs) - lo);
+  const int nvec = n / W;                                   // n is a multiple of 8
+
+  int k = 0;
+  for (; k <= K; ++k) {
+    const bool has_q = kRej && k < K;
+    const elem* trow = static_cast<const elem*>(L.target) + ((long long)i * (K + 1) + k) * L.ld;
+    const elem* qrow = has_q ? static_cast<const elem*>(L.draft) + ((long long)i * K + k) * L.ld : trow;
+    // the logits at the draft token, needed by every CTA's decision: in flight meanwhile
+    float xt_d = 0.f, xq_d = 0.f;
+    int d = -1;
+    if (k < K && warp == 0) {
+      d = L.draft_tokens[(long long)i * K + k];
+      if (kRej && d >= 0 && d < L.V) {
+        xt_d = load_scalar(trow, d);
+        xq_d = load_scalar(qrow, d);
+      }
+    }
+    // ---- stream this CTA's slice of the position's rows
+    MSAcc at = msacc_init(), aq = msacc_init();
+    VI best{-INFINITY, kNoIndex};
+    const uint4* tv = reinterpret_cast<const uint4*>(trow + lo);
+    const uint4* qv = reinterpret_cast<const uint4*>(qrow + lo);
+    int v0 = tid;
+    for (; v0 + (U - 1) * kThreads < nvec; v0 += U * kThreads) {   // full batches
+      uint4 bt[U], bq[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        bt[u] = ld_stream(tv + v0 + u * kThreads);
+        if (has_q) bq[u] = ld_stream(qv + v0 + u * kThreads);
+      }
+      if constexpr (kRej) {
+        consume_ms_batch<Tag, U>(bt, at);
+        if (has_q) consume_ms_batch<Tag, U>(bq, aq);
+      } else {
+#pragma unroll
+        for (int u = 0; u < U; ++u) consume_argmax<Tag>(bt[u], lo + (long long)(v0 + u * kThreads) * W, best);
+      }
+    }
+    for (; v0 < nvec; v0 += kThreads) {                            // the rest, one by one
+      const uint4 x = ld_stream(tv + v0);
+      if constexpr (kRej) {
+        consume_ms<Tag>(x, at);
+        if (has_q) consume_ms<Tag>(ld_stream(qv + v0), aq);
+      } else {
+        consume_argmax<Tag>(x, lo + (long long)v0 * W, best);
+      }
+    }
+    MS mt = msacc_final(at), mq = msacc_final(aq);
+    if constexpr (kRej) {
+      mt = warp_merge_ms(mt);
+      mq = warp_merge_ms(mq);
+      if (lane == 0) { s_ms[0][warp] = mt; s_ms[1][warp] = mq; }
+    } else {
+      best = warp_argmax(best);
+      if (lane == 0) s_vi[warp] = best;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      EEPart& pp = part[k & 1];
+      if constexpr (kRej) {
+        MS a = s_ms[0][0], b = s_ms[1][0];
+        for (int w = 1; w < kWarps; ++w) { a = ms_merge(a, s_ms[0][w]); b = ms_merge(b, s_ms[1][w]); }
+        pp.mt = a.m; pp.st = a.s; pp.mq = b.m; pp.sq = b.s;
+      } else {
+        VI a = s_vi[0];
+        for (int w = 1; w < kWarps; ++w)
+          if (vi_better(s_vi[w], a)) a = s_vi[w];
+        pp.bv = a.v; pp.bi = a.i;
+      }
+    }
+    cluster.sync();                                          // A: this position's partials
+
+    // ---- every CTA takes the same decision from the same partials (rank order, fixed
+    // shuffle tree): no second barrier and no broadcast are needed
+    if (warp == 0) {
+      EEPart p{};
+      if (lane < G) p = *cluster.map_shared_rank(&part[k & 1], (unsigned)lane);
+      int stop = 0, a = k;
+      if constexpr (kRej) {
+        float Mt = lane < G ? p.mt : -INFINITY, Mq = lane < G ? p.mq : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          Mt = fmaxf(Mt, __shfl_xor_sync(0xffffffffu, Mt, o));
+          Mq = fmaxf(Mq, __shfl_xor_sync(0xffffffffu, Mq, o));
+        }
+        double st = (lane < G && p.mt != -INFINITY) ? (double)p.st * exp2((double)p.mt - (double)Mt) : 0.0;
+        double sq = (lane < G && has_q && p.mq != -INFINITY) ? (double)p.sq * exp2((double)p.mq - (double)Mq) : 0.0;
+        st = warp_sum_d(st);
+        sq = warp_sum_d(sq);
+        d = __shfl_sync(0xffffffffu, d, 0);
+        xt_d = __shfl_sync(0xffffffffu, xt_d, 0);
+        xq_d = __shfl_sync(0xffffffffu, xq_d, 0);
+        bool accept = false;
+        if (k < K && d >= 0 && d < L.V) {
+          const double pp = (Mt != -INFINITY && xt_d != -INFINITY)
+                                ? exp2((double)xt_d * (double)kLog2e - (double)Mt) / st : 0.0;
+          const double qq = (Mq != -INFINITY && xq_d != -INFINITY)
+                                ? exp2((double)xq_d * (double)kLog2e - (double)Mq) / sq : 0.0;
+          const double u = (double)L.uniforms[(long long)i * (K + 1) + k];
+          accept = qq > 0.0 ? (u * qq < pp) : (pp > 0.0);
+        }
+        if (!accept) {
+          stop = 1;
+          if (lane == 0) {
+            s_dec[0] = Mt;
+            s_dec[1] = st > 0.0 ? (float)(1.0 / st) : 0.f;
+            s_dec[2] = Mq;
+            s_dec[3] = sq > 0.0 ? (float)(1.0 / sq) : 0.f;
+          }
+        }
+      } else {
+        VI b = lane < G ? VI{p.bv, p.bi} : VI{-INFINITY, kNoIndex};
+        b = warp_argmax(b);                 // largest value, lowest index among equals
+        const int gk = b.i == kNoIndex ? 0 : b.i;
+        d = __shfl_sync(0xffffffffu, d, 0);
+        const bool match = k < K && d >= 0 && d < L.V && d == gk;
+        if (!match) {
+          stop = 1;
+          if (g == 0 && lane == 0) { L.bonus[i] = gk; L.out_tokens[(long long)i * (K + 1) + k] = gk; }
+        }
+      }
+      if (stop && g == 0) {
+        // outputs the two rules share: accepted drafts, the -1 tail, the count, range errors
+        int bad = 0;
+        if (lane < K) {
+          const int dj = L.draft_tokens[(long long)i * K + lane];
+          bad = dj < 0 || dj >= L.V;
+          if (lane < a) L.out_tokens[(long long)i * (K + 1) + lane] = dj;
+        }
+        if (lane <= K && lane > a) L.out_tokens[(long long)i * (K + 1) + lane] = -1;
+        if (__any_sync(0xffffffffu, bad) && lane == 0) set_err(L.err, PSPEC_DEVERR_TOKEN_RANGE);
+        if (lane == 0) L.accepted_len[i] = a;
+      }
+      if (lane == 0) s_stop = stop;
+    }
+    __syncthreads();
+    if (s_stop) break;
+  }
+
+  if constexpr (kRej) {
+    // ---- the draw at the stop position a = k: r = max(0, p_a - q_a), or p_K after K passes
+    const int a = k;
+    DrawRow D;
+    D.trow = static_cast<const elem*>(L.target) + ((long long)i * (K + 1) + a) * L.ld;
+    D.resid = a < K;
+    D.qrow = D.resid ? static_cast<const elem*>(L.draft) + ((long long)i * K + a) * L.ld : D.trow;
+    D.mt = s_dec[0]; D.inv_st = s_dec[1]; D.mq = s_dec[2]; D.inv_sq = s_dec[3];
+    const int ntiles = (n + 255) / 256;
+    const double u = (double)L.uniforms[(long long)i * (K + 1) + K];
+    double Z = 0.0;
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int t = warp; t < ntiles; t += kWarps) {
+        float r[8];
+        slice_r8<Tag>(D, lo, n, t * 256 + lane * 8, r);
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sum += r[j];
+        const double ts = warp_sum_d((double)sum);
+        if (lane == 0) tsum[t] = ts;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        double tt = 0.0;
+        for (int t = 0; t < ntiles; ++t) tt += tsum[t];
+        tot_slice = tt;
+      }
+      cluster.sync();                                        // C: slice totals in place
+      Z = 0.0;
+      for (int h = 0; h < G; ++h) Z += *cluster.map_shared_rank(&tot_slice, (unsigned)h);
+      if (Z > 0.0 || !D.resid) break;
+      D.resid = false;                                       // residual vanished: draw from p
+      D.qrow = D.trow;
+      cluster.sync();                                        // every CTA has read the totals
+    }
+    const double thr = u * Z;
+    int owner = -1, last_pos = -1;
+    double base = 0.0, run = 0.0;
+    for (int h = 0; h < G; ++h) {
+      const double th = *cluster.map_shared_rank(&tot_slice, (unsigned)h);
+      if (th > 0.0) last_pos = h;
+      if (owner < 0 && th > 0.0 && run + th > thr) { owner = h; base = run; }
+      run += th;
+    }
+    const bool crossing = owner >= 0;
+    if (!crossing && Z > 0.0) owner = last_pos;              // rounding: last slice with mass
+    if (g == owner) {
+      if (tid == 0) {
+        int tile = -1, last_tile = -1;
+        double b2 = base, tb = base;
+        for (int t = 0; t < ntiles; ++t) {
+          if (tsum[t] > 0.0) last_tile = t;
+          if (tile < 0 && crossing && tsum[t] > 0.0 && b2 + tsum[t] > thr) { tile = t; tb = b2; }
+          b2 += tsum[t];
+        }
+        if (tile < 0) { tile = last_tile; tb = thr; }       // no crossing: its last positive r
+        s_tile = tile;
+        s_base = tb;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int token = 0;
+        const int tile = s_tile;
+        if (tile >= 0) {
+          const int e0 = tile * 256 + lane * 8;
+          float r[8];
+          slice_r8<Tag>(D, lo, n, e0, r);
+          float incl[8], acc = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) { acc += r[j]; incl[j] = acc; }
+          double inc = acc;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const double v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+          }
+          const double ex = inc - (double)acc;
+          const double tb = s_base;
+          int cand = 0x7fffffff, lastp = -1;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (r[j] > 0.f) lastp = (int)(lo + e0 + j);
+            if (cand == 0x7fffffff && tb + ex + (double)incl[j] > thr) cand = (int)(lo + e0 + j);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
+            lastp = max(lastp, __shfl_xor_sync(0xffffffffu, lastp, o));
+          }
+          token = cand != 0x7fffffff ? cand : (lastp >= 0 ? lastp : 0);
+        }
+        if (lane == 0) {
+          L.out_tokens[(long long)i * (K + 1) + a] = token;
+          L.bonus[i] = token;
+          if (L.residual_mass) L.residual_mass[i] = (float)Z;
+        }
+      }
+    } else if (owner < 0 && g == 0 && tid == 0) {            // no mass anywhere: token 0
+      L.out_tokens[(long long)i * (K + 1) + a] = 0;
+      L.bonus[i] = 0;
+      if (L.residual_mass) L.residual_mass[i] = 0.f;
+    }
+  }
+  cluster.sync();                                            // D: no remote reads after exit
+}
+
+template <typename Tag, int G, bool kRej>
+cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream) {
+  auto kern = ee_kernel<Tag, G, kRej>;
+  cudaError_t e = cudaSuccess;
+  if (G > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)L.B * G), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, L);
+}
+
+}  // namespace
+
+cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream) {
+  const bool bf = L.dtype == PSPEC_BF16;
+  if (L.G == 8) {
+    if (L.rejection) return bf ? launch_ee<BF16Tag, 8, true>(L, stream) : launch_ee<F32Tag, 8, true>(L, stream);
+    return bf ? launch_ee<BF16Tag, 8, false>(L, stream) : launch_ee<F32Tag, 8, false>(L, stream);
+  }
+  if (L.rejection) return bf ? launch_ee<BF16Tag, 16, true>(L, stream) : launch_ee<F32Tag, 16, true>(L, stream);
+  return bf ? launch_ee<BF16Tag, 16, false>(L, stream) : launch_ee<F32Tag, 16, false>(L, stream);
+}
+
+}  // namespace pspec

@@ -8,60 +8,19 @@
 // Design: the grid is B*(K+1) rows x S segments, one CTA per segment, 16-byte streaming
 // loads with four vectors in flight per thread.  The bf16 max of each vector is taken
 // on packed pairs (max.bf16x2), and only a vector that beats the running best is
-// unpacked to find the first position of its maximum.  Each CTA writes one partial;
+// unpacked to find the first position of its maximum.  The optional log-sum-exp uses the
+// base-2 online normaliser of verify_common.cuh.  Each CTA writes one partial;
 // an atomic ticket per sequence elects the CTA that finishes the sequence last, and that
 // CTA merges the partials in segment order (deterministic, lowest id wins ties) and
 // writes the accepted length, the bonus token and the output tokens.  No CTA waits.
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
+#include "verify_common.cuh"
 
 namespace pspec {
 
 namespace {
-
-__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-__device__ __forceinline__ float vec_max(const uint4& v, BF16Tag) {
-  uint32_t m = bmax2(bmax2(v.x, v.y), bmax2(v.z, v.w));
-  return fmaxf(bf16_lo(m), bf16_hi(m));
-}
-__device__ __forceinline__ float vec_max(const uint4& v, F32Tag) {
-  return fmaxf(fmaxf(__uint_as_float(v.x), __uint_as_float(v.y)),
-               fmaxf(__uint_as_float(v.z), __uint_as_float(v.w)));
-}
-
-template <typename Tag, bool kLse>
-__device__ __forceinline__ void consume(const uint4& v, long long idx0, VI& best, MS& ms) {
-  constexpr int W = Tag::kVec;
-  float vmax = vec_max(v, Tag{});
-  if (kLse || vmax > best.v) {
-    float x[W];
-    unpack(v, x, Tag{});
-    if (vmax > best.v) {
-      int j = 0;
-#pragma unroll
-      for (int t = W - 1; t >= 0; --t)
-        if (x[t] == vmax) j = t;
-      best.v = vmax;
-      best.i = (int)(idx0 + j);
-    }
-    if (kLse && vmax != -INFINITY) {
-      if (vmax > ms.m) {
-        ms.s = ms.m == -INFINITY ? 0.f : ms.s * ex2((ms.m - vmax) * kLog2e);
-        ms.m = vmax;
-      }
-      float acc = 0.f;
-#pragma unroll
-      for (int t = 0; t < W; ++t) acc += ex2((x[t] - ms.m) * kLog2e);
-      ms.s += acc;
-    }
-  }
-}
 
 template <typename Tag, bool kLse>
 __global__ void __launch_bounds__(kThreads)
@@ -76,14 +35,18 @@ greedy_sweep_kernel(const GreedyLaunch L) {
   const long long hi = min((long long)L.V, lo + L.seg);
 
   VI best{-INFINITY, kNoIndex};
-  MS ms{-INFINITY, 0.f};
+  MSAcc acc = msacc_init();
   sweep_segment<Tag, 4>(
       row, lo, hi,
-      [&](const uint4& v, long long idx0) { consume<Tag, kLse>(v, idx0, best, ms); },
+      [&](const uint4& v, long long idx0) {
+        consume_argmax<Tag>(v, idx0, best);
+        if (kLse) consume_ms<Tag>(v, acc);
+      },
       [&](float x, long long t) {
         if (x > best.v) { best.v = x; best.i = (int)t; }
-        if (kLse && x != -INFINITY) ms = ms_merge(ms, MS{x, 1.f});
+        if (kLse) consume_one(x, acc);
       });
+  MS ms = msacc_final(acc);
 
   // CTA reduction
   __shared__ VI s_vi[kWarps];
@@ -132,9 +95,9 @@ greedy_sweep_kernel(const GreedyLaunch L) {
       if (M != -INFINITY)
         for (int t = 0; t < L.S; ++t) {
           GreedyPart q = ld_cg(part + (long long)lane * L.S + t);
-          if (q.m != -INFINITY) S += (double)q.s * exp((double)q.m - (double)M);
+          if (q.m != -INFINITY) S += (double)q.s * exp2((double)q.m - (double)M);
         }
-      lse = M == -INFINITY ? -INFINITY : (double)M + log(S);
+      lse = M == -INFINITY ? -INFINITY : ((double)M + log2(S)) / (double)kLog2e;
     }
   }
   int d = -1;

@@ -20,29 +20,11 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
+#include "verify_common.cuh"
 
 namespace pspec {
 
 namespace {
-
-template <typename Tag>
-__device__ __forceinline__ void consume_ms(const uint4& v, MS& ms) {
-  constexpr int W = Tag::kVec;
-  float x[W];
-  unpack(v, x, Tag{});
-  float vmax = x[0];
-#pragma unroll
-  for (int t = 1; t < W; ++t) vmax = fmaxf(vmax, x[t]);
-  if (vmax == -INFINITY) return;
-  if (vmax > ms.m) {
-    ms.s = ms.m == -INFINITY ? 0.f : ms.s * ex2((ms.m - vmax) * kLog2e);
-    ms.m = vmax;
-  }
-  float acc = 0.f;
-#pragma unroll
-  for (int t = 0; t < W; ++t) acc += ex2((x[t] - ms.m) * kLog2e);
-  ms.s += acc;
-}
 
 // Row r of sequence i in the sweep order: target rows 0..K, then draft rows 0..K-1.
 template <typename elem>
@@ -57,13 +39,6 @@ __device__ __forceinline__ const elem* sweep_row(const RejectionLaunch& L, int i
 // each probability computed in fp32 as 2^((x - M) log2 e) / S.  The tile sums and the
 // rescan compute r through the same code, so both see bit-identical values.
 constexpr int kWTile = 256;   // one warp tile: 32 lanes x 8 consecutive elements
-
-struct DrawRow {
-  const void* trow;
-  const void* qrow;
-  float mt, inv_st, mq, inv_sq;
-  bool resid;
-};
 
 __device__ __forceinline__ DrawRow make_draw_row(const RejectionLaunch& L, int elem_bytes, int i,
                                                  int a, double mt, double st, double mq,
@@ -119,13 +94,6 @@ __device__ __forceinline__ void raw8_values(const void* rowp, int V, long long t
   }
 }
 
-__device__ __forceinline__ float draw_r(const DrawRow& D, float xt, float xq) {
-  const float pt = (D.mt == -INFINITY || xt == -INFINITY) ? 0.f : ex2((xt - D.mt) * kLog2e) * D.inv_st;
-  if (!D.resid) return pt;
-  const float pq = (D.mq == -INFINITY || xq == -INFINITY) ? 0.f : ex2((xq - D.mq) * kLog2e) * D.inv_sq;
-  return fmaxf(pt - pq, 0.f);
-}
-
 template <typename Tag>
 __device__ __forceinline__ void r8(const DrawRow& D, int V, long long t0, float (&r)[8]) {
   Raw8<Tag> T, Q;
@@ -134,8 +102,7 @@ __device__ __forceinline__ void r8(const DrawRow& D, int V, long long t0, float 
   float xt[8], xq[8];
   raw8_values<Tag>(D.trow, V, t0, T, xt);
   if (D.resid) raw8_values<Tag>(D.qrow, V, t0, Q, xq);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) r[j] = draw_r(D, xt[j], D.resid ? xq[j] : 0.f);
+  draw_r8(D, xt, xq, r);
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -161,17 +128,19 @@ __device__ void warp_tile_sums(const DrawRow& D, int V, long long t_begin, long 
       raw8_load<Tag>(D.trow, V, e2, T2);
       if (D.resid) raw8_load<Tag>(D.qrow, V, e2, Q2);
     }
-    float x[8], y[8];
+    float x[8], y[8], r[8];
     float s1 = 0.f, s2 = 0.f;
     raw8_values<Tag>(D.trow, V, e1, T1, x);
     if (D.resid) raw8_values<Tag>(D.qrow, V, e1, Q1, y);
+    draw_r8(D, x, y, r);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) s1 += draw_r(D, x[j], D.resid ? y[j] : 0.f);
+    for (int j = 0; j < 8; ++j) s1 += r[j];
     if (two) {
       raw8_values<Tag>(D.trow, V, e2, T2, x);
       if (D.resid) raw8_values<Tag>(D.qrow, V, e2, Q2, y);
+      draw_r8(D, x, y, r);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s2 += draw_r(D, x[j], D.resid ? y[j] : 0.f);
+      for (int j = 0; j < 8; ++j) s2 += r[j];
     }
     const double d1 = warp_sum((double)s1);
     const double d2 = warp_sum((double)s2);
@@ -330,12 +299,12 @@ rej_stats_kernel(const RejectionLaunch L) {
   const long long lo = (long long)s * L.seg;
   const long long hi = min((long long)L.V, lo + L.seg);
 
-  MS ms{-INFINITY, 0.f};
-  sweep_segment<Tag, 4>(
-      row, lo, hi, [&](const uint4& v, long long) { consume_ms<Tag>(v, ms); },
-      [&](float x, long long) {
-        if (x != -INFINITY) ms = ms_merge(ms, MS{x, 1.f});
-      });
+  MSAcc acc = msacc_init();
+  sweep_segment_batched<Tag, 4>(
+      row, lo, hi, [&](const uint4 (&v)[4]) { consume_ms_batch<Tag, 4>(v, acc); },
+      [&](const uint4& v, long long) { consume_ms<Tag>(v, acc); },
+      [&](float x, long long) { consume_one(x, acc); });
+  MS ms = msacc_final(acc);
 
   __shared__ MS s_ms[kWarps];
   __shared__ int s_last;
@@ -357,7 +326,9 @@ rej_stats_kernel(const RejectionLaunch L) {
   if (!s_last) return;
   __threadfence();
 
-  // ---- last CTA of sequence i: merge partials (double), accept test, stats of row a_i
+  // ---- last CTA of sequence i: merge partials (double), accept test, stats of row a_i.
+  // Partials are in base-2 units (MS); p(d) uses the same kLog2e, so the normaliser and
+  // the numerator describe one and the same softmax.
   __shared__ double s_M[2 * PSPEC_MAX_K + 1];
   __shared__ double s_S[2 * PSPEC_MAX_K + 1];
   const RejPart* part = reinterpret_cast<const RejPart*>(L.part) + (long long)i * R * L.S;
@@ -369,7 +340,7 @@ rej_stats_kernel(const RejectionLaunch L) {
     if (M != -INFINITY)
       for (int t = 0; t < L.S; ++t) {
         RejPart q = ld_cg(pr + t);
-        if (q.m != -INFINITY) S += (double)q.s * exp((double)q.m - (double)M);
+        if (q.m != -INFINITY) S += (double)q.s * exp2((double)q.m - (double)M);
       }
     s_M[threadIdx.x] = M;
     s_S[threadIdx.x] = S;
@@ -389,8 +360,8 @@ rej_stats_kernel(const RejectionLaunch L) {
       const double Mq = s_M[K + 1 + lane], Sq = s_S[K + 1 + lane];
       const float xt = load_scalar(sweep_row<elem>(L, i, lane), d);
       const float xq = load_scalar(sweep_row<elem>(L, i, K + 1 + lane), d);
-      if (Mt != -INFINITY && xt != -INFINITY) p = exp((double)xt - Mt) / St;
-      if (Mq != -INFINITY && xq != -INFINITY) q = exp((double)xq - Mq) / Sq;
+      if (Mt != -INFINITY && xt != -INFINITY) p = exp2((double)xt * (double)kLog2e - Mt) / St;
+      if (Mq != -INFINITY && xq != -INFINITY) q = exp2((double)xq * (double)kLog2e - Mq) / Sq;
       const double u = (double)L.uniforms[(long long)i * (K + 1) + lane];
       accept = q > 0.0 ? (u * q < p) : (p > 0.0);
     }
@@ -404,13 +375,15 @@ rej_stats_kernel(const RejectionLaunch L) {
     if (L.q_at_draft) L.q_at_draft[(long long)i * K + lane] = (float)q;
     if (L.draft_lse) {
       const double M = s_M[K + 1 + lane];
-      L.draft_lse[(long long)i * K + lane] = (float)(M == -INFINITY ? M : M + log(s_S[K + 1 + lane]));
+      L.draft_lse[(long long)i * K + lane] =
+          (float)(M == -INFINITY ? M : (M + log2(s_S[K + 1 + lane])) / (double)kLog2e);
     }
   }
   if (lane <= K) {
     if (L.target_lse) {
       const double M = s_M[lane];
-      L.target_lse[(long long)i * (K + 1) + lane] = (float)(M == -INFINITY ? M : M + log(s_S[lane]));
+      L.target_lse[(long long)i * (K + 1) + lane] =
+          (float)(M == -INFINITY ? M : (M + log2(s_S[lane])) / (double)kLog2e);
     }
     if (lane != a) L.out_tokens[(long long)i * (K + 1) + lane] = lane < a ? d : -1;
   }

@@ -41,7 +41,10 @@ def test_status_strings_and_launch_counts():
     assert ps.pspec_status_string(0) == "PSPEC_OK"
     assert ps.pspec_status_string(4) == "PSPEC_ERR_WORKSPACE"
     assert ps.pspec_status_string(99) == "PSPEC_ERR_UNKNOWN"
-    assert [ps.pspec_launches_per_call(i) for i in range(4)] == [1, 1, 2, -1]
+    assert ps.pspec_last_launches() == 0          # no successful call on this thread yet
+    for path in (1, 2, 0, 7):
+        ps.pspec_set_verify_path(path)                # setter only; 7 falls back to automatic
+    ps.pspec_set_verify_path(0)
 
 
 def test_workspace_sizes():

@@ -25,10 +25,31 @@ def _sample(B, n, seed):
     return np.sort(np.random.default_rng(seed).choice(B, size=n, replace=False))
 
 
+class verify_path:
+    """Force the full sweep (1) or the early-exit path (2) inside a with-block."""
+
+    def __init__(self, path):
+        self.path = path
+
+    def __enter__(self):
+        ps.pspec_set_verify_path(self.path)
+
+    def __exit__(self, *a):
+        ps.pspec_set_verify_path(0)
+
+
+def early_exit_allowed(t):
+    return t.shape[2] % 8 == 0 and t.data_ptr() % 16 == 0 and (t.stride(1) * t.element_size()) % 16 == 0
+
+
 def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True):
+    """Both verify rules, on both paths, against the oracle: the full sweep with every
+    diagnostic, then (where its shape rules allow) the early-exit path, which reads rows
+    only up to the first rejection and must give the same tokens."""
     V = target.shape[2]
-    gr = ps.verify_greedy(target, greedy_drafts, want_lse=diag)
-    rj = ps.verify_rejection(target, draft, sampled, u, diagnostics=diag)
+    with verify_path(1):
+        gr = ps.verify_greedy(target, greedy_drafts, want_lse=diag)
+        rj = ps.verify_rejection(target, draft, sampled, u, diagnostics=diag)
     torch.cuda.synchronize()
     U.check_verify_invariants(gr, greedy_drafts, V)
     U.check_verify_invariants(rj, sampled, V)
@@ -36,6 +57,17 @@ def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True)
     U.compare_greedy(gr, og, seqs)
     orj = U.oracle_rejection(target, draft, sampled, u, seqs)
     U.compare_rejection(rj, orj, seqs)
+    if early_exit_allowed(target):
+        with verify_path(2):
+            ge = ps.verify_greedy(target, greedy_drafts)
+            assert ps.pspec_last_launches() == 1
+            re = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
+            assert ps.pspec_last_launches() == 1
+        torch.cuda.synchronize()
+        U.check_verify_invariants(ge, greedy_drafts, V)
+        U.check_verify_invariants(re, sampled, V)
+        U.compare_greedy(ge, og, seqs)
+        U.compare_rejection(re, orj, seqs)
     return gr, rj, orj
 
 
@@ -93,7 +125,7 @@ def test_depth_sweep_sampled(K, sigma):
 # --------------------------------------------------------------------------- shapes
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("V,seg", [(1, 0), (7, 0), (8, 0), (2047, 0), (5003, 1024), (70001, 4096),
-                                   (70001, 0)])
+                                   (70001, 0), (5000, 1024), (70000, 0), (262144, 0)])
 @pytest.mark.parametrize("K", [1, 4])
 def test_ragged_multi_segment(dtype, V, seg, K):
     B = 5
@@ -156,8 +188,14 @@ def test_neg_inf_rows_and_entries():
     gr = ps.verify_greedy(target, d, want_lse=True)
     rj = ps.verify_rejection(target, draft, d, u, diagnostics=True)
     U.compare_greedy(gr, U.oracle_greedy(target, d))
-    U.compare_rejection(rj, U.oracle_rejection(target, draft, d, u))
+    o = U.oracle_rejection(target, draft, d, u)
+    U.compare_rejection(rj, o)
     assert rj["accepted_len"][3].item() == 0
+    with verify_path(2):
+        ge = ps.verify_greedy(target, d)
+        re = ps.verify_rejection(target, draft, d, u, residual_mass=True)
+    U.compare_greedy(ge, U.oracle_greedy(target, d, want_lse=False))
+    U.compare_rejection(re, o)
 
 
 def test_out_of_range_draft_tokens():
@@ -173,8 +211,50 @@ def test_out_of_range_draft_tokens():
     assert gr["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
     assert rj["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
     U.compare_greedy(gr, U.oracle_greedy(target, bad, want_lse=False))
-    U.compare_rejection(rj, U.oracle_rejection(target, draft, bad, u))
+    o = U.oracle_rejection(target, draft, bad, u)
+    U.compare_rejection(rj, o)
     assert gr["accepted_len"][0].item() == 0 and rj["accepted_len"][0].item() == 0
+    with verify_path(2):
+        ge = ps.verify_greedy(target, bad)
+        re = ps.verify_rejection(target, draft, bad, u)
+    assert ge["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
+    assert re["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
+    U.compare_greedy(ge, U.oracle_greedy(target, bad, want_lse=False))
+    U.compare_rejection(re, o)
+
+
+@pytest.mark.parametrize("B", [1, 63, 64, 200])
+def test_automatic_path_selection(B):
+    """Automatic selection: the early exit (one launch) from 64 sequences on when no per-row
+    diagnostic is requested; the full sweep (two launches) otherwise; same tokens."""
+    w = I.Workload("t", B, 5, 4096, 16, 4, torch.bfloat16, seed=B, sigma_t=2.0, sigma_d=0.6)
+    target, draft = I.logits(w, DEV)
+    sampled, _ = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    a = ps.verify_rejection(target, draft, sampled, u)
+    n_auto = ps.pspec_last_launches()
+    b = ps.verify_rejection(target, draft, sampled, u, diagnostics=True)
+    assert ps.pspec_last_launches() == 2
+    assert n_auto == (1 if B >= 64 else 2)
+    o = U.oracle_rejection(target, draft, sampled, u)
+    U.compare_rejection(a, o)
+    U.compare_rejection(b, o)
+
+
+def test_early_exit_refuses_what_it_cannot_take():
+    w = I.Workload("t", 4, 3, 1001, 16, 4, torch.bfloat16, seed=5, sigma_t=2.0, sigma_d=0.6)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    with verify_path(2):
+        with pytest.raises(ps.PspecError):
+            ps.verify_rejection(target, draft, sampled, u)          # V not a multiple of 8
+    w = I.Workload("t", 4, 3, 1000, 16, 4, torch.bfloat16, seed=5, sigma_t=2.0, sigma_d=0.6)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    with verify_path(2):
+        with pytest.raises(ps.PspecError):
+            ps.verify_rejection(target, draft, sampled, I.uniforms(w, DEV), diagnostics=True)
 
 
 def test_determinism_and_workspace_reuse():
@@ -192,6 +272,11 @@ def test_determinism_and_workspace_reuse():
     r = ps.verify_rejection(target[:5], draft[:5], sampled[:5], u[:5], workspace=ws)
     for k in ("out_tokens", "accepted_len", "bonus"):
         assert torch.equal(r[k], outs[0][k][:5]), k
+    with verify_path(2):
+        e1 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
+        e2 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
+    for k in e1:
+        assert torch.equal(e1[k], e2[k]), k
     wsg = ps.Workspace(w.B, w.K, w.V, False)
     g1 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
     g2 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
