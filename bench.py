@@ -44,6 +44,7 @@ def parse_args():
     p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
     p.add_argument("--path", choices=["auto", "sweep", "early"], default="auto",
                    help="verify path: automatic selection, full sweep, or early exit")
+    p.add_argument("--cluster", type=int, default=0, help="early-exit cluster size (0 auto)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -218,6 +219,7 @@ def run_pspec(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2}[args.path])
+    ps.pspec_set_cluster_size(args.cluster)
     w, d = make_workload(args.workload, dev, rank)
     rej = args.mode == "rejection"
     ws = ps.Workspace(w.B, w.K, w.V, rej, dev)

@@ -272,6 +272,11 @@ PSPEC_API int pspec_last_launches(void);
    Both paths give the same outputs; they differ in which rows they read. */
 PSPEC_API void pspec_set_verify_path(int path);
 
+/* Tuning: CTAs per thread-block cluster on the early-exit path (2, 4, 8 or 16; each CTA
+   streams a 1/G slice of a row); 0 restores the automatic choice (4, or 16 when a slice
+   of 4 would exceed 262144 elements).  Process-wide. */
+PSPEC_API void pspec_set_cluster_size(int G);
+
 /* The path the most recent successful verify call on this host thread took: 1 full sweep,
    2 early exit, 0 none yet. */
 PSPEC_API int pspec_last_verify_path(void);

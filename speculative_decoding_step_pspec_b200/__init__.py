@@ -9,7 +9,7 @@ the library has not been built: there is no CPU fallback.
 from ._binding import (  # noqa: F401
     EXPORTED, LIB, PspecError, library_path, pspec_build_draft_batch,
     pspec_last_launches, pspec_set_segment_elems, pspec_set_split_event,
-    pspec_set_verify_path, pspec_last_verify_path,
+    pspec_set_verify_path, pspec_last_verify_path, pspec_set_cluster_size,
     pspec_status_string,
     pspec_verify_greedy, pspec_verify_rejection, pspec_verify_workspace_bytes,
 )

@@ -26,7 +26,7 @@ PSPEC_MAX_K = 31
 EXPORTED = (
     "pspec_verify_workspace_bytes", "pspec_verify_greedy", "pspec_verify_rejection",
     "pspec_build_draft_batch", "pspec_status_string", "pspec_last_launches",
-    "pspec_set_verify_path", "pspec_last_verify_path",
+    "pspec_set_verify_path", "pspec_last_verify_path", "pspec_set_cluster_size",
     "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
 )
 
@@ -82,6 +82,8 @@ def _load():
     lib.pspec_last_launches.restype = _I
     lib.pspec_set_verify_path.argtypes = [_I]
     lib.pspec_set_verify_path.restype = None
+    lib.pspec_set_cluster_size.argtypes = [_I]
+    lib.pspec_set_cluster_size.restype = None
     lib.pspec_last_verify_path.argtypes = []
     lib.pspec_last_verify_path.restype = _I
     lib.pspec_set_segment_elems.argtypes = [ctypes.c_longlong]
@@ -143,6 +145,11 @@ def pspec_status_string(status: int) -> str:
 def pspec_last_launches() -> int:
     """Kernel launches the most recent successful call on this thread issued."""
     return LIB.pspec_last_launches()
+
+
+def pspec_set_cluster_size(G: int) -> None:
+    """CTAs per cluster on the early-exit path: 4, 8, 16, or 0 for automatic."""
+    LIB.pspec_set_cluster_size(int(G))
 
 
 def pspec_last_verify_path() -> int:

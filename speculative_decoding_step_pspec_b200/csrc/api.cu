@@ -16,6 +16,7 @@ using namespace pspec;
 long long g_seg_override = 0;   // 0 = automatic segment length
 cudaEvent_t g_split_event = nullptr;
 int g_verify_path = 0;          // 0 automatic, 1 full sweep, 2 early exit
+int g_cluster = 0;              // early-exit cluster size; 0 = automatic
 thread_local int t_last_launches = 0;
 thread_local int t_last_path = 0;
 
@@ -53,8 +54,8 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   if (g_verify_path == 1) return false;
   if (g_verify_path == 0 && (a->B < kEarlyExitMinB || diagnostics)) return false;
   const int eb = (int)elem_bytes(a->dtype);
-  EarlyExitPlan ep = make_early_exit_plan(a->V, kEarlyExitCluster);
-  if (!ep.ok) ep = make_early_exit_plan(a->V, 16);
+  EarlyExitPlan ep = make_early_exit_plan(a->V, g_cluster ? g_cluster : kEarlyExitCluster);
+  if (!ep.ok && g_cluster == 0) ep = make_early_exit_plan(a->V, 16);
   const bool aligned = aligned16(a->target_logits) && (!rejection || aligned16(a->draft_logits)) &&
                        (a->ld * eb) % 16 == 0;
   if (!ep.ok || !aligned || diagnostics) {
@@ -221,6 +222,8 @@ int pspec_last_launches(void) { return t_last_launches; }
 int pspec_last_verify_path(void) { return t_last_path; }
 
 void pspec_set_verify_path(int path) { g_verify_path = (path == 1 || path == 2) ? path : 0; }
+
+void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || G == 16) ? G : 0; }
 
 void pspec_set_segment_elems(long long elems) { g_seg_override = elems > 0 ? elems : 0; }
 

@@ -18,7 +18,7 @@ constexpr int kTargetCtas = kNumSMs * 32;
 constexpr int kResampleTargetCtas = kNumSMs * 8;
 constexpr int kDrawTilesPerCta = 64;     // separate draw launch: at most 8 tiles per warp
 constexpr int kEarlyExitMinB = 64;       // automatic path: early exit from this many sequences
-constexpr int kEarlyExitCluster = 8;     // CTAs per sequence on the early-exit path
+constexpr int kEarlyExitCluster = 4;     // CTAs per sequence on the early-exit path
 
 // Per-(row, segment) partial of the greedy sweep.
 struct GreedyPart {
@@ -104,7 +104,7 @@ inline VerifyPlan make_verify_plan(int B, int K, int V, int rejection, long long
 // Early-exit verify: one cluster of G CTAs per sequence, each CTA streaming a 1/G slice
 // of the position's rows.  Needs V a multiple of 8 and 16-byte aligned rows; the slice
 // must hold at most kMaxSliceTiles 256-element tiles.
-constexpr int kMaxSliceTiles = 512;
+constexpr int kMaxSliceTiles = 1024;
 
 struct EarlyExitPlan {
   bool ok;
@@ -118,8 +118,7 @@ inline EarlyExitPlan make_early_exit_plan(int V, int G) {
   p.G = G;
   p.vs = ((long long)V + G - 1) / G;
   p.vs = (p.vs + 7) / 8 * 8;
-  p.ok = (p.vs + 255) / 256 <= kMaxSliceTiles || G >= 16;
-  if ((p.vs + 255) / 256 > kMaxSliceTiles) p.ok = false;
+  p.ok = (p.vs + 255) / 256 <= kMaxSliceTiles;
   return p;
 }
 

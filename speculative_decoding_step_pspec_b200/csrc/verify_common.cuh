@@ -103,20 +103,42 @@ struct DrawRow {
   bool resid;
 };
 
-__device__ __forceinline__ float draw_r(const DrawRow& D, float xt, float xq) {
-  const float pt =
-      (D.mt == -INFINITY || xt == -INFINITY) ? 0.f : ex2(fmaf(xt, kLog2e, -D.mt)) * D.inv_st;
-  if (!D.resid) return pt;
-  const float pq =
-      (D.mq == -INFINITY || xq == -INFINITY) ? 0.f : ex2(fmaf(xq, kLog2e, -D.mq)) * D.inv_sq;
-  return fmaxf(pt - pq, 0.f);
+
+// r of eight consecutive elements, computed on packed fp32 pairs.  Every pass over the
+// same elements (tile sums, rescans) goes through this function, so all of them see
+// bit-identical values.
+__device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b));
 }
 
-// r of eight consecutive elements.
 __device__ __forceinline__ void draw_r8(const DrawRow& D, const float (&xt)[8], const float (&xq)[8],
                                         float (&r)[8]) {
+  if (D.mt == -INFINITY) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) r[j] = draw_r(D, xt[j], D.resid ? xq[j] : 0.f);
+    for (int j = 0; j < 8; ++j) r[j] = 0.f;
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    float a0, a1;
+    ffma2(a0, a1, xt[j], xt[j + 1], kLog2e, -D.mt);        // -inf logits give 2^-inf = 0
+    float p0, p1;
+    fmul2(p0, p1, ex2(a0), ex2(a1), D.inv_st);
+    if (D.resid && D.mq != -INFINITY) {
+      float b0, b1, q0, q1;
+      ffma2(b0, b1, xq[j], xq[j + 1], kLog2e, -D.mq);
+      fmul2(q0, q1, ex2(b0), ex2(b1), D.inv_sq);
+      r[j] = fmaxf(p0 - q0, 0.f);
+      r[j + 1] = fmaxf(p1 - q1, 0.f);
+    } else {
+      r[j] = p0;
+      r[j + 1] = p1;
+    }
+  }
 }
 
 // ---- argmax over 16-byte vectors: the vector's max on packed pairs, and only a vector

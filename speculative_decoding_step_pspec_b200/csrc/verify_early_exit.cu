@@ -7,7 +7,7 @@
 // 60-80 % acceptance is well under half of the full sweep's bytes, and its outputs are
 // the full sweep's outputs.
 //
-// Design (one thread-block cluster of G CTAs per sequence, G = 8 or 16):
+// Design (one thread-block cluster of G CTAs per sequence, G = 2, 4, 8 or 16):
 //   * position k = 0, 1, ...: each CTA streams its 1/G slice of target row k (and of draft
 //     row k for the rejection rule) with 16-byte loads, four vectors per row in flight per
 //     thread, and reduces it to (max, sum exp) or to its argmax;
@@ -15,10 +15,12 @@
 //     shared memory in rank order and takes the same decision (u q < p, or draft ==
 //     argmax), so no second barrier or broadcast is needed (partials are double-buffered
 //     by position parity, so the next position cannot overwrite what a slower CTA reads);
-//   * rejection rule: at the stop position each CTA sums r = max(0, p - q) (or p) over
+//   * rejection rule: at the stop position each CTA sums r = max(0, p - q) over
 //     256-element warp tiles of its slice, re-read right after the statistics pass
 //     (usually from L2); the slice totals are prefix-summed in rank order on every CTA, and
-//     the CTA whose slice holds u_K * Z rescans one tile.
+//     the CTA whose slice holds u_K * Z rescans one tile.  When the draw is from the target
+//     row itself (all drafts passed), the slice totals follow from the statistics already
+//     merged and only the CTA holding u_K * Z goes over its slice.
 // Rows are held in registers, not shared memory, so that six CTAs fit per SM and about a
 // hundred sequences are in flight: measured on B200, caching each 100 KB slice pair in
 // shared memory (two CTAs per SM) left HBM idle between positions.
@@ -58,19 +60,19 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
-// r over eight consecutive row elements [t0, t0+8) of this CTA's slice (global memory,
-// usually still in L2 from the statistics pass), 0 at or past the slice end n.
+// Eight consecutive logits [e0, e0+8) of this CTA's slice of the draw rows (global memory,
+// usually still in L2 from the statistics pass); -inf at or past the slice end n.
 template <typename Tag>
-__device__ __forceinline__ void slice_r8(const DrawRow& D, long long lo, int n, int e0, float (&r)[8]) {
+__device__ __forceinline__ void slice_x8(const DrawRow& D, long long lo, int n, int e0,
+                                         float (&xt)[8], float (&xq)[8]) {
   if (e0 >= n) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) r[j] = 0.f;
+    for (int j = 0; j < 8; ++j) xt[j] = xq[j] = -INFINITY;
     return;
   }
   using elem = typename Tag::elem;
   const elem* tp = static_cast<const elem*>(D.trow) + lo + e0;
   const elem* qp = static_cast<const elem*>(D.qrow) + lo + e0;
-  float xt[8], xq[8];
   if constexpr (Tag::kVec == 8) {
     unpack(ld_stream(tp), xt, BF16Tag{});
     if (D.resid) unpack(ld_stream(qp), xq, BF16Tag{});
@@ -87,7 +89,6 @@ __device__ __forceinline__ void slice_r8(const DrawRow& D, long long lo, int n, 
       for (int j = 0; j < 4; ++j) { xq[j] = a[j]; xq[4 + j] = b[j]; }
     }
   }
-  draw_r8(D, xt, xq, r);
 }
 
 template <typename Tag, int G, bool kRej>
@@ -108,6 +109,8 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
   __shared__ VI s_vi[kWarps];
   __shared__ int s_stop;
   __shared__ float s_dec[4];
+  __shared__ double s_St;                                    // target row's S at the stop
+  __shared__ double s_tot[16];                               // per-slice draw totals
   __shared__ int s_tile;
   __shared__ double s_base;
 
@@ -221,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
             s_dec[1] = st > 0.0 ? (float)(1.0 / st) : 0.f;
             s_dec[2] = Mq;
             s_dec[3] = sq > 0.0 ? (float)(1.0 / sq) : 0.f;
+            s_St = st;
           }
         }
       } else {
@@ -262,17 +266,23 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
     D.mt = s_dec[0]; D.inv_st = s_dec[1]; D.mq = s_dec[2]; D.inv_sq = s_dec[3];
     const int ntiles = (n + 255) / 256;
     const double u = (double)L.uniforms[(long long)i * (K + 1) + K];
-    double Z = 0.0;
-    for (int pass = 0; pass < 2; ++pass) {
+
+    // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8).
+    auto tile_pass = [&]() {
       for (int t = warp; t < ntiles; t += kWarps) {
-        float r[8];
-        slice_r8<Tag>(D, lo, n, t * 256 + lane * 8, r);
+        float xt[8], xq[8], r[8];
+        slice_x8<Tag>(D, lo, n, t * 256 + lane * 8, xt, xq);
+        draw_r8(D, xt, xq, r);
         float sum = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) sum += r[j];
         const double ts = warp_sum_d((double)sum);
         if (lane == 0) tsum[t] = ts;
       }
+    };
+    bool own_pass_done = false;
+    if (D.resid) {
+      tile_pass();
       __syncthreads();
       if (tid == 0) {
         double tt = 0.0;
@@ -280,18 +290,36 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
         tot_slice = tt;
       }
       cluster.sync();                                        // C: slice totals in place
-      Z = 0.0;
-      for (int h = 0; h < G; ++h) Z += *cluster.map_shared_rank(&tot_slice, (unsigned)h);
-      if (Z > 0.0 || !D.resid) break;
-      D.resid = false;                                       // residual vanished: draw from p
-      D.qrow = D.trow;
-      cluster.sync();                                        // every CTA has read the totals
+      if (tid < G) s_tot[tid] = *cluster.map_shared_rank(&tot_slice, (unsigned)tid);
+      __syncthreads();
+      double Z0 = 0.0;
+      for (int h = 0; h < G; ++h) Z0 += s_tot[h];
+      own_pass_done = true;
+      if (Z0 == 0.0) {                                       // residual vanished: draw from p
+        D.resid = false;
+        D.qrow = D.trow;
+        own_pass_done = false;
+      }
     }
+    if (!D.resid) {
+      // Drawing from the target row itself (all K drafts passed, or the residual was
+      // empty): its slice totals s_g 2^(m_g - M) / S come from the statistics already
+      // merged, so only the CTA that holds u*Z has to go over its slice again.
+      if (tid < G) {
+        const EEPart ph = *cluster.map_shared_rank(&part[a & 1], (unsigned)tid);
+        const double Mt = (double)D.mt;
+        s_tot[tid] = (ph.mt == -INFINITY || s_St <= 0.0) ? 0.0
+                                                         : (double)ph.st * exp2((double)ph.mt - Mt) / s_St;
+      }
+      __syncthreads();
+    }
+    double Z = 0.0;
+    for (int h = 0; h < G; ++h) Z += s_tot[h];
     const double thr = u * Z;
     int owner = -1, last_pos = -1;
     double base = 0.0, run = 0.0;
     for (int h = 0; h < G; ++h) {
-      const double th = *cluster.map_shared_rank(&tot_slice, (unsigned)h);
+      const double th = s_tot[h];
       if (th > 0.0) last_pos = h;
       if (owner < 0 && th > 0.0 && run + th > thr) { owner = h; base = run; }
       run += th;
@@ -299,6 +327,10 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
     const bool crossing = owner >= 0;
     if (!crossing && Z > 0.0) owner = last_pos;              // rounding: last slice with mass
     if (g == owner) {
+      if (!own_pass_done) {
+        tile_pass();
+        __syncthreads();
+      }
       if (tid == 0) {
         int tile = -1, last_tile = -1;
         double b2 = base, tb = base;
@@ -317,8 +349,9 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
         const int tile = s_tile;
         if (tile >= 0) {
           const int e0 = tile * 256 + lane * 8;
-          float r[8];
-          slice_r8<Tag>(D, lo, n, e0, r);
+          float xt[8], xq[8], r[8];
+          slice_x8<Tag>(D, lo, n, e0, xt, xq);
+          draw_r8(D, xt, xq, r);
           float incl[8], acc = 0.f;
 #pragma unroll
           for (int j = 0; j < 8; ++j) { acc += r[j]; incl[j] = acc; }
@@ -385,6 +418,14 @@ cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream) {
 
 cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream) {
   const bool bf = L.dtype == PSPEC_BF16;
+  if (L.G == 2) {
+    if (L.rejection) return bf ? launch_ee<BF16Tag, 2, true>(L, stream) : launch_ee<F32Tag, 2, true>(L, stream);
+    return bf ? launch_ee<BF16Tag, 2, false>(L, stream) : launch_ee<F32Tag, 2, false>(L, stream);
+  }
+  if (L.G == 4) {
+    if (L.rejection) return bf ? launch_ee<BF16Tag, 4, true>(L, stream) : launch_ee<F32Tag, 4, true>(L, stream);
+    return bf ? launch_ee<BF16Tag, 4, false>(L, stream) : launch_ee<F32Tag, 4, false>(L, stream);
+  }
   if (L.G == 8) {
     if (L.rejection) return bf ? launch_ee<BF16Tag, 8, true>(L, stream) : launch_ee<F32Tag, 8, true>(L, stream);
     return bf ? launch_ee<BF16Tag, 8, false>(L, stream) : launch_ee<F32Tag, 8, false>(L, stream);
