@@ -48,9 +48,11 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-sample", type=int, default=192,
+    p.add_argument("--cpu-sample", type=int, default=512,
                    help="sequences of the workload the CPU oracle baseline verifies")
     p.add_argument("--workload", default="b1024", help="b1024 (default), c64 or c1")
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the workload's number of sequences (profiling and scaling aid)")
     p.add_argument("--build-only", action="store_true",
                    help="time the draft-batch construction alone (profiling aid: no logits)")
     return p.parse_args()
@@ -165,12 +167,31 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sms), "source": "nvml, 10 ms period"}
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's elapsed time: every rank contributes its own device-timed ms."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job throughput: every rank ran `steps` steps of its own batch (weak scaling)
+    within the slowest rank's elapsed time."""
+    return world * steps / (elapsed_ms * 1e-3)
+
+
 # ----------------------------------------------------------------------------- workload
-def make_workload(name, device, rank):
+def make_workload(name, device, rank, batch=0):
     import torch
     from speculative_decoding_step_pspec_b200 import inputs as I
     w = dict(b1024=I.B1024, c64=I.C64, c1=I.C1)[name]
     w = I.scaled(w, seed=w.seed + 1000 * rank)      # each replica draws its own batch
+    if batch:
+        w = I.scaled(w, B=batch)
     target, draft = I.logits(w, device)
     sampled, greedy = I.draft_tokens(w, draft)
     u = I.uniforms(w, device)
@@ -220,7 +241,7 @@ def run_pspec(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2}[args.path])
     ps.pspec_set_cluster_size(args.cluster)
-    w, d = make_workload(args.workload, dev, rank)
+    w, d = make_workload(args.workload, dev, rank, args.batch)
     rej = args.mode == "rejection"
     ws = ps.Workspace(w.B, w.K, w.V, rej, dev)
     vout = ps.api.verify_outputs(w.B, w.K, dev, False, rej)
@@ -275,11 +296,7 @@ def run_pspec(args, rank, world, local_rank):
     ps.pspec_set_split_event(None)
     if world > 1:
         dist.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
 
     verify_ms = [e[0].elapsed_time(e[2]) for e in ev]
     build_ms = [e[2].elapsed_time(e[3]) for e in ev]
@@ -310,12 +327,12 @@ def run_pspec(args, rank, world, local_rank):
     traffic = profiled_traffic(dom_kernel, args.workload, src_hash)
 
     line = {
-        "metric": METRIC, "value": round(world * K / (elapsed_ms * 1e-3), 3), "unit": UNIT,
+        "metric": METRIC, "value": round(aggregate_value(K, world, elapsed_ms), 3), "unit": UNIT,
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": f"{args.workload}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
+            "workload": f"{args.workload}{'' if not args.batch else ' (B overridden)'}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
                         f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
             "verify_path": "early exit (cluster per sequence)" if early else "full sweep",
@@ -417,13 +434,9 @@ def run_e2e(args, w, d, ps, dev, world):
         step()
     b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(a.elapsed_time(b), world, dev)
     del host, dv
-    return {"value": round(world * n / (ms * 1e-3), 3), "unit": UNIT,
+    return {"value": round(aggregate_value(n, world, ms), 3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": n, "ms_per_step": round(ms / n, 3),
             "path": "pinned host buffers -> cudaMemcpyAsync -> C-ABI verify + build -> results to host"}
