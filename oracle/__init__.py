@@ -58,6 +58,8 @@ def _bind(path: str):
     lib.oracle_verify_rejection.restype = i32
     lib.oracle_build_draft_batch.argtypes = [i32] * 10 + [P] * 17
     lib.oracle_build_draft_batch.restype = i32
+    lib.oracle_sample_rows.argtypes = [i32, i32, i64, i32, P, P, P, P, P, f64]
+    lib.oracle_sample_rows.restype = i32
     return lib
 
 
@@ -174,6 +176,33 @@ class OracleLib:
         out["err"] = int(np.bitwise_or.reduce(np.array(errs or [0])))
         return out
 
+    def sample_rows(self, logits: np.ndarray, uniforms=None, tie_eps: float = TIE_EPS,
+                    threads: int = 1) -> dict:
+        """Sample one token per row of logits [..., V] (float32 or raw bf16 bits) by inverse
+        CDF at uniforms [...] (float32), or take the argmax when uniforms is None."""
+        lib = self.lib
+        logits = np.ascontiguousarray(logits)
+        shape = logits.shape[:-1]
+        V = logits.shape[-1]
+        flat = logits.reshape(-1, V)
+        N = flat.shape[0]
+        u = None if uniforms is None else np.ascontiguousarray(uniforms, np.float32).reshape(-1)
+        assert u is None or u.shape == (N,)
+        dt = _logits_dtype(flat)
+        out = {"tokens": np.empty(N, np.int32), "probs": np.empty(N, np.float64),
+               "flags": np.empty(N, np.int32)}
+
+        def run(b0, b1):
+            rc = lib.oracle_sample_rows(
+                b1 - b0, V, V, dt, _ptr(flat[b0:b1]), _ptr(u[b0:b1]) if u is not None else None,
+                _ptr(out["tokens"][b0:b1]), _ptr(out["probs"][b0:b1]), _ptr(out["flags"][b0:b1]),
+                ctypes.c_double(tie_eps))
+            if rc != 0:
+                raise ValueError("oracle_sample_rows rejected its arguments")
+
+        _run_parallel(run, N, threads)
+        return {k: v.reshape(shape) for k, v in out.items()}
+
     def build_draft_batch(self, *, K: int, block_size: int, mask_id: int, pad_id: int,
                           T_cap: int, qsl_in, verify_tokens, verify_pos, accepted_len, bonus,
                           block_table, verify_hidden=None, h_shared=None,
@@ -250,6 +279,11 @@ def verify_greedy(*args, **kw) -> dict:
 def verify_rejection(*args, **kw) -> dict:
     """Rejection-rule verify with the default oracle (see ``OracleLib.verify_rejection``)."""
     return default().verify_rejection(*args, **kw)
+
+
+def sample_rows(*args, **kw) -> dict:
+    """Draft sampling with the default oracle (see ``OracleLib.sample_rows``)."""
+    return default().sample_rows(*args, **kw)
 
 
 def build_draft_batch(**kw) -> dict:

@@ -43,6 +43,9 @@
  *       (h_context), MASK row m carries mask_id with h_shared at position NTP + m, and the
  *       rejected rows carry pad_id, their old verify position and slot -1.  Padding rows
  *       after the last span carry pad_id, position 0 and slot -1.
+ *   R8  draft sampling draws each of the drafter's K output rows by the same inverse-CDF
+ *       convention as R3 (u in [0,1), token-id order) from softmax(row); without uniforms
+ *       it takes the argmax (R4).  A draw within tie_eps of a CDF boundary is flagged.
  *   R7  invalid values never stop the oracle: accepted counts are clamped into [0, K]
  *       (error bit 0x2), out-of-range block lookups give slot -1 (error bit 0x4), a
  *       sequence with L_i < K+1 keeps its span as padding rows with seq_len 0 and sample
@@ -265,6 +268,45 @@ int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
     free(qk);
     free(r);
     if (err) *err |= e;
+    return 0;
+}
+
+int oracle_sample_rows(int N, int V, long long ld, int dtype, const void *logits,
+                       const float *uniforms, int *tokens, double *probs, int *flags,
+                       double tie_eps)
+{
+    if (N < 0 || V < 1 || ld < V) return 1;
+    for (int n = 0; n < N; ++n) {
+        long long off = (long long)n * ld;
+        double lse = row_logsumexp(logits, dtype, off, V);
+        int tok, flag = 0;
+        if (!uniforms) {
+            tok = row_argmax(logits, dtype, off, V);
+        } else {
+            /* inverse CDF of the softmax in token-id order (R3, R8) */
+            double Z = 0.0;
+            for (int t = 0; t < V; ++t) Z += row_prob(logits, dtype, off, t, lse);
+            double thr = (double)uniforms[n] * Z, cum = 0.0, prev = 0.0;
+            int last_pos = -1;
+            tok = -1;
+            for (int t = 0; t < V; ++t) {
+                double p = row_prob(logits, dtype, off, t, lse);
+                if (p > 0.0) last_pos = t;
+                prev = cum;
+                cum += p;
+                if (cum > thr) { tok = t; break; }
+            }
+            if (tok < 0) {
+                tok = last_pos >= 0 ? last_pos : 0;
+                flag = 2;
+            } else if (thr - prev < tie_eps * Z || cum - thr < tie_eps * Z) {
+                flag = 2;
+            }
+        }
+        tokens[n] = tok;
+        if (probs) probs[n] = row_prob(logits, dtype, off, tok, lse);
+        if (flags) flags[n] = flag;
+    }
     return 0;
 }
 

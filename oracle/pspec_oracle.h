@@ -40,6 +40,15 @@ int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
                             double *target_lse, double *draft_lse,
                             double *residual_mass, int *flags, double tie_eps, int *err);
 
+/* Draft sampling from the drafter's output rows: N rows of logits [N, ld] (V valid).
+   With uniforms [N] in [0,1): tokens[n] = the smallest t whose cumulative softmax exceeds
+   u_n (token-id order; if rounding leaves none, the last t with positive probability);
+   flags[n] bit 1 marks a draw within tie_eps of a boundary.  With uniforms NULL: the
+   argmax, lowest id on ties.  probs[n] (optional) = softmax probability of the token. */
+int oracle_sample_rows(int N, int V, long long ld, int dtype, const void *logits,
+                       const float *uniforms, int *tokens, double *probs, int *flags,
+                       double tie_eps);
+
 /* P-EAGLE draft-batch construction.  Inputs: qsl_in [B+1], verify_tokens [T_in],
    verify_pos [T_in], accepted_len [B], bonus [B], block_table [B, max_blocks],
    verify_hidden [T_in, H] and h_shared [H] (hidden_elem_bytes per element; NULL

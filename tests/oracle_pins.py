@@ -465,9 +465,38 @@ def pin_build_invalid_values(o):
     assert r["err"] == 0x8
 
 
+# ----------------------------------------------------------------------------- sampling
+def pin_sampling(o):
+    """Drafter-row sampling: the worked example, greedy = numpy argmax, never a zero-
+    probability token, and the law read off by bisection equals the softmax."""
+    g = _load("verify_worked_examples.json")["sampling"]
+    x = np.log(np.array(g["p"], np.float64)).astype(np.float32)
+    for u, tok in zip(g["u"], g["tokens"]):
+        r = o.sample_rows(x[None], np.array([u], np.float32))
+        assert int(r["tokens"][0]) == tok, (u, r["tokens"])
+    rng = np.random.default_rng(31)
+    L = rng.normal(0, 2, size=(50, 37)).astype(np.float32)
+    L[::3, 5] = -np.inf
+    r = o.sample_rows(L)
+    assert (r["tokens"] == np.argmax(L, axis=1)).all()
+    r = o.sample_rows(L, rng.random(50, dtype=np.float32))
+    assert np.isfinite(L[np.arange(50), r["tokens"]]).all()
+    P = sps.softmax(L.astype(np.float64), axis=1)
+    np.testing.assert_allclose(r["probs"], P[np.arange(50), r["tokens"]], rtol=1e-12)
+    # exact law: the CDF boundaries of the inverse-CDF draw are the softmax's cumulative sums
+    rows = L[:6]
+    Pc = np.cumsum(sps.softmax(rows.astype(np.float64), axis=1), axis=1)
+    for n in range(rows.shape[0]):
+        for t in range(rows.shape[1] - 1):
+            if Pc[n, t + 1] - Pc[n, t] <= 0:
+                continue
+            thr = _threshold(lambda u, n=n, t=t: o.sample_rows(rows[n:n + 1], np.array([u], np.float32))["tokens"][0] > t)
+            assert abs(thr - Pc[n, t]) < 2e-7, (n, t, thr, Pc[n, t])
+
+
 ALL_PINS = [
     pin_worked_examples, pin_greedy_matches_numpy_argmax, pin_bf16_decoding,
     pin_probabilities_match_scipy, pin_residual_mass_closed_form, pin_special_cases,
     pin_exact_distribution, pin_build_worked_example, pin_build_invariants,
-    pin_build_invalid_values,
+    pin_build_invalid_values, pin_sampling,
 ]

@@ -24,7 +24,8 @@ MUTANTS = [
      "                              row_prob(draft_logits, dtype, qoff, t, lse_q[a]);",
      "double diff = row_prob(draft_logits, dtype, qoff, t, lse_q[a]) -\n"
      "                              row_prob(target_logits, dtype, toff, t, lse_t[a]);"),
-    ("inverse_cdf_ge", "if (cum > thr) { tok = t; break; }", "if (cum >= thr + 0.01) { tok = t; break; }"),
+    ("inverse_cdf_ge", "cum += r[t];\n            if (cum > thr) { tok = t; break; }",
+     "cum += r[t];\n            if (cum >= thr + 0.01) { tok = t; break; }"),
     ("bonus_from_row_k_minus_1", "long long toff = ((long long)i * (K + 1) + a) * ld;",
      "long long toff = ((long long)i * (K + 1) + (a == K ? K - 1 : a)) * ld;"),
     ("lse_dropped_shift", "for (int t = 0; t < V; ++t) s += exp(logit_at(base, dtype, off + t) - m);\n    return m + log(s);",
@@ -41,6 +42,10 @@ MUTANTS = [
      "src = s + j - 1;\n                kind = ORACLE_ROW_NTP;"),
     ("slot_formula_swapped", "return (long long)id * block_size + pos % block_size;",
      "return (long long)id * block_size + pos / block_size;"),
+    ("sample_cdf_ge", "if (cum > thr) { tok = t; break; }\n            }\n            if (tok < 0) {\n                tok = last_pos >= 0 ? last_pos : 0;\n                flag = 2;\n            } else if (thr - prev < tie_eps * Z",
+     "if (cum + 0.05 > thr) { tok = t; break; }\n            }\n            if (tok < 0) {\n                tok = last_pos >= 0 ? last_pos : 0;\n                flag = 2;\n            } else if (thr - prev < tie_eps * Z"),
+    ("sample_greedy_last_tie", "            tok = row_argmax(logits, dtype, off, V);\n        } else {",
+     "            tok = row_argmax(logits, dtype, off, V) + (V > 1);\n        } else {"),
     ("offsets_without_masks", "off += (qsl_in[i + 1] - qsl_in[i]) + K - 1;", "off += (qsl_in[i + 1] - qsl_in[i]) + K;"),
 ]
 
