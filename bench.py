@@ -55,6 +55,8 @@ def parse_args():
                    help="override the workload's number of sequences (profiling and scaling aid)")
     p.add_argument("--build-only", action="store_true",
                    help="time the draft-batch construction alone (profiling aid: no logits)")
+    p.add_argument("--sample-only", choices=["sample", "argmax"], default=None,
+                   help="time draft-token sampling alone over the workload's drafter rows")
     return p.parse_args()
 
 
@@ -540,6 +542,68 @@ def run_build_only(args, local_rank):
                       "err": int(out["err"].item())}), flush=True)
 
 
+def run_sample_only(args, local_rank):
+    """Draft-token sampling alone over the workload's B*K drafter rows (the step after the
+    drafter forward): inverse-CDF draws with seeded uniforms, or the argmax.  The rows are
+    larger than L2 at the large-batch size; smaller workloads flush L2 between launches."""
+    import torch
+
+    import speculative_decoding_step_pspec_b200 as ps
+    from speculative_decoding_step_pspec_b200 import inputs as I
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = dict(b1024=I.B1024, c64=I.C64, c1=I.C1)[args.workload]
+    if args.batch:
+        w = I.scaled(w, B=args.batch)
+    g = torch.Generator(device=dev).manual_seed(w.seed)
+    draft = torch.empty((w.B, w.K, w.V), dtype=w.dtype, device=dev)
+    for b0 in range(0, w.B, 64):                   # drafter rows N(0, sigma_t), chunked
+        b1 = min(w.B, b0 + 64)
+        draft[b0:b1] = (torch.randn((b1 - b0, w.K, w.V), generator=g, device=dev)
+                        * w.sigma_t).to(w.dtype)
+    u = I.uniforms(w, dev)[:, :w.K].contiguous() if args.sample_only == "sample" else None
+    ws = torch.zeros(ps._binding.pspec_sample_workspace_bytes(w.B, w.K, w.V), dtype=torch.uint8,
+                     device=dev)
+    out = ps.sample_drafts(draft, u, workspace=ws)
+    nbytes = draft.numel() * draft.element_size()
+    flush = None if nbytes > (256 << 20) else torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        ps.sample_drafts(draft, u, workspace=ws, out=out)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        for a, b in ev:
+            if flush is not None:
+                flush.fill_(1)
+            a.record()
+            ps.sample_drafts(draft, u, workspace=ws, out=out)
+            b.record()
+        torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in ev]
+    assert int(out["err"].item()) == 0
+    ms = statistics.mean(times)
+    hbm, peak_src = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    src = ["speculative_decoding_step_pspec_b200/csrc/sample_drafts.cu",
+           "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
+           "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
+    print(json.dumps({
+        "metric": "draft-token sampling alone: rows/s and achieved HBM GB/s",
+        "workload": f"{args.workload}: B={w.B}, K={w.K}, V={w.V}, {str(w.dtype).split('.')[-1]} drafter rows",
+        "mode": args.sample_only, "rows": w.B * w.K, "steps": args.steps,
+        "ms_mean": round(ms, 5), "ms_median": round(statistics.median(times), 5),
+        "rows_per_s": round(w.B * w.K / (ms * 1e-3), 1),
+        "l2": "rows larger than L2; no flush" if flush is None else "256 MB flush between launches",
+        "roofline": {"kernel": "sample_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                     "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                     "traffic": profiled_traffic("sample_kernel", args.workload,
+                                                 kernel_source_hash(src)),
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": int(nbytes)},
+        "gpu_launches": args.steps, "clocks": sampler.summary()}), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, rank):
     """The CPU oracle as the reference arm: each step verifies a rotating bounded sample of
@@ -619,6 +683,8 @@ def main():
     try:
         if args.build_only:
             run_build_only(args, local_rank)
+        elif args.sample_only:
+            run_sample_only(args, local_rank)
         else:
             run_pspec(args, rank, world, local_rank)
     finally:

@@ -165,6 +165,40 @@ PSPEC_API pspec_status pspec_verify_rejection(const pspec_verify_args *args, voi
                                     size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Draft-token sampling ("Eagle parallel speculative decoding, vLLM, TorchSpec", section
+ * "Parallel architecture": the P-EAGLE drafter predicts its K draft tokens from K output
+ * rows of one forward pass).  For every row (i, k) of logits [B, K, ld] (V valid, any
+ * alignment of the base to its element size): with uniforms, draft_tokens[i][k] = the
+ * smallest token t whose cumulative softmax probability exceeds u_{i,k} (token-id order;
+ * if rounding leaves none, the last token with positive probability), the same inverse-CDF
+ * convention as the verify draw; with uniforms NULL, the argmax (lowest id on ties).
+ * q_at_draft (optional) receives each drafted token's softmax probability.  One launch,
+ * one pass over the logits: per chunk of 2048 (bf16) or 1024 (fp32) elements the sweep
+ * keeps (max, sum exp) or (max, first index); the CTA finishing a row turns the chunk
+ * partials into the token and rescans one chunk.  Workspace:
+ * pspec_sample_workspace_bytes(B, K, V) bytes (enough for either dtype), 256-byte aligned,
+ * zero-filled once before first use (each call leaves its counters at zero).  Returns
+ * PSPEC_ERR_INVALID_ARG for bad sizes, pointers or dtype, PSPEC_ERR_WORKSPACE for a
+ * missing, misaligned or short workspace, PSPEC_ERR_CUDA when the launch fails.
+ */
+typedef struct {
+  int B;                       /* sequences; B = 0 is a no-op */
+  int K;                       /* drafter output rows per sequence, >= 1 */
+  int V;                       /* vocabulary size, >= 1 */
+  long long ld;                /* row stride in elements, >= V */
+  pspec_dtype dtype;
+  const void *logits;          /* [B, K, ld] */
+  const float *uniforms;       /* [B, K] in [0,1), or NULL for the argmax */
+  int32_t *draft_tokens;       /* [B, K] out */
+  float *q_at_draft;           /* [B, K] out, optional */
+  int32_t *err;                /* device error word (required) */
+} pspec_sample_args;
+
+PSPEC_API size_t pspec_sample_workspace_bytes(int B, int K, int V);
+PSPEC_API pspec_status pspec_sample_drafts(const pspec_sample_args *args, void *workspace,
+                                           size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Draft-batch construction arguments.
  *
  * Verify batch: sequence i owns rows [qsl_in[i], qsl_in[i+1]) of the verify arrays, with

@@ -13,4 +13,7 @@ from ._binding import (  # noqa: F401
     pspec_status_string,
     pspec_verify_greedy, pspec_verify_rejection, pspec_verify_workspace_bytes,
 )
-from .api import Workspace, build_draft_batch, verify_greedy, verify_rejection  # noqa: F401
+from ._binding import pspec_sample_drafts, pspec_sample_workspace_bytes  # noqa: F401
+from .api import (  # noqa: F401
+    Workspace, build_draft_batch, sample_drafts, verify_greedy, verify_rejection,
+)

@@ -27,6 +27,7 @@ EXPORTED = (
     "pspec_verify_workspace_bytes", "pspec_verify_greedy", "pspec_verify_rejection",
     "pspec_build_draft_batch", "pspec_status_string", "pspec_last_launches",
     "pspec_set_verify_path", "pspec_last_verify_path", "pspec_set_cluster_size",
+    "pspec_sample_workspace_bytes", "pspec_sample_drafts",
     "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
 )
 
@@ -48,6 +49,13 @@ class pspec_verify_args(ctypes.Structure):
         ("out_tokens", _P), ("accepted_len", _P), ("bonus", _P),
         ("target_lse", _P), ("draft_lse", _P), ("p_at_draft", _P), ("q_at_draft", _P),
         ("residual_mass", _P), ("err", _P),
+    ]
+
+
+class pspec_sample_args(ctypes.Structure):
+    _fields_ = [
+        ("B", _I), ("K", _I), ("V", _I), ("ld", ctypes.c_longlong), ("dtype", _I),
+        ("logits", _P), ("uniforms", _P), ("draft_tokens", _P), ("q_at_draft", _P), ("err", _P),
     ]
 
 
@@ -74,6 +82,10 @@ def _load():
     for fn in ("pspec_verify_greedy", "pspec_verify_rejection"):
         getattr(lib, fn).argtypes = [ctypes.POINTER(pspec_verify_args), _P, ctypes.c_size_t, _P]
         getattr(lib, fn).restype = _I
+    lib.pspec_sample_workspace_bytes.argtypes = [_I, _I, _I]
+    lib.pspec_sample_workspace_bytes.restype = ctypes.c_size_t
+    lib.pspec_sample_drafts.argtypes = [ctypes.POINTER(pspec_sample_args), _P, ctypes.c_size_t, _P]
+    lib.pspec_sample_drafts.restype = _I
     lib.pspec_build_draft_batch.argtypes = [ctypes.POINTER(pspec_build_args), _P]
     lib.pspec_build_draft_batch.restype = _I
     lib.pspec_status_string.argtypes = [_I]
@@ -132,9 +144,10 @@ def _logits_layout(t: torch.Tensor, rows: int, name: str):
     if t.dtype not in _DT:
         raise TypeError(f"{name} must be float32 or bfloat16, got {t.dtype}")
     B, _, V = t.shape
-    if t.stride(2) != 1 or (B > 0 and t.stride(0) != rows * t.stride(1)) or t.stride(1) < V:
+    ld = t.stride(1) if rows > 1 else t.stride(0)      # one row per sequence: the batch stride
+    if (V > 1 and t.stride(2) != 1) or (B > 1 and t.stride(0) != rows * ld) or ld < V:
         raise ValueError(f"{name} must be row-major with a uniform row stride")
-    return B, V, t.stride(1), _DT[t.dtype]
+    return B, V, ld, _DT[t.dtype]
 
 
 # --------------------------------------------------------------------------- entry points
@@ -225,6 +238,27 @@ def pspec_verify_rejection(*, target_logits, draft_logits, draft_tokens, uniform
                                     workspace.numel(), _stream(stream))
     if st != PSPEC_OK:
         raise PspecError("pspec_verify_rejection", st)
+
+
+def pspec_sample_workspace_bytes(B: int, K: int, V: int) -> int:
+    return int(LIB.pspec_sample_workspace_bytes(int(B), int(K), int(V)))
+
+
+def pspec_sample_drafts(*, logits, draft_tokens, err, workspace, uniforms=None, q_at_draft=None,
+                        stream=None) -> None:
+    K = int(logits.shape[1])
+    Bn, V, ld, dt = _logits_layout(logits, K, "logits")
+    a = pspec_sample_args()
+    a.B, a.K, a.V, a.ld, a.dtype = Bn, K, V, ld, dt
+    a.logits = logits.data_ptr()
+    a.uniforms = _ptr(uniforms, torch.float32, "uniforms")
+    a.draft_tokens = _ptr(draft_tokens, torch.int32, "draft_tokens")
+    a.q_at_draft = _ptr(q_at_draft, torch.float32, "q_at_draft")
+    a.err = _ptr(err, torch.int32, "err")
+    st = LIB.pspec_sample_drafts(ctypes.byref(a), _ptr(workspace, torch.uint8, "workspace"),
+                                 workspace.numel(), _stream(stream))
+    if st != PSPEC_OK:
+        raise PspecError("pspec_sample_drafts", st)
 
 
 def pspec_build_draft_batch(*, K, block_size, mask_id, pad_id, T_cap, qsl_in, verify_tokens,

@@ -81,6 +81,27 @@ def verify_rejection(target_logits: torch.Tensor, draft_logits: torch.Tensor,
     return o
 
 
+def sample_drafts(logits: torch.Tensor, uniforms: torch.Tensor | None = None, *,
+                  want_probs: bool = False, workspace: torch.Tensor | None = None,
+                  out=None, stream=None) -> dict:
+    """Draft tokens from drafter logits [B, K, V]: inverse-CDF sampling with uniforms
+    [B, K], or the argmax when uniforms is None.  Returns draft_tokens, err (+ q_at_draft)."""
+    Bn, K, V = logits.shape
+    dev = logits.device
+    o = out if out is not None else {
+        "draft_tokens": torch.empty((Bn, K), dtype=torch.int32, device=dev),
+        "err": torch.zeros((1,), dtype=torch.int32, device=dev),
+    }
+    if want_probs and "q_at_draft" not in o:
+        o["q_at_draft"] = torch.empty((Bn, K), dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else torch.zeros(
+        max(256, _b.pspec_sample_workspace_bytes(Bn, K, V)), dtype=torch.uint8, device=dev)
+    _b.pspec_sample_drafts(logits=logits, draft_tokens=o["draft_tokens"], err=o["err"],
+                           workspace=ws, uniforms=uniforms, q_at_draft=o.get("q_at_draft"),
+                           stream=stream)
+    return o
+
+
 def build_outputs(Bn: int, K: int, H: int, T_cap: int, hidden_dtype, device) -> dict:
     i32 = dict(dtype=torch.int32, device=device)
     return {

@@ -206,6 +206,43 @@ pspec_status pspec_build_draft_batch(const pspec_build_args* a, cudaStream_t str
   return PSPEC_OK;
 }
 
+size_t pspec_sample_workspace_bytes(int B, int K, int V) {
+  if (B < 0 || K < 1 || V < 1) return 0;
+  // sized for the smaller fp32 chunks, so one workspace serves either dtype
+  return make_sample_plan((long long)B * K, V, sample_chunk_elems(PSPEC_F32)).bytes;
+}
+
+pspec_status pspec_sample_drafts(const pspec_sample_args* a, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  if (!a) return PSPEC_ERR_INVALID_ARG;
+  if (a->B < 0 || a->K < 1 || a->V < 1 || a->ld < a->V) return PSPEC_ERR_INVALID_ARG;
+  if (!dtype_ok(a->dtype) || !a->err) return PSPEC_ERR_INVALID_ARG;
+  if (a->B == 0) { t_last_launches = 0; return PSPEC_OK; }
+  if (!a->logits || !a->draft_tokens) return PSPEC_ERR_INVALID_ARG;
+  if (!aligned_to(a->logits, elem_bytes(a->dtype))) return PSPEC_ERR_INVALID_ARG;
+  const long long rows = (long long)a->B * a->K;
+  const SamplePlan p = make_sample_plan(rows, a->V, sample_chunk_elems(a->dtype));
+  if (rows * p.S >= 0x7fffffffLL) return PSPEC_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < p.bytes)
+    return PSPEC_ERR_WORKSPACE;
+  SampleLaunch L{};
+  L.rows = rows; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
+  L.tiles = p.tiles; L.tiles_per_seg = p.tiles_per_seg; L.S = p.S;
+  L.logits = a->logits;
+  L.uniforms = a->uniforms;
+  L.tokens = a->draft_tokens;
+  L.probs = a->q_at_draft;
+  L.err = a->err;
+  char* ws = static_cast<char*>(workspace);
+  L.cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+  L.parts = ws + p.off_parts;
+  L.maxes = ws + p.off_maxes;
+  if (launch_sample(L, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
+  t_last_launches = 1;
+  return PSPEC_OK;
+}
+
 const char* pspec_status_string(pspec_status s) {
   switch (s) {
     case PSPEC_OK: return "PSPEC_OK";

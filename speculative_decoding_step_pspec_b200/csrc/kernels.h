@@ -73,6 +73,24 @@ struct EarlyExitLaunch {
   int32_t* err;
 };
 
+struct SampleLaunch {
+  long long rows;        // B*K drafter rows
+  int V;
+  long long ld;
+  pspec_dtype dtype;
+  int tiles;             // chunks per row (2048 bf16 / 1024 fp32 elements)
+  int tiles_per_seg;     // chunks per CTA
+  int S;                 // CTAs per row
+  const void* logits;
+  const float* uniforms; // NULL: argmax
+  int32_t* tokens;
+  float* probs;          // optional
+  int32_t* err;
+  int* cnt;              // workspace: tickets [rows]
+  void* parts;           // workspace: (m, s) per chunk [rows*tiles]
+  void* maxes;           // workspace: (max, index) per chunk [rows*tiles]
+};
+
 struct BuildLaunch {
   pspec_build_args a;
   long long row_vecs;    // 16-byte vectors per hidden row
@@ -85,5 +103,6 @@ cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream);
 cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream, cudaEvent_t split_event);
 cudaError_t launch_build(const BuildLaunch& L, cudaStream_t stream);
 cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream);
+cudaError_t launch_sample(const SampleLaunch& L, cudaStream_t stream);
 
 }  // namespace pspec

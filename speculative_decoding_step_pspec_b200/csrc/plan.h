@@ -122,4 +122,34 @@ inline EarlyExitPlan make_early_exit_plan(int V, int G) {
   return p;
 }
 
+// Draft sampling: rows x S CTAs over chunks of 32 lanes x kSampleGroups(dtype) groups of 8
+// elements (2048 bf16 / 1024 fp32 elements: eight 16-byte loads per lane), each warp taking
+// every eighth chunk of its CTA's segment; workspace = tickets + two partials per chunk.
+inline int sample_chunk_elems(pspec_dtype dt) { return dt == PSPEC_BF16 ? 2048 : 1024; }
+
+struct SamplePlan {
+  int tiles, tiles_per_seg, S;    // chunks per row, chunks per CTA, CTAs per row
+  size_t off_cnt, off_parts, off_maxes, bytes;
+};
+
+inline SamplePlan make_sample_plan(long long rows, int V, int chunk_elems) {
+  SamplePlan p{};
+  p.tiles = (int)(((long long)V + chunk_elems - 1) / chunk_elems);
+  long long S = rows > 0 ? (kTargetCtas + rows - 1) / rows : 1;
+  const long long s_hi = (p.tiles + kWarps - 1) / kWarps;   // at least one chunk per warp
+  if (S > s_hi) S = s_hi;
+  if (S < 1) S = 1;
+  p.tiles_per_seg = (int)((p.tiles + S - 1) / S);
+  p.S = (p.tiles + p.tiles_per_seg - 1) / p.tiles_per_seg;
+  size_t off = 0;
+  p.off_cnt = off;
+  off = align256(off + sizeof(int32_t) * (size_t)rows);
+  p.off_parts = off;
+  off = align256(off + 8 * (size_t)rows * p.tiles);
+  p.off_maxes = off;
+  off = align256(off + 8 * (size_t)rows * p.tiles);
+  p.bytes = off;
+  return p;
+}
+
 }  // namespace pspec

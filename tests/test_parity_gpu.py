@@ -453,3 +453,102 @@ def test_build_empty_batch_pads():
                verify_hidden=torch.zeros((0, 8), dtype=torch.float32, device=DEV),
                h_shared=torch.zeros(8, dtype=torch.float32, device=DEV))
     _build_and_compare(inp)
+
+
+# --------------------------------------------------------------------------- draft sampling
+def _sample_both(logits, u, seqs=None):
+    """Inverse-CDF sampling and argmax of drafter rows [B, K, V] against the oracle."""
+    B, K, V = logits.shape
+    s = ps.sample_drafts(logits, u, want_probs=True)
+    g = ps.sample_drafts(logits, None, want_probs=True)
+    torch.cuda.synchronize()
+    assert s["err"].item() == 0 and g["err"].item() == 0
+    idx = slice(None) if seqs is None else torch.as_tensor(seqs, device=logits.device)
+    host = U.host_logits(logits[idx])
+    os_ = oracle.sample_rows(host, u[idx].cpu().numpy(), threads=U.THREADS)
+    og = oracle.sample_rows(host, None, threads=U.THREADS)
+    sel = slice(None) if seqs is None else np.asarray(seqs)
+    st = s["draft_tokens"].cpu().numpy()[sel]
+    gt = g["draft_tokens"].cpu().numpy()[sel]
+    assert np.array_equal(gt, og["tokens"]), np.argwhere(gt != og["tokens"])[:5]
+    clean = os_["flags"] == 0
+    bad = np.argwhere((st != os_["tokens"]) & clean)
+    assert bad.size == 0, (bad[:5], st[tuple(bad[:5].T)], os_["tokens"][tuple(bad[:5].T)])
+    for out, o in ((s, os_), (g, og)):
+        pr = out["q_at_draft"].cpu().numpy()[sel]
+        same = out["draft_tokens"].cpu().numpy()[sel] == o["tokens"]
+        ok = U._rel_ok(pr, o["probs"]) | ~same
+        assert ok.all(), (pr[~ok][:5], o["probs"][~ok][:5])
+    x = logits.float()
+    tok = s["draft_tokens"].long()
+    live = torch.isfinite(x).any(-1)                  # rows with some mass never pick -inf
+    assert torch.isfinite(torch.gather(x, 2, tok[..., None]))[..., 0][live].all()
+    print(f"[sampling] {clean.size} rows, {int((~clean).sum())} flagged near-ties")
+
+
+@pytest.mark.parametrize("name", ["tiny", "c1", "c64"])
+def test_sampling_workloads(name):
+    if name == "tiny":
+        t = I.tiny_verify_numpy()
+        logits = torch.from_numpy(t["draft"]).to(DEV)
+        u = torch.from_numpy(t["uniforms"][:, :logits.shape[1]].copy()).to(DEV)
+    else:
+        w = I.WORKLOADS[name]
+        _, logits = I.logits(w, DEV)
+        u = I.uniforms(w, DEV)[:, :w.K].contiguous()
+    _sample_both(logits, u)
+
+
+def test_sampling_b1024_sampled():
+    w = I.B1024
+    _, logits = I.logits(w, DEV)
+    u = I.uniforms(w, DEV)[:, :w.K].contiguous()
+    _sample_both(logits, u, seqs=_sample(w.B, 32, 11))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("V", [1, 7, 8, 255, 257, 2047, 5003, 70001, 262144])
+def test_sampling_ragged(dtype, V):
+    w = I.Workload("t", 3, 4, V, 16, 4, dtype, seed=V, sigma_t=2.0, sigma_d=0.6)
+    _, logits = I.logits(w, DEV)
+    _sample_both(logits, I.uniforms(w, DEV)[:, :4].contiguous())
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_sampling_padded_stride_and_neg_inf(dtype):
+    B, K, V, ld = 4, 3, 3001, 3016
+    g = torch.Generator(device=DEV).manual_seed(3)
+    buf = torch.full((B, K, ld), 77.0, dtype=dtype, device=DEV)
+    buf[:, :, :V] = (torch.randn((B, K, V), generator=g, device=DEV) * 2).to(dtype)
+    buf[0, 0, :V:2] = -float("inf")
+    buf[1, 2, :] = -float("inf")                     # a row with no mass: token 0, p 0
+    logits = buf[:, :, :V]
+    u = torch.rand((B, K), generator=g, device=DEV)
+    _sample_both(logits, u)
+
+
+def test_sampling_threshold_probing():
+    """The token at the middle of every CDF interval is that interval's token."""
+    import scipy.special as sps
+    rng = np.random.default_rng(8)
+    rows = rng.normal(0, 1.5, size=(5, 8)).astype(np.float32)
+    P = sps.softmax(rows.astype(np.float64), axis=1)
+    F = np.concatenate([np.zeros((5, 1)), np.cumsum(P, axis=1)], axis=1)
+    lg, uu, want = [], [], []
+    for n in range(5):
+        for t in range(8):
+            if F[n, t + 1] - F[n, t] < 1e-5:
+                continue
+            lg.append(rows[n]); uu.append((F[n, t] + F[n, t + 1]) / 2); want.append(t)
+    L = torch.from_numpy(np.stack(lg)[:, None, :]).to(DEV)
+    U_ = torch.tensor(np.array(uu, np.float32)[:, None], device=DEV)
+    got = ps.sample_drafts(L, U_)["draft_tokens"][:, 0].cpu().numpy()
+    assert np.array_equal(got, np.array(want))
+
+
+def test_sampling_empty_and_errors():
+    L = torch.empty((0, 3, 100), dtype=torch.bfloat16, device=DEV)
+    ps.sample_drafts(L, None)
+    with pytest.raises(ps.PspecError):
+        ws = torch.zeros(256, dtype=torch.uint8, device=DEV)       # too small
+        ps.sample_drafts(torch.zeros((2, 3, 100), device=DEV), None, workspace=ws)
