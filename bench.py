@@ -42,8 +42,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["pspec", "reference"], default="pspec")
     p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
-    p.add_argument("--path", choices=["auto", "sweep", "early"], default="auto",
-                   help="verify path: automatic selection, full sweep, or early exit")
+    p.add_argument("--path", choices=["auto", "sweep", "early", "queue"], default="auto",
+                   help="verify path: automatic selection, full sweep, early exit, or work queue")
     p.add_argument("--cluster", type=int, default=0, help="early-exit cluster size (0 auto)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
@@ -241,7 +241,7 @@ def run_pspec(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2}[args.path])
+    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3}[args.path])
     ps.pspec_set_cluster_size(args.cluster)
     w, d = make_workload(args.workload, dev, rank, args.batch)
     rej = args.mode == "rejection"
@@ -306,13 +306,19 @@ def run_pspec(args, rank, world, local_rank):
     draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if rej else None
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
     acc = vout["accepted_len"].cpu().numpy()
-    early = path == 2
+    early = path in (2, 3)                  # paths that read rows only up to a_i
     vbytes, bbytes = algorithmic_bytes(w, args.mode, acc, early)
     full_vbytes, _ = algorithmic_bytes(w, args.mode, acc, False)
     hbm, peak_src = peaks()
     ms_step = elapsed_ms / K
     step_gbs = (vbytes + bbytes) / (ms_step * 1e-3) / 1e9
-    if early:
+    if path == 3:
+        dom_kernel = "queue_kernel"
+        src = ["speculative_decoding_step_pspec_b200/csrc/verify_queue.cu",
+               "speculative_decoding_step_pspec_b200/csrc/verify_draw.cuh",
+               "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
+               "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
+    elif early:
         dom_kernel = "ee_kernel"
         src = ["speculative_decoding_step_pspec_b200/csrc/verify_early_exit.cu",
                "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
@@ -337,7 +343,8 @@ def run_pspec(args, rank, world, local_rank):
             "workload": f"{args.workload}{'' if not args.batch else ' (B overridden)'}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
                         f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
-            "verify_path": "early exit (cluster per sequence)" if early else "full sweep",
+            "verify_path": {1: "full sweep", 2: "early exit (cluster per sequence)",
+                            3: "work queue (persistent, position order)"}[path],
             "l2": "inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9),
             "parallelism": f"replicas x{world} (independent sequences, no collective)",
         },

@@ -126,8 +126,12 @@ typedef struct {
  * Workspace for the verify calls: scratch device memory owned by the caller, at least
  * pspec_verify_workspace_bytes(B, K, V, rejection) bytes, 256-byte aligned.  It must be
  * zero-filled once (cudaMemsetAsync) before its first use; every call leaves its
- * per-sequence counters back at zero, so later calls need no re-initialisation.  Calls
- * that share one workspace must not overlap on the GPU (use one workspace per stream).
+ * counters back at zero, so later calls need no re-initialisation.  The counters sit at
+ * the end of the workspace (the address plus the byte count passed with each call, so
+ * pass the same count every time), at addresses that depend on neither B nor K: a
+ * workspace sized for B sequences serves every later call with at most B sequences, on
+ * any verify path.  Calls that share one workspace must not overlap on the GPU (use one
+ * workspace per stream).
  */
 PSPEC_API size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection);
 
@@ -177,7 +181,9 @@ PSPEC_API pspec_status pspec_verify_rejection(const pspec_verify_args *args, voi
  * keeps (max, sum exp) or (max, first index); the CTA finishing a row turns the chunk
  * partials into the token and rescans one chunk.  Workspace:
  * pspec_sample_workspace_bytes(B, K, V) bytes (enough for either dtype), 256-byte aligned,
- * zero-filled once before first use (each call leaves its counters at zero).  Returns
+ * zero-filled once before first use (each call leaves its counters at zero; they sit at
+ * the end of the workspace, one per row, so a workspace sized for B*K rows serves any
+ * call with fewer rows when the same byte count is passed).  Returns
  * PSPEC_ERR_INVALID_ARG for bad sizes, pointers or dtype, PSPEC_ERR_WORKSPACE for a
  * missing, misaligned or short workspace, PSPEC_ERR_CUDA when the launch fails.
  */
@@ -302,8 +308,16 @@ PSPEC_API int pspec_last_launches(void);
      requested (target_lse, draft_lse, p_at_draft, q_at_draft all NULL), V is a multiple
      of 8 and the logits rows start on 16-byte boundaries; otherwise the full sweep;
    1 always the full sweep;
-   2 always the early-exit path (PSPEC_ERR_UNSUPPORTED when the arguments do not allow it).
-   Both paths give the same outputs; they differ in which rows they read. */
+   2 always the early-exit path (PSPEC_ERR_UNSUPPORTED when the arguments do not allow it);
+   3 always the work-queue path: one persistent launch whose CTAs pull (sequence,
+     position) items cut into row segments from an on-device queue, in position order; the
+     CTA completing an item applies the rule and appends the next position, or the draw,
+     as new units (PSPEC_ERR_UNSUPPORTED with a per-row diagnostic requested,
+     PSPEC_ERR_WORKSPACE when the workspace is smaller than
+     pspec_verify_workspace_bytes).  Any V, ld and element alignment.  Every wait in that
+     kernel is bounded: when one runs out it sets PSPEC_DEVERR_TIMEOUT, the outputs are
+     undefined, and the kernel clears the queue state before it ends.
+   All paths give the same outputs; they differ in which rows they read. */
 PSPEC_API void pspec_set_verify_path(int path);
 
 /* Tuning: CTAs per thread-block cluster on the early-exit path (2, 4, 8 or 16; each CTA
@@ -312,7 +326,7 @@ PSPEC_API void pspec_set_verify_path(int path);
 PSPEC_API void pspec_set_cluster_size(int G);
 
 /* The path the most recent successful verify call on this host thread took: 1 full sweep,
-   2 early exit, 0 none yet. */
+   2 early exit, 3 work queue, 0 none yet. */
 PSPEC_API int pspec_last_verify_path(void);
 
 /* Tuning: force the verify sweeps' segment length (elements of one row handled by one

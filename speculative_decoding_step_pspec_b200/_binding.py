@@ -166,12 +166,13 @@ def pspec_set_cluster_size(G: int) -> None:
 
 
 def pspec_last_verify_path() -> int:
-    """1 full sweep, 2 early exit: the path of the most recent verify call on this thread."""
+    """1 full sweep, 2 early exit, 3 work queue: the path of the most recent verify call on
+    this thread."""
     return LIB.pspec_last_verify_path()
 
 
 def pspec_set_verify_path(path: int) -> None:
-    """0 automatic, 1 full sweep, 2 early exit (see include/pspec.h)."""
+    """0 automatic, 1 full sweep, 2 early exit, 3 work queue (see include/pspec.h)."""
     LIB.pspec_set_verify_path(int(path))
 
 

@@ -15,7 +15,7 @@ using namespace pspec;
 
 long long g_seg_override = 0;   // 0 = automatic segment length
 cudaEvent_t g_split_event = nullptr;
-int g_verify_path = 0;          // 0 automatic, 1 full sweep, 2 early exit
+int g_verify_path = 0;          // 0 automatic, 1 full sweep, 2 early exit, 3 work queue
 int g_cluster = 0;              // early-exit cluster size; 0 = automatic
 thread_local int t_last_launches = 0;
 thread_local int t_last_path = 0;
@@ -87,10 +87,66 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   return true;
 }
 
-pspec_status check_workspace(void* ws, size_t bytes, const VerifyPlan& p) {
-  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < p.bytes)
-    return PSPEC_ERR_WORKSPACE;
+// The caller's workspace: 256-byte aligned, `scratch` bytes from its start and the zero area
+// of B sequences below its (aligned) end; *z receives the zero area.
+pspec_status check_workspace(void* ws, size_t bytes, size_t scratch, long long B, ZeroArea* z) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return PSPEC_ERR_WORKSPACE;
+  if (bytes < align256(scratch) + zero_area_bytes(B)) return PSPEC_ERR_WORKSPACE;
+  *z = zero_area(ws, bytes, B);
+  if (static_cast<char*>(ws) + scratch > z->lowest) return PSPEC_ERR_WORKSPACE;
   return PSPEC_OK;
+}
+
+// The work-queue path (one persistent launch), when forced.  Returns true and sets *st
+// when it handled the call.
+bool try_queue(const pspec_verify_args* a, bool rejection, void* workspace, size_t bytes,
+               cudaStream_t stream, pspec_status* st) {
+  if (g_verify_path != 3) return false;
+  const bool diagnostics = a->target_lse || a->draft_lse || a->p_at_draft || a->q_at_draft;
+  if (diagnostics) {
+    *st = PSPEC_ERR_UNSUPPORTED;              // rows after a_i are never read on this path
+    return true;
+  }
+  if (a->B >= (1 << 26)) {                     // items pack i << 5 | k into an int
+    *st = PSPEC_ERR_UNSUPPORTED;
+    return true;
+  }
+  const QueuePlan p = make_queue_plan(a->B, a->K, a->V, rejection);
+  ZeroArea z;
+  *st = check_workspace(workspace, bytes, p.bytes, a->B, &z);
+  if (*st != PSPEC_OK) return true;
+  QueueLaunch L{};
+  L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
+  L.rejection = rejection;
+  L.S = p.S; L.seg = p.seg;
+  L.tiles = p.tiles; L.tiles_per_unit = p.tiles_per_unit; L.C = p.C;
+  L.target = a->target_logits;
+  L.draft = a->draft_logits;
+  L.draft_tokens = a->draft_tokens;
+  L.uniforms = a->uniforms;
+  L.out_tokens = a->out_tokens;
+  L.accepted_len = a->accepted_len;
+  L.bonus = a->bonus;
+  L.residual_mass = rejection ? a->residual_mass : nullptr;
+  L.err = a->err;
+  char* ws = static_cast<char*>(workspace);
+  L.ctr = z.ctr;
+  L.items = z.line0 + kZwItems;
+  L.draws = z.line0 + kZwDraw;
+  L.cnt = z.line0 + kZwQCnt;
+  L.cnt2 = z.line0 + kZwQCnt2;
+  L.part = ws + p.off_part;
+  L.seq = ws + p.off_seq;
+  L.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
+  if (launch_queue(L, stream) != cudaSuccess) {
+    *st = PSPEC_ERR_CUDA;
+    return true;
+  }
+  if (rejection && g_split_event) cudaEventRecord(g_split_event, stream);
+  t_last_launches = 1;
+  t_last_path = 3;
+  *st = PSPEC_OK;
+  return true;
 }
 
 }  // namespace
@@ -99,7 +155,9 @@ extern "C" {
 
 size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection) {
   if (B < 0 || K < 1 || K > PSPEC_MAX_K || V < 1) return 0;
-  return make_verify_plan(B, K, V, rejection, g_seg_override).bytes;
+  const size_t sweep = align256(make_verify_plan(B, K, V, rejection, g_seg_override).bytes);
+  const size_t queue = align256(make_queue_plan(B, K, V, rejection).bytes);
+  return (sweep > queue ? sweep : queue) + zero_area_bytes(B);
 }
 
 pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
@@ -108,8 +166,10 @@ pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
   if (st != PSPEC_OK) return st;
   if (a->B == 0) { t_last_launches = 0; return st; }
   const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 0, g_seg_override);
-  st = check_workspace(workspace, workspace_bytes, p);
+  ZeroArea z;
+  st = check_workspace(workspace, workspace_bytes, p.bytes, a->B, &z);
   if (st != PSPEC_OK) return st;
+  if (try_queue(a, false, workspace, workspace_bytes, stream, &st)) return st;
   if (try_early_exit(a, false, stream, &st)) return st;
   GreedyLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
@@ -122,7 +182,7 @@ pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
   L.target_lse = a->target_lse;
   L.err = a->err;
   char* ws = static_cast<char*>(workspace);
-  L.cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+  L.cnt = z.line0 + kZwSCnt;
   L.part = ws + p.off_part;
   if (launch_greedy(L, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
   t_last_launches = 1;
@@ -136,8 +196,10 @@ pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
   if (st != PSPEC_OK) return st;
   if (a->B == 0) { t_last_launches = 0; return st; }
   const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 1, g_seg_override);
-  st = check_workspace(workspace, workspace_bytes, p);
+  ZeroArea z;
+  st = check_workspace(workspace, workspace_bytes, p.bytes, a->B, &z);
   if (st != PSPEC_OK) return st;
+  if (try_queue(a, true, workspace, workspace_bytes, stream, &st)) return st;
   if (try_early_exit(a, true, stream, &st)) return st;
   RejectionLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
@@ -157,8 +219,8 @@ pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
   L.residual_mass = a->residual_mass;
   L.err = a->err;
   char* ws = static_cast<char*>(workspace);
-  L.cnt = reinterpret_cast<int*>(ws + p.off_cnt);
-  L.cnt2 = reinterpret_cast<int*>(ws + p.off_cnt2);
+  L.cnt = z.line0 + kZwSCnt;
+  L.cnt2 = z.line0 + kZwSCnt2;
   L.part = ws + p.off_part;
   L.seq = ws + p.off_seq;
   L.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
@@ -226,6 +288,9 @@ pspec_status pspec_sample_drafts(const pspec_sample_args* a, void* workspace,
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < p.bytes)
     return PSPEC_ERR_WORKSPACE;
+  // tickets at the aligned end, one per row, so calls with other batch sizes find them at 0
+  int32_t* tickets_end = reinterpret_cast<int32_t*>(
+      (reinterpret_cast<uintptr_t>(workspace) + workspace_bytes) & ~uintptr_t(255));
   SampleLaunch L{};
   L.rows = rows; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.tiles = p.tiles; L.tiles_per_seg = p.tiles_per_seg; L.S = p.S;
@@ -235,7 +300,7 @@ pspec_status pspec_sample_drafts(const pspec_sample_args* a, void* workspace,
   L.probs = a->q_at_draft;
   L.err = a->err;
   char* ws = static_cast<char*>(workspace);
-  L.cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+  L.cnt = tickets_end;
   L.parts = ws + p.off_parts;
   L.maxes = ws + p.off_maxes;
   if (launch_sample(L, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
@@ -258,7 +323,7 @@ int pspec_last_launches(void) { return t_last_launches; }
 
 int pspec_last_verify_path(void) { return t_last_path; }
 
-void pspec_set_verify_path(int path) { g_verify_path = (path == 1 || path == 2) ? path : 0; }
+void pspec_set_verify_path(int path) { g_verify_path = (path >= 1 && path <= 3) ? path : 0; }
 
 void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || G == 16) ? G : 0; }
 

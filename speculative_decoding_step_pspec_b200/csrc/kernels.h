@@ -24,7 +24,7 @@ struct GreedyLaunch {
   int32_t* bonus;
   float* target_lse;     // optional
   int32_t* err;
-  int* cnt;              // workspace: tickets [B]
+  int* cnt;              // zero area: ticket column (entry i = zcol(cnt, i))
   void* part;            // workspace: GreedyPart [B*(K+1)*S]
 };
 
@@ -48,8 +48,8 @@ struct RejectionLaunch {
   float* q_at_draft;     // optional
   float* residual_mass;  // optional
   int32_t* err;
-  int* cnt;              // workspace: sweep tickets [B]
-  int* cnt2;             // workspace: resample tickets [B]
+  int* cnt;              // zero area: sweep ticket column (zcol)
+  int* cnt2;             // zero area: resample ticket column (zcol)
   void* part;            // workspace: RejPart [B*(2K+1)*S]
   void* seq;             // workspace: SeqInfo [B]
   double* tile_sums;     // workspace: [B*tiles] sums of r over 256-element tiles
@@ -86,9 +86,39 @@ struct SampleLaunch {
   int32_t* tokens;
   float* probs;          // optional
   int32_t* err;
-  int* cnt;              // workspace: tickets [rows]
+  int* cnt;              // end of the workspace: ticket of row r = zrow(cnt, r)
   void* parts;           // workspace: (m, s) per chunk [rows*tiles]
   void* maxes;           // workspace: (max, index) per chunk [rows*tiles]
+};
+
+struct QueueLaunch {
+  int B, K, V;
+  long long ld;
+  pspec_dtype dtype;
+  int rejection;         // 1: rejection rule, 0: greedy
+  int S;                 // segments per row
+  long long seg;         // elements per segment
+  int tiles;             // 256-element draw tiles per row
+  int tiles_per_unit;    // draw tiles per draw unit
+  int C;                 // draw units per sequence
+  const void* target;
+  const void* draft;
+  const int32_t* draft_tokens;
+  const float* uniforms;
+  int32_t* out_tokens;
+  int32_t* accepted_len;
+  int32_t* bonus;
+  float* residual_mass;  // optional
+  int32_t* err;
+  unsigned long long* ctr;  // zero area: queue counters [8]
+  int* items;            // zero area: line 0 (item slot s = zitem(items, s)), holding
+                         // (i*32 + k) + 1 once published, 0 before
+  int* draws;            // zero area: draw slot column (zcol), i + 1 once published
+  int* cnt;              // zero area: stream-unit ticket column (zcol)
+  int* cnt2;             // zero area: draw-unit ticket column (zcol)
+  void* part;            // workspace: 8-byte partials [B*R*S]
+  void* seq;             // workspace: SeqInfo [B]
+  double* tile_sums;     // workspace: [B*tiles]
 };
 
 struct BuildLaunch {
@@ -101,6 +131,7 @@ struct BuildLaunch {
 cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream);
 // split_event (may be null) is recorded between the statistics sweep and the draw.
 cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream, cudaEvent_t split_event);
+cudaError_t launch_queue(const QueueLaunch& L, cudaStream_t stream);
 cudaError_t launch_build(const BuildLaunch& L, cudaStream_t stream);
 cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream);
 cudaError_t launch_sample(const SampleLaunch& L, cudaStream_t stream);

@@ -67,13 +67,15 @@ extern "C" pspec_status pspec_verify_greedy_noalloc(const pspec_verify_args* a,
 
   // Always the automatic segment length: the scratch bound must not move with tuning.
   const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 0, 0);
-  if (p.bytes > kNoAllocScratchBytes) return PSPEC_ERR_UNSUPPORTED;
+  if (align256(p.bytes) + zero_area_bytes(a->B) > kNoAllocScratchBytes) return PSPEC_ERR_UNSUPPORTED;
 
   void* scratch = nullptr;
   if (scratch_of_current_device(&scratch) != cudaSuccess) return PSPEC_ERR_CUDA;
   char* ws = static_cast<char*>(scratch);
-  // the tickets must start at zero whatever an earlier call left behind
-  if (cudaMemsetAsync(ws + p.off_cnt, 0, sizeof(int) * (size_t)a->B, stream) != cudaSuccess)
+  const ZeroArea z = zero_area(scratch, kNoAllocScratchBytes, a->B);
+  // the tickets (the zero area's lines of sequences 0..B-1) must start at zero whatever an
+  // earlier call left behind
+  if (cudaMemsetAsync(z.lowest, 0, kLineBytes * (size_t)a->B, stream) != cudaSuccess)
     return PSPEC_ERR_CUDA;
 
   GreedyLaunch L{};
@@ -86,7 +88,7 @@ extern "C" pspec_status pspec_verify_greedy_noalloc(const pspec_verify_args* a,
   L.bonus = a->bonus;
   L.target_lse = a->target_lse;
   L.err = a->err;
-  L.cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+  L.cnt = z.line0 + kZwSCnt;
   L.part = ws + p.off_part;
   return launch_greedy(L, stream) == cudaSuccess ? PSPEC_OK : PSPEC_ERR_CUDA;
 }

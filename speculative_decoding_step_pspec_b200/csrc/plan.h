@@ -49,15 +49,63 @@ struct VerifyPlan {
   int tiles;              // draw tiles per row
   int tiles_per_chunk;    // draw tiles per CTA of the separate draw launch
   int C;                  // CTAs per sequence of the separate draw launch
-  size_t off_cnt;         // int32[B]  sweep tickets
-  size_t off_cnt2;        // int32[B]  resample tickets
   size_t off_part;        // partials [B*rows*S]
   size_t off_seq;         // SeqInfo[B]
   size_t off_tiles;       // double[B*tiles]
-  size_t bytes;           // total
+  size_t bytes;           // scratch bytes (the zero area comes on top, see zero_area)
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Words that must be zero when a call starts (tickets, queue slots, queue counters) live at
+// the END of the caller's workspace, and scratch (partials, statistics, tile sums) grows
+// from its start.  The zero words are laid out backwards from the end, one line of
+// kLineWords words per index, so that their addresses depend on neither B nor K: a call
+// with a smaller batch finds every counter a larger call left at zero, and its scratch
+// never reaches them.  Line j (j = 0, 1, ...) holds queue item slots 32j .. 32j+31 and the
+// per-sequence words of sequence j.
+constexpr int kLineWords = 40;
+constexpr size_t kLineBytes = kLineWords * sizeof(int32_t);
+constexpr size_t kCtrBytes = 256;        // queue counters, just below the aligned end
+enum : int {
+  kZwItems = 0,     // 32 queue item slots
+  kZwDraw = 32,     // queue draw slot
+  kZwQCnt = 33,     // queue stream-unit ticket
+  kZwQCnt2 = 34,    // queue draw-unit ticket
+  kZwSCnt = 35,     // sweep ticket
+  kZwSCnt2 = 36,    // sweep draw ticket
+};
+
+// Bytes of zero area for B sequences (with slack for aligning the end down to 256 bytes).
+inline size_t zero_area_bytes(long long B) {
+  return kCtrBytes + ((size_t)B * kLineBytes + 255) / 256 * 256 + 256;
+}
+
+struct ZeroArea {
+  unsigned long long* ctr;   // 8 queue counters
+  int32_t* line0;            // word 0 of line 0; line j starts kLineWords * j words lower
+  char* lowest;              // first byte of line B-1 (scratch must end at or below it)
+};
+
+inline ZeroArea zero_area(void* ws, size_t bytes, long long B) {
+  const uintptr_t end = (reinterpret_cast<uintptr_t>(ws) + bytes) & ~uintptr_t(255);
+  ZeroArea z;
+  z.ctr = reinterpret_cast<unsigned long long*>(end - kCtrBytes);
+  z.line0 = reinterpret_cast<int32_t*>(end - kCtrBytes - kLineBytes);
+  z.lowest = reinterpret_cast<char*>(end - kCtrBytes) - (size_t)(B > 0 ? B : 1) * kLineBytes;
+  return z;
+}
+
+// Entry i of a zero-area column (col = line0 + word): entries run backwards, a line apart.
+__host__ __device__ __forceinline__ int32_t* zcol(int32_t* col, long long i) {
+  return col - i * kLineWords;
+}
+// Queue item slot s.
+__host__ __device__ __forceinline__ int32_t* zitem(int32_t* line0, long long s) {
+  return zcol(line0 + (s & 31), s >> 5);
+}
+// Entry r of a plain backward array ending at `end` (the sampling tickets).
+__host__ __device__ __forceinline__ int32_t* zrow(int32_t* end, long long r) { return end - 1 - r; }
 
 // seg_override > 0 forces the segment length (rounded up to a multiple of 8).
 inline VerifyPlan make_verify_plan(int B, int K, int V, int rejection, long long seg_override) {
@@ -86,10 +134,6 @@ inline VerifyPlan make_verify_plan(int B, int K, int V, int rejection, long long
   p.C = (p.tiles + p.tiles_per_chunk - 1) / p.tiles_per_chunk;
 
   size_t off = 0;
-  p.off_cnt = off;
-  off = align256(off + sizeof(int32_t) * (size_t)B);
-  p.off_cnt2 = off;
-  off = align256(off + (rejection ? sizeof(int32_t) * (size_t)B : 0));
   p.off_part = off;
   size_t part_sz = rejection ? sizeof(RejPart) : sizeof(GreedyPart);
   off = align256(off + part_sz * (size_t)B * p.rows * p.S);
@@ -122,6 +166,55 @@ inline EarlyExitPlan make_early_exit_plan(int V, int G) {
   return p;
 }
 
+// Work-queue verify: units are segments of about kQueueSeg elements of one row of one
+// (sequence, position) item, draws are cut into units of kQueueDrawTiles warp tiles.
+#ifndef PSPEC_QUEUE_SEG
+#define PSPEC_QUEUE_SEG 65536
+#endif
+constexpr long long kQueueSeg = PSPEC_QUEUE_SEG;
+#ifndef PSPEC_QUEUE_DRAW_TILES
+#define PSPEC_QUEUE_DRAW_TILES 256
+#endif
+constexpr int kQueueDrawTiles = PSPEC_QUEUE_DRAW_TILES;
+
+struct QueuePlan {
+  int R;                  // rows per item: 2 (target + draft, rejection) or 1 (greedy)
+  int S;                  // segments per row
+  long long seg;          // elements per segment
+  int tiles;              // 256-element draw tiles per row
+  int tiles_per_unit;     // draw tiles per draw unit
+  int C;                  // draw units per sequence
+  size_t off_part;        // 8-byte partials [B*R*S]
+  size_t off_seq;         // SeqInfo[B]
+  size_t off_tiles;       // double[B*tiles]
+  size_t bytes;
+};
+
+inline QueuePlan make_queue_plan(int B, int K, int V, int rejection) {
+  QueuePlan p{};
+  p.R = rejection ? 2 : 1;
+  long long S = (V + kQueueSeg - 1) / kQueueSeg;
+  if (S < 1) S = 1;
+  long long seg = (V + S - 1) / S;
+  seg = (seg + 7) / 8 * 8;
+  p.seg = seg;
+  p.S = (int)((V + seg - 1) / seg);
+  p.tiles = (V + kDrawTile - 1) / kDrawTile;
+  int C = (p.tiles + kQueueDrawTiles - 1) / kQueueDrawTiles;
+  if (C < 1) C = 1;
+  p.tiles_per_unit = (p.tiles + C - 1) / C;
+  p.C = (p.tiles + p.tiles_per_unit - 1) / p.tiles_per_unit;
+  size_t off = 0;
+  p.off_part = off;
+  off = align256(off + 8 * (size_t)B * p.R * p.S);
+  p.off_seq = off;
+  off = align256(off + (rejection ? sizeof(SeqInfo) * (size_t)B : 0));
+  p.off_tiles = off;
+  off = align256(off + (rejection ? sizeof(double) * (size_t)B * p.tiles : 0));
+  p.bytes = off;
+  return p;
+}
+
 // Draft sampling: rows x S CTAs over chunks of 32 lanes x kSampleGroups(dtype) groups of 8
 // elements (2048 bf16 / 1024 fp32 elements: eight 16-byte loads per lane), each warp taking
 // every eighth chunk of its CTA's segment; workspace = tickets + two partials per chunk.
@@ -129,7 +222,9 @@ inline int sample_chunk_elems(pspec_dtype dt) { return dt == PSPEC_BF16 ? 2048 :
 
 struct SamplePlan {
   int tiles, tiles_per_seg, S;    // chunks per row, chunks per CTA, CTAs per row
-  size_t off_cnt, off_parts, off_maxes, bytes;
+  size_t off_parts, off_maxes;    // scratch, from the start of the workspace
+  size_t scratch;                 // scratch bytes
+  size_t bytes;                   // scratch + tickets at the end (one int per row) + slack
 };
 
 inline SamplePlan make_sample_plan(long long rows, int V, int chunk_elems) {
@@ -142,13 +237,12 @@ inline SamplePlan make_sample_plan(long long rows, int V, int chunk_elems) {
   p.tiles_per_seg = (int)((p.tiles + S - 1) / S);
   p.S = (p.tiles + p.tiles_per_seg - 1) / p.tiles_per_seg;
   size_t off = 0;
-  p.off_cnt = off;
-  off = align256(off + sizeof(int32_t) * (size_t)rows);
   p.off_parts = off;
   off = align256(off + 8 * (size_t)rows * p.tiles);
   p.off_maxes = off;
   off = align256(off + 8 * (size_t)rows * p.tiles);
-  p.bytes = off;
+  p.scratch = off;
+  p.bytes = off + (sizeof(int32_t) * (size_t)rows + 255) / 256 * 256 + 256;
   return p;
 }
 

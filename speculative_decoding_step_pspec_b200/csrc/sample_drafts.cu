@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, kSampleMinBlocks) sample_kernel(cons
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    const int tk = atomicAdd(L.cnt + row, 1);
+    const int tk = atomicAdd(zrow(L.cnt, row), 1);
     s_last = (tk == L.S - 1);
   }
   __syncthreads();
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, kSampleMinBlocks) sample_kernel(cons
                          ? 0.f
                          : (float)(exp2((double)x * (double)kLog2e - (double)M) / S);
     }
-    L.cnt[row] = 0;
+    *zrow(L.cnt, row) = 0;
   }
 }
 

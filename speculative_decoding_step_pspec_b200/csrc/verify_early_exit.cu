@@ -91,6 +91,59 @@ __device__ __forceinline__ void slice_x8(const DrawRow& D, long long lo, int n, 
   }
 }
 
+// The same eight elements in two steps, so that several groups' loads can be in flight
+// before any of them is unpacked.
+template <typename Tag>
+struct SliceRaw {
+  uint4 t[8 / Tag::kVec], q[8 / Tag::kVec];
+  bool live;
+};
+
+template <typename Tag>
+__device__ __forceinline__ void slice_load(const DrawRow& D, long long lo, int n, int e0,
+                                           SliceRaw<Tag>& R) {
+  R.live = e0 < n;
+  if (!R.live) return;
+  using elem = typename Tag::elem;
+  const elem* tp = static_cast<const elem*>(D.trow) + lo + e0;
+  const elem* qp = static_cast<const elem*>(D.qrow) + lo + e0;
+#pragma unroll
+  for (int k = 0; k < 8 / Tag::kVec; ++k) {
+    R.t[k] = ld_stream(tp + k * Tag::kVec);
+    if (D.resid) R.q[k] = ld_stream(qp + k * Tag::kVec);
+  }
+}
+
+template <typename Tag>
+__device__ __forceinline__ void slice_values(const DrawRow& D, const SliceRaw<Tag>& R,
+                                             float (&xt)[8], float (&xq)[8]) {
+  if (!R.live) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xt[j] = xq[j] = -INFINITY;
+    return;
+  }
+  if constexpr (Tag::kVec == 8) {
+    unpack(R.t[0], xt, BF16Tag{});
+    if (D.resid) unpack(R.q[0], xq, BF16Tag{});
+  } else {
+    float a[4], b[4];
+    unpack(R.t[0], a, F32Tag{});
+    unpack(R.t[1], b, F32Tag{});
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { xt[j] = a[j]; xt[4 + j] = b[j]; }
+    if (D.resid) {
+      unpack(R.q[0], a, F32Tag{});
+      unpack(R.q[1], b, F32Tag{});
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { xq[j] = a[j]; xq[4 + j] = b[j]; }
+    }
+  }
+}
+
+#ifndef PSPEC_EE_DRAW_U
+#define PSPEC_EE_DRAW_U 1
+#endif
+
 template <typename Tag, int G, bool kRej>
 __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyExitLaunch L) {
   using elem = typename Tag::elem;
@@ -267,17 +320,39 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
     const int ntiles = (n + 255) / 256;
     const double u = (double)L.uniforms[(long long)i * (K + 1) + K];
 
-    // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8).
+    // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8).  Measured on
+    // B200 at B=1024: walking the slice last tile first (the part streamed most recently)
+    // and two or four tiles in flight per warp were both slower or no faster, so the
+    // defaults are first tile first, one tile per warp and iteration.
+#ifndef PSPEC_EE_DRAW_REVERSE
+#define PSPEC_EE_DRAW_REVERSE 0
+#endif
+    // PSPEC_EE_DRAW_U tiles per warp and iteration, all their loads issued first.
     auto tile_pass = [&]() {
-      for (int t = warp; t < ntiles; t += kWarps) {
-        float xt[8], xq[8], r[8];
-        slice_x8<Tag>(D, lo, n, t * 256 + lane * 8, xt, xq);
-        draw_r8(D, xt, xq, r);
-        float sum = 0.f;
+      constexpr int U = PSPEC_EE_DRAW_U;
+      for (int t0 = warp; t0 < ntiles; t0 += kWarps * U) {
+        SliceRaw<Tag> R[U];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sum += r[j];
-        const double ts = warp_sum_d((double)sum);
-        if (lane == 0) tsum[t] = ts;
+        for (int u = 0; u < U; ++u) {
+          const int tu = t0 + u * kWarps;
+          const int t = PSPEC_EE_DRAW_REVERSE ? ntiles - 1 - tu : tu;
+          R[u].live = false;
+          if (tu < ntiles) slice_load<Tag>(D, lo, n, t * 256 + lane * 8, R[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int tu = t0 + u * kWarps;
+          if (tu >= ntiles) break;                   // the same on every lane
+          const int t = PSPEC_EE_DRAW_REVERSE ? ntiles - 1 - tu : tu;
+          float xt[8], xq[8], r[8];
+          slice_values<Tag>(D, R[u], xt, xq);
+          draw_r8(D, xt, xq, r);
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sum += r[j];
+          const double ts = warp_sum_d((double)sum);
+          if (lane == 0) tsum[t] = ts;
+        }
       }
     };
     bool own_pass_done = false;
@@ -339,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
           if (tile < 0 && crossing && tsum[t] > 0.0 && b2 + tsum[t] > thr) { tile = t; tb = b2; }
           b2 += tsum[t];
         }
-        if (tile < 0) { tile = last_tile; tb = thr; }       // no crossing: its last positive r
+        if (tile < 0) { tile = last_tile; tb = -INFINITY; } // no crossing: its last positive r
         s_tile = tile;
         s_base = tb;
       }
@@ -367,7 +442,8 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             if (r[j] > 0.f) lastp = (int)(lo + e0 + j);
-            if (cand == 0x7fffffff && tb + ex + (double)incl[j] > thr) cand = (int)(lo + e0 + j);
+            if (cand == 0x7fffffff && r[j] > 0.f && tb + ex + (double)incl[j] > thr)
+              cand = (int)(lo + e0 + j);             // only a token with mass can cross
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {

@@ -66,7 +66,7 @@ greedy_sweep_kernel(const GreedyLaunch L) {
       GreedyPart* part = reinterpret_cast<GreedyPart*>(L.part);
       part[item] = GreedyPart{best.v, best.i, ms.m, ms.s};
       __threadfence();
-      int t = atomicAdd(L.cnt + i, 1);
+      int t = atomicAdd(zcol(L.cnt, i), 1);
       s_last = (t == L.S * (L.K + 1) - 1);
     }
   }
@@ -119,7 +119,7 @@ greedy_sweep_kernel(const GreedyLaunch L) {
     L.accepted_len[i] = a;
     L.bonus[i] = bonus;
     if (anybad) set_err(L.err, PSPEC_DEVERR_TOKEN_RANGE);
-    L.cnt[i] = 0;                        // ticket back to zero for the next call
+    *zcol(L.cnt, i) = 0;                       // ticket back to zero for the next call
   }
 }
 

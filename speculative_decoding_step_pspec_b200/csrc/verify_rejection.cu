@@ -21,6 +21,7 @@
 #include "kernels.h"
 #include "plan.h"
 #include "verify_common.cuh"
+#include "verify_draw.cuh"
 
 namespace pspec {
 
@@ -32,256 +33,6 @@ __device__ __forceinline__ const elem* sweep_row(const RejectionLaunch& L, int i
   if (r <= L.K)
     return static_cast<const elem*>(L.target) + ((long long)i * (L.K + 1) + r) * L.ld;
   return static_cast<const elem*>(L.draft) + ((long long)i * L.K + (r - L.K - 1)) * L.ld;
-}
-
-// ---------------------------------------------------------------------------------------
-// The draw.  r(t) for t in [0, V): max(0, p(t) - q(t)) (resid) or p(t) (target only),
-// each probability computed in fp32 as 2^((x - M) log2 e) / S.  The tile sums and the
-// rescan compute r through the same code, so both see bit-identical values.
-constexpr int kWTile = 256;   // one warp tile: 32 lanes x 8 consecutive elements
-
-__device__ __forceinline__ DrawRow make_draw_row(const RejectionLaunch& L, int elem_bytes, int i,
-                                                 int a, double mt, double st, double mq,
-                                                 double sq) {
-  DrawRow D;
-  const char* t = static_cast<const char*>(L.target);
-  const char* q = static_cast<const char*>(L.draft);
-  D.trow = t + ((long long)i * (L.K + 1) + a) * L.ld * elem_bytes;
-  D.resid = a < L.K;
-  D.qrow = D.resid ? q + ((long long)i * L.K + a) * L.ld * elem_bytes : D.trow;
-  D.mt = (float)mt;
-  D.inv_st = st > 0.0 ? (float)(1.0 / st) : 0.f;
-  D.mq = (float)mq;
-  D.inv_sq = sq > 0.0 ? (float)(1.0 / sq) : 0.f;
-  return D;
-}
-
-// Eight consecutive elements [t0, t0+8) of a row: 16-byte loads when the group lies inside
-// the row on a 16-byte boundary, else scalar loads (-inf past V) when the values are read.
-template <typename Tag>
-struct Raw8 {
-  uint4 v[8 / Tag::kVec];
-  bool fast;
-};
-
-template <typename Tag>
-__device__ __forceinline__ void raw8_load(const void* rowp, int V, long long t0, Raw8<Tag>& R) {
-  const typename Tag::elem* row = static_cast<const typename Tag::elem*>(rowp);
-  R.fast = t0 + 8 <= V && (reinterpret_cast<uintptr_t>(row + t0) & 15u) == 0;
-  if (R.fast) {
-#pragma unroll
-    for (int k = 0; k < 8 / Tag::kVec; ++k) R.v[k] = ld_stream(row + t0 + k * Tag::kVec);
-  }
-}
-
-template <typename Tag>
-__device__ __forceinline__ void raw8_values(const void* rowp, int V, long long t0,
-                                            const Raw8<Tag>& R, float (&x)[8]) {
-  const typename Tag::elem* row = static_cast<const typename Tag::elem*>(rowp);
-  if (R.fast) {
-    if constexpr (Tag::kVec == 8) {
-      unpack(R.v[0], x, BF16Tag{});
-    } else {
-      float lo[4], hi[4];
-      unpack(R.v[0], lo, F32Tag{});
-      unpack(R.v[1], hi, F32Tag{});
-#pragma unroll
-      for (int j = 0; j < 4; ++j) { x[j] = lo[j]; x[4 + j] = hi[j]; }
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) x[j] = t0 + j < V ? load_scalar(row, t0 + j) : -INFINITY;
-  }
-}
-
-template <typename Tag>
-__device__ __forceinline__ void r8(const DrawRow& D, int V, long long t0, float (&r)[8]) {
-  Raw8<Tag> T, Q;
-  raw8_load<Tag>(D.trow, V, t0, T);
-  if (D.resid) raw8_load<Tag>(D.qrow, V, t0, Q);
-  float xt[8], xq[8];
-  raw8_values<Tag>(D.trow, V, t0, T, xt);
-  if (D.resid) raw8_values<Tag>(D.qrow, V, t0, Q, xq);
-  draw_r8(D, xt, xq, r);
-}
-
-__device__ __forceinline__ double warp_sum(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// This warp's share of the tile sums: tiles t_begin, t_begin + stride, ... below t_end,
-// two tiles per iteration with all their loads issued before any arithmetic.
-template <typename Tag>
-__device__ void warp_tile_sums(const DrawRow& D, int V, long long t_begin, long long t_end,
-                               long long stride, double* ts) {
-  const int lane = threadIdx.x & 31;
-  for (long long t = t_begin; t < t_end; t += 2 * stride) {
-    const long long t2 = t + stride;
-    const bool two = t2 < t_end;
-    const long long e1 = t * kWTile + lane * 8, e2 = t2 * kWTile + lane * 8;
-    Raw8<Tag> T1, Q1, T2, Q2;
-    raw8_load<Tag>(D.trow, V, e1, T1);
-    if (D.resid) raw8_load<Tag>(D.qrow, V, e1, Q1);
-    if (two) {
-      raw8_load<Tag>(D.trow, V, e2, T2);
-      if (D.resid) raw8_load<Tag>(D.qrow, V, e2, Q2);
-    }
-    float x[8], y[8], r[8];
-    float s1 = 0.f, s2 = 0.f;
-    raw8_values<Tag>(D.trow, V, e1, T1, x);
-    if (D.resid) raw8_values<Tag>(D.qrow, V, e1, Q1, y);
-    draw_r8(D, x, y, r);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s1 += r[j];
-    if (two) {
-      raw8_values<Tag>(D.trow, V, e2, T2, x);
-      if (D.resid) raw8_values<Tag>(D.qrow, V, e2, Q2, y);
-      draw_r8(D, x, y, r);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) s2 += r[j];
-    }
-    const double d1 = warp_sum((double)s1);
-    const double d2 = warp_sum((double)s2);
-    if (lane == 0) {
-      ts[t] = d1;
-      if (two) ts[t2] = d2;
-    }
-  }
-}
-
-__device__ __forceinline__ double block_sum(double v, double* s_red) {
-  v = warp_sum(v);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) s_red[warp] = v;
-  __syncthreads();
-  double t = 0.0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) t += s_red[w];
-  return t;
-}
-
-// Exclusive prefix over the CTA of one double per thread; returns the prefix and sets *total.
-__device__ __forceinline__ double block_exclusive_scan(double v, double* s_red, double* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    double n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  __syncthreads();
-  if (lane == 31) s_red[warp] = incl;
-  __syncthreads();
-  double base = 0.0, all = 0.0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    if (w < warp) base += s_red[w];
-    all += s_red[w];
-  }
-  *total = all;
-  return base + incl - v;
-}
-
-struct DrawShared {
-  double red[kWarps + 1];
-  int found;
-  int token;
-};
-
-// One CTA, all threads, once the tile sums ts[0..tiles) of row a_i are in place: Z, the
-// first tile whose inclusive prefix exceeds u*Z, and the first token of that tile whose
-// running sum does (the last positive r of the tile if rounding leaves none; token 0 if
-// the row holds no mass at all).  A residual that sums to zero is redrawn from p itself.
-template <typename Tag>
-__device__ int draw_finish(DrawRow& D, int V, int tiles, double u, double* ts, DrawShared& sh,
-                           double* Zout) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  double Z = 0.0;
-  for (int t0 = 0; t0 < tiles; t0 += kThreads)
-    Z += block_sum(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
-  if (Z == 0.0 && D.resid) {
-    D.resid = false;                       // max(0, p - q) vanished: draw from p
-    D.qrow = D.trow;
-    __syncthreads();
-    warp_tile_sums<Tag>(D, V, warp, tiles, kWarps, ts);
-    __syncthreads();
-    Z = 0.0;
-    for (int t0 = 0; t0 < tiles; t0 += kThreads)
-      Z += block_sum(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
-  }
-  const double thr = u * Z;
-
-  int tile = -1;
-  double tile_base = 0.0;
-  double base = 0.0;
-  for (int t0 = 0; t0 < tiles; t0 += kThreads) {
-    const int t = t0 + tid;
-    const double v = t < tiles ? ld_cg(ts + t) : 0.0;
-    double tot;
-    const double ex = block_exclusive_scan(v, sh.red, &tot);
-    if (tid == 0) sh.found = 0x7fffffff;
-    __syncthreads();
-    if (t < tiles && v > 0.0 && base + ex + v > thr) atomicMin(&sh.found, t);
-    __syncthreads();
-    const int f = sh.found;
-    if (f != 0x7fffffff) {
-      if (t == f) sh.red[kWarps] = base + ex;
-      __syncthreads();
-      tile = f;
-      tile_base = sh.red[kWarps];
-      break;                               // f is the same on every thread
-    }
-    base += tot;
-  }
-  if (tile < 0 && Z > 0.0) {
-    // rounding kept every prefix at or below u*Z: the last tile holding any mass
-    if (tid == 0) sh.found = -1;
-    __syncthreads();
-    for (int t = tid; t < tiles; t += kThreads)
-      if (ld_cg(ts + t) > 0.0) atomicMax(&sh.found, t);
-    __syncthreads();
-    tile = sh.found;
-    if (tile >= 0) {
-      tile_base = thr;                     // no crossing inside: take its last positive r
-    }
-  }
-  if (warp == 0) {
-    int token = 0;
-    if (tile >= 0) {
-      const long long e0 = (long long)tile * kWTile + lane * 8;
-      float r[8];
-      r8<Tag>(D, V, e0, r);
-      float incl[8], run = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { run += r[j]; incl[j] = run; }
-      double inc = run;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const double n = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += n;
-      }
-      const double ex = inc - (double)run;
-      int cand = 0x7fffffff, lastpos = -1;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (r[j] > 0.f) lastpos = (int)(e0 + j);
-        if (cand == 0x7fffffff && tile_base + ex + (double)incl[j] > thr) cand = (int)(e0 + j);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        cand = min(cand, __shfl_xor_sync(0xffffffffu, cand, o));
-        lastpos = max(lastpos, __shfl_xor_sync(0xffffffffu, lastpos, o));
-      }
-      token = cand != 0x7fffffff ? cand : (lastpos >= 0 ? lastpos : 0);
-    }
-    if (lane == 0) sh.token = token;
-  }
-  __syncthreads();
-  *Zout = Z;
-  return sh.token;
 }
 
 template <typename Tag>
@@ -318,7 +69,7 @@ rej_stats_kernel(const RejectionLaunch L) {
     if (lane == 0) {
       reinterpret_cast<RejPart*>(L.part)[item] = RejPart{ms.m, ms.s};
       __threadfence();
-      int t = atomicAdd(L.cnt + i, 1);
+      int t = atomicAdd(zcol(L.cnt, i), 1);
       s_last = (t == L.S * R - 1);
     }
   }
@@ -398,7 +149,7 @@ rej_stats_kernel(const RejectionLaunch L) {
     reinterpret_cast<SeqInfo*>(L.seq)[i] = si;
     L.accepted_len[i] = a;
     if (anybad) set_err(L.err, PSPEC_DEVERR_TOKEN_RANGE);
-    L.cnt[i] = 0;
+    *zcol(L.cnt, i) = 0;
   }
   }  // warp 0
 }
@@ -416,7 +167,8 @@ rej_draw_kernel(const RejectionLaunch L) {
   __shared__ DrawShared sh;
 
   const SeqInfo si = reinterpret_cast<const SeqInfo*>(L.seq)[i];  // previous launch
-  DrawRow D = make_draw_row(L, sizeof(elem), i, si.a, si.mt, si.st, si.mq, si.sq);
+  DrawRow D = make_draw_row(L.target, L.draft, L.ld, K, (int)sizeof(elem), i, si.a, si.mt, si.st,
+                            si.mq, si.sq);
   double* ts = L.tile_sums + (long long)i * L.tiles;
   const long long t_lo = (long long)c * L.tiles_per_chunk;
   const long long t_hi = min((long long)L.tiles, t_lo + L.tiles_per_chunk);
@@ -424,7 +176,7 @@ rej_draw_kernel(const RejectionLaunch L) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    const int t = atomicAdd(L.cnt2 + i, 1);
+    const int t = atomicAdd(zcol(L.cnt2, i), 1);
     s_last = (t == L.C - 1);
   }
   __syncthreads();
@@ -437,7 +189,7 @@ rej_draw_kernel(const RejectionLaunch L) {
     L.out_tokens[(long long)i * (K + 1) + si.a] = token;
     L.bonus[i] = token;
     if (L.residual_mass) L.residual_mass[i] = (float)Z;
-    L.cnt2[i] = 0;
+    *zcol(L.cnt2, i) = 0;
   }
 }
 

@@ -26,7 +26,8 @@ def _sample(B, n, seed):
 
 
 class verify_path:
-    """Force the full sweep (1) or the early-exit path (2) inside a with-block."""
+    """Force the full sweep (1), the early-exit path (2) or the work-queue path (3) inside a
+    with-block."""
 
     def __init__(self, path):
         self.path = path
@@ -57,13 +58,16 @@ def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True)
     U.compare_greedy(gr, og, seqs)
     orj = U.oracle_rejection(target, draft, sampled, u, seqs)
     U.compare_rejection(rj, orj, seqs)
-    if early_exit_allowed(target):
-        with verify_path(2):
+    for path in (2, 3):                    # early exit where its shape rules allow; queue always
+        if path == 2 and not early_exit_allowed(target):
+            continue
+        with verify_path(path):
             ge = ps.verify_greedy(target, greedy_drafts)
-            assert ps.pspec_last_launches() == 1
+            assert ps.pspec_last_launches() == 1 and ps.pspec_last_verify_path() == path
             re = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
-            assert ps.pspec_last_launches() == 1
+            assert ps.pspec_last_launches() == 1 and ps.pspec_last_verify_path() == path
         torch.cuda.synchronize()
+        assert ge["err"].item() == 0 and re["err"].item() == 0, path
         U.check_verify_invariants(ge, greedy_drafts, V)
         U.check_verify_invariants(re, sampled, V)
         U.compare_greedy(ge, og, seqs)
@@ -191,11 +195,12 @@ def test_neg_inf_rows_and_entries():
     o = U.oracle_rejection(target, draft, d, u)
     U.compare_rejection(rj, o)
     assert rj["accepted_len"][3].item() == 0
-    with verify_path(2):
-        ge = ps.verify_greedy(target, d)
-        re = ps.verify_rejection(target, draft, d, u, residual_mass=True)
-    U.compare_greedy(ge, U.oracle_greedy(target, d, want_lse=False))
-    U.compare_rejection(re, o)
+    for path in (2, 3):
+        with verify_path(path):
+            ge = ps.verify_greedy(target, d)
+            re = ps.verify_rejection(target, draft, d, u, residual_mass=True)
+        U.compare_greedy(ge, U.oracle_greedy(target, d, want_lse=False))
+        U.compare_rejection(re, o)
 
 
 def test_out_of_range_draft_tokens():
@@ -214,13 +219,14 @@ def test_out_of_range_draft_tokens():
     o = U.oracle_rejection(target, draft, bad, u)
     U.compare_rejection(rj, o)
     assert gr["accepted_len"][0].item() == 0 and rj["accepted_len"][0].item() == 0
-    with verify_path(2):
-        ge = ps.verify_greedy(target, bad)
-        re = ps.verify_rejection(target, draft, bad, u)
-    assert ge["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
-    assert re["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
-    U.compare_greedy(ge, U.oracle_greedy(target, bad, want_lse=False))
-    U.compare_rejection(re, o)
+    for path in (2, 3):
+        with verify_path(path):
+            ge = ps.verify_greedy(target, bad)
+            re = ps.verify_rejection(target, draft, bad, u)
+        assert ge["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
+        assert re["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
+        U.compare_greedy(ge, U.oracle_greedy(target, bad, want_lse=False))
+        U.compare_rejection(re, o)
 
 
 @pytest.mark.parametrize("B", [1, 63, 64, 200])
@@ -277,11 +283,52 @@ def test_determinism_and_workspace_reuse():
         e2 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
     for k in e1:
         assert torch.equal(e1[k], e2[k]), k
+    # paths take turns on one workspace: queue, sweep, queue, smaller batch on the queue
+    with verify_path(3):
+        q1 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
+    with verify_path(1):
+        s1 = ps.verify_rejection(target, draft, sampled, u, diagnostics=True, workspace=ws)
+    with verify_path(3):
+        q2 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
+        q3 = ps.verify_rejection(target[:5], draft[:5], sampled[:5], u[:5], workspace=ws)
+    for k in q1:
+        assert torch.equal(q1[k], q2[k]), k                  # same path: bit-identical
+    for k in ("out_tokens", "accepted_len", "bonus"):
+        assert torch.equal(q1[k], e1[k]), k
+    # residual mass is summed in a different order on each path: fp32 within 1e-5
+    assert torch.allclose(q1["residual_mass"], e1["residual_mass"], rtol=1e-5, atol=0)
+    for k in ("out_tokens", "accepted_len", "bonus"):
+        assert torch.equal(s1[k], q1[k]), k
+        assert torch.equal(q3[k], q1[k][:5]), k
     wsg = ps.Workspace(w.B, w.K, w.V, False)
     g1 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
     g2 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
     for k in g1:
         assert torch.equal(g1[k], g2[k]), k
+    with verify_path(3):
+        h1 = ps.verify_greedy(target, greedy, workspace=wsg)
+        h2 = ps.verify_greedy(target, greedy, workspace=wsg)
+    g3 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
+    for k in ("out_tokens", "accepted_len", "bonus"):
+        assert torch.equal(h1[k], g1[k]) and torch.equal(h2[k], g1[k]) and torch.equal(g3[k], g1[k]), k
+
+
+def test_queue_refuses_diagnostics_and_short_workspace():
+    w = I.Workload("t", 4, 3, 1001, 16, 4, torch.bfloat16, seed=5, sigma_t=2.0, sigma_d=0.6)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    with verify_path(3):
+        with pytest.raises(ps.PspecError):
+            ps.verify_rejection(target, draft, sampled, u, diagnostics=True)
+        with pytest.raises(ps.PspecError):
+            ps.verify_greedy(target, greedy, want_lse=True)
+        short = ps.Workspace(w.B, w.K, w.V, True)
+        short.tensor = short.tensor[:512]                          # below the queue's need
+        with pytest.raises(ps.PspecError):
+            ps.verify_rejection(target, draft, sampled, u, workspace=short)
+        r = ps.verify_rejection(target, draft, sampled, u)         # odd V is fine here
+    U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u))
 
 
 def test_empty_batch():
@@ -346,21 +393,23 @@ def test_threshold_probing_exact_rule():
     Qd = torch.from_numpy(np.stack(rows_q)).to(DEV)
     D = torch.from_numpy(np.stack(rows_d)).to(DEV)
     Uu = torch.from_numpy(np.stack(rows_u)).to(DEV)
-    r = ps.verify_rejection(T, Qd, D, Uu)
-    a = r["accepted_len"].cpu().numpy()
-    bonus = r["bonus"].cpu().numpy()
     o = oracle.verify_rejection(np.stack(rows_t), np.stack(rows_q), np.stack(rows_d), np.stack(rows_u))
-    for n, ((k, acc), tok) in enumerate(zip(expect_a, expect_tok)):
-        if acc is True:
-            assert a[n] > k, n
-        elif acc is False:
-            assert a[n] == k, n
-        else:
-            assert a[n] == K, n
-        if tok >= 0:
-            assert bonus[n] == tok, (n, bonus[n], tok)
-            assert o["bonus"][n] == tok
-    assert np.array_equal(a, o["accepted_len"])
+    for path in (1, 2, 3):
+        with verify_path(path):
+            r = ps.verify_rejection(T, Qd, D, Uu)
+        a = r["accepted_len"].cpu().numpy()
+        bonus = r["bonus"].cpu().numpy()
+        for n, ((k, acc), tok) in enumerate(zip(expect_a, expect_tok)):
+            if acc is True:
+                assert a[n] > k, (path, n)
+            elif acc is False:
+                assert a[n] == k, (path, n)
+            else:
+                assert a[n] == K, (path, n)
+            if tok >= 0:
+                assert bonus[n] == tok, (path, n, bonus[n], tok)
+                assert o["bonus"][n] == tok
+        assert np.array_equal(a, o["accepted_len"]), path
 
 
 # --------------------------------------------------------------------------- build
@@ -552,3 +601,20 @@ def test_sampling_empty_and_errors():
     with pytest.raises(ps.PspecError):
         ws = torch.zeros(256, dtype=torch.uint8, device=DEV)       # too small
         ps.sample_drafts(torch.zeros((2, 3, 100), device=DEV), None, workspace=ws)
+
+
+def test_sampling_workspace_serves_smaller_batches():
+    """One workspace sized for the largest batch: large, small, large again give the same
+    tokens as fresh workspaces (the tickets sit at addresses independent of B)."""
+    w = I.Workload("t", 24, 5, 30011, 16, 4, torch.bfloat16, seed=21, sigma_t=2.0, sigma_d=0.6)
+    _, logits = I.logits(w, DEV)
+    u = I.uniforms(w, DEV)[:, :w.K].contiguous()
+    ws = torch.zeros(ps._binding.pspec_sample_workspace_bytes(w.B, w.K, w.V), dtype=torch.uint8,
+                     device=DEV)
+    ref = ps.sample_drafts(logits, u, want_probs=True)
+    a = ps.sample_drafts(logits, u, want_probs=True, workspace=ws)
+    b = ps.sample_drafts(logits[:7], u[:7], want_probs=True, workspace=ws)
+    c = ps.sample_drafts(logits, u, want_probs=True, workspace=ws)
+    for k in ("draft_tokens", "q_at_draft"):
+        assert torch.equal(a[k], ref[k]) and torch.equal(c[k], ref[k]), k
+        assert torch.equal(b[k], ref[k][:7]), k
