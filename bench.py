@@ -53,6 +53,10 @@ def parse_args():
     p.add_argument("--workload", default="b1024", help="b1024 (default), c64 or c1")
     p.add_argument("--batch", type=int, default=0,
                    help="override the workload's number of sequences (profiling and scaling aid)")
+    p.add_argument("--graph", action="store_true",
+                   help="capture one step in a CUDA graph and time its replays")
+    p.add_argument("--separate", action="store_true",
+                   help="time verify and build as two calls even where one fused launch can do both")
     p.add_argument("--build-only", action="store_true",
                    help="time the draft-batch construction alone (profiling aid: no logits)")
     p.add_argument("--sample-only", choices=["sample", "argmax"], default=None,
@@ -265,14 +269,41 @@ def run_pspec(args, rank, world, local_rank):
                              block_table=bi["block_table"], verify_hidden=bi["verify_hidden"],
                              h_shared=bi["h_shared"], out=bout)
 
+    def fused_step():
+        ps.step(d["target"], drafts, bi, draft_logits=d["draft"] if rej else None,
+                uniforms=d["u"] if rej else None, workspace=ws, out=vout, build_out=bout)
+
+    # one call of the public step API: where a single launch verifies and builds, that is
+    # the step that is timed; otherwise the two calls are timed apart
+    fused_step()
+    fused = (not args.separate) and ps.pspec_last_launches() == 1
     for _ in range(max(3, args.warmup)):
-        verify()
-        lv = ps.pspec_last_launches()
+        if fused:
+            fused_step()
+            lv, lb = 1, 0
+        else:
+            verify()
+            lv = ps.pspec_last_launches()
+            build()
+            lb = ps.pspec_last_launches()
         path = ps.pspec_last_verify_path()
-        build()
-        lb = ps.pspec_last_launches()
     launches_per_step = lv + lb
     torch.cuda.synchronize()
+    graph = None
+    if args.graph:                     # the step's launches, captured once and replayed
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph):
+                if fused:
+                    fused_step()
+                else:
+                    verify()
+                    build()
+        torch.cuda.current_stream().wait_stream(side)
+        graph.replay()
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
 
@@ -287,12 +318,21 @@ def run_pspec(args, rank, world, local_rank):
         t0.record()
         for s in range(K):
             ev[s][0].record()
-            if rej:
-                ps.pspec_set_split_event(ev[s][1])
-            verify()
-            ev[s][2].record()
-            build()
-            ev[s][3].record()
+            if graph is not None:
+                graph.replay()
+                ev[s][2].record()
+                ev[s][3].record()
+            elif fused:
+                fused_step()
+                ev[s][2].record()
+                ev[s][3].record()
+            else:
+                if rej:
+                    ps.pspec_set_split_event(ev[s][1])
+                verify()
+                ev[s][2].record()
+                build()
+                ev[s][3].record()
         t1.record()
         torch.cuda.synchronize()
     ps.pspec_set_split_event(None)
@@ -302,8 +342,9 @@ def run_pspec(args, rank, world, local_rank):
 
     verify_ms = [e[0].elapsed_time(e[2]) for e in ev]
     build_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    stats_ms = [e[0].elapsed_time(e[1]) for e in ev] if rej else verify_ms
-    draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if rej else None
+    split = rej and not fused and graph is None             # library-recorded split event
+    stats_ms = [e[0].elapsed_time(e[1]) for e in ev] if split else verify_ms
+    draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if split else None
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
     acc = vout["accepted_len"].cpu().numpy()
     early = path in (2, 3)                  # paths that read rows only up to a_i
@@ -323,6 +364,8 @@ def run_pspec(args, rank, world, local_rank):
         src = ["speculative_decoding_step_pspec_b200/csrc/verify_early_exit.cu",
                "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
                "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
+        if fused:
+            src.append("speculative_decoding_step_pspec_b200/csrc/build_common.cuh")
     else:
         dom_kernel = "rej_stats_kernel" if rej else "greedy_sweep_kernel"
         src = ["speculative_decoding_step_pspec_b200/csrc/verify_rejection.cu" if rej else
@@ -331,7 +374,9 @@ def run_pspec(args, rank, world, local_rank):
                "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
     src_hash = kernel_source_hash(src)
     dom_ms = statistics.mean(stats_ms)
-    achieved = vbytes / (dom_ms * 1e-3) / 1e9
+    whole = fused or graph is not None                     # one timed unit: the whole step
+    dom_bytes = vbytes + bbytes if whole else vbytes       # a fused launch also builds
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     traffic = profiled_traffic(dom_kernel, args.workload, src_hash)
 
     line = {
@@ -345,6 +390,8 @@ def run_pspec(args, rank, world, local_rank):
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
             "verify_path": {1: "full sweep", 2: "early exit (cluster per sequence)",
                             3: "work queue (persistent, position order)"}[path],
+            "step": ("one launch (verify + build fused)" if fused else "verify launches + build launch")
+                    + (", CUDA graph replay" if graph is not None else ""),
             "l2": "inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9),
             "parallelism": f"replicas x{world} (independent sequences, no collective)",
         },
@@ -353,16 +400,17 @@ def run_pspec(args, rank, world, local_rank):
         "algorithmic_bytes_per_step": {"verify": int(vbytes), "build": int(bbytes),
                                        "verify_full_sweep": int(full_vbytes)},
         "kernels_ms": {
-            dom_kernel: round(dom_ms, 5),
-            **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if rej and not early else {}),
-            "build_kernel": round(statistics.mean(build_ms), 5),
+            dom_kernel + (" (verify + build, one launch)" if fused else "")
+            + (" (CUDA graph replay of the step)" if graph is not None else ""): round(dom_ms, 5),
+            **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if draw_ms else {}),
+            **({} if whole else {"build_kernel": round(statistics.mean(build_ms), 5)}),
         },
-        "build_gbs": round(bbytes / (statistics.mean(build_ms) * 1e-3) / 1e9, 1),
+        **({} if whole else {"build_gbs": round(bbytes / (statistics.mean(build_ms) * 1e-3) / 1e9, 1)}),
         "roofline": {
             "kernel": dom_kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
             "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
-            "algorithmic_bytes_per_launch": int(vbytes),
+            "algorithmic_bytes_per_launch": int(dom_bytes),
         },
         "gpu_launches": K * launches_per_step,
         "launches_per_step": launches_per_step,
@@ -417,16 +465,12 @@ def run_e2e(args, w, d, ps, dev, world):
     def step():
         for k, t in host.items():
             dv[k].copy_(t, non_blocking=True)
-        if rej:
-            ps.verify_rejection(dv["target"], dv["draft"], dv["drafts"], dv["u"], workspace=ws, out=vout)
-        else:
-            ps.verify_greedy(dv["target"], dv["drafts"], workspace=ws, out=vout)
-        ps.build_draft_batch(K=w.K, block_size=w.block_size, mask_id=bi["mask_id"],
-                             pad_id=bi["pad_id"], T_cap=bi["T_cap"], qsl_in=dv["b_qsl_in"],
-                             verify_tokens=dv["b_verify_tokens"], verify_pos=dv["b_verify_pos"],
-                             accepted_len=vout["accepted_len"], bonus=vout["bonus"],
-                             block_table=dv["b_block_table"], verify_hidden=dv["b_verify_hidden"],
-                             h_shared=dv["b_h_shared"], out=bout)
+        binp = dict(K=w.K, block_size=w.block_size, mask_id=bi["mask_id"], pad_id=bi["pad_id"],
+                    T_cap=bi["T_cap"], qsl_in=dv["b_qsl_in"], verify_tokens=dv["b_verify_tokens"],
+                    verify_pos=dv["b_verify_pos"], block_table=dv["b_block_table"],
+                    verify_hidden=dv["b_verify_hidden"], h_shared=dv["b_h_shared"])
+        ps.step(dv["target"], dv["drafts"], binp, draft_logits=dv["draft"] if rej else None,
+                uniforms=dv["u"] if rej else None, workspace=ws, out=vout, build_out=bout)
         for k in res_names:
             hres[k].copy_(vout[k], non_blocking=True)
         for k in bres_names:
@@ -448,7 +492,7 @@ def run_e2e(args, w, d, ps, dev, world):
     return {"value": round(aggregate_value(n, world, ms), 3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": n, "ms_per_step": round(ms / n, 3),
-            "path": "pinned host buffers -> cudaMemcpyAsync -> C-ABI verify + build -> results to host"}
+            "path": "pinned host buffers -> cudaMemcpyAsync -> C-ABI step (verify + build) -> results to host"}
 
 
 def _oracle_inputs(d, seqs):

@@ -296,6 +296,30 @@ PSPEC_API pspec_status pspec_verify_greedy_noalloc(const pspec_verify_args *args
  */
 PSPEC_API pspec_status pspec_build_draft_batch(const pspec_build_args *args, cudaStream_t stream);
 
+/*
+ * One speculative-decoding step: target verification followed by the P-EAGLE draft-batch
+ * construction for the next step ("Eagle parallel speculative decoding, vLLM, TorchSpec",
+ * sections "Parallel architecture" and "TorchSpec integration": the batch metadata and the
+ * hidden-state fill are rebuilt on the GPU right after verification).  Computes exactly
+ * pspec_verify_greedy / pspec_verify_rejection(v, ...) followed by
+ * pspec_build_draft_batch(b) with b's accepted_len and bonus taken from v's outputs
+ * (b->accepted_len and b->bonus must be NULL or v->accepted_len and v->bonus; b->B and b->K
+ * must equal v->B and v->K).  When the early-exit path takes the verification and fusion
+ * is on (pspec_set_step_fusion; automatic: fewer than 256 sequences, where the saved launch
+ * measured faster than building each span at the end of its cluster's work), ONE launch
+ * does both: the cluster that decides sequence i writes sequence i's span of the draft
+ * batch (its metadata and its hidden rows), and the cluster of the last sequence writes
+ * the padding rows; otherwise the verify launches are followed by the build launch.
+ * pspec_last_launches() reports which.  Errors: those of the two calls it stands for; the
+ * build's device-side error bits go to b->err, the verify's to v->err.
+ */
+PSPEC_API pspec_status pspec_step_greedy(const pspec_verify_args *v, const pspec_build_args *b,
+                                         void *workspace, size_t workspace_bytes,
+                                         cudaStream_t stream);
+PSPEC_API pspec_status pspec_step_rejection(const pspec_verify_args *v, const pspec_build_args *b,
+                                            void *workspace, size_t workspace_bytes,
+                                            cudaStream_t stream);
+
 /* Human-readable name of a status code (static storage). */
 PSPEC_API const char *pspec_status_string(pspec_status status);
 
@@ -324,6 +348,10 @@ PSPEC_API void pspec_set_verify_path(int path);
    streams a 1/G slice of a row); 0 restores the automatic choice (4, or 16 when a slice
    of 4 would exceed 262144 elements).  Process-wide. */
 PSPEC_API void pspec_set_cluster_size(int G);
+
+/* Tuning: fusion of the two halves of pspec_step_* into one launch (early-exit path only):
+   0 automatic (fewer than 256 sequences), 1 always, 2 never.  Process-wide. */
+PSPEC_API void pspec_set_step_fusion(int mode);
 
 /* The path the most recent successful verify call on this host thread took: 1 full sweep,
    2 early exit, 3 work queue, 0 none yet. */

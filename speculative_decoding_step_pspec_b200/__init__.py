@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     pspec_verify_greedy, pspec_verify_rejection, pspec_verify_workspace_bytes,
 )
 from ._binding import pspec_sample_drafts, pspec_sample_workspace_bytes  # noqa: F401
+from ._binding import pspec_set_step_fusion, pspec_step_greedy, pspec_step_rejection  # noqa: F401
 from .api import (  # noqa: F401
-    Workspace, build_draft_batch, sample_drafts, verify_greedy, verify_rejection,
+    Workspace, build_draft_batch, sample_drafts, step, verify_greedy, verify_rejection,
 )

@@ -29,6 +29,7 @@ EXPORTED = (
     "pspec_set_verify_path", "pspec_last_verify_path", "pspec_set_cluster_size",
     "pspec_sample_workspace_bytes", "pspec_sample_drafts",
     "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
+    "pspec_step_greedy", "pspec_step_rejection", "pspec_set_step_fusion",
 )
 
 
@@ -88,12 +89,18 @@ def _load():
     lib.pspec_sample_drafts.restype = _I
     lib.pspec_build_draft_batch.argtypes = [ctypes.POINTER(pspec_build_args), _P]
     lib.pspec_build_draft_batch.restype = _I
+    for fn in (lib.pspec_step_greedy, lib.pspec_step_rejection):
+        fn.argtypes = [ctypes.POINTER(pspec_verify_args), ctypes.POINTER(pspec_build_args), _P,
+                       ctypes.c_size_t, _P]
+        fn.restype = _I
     lib.pspec_status_string.argtypes = [_I]
     lib.pspec_status_string.restype = ctypes.c_char_p
     lib.pspec_last_launches.argtypes = []
     lib.pspec_last_launches.restype = _I
     lib.pspec_set_verify_path.argtypes = [_I]
     lib.pspec_set_verify_path.restype = None
+    lib.pspec_set_step_fusion.argtypes = [_I]
+    lib.pspec_set_step_fusion.restype = None
     lib.pspec_set_cluster_size.argtypes = [_I]
     lib.pspec_set_cluster_size.restype = None
     lib.pspec_last_verify_path.argtypes = []
@@ -174,6 +181,11 @@ def pspec_last_verify_path() -> int:
 def pspec_set_verify_path(path: int) -> None:
     """0 automatic, 1 full sweep, 2 early exit, 3 work queue (see include/pspec.h)."""
     LIB.pspec_set_verify_path(int(path))
+
+
+def pspec_set_step_fusion(mode: int) -> None:
+    """Fusion of pspec_step_*'s two halves into one launch: 0 automatic, 1 always, 2 never."""
+    LIB.pspec_set_step_fusion(int(mode))
 
 
 def pspec_set_segment_elems(elems: int) -> None:
@@ -262,11 +274,10 @@ def pspec_sample_drafts(*, logits, draft_tokens, err, workspace, uniforms=None, 
         raise PspecError("pspec_sample_drafts", st)
 
 
-def pspec_build_draft_batch(*, K, block_size, mask_id, pad_id, T_cap, qsl_in, verify_tokens,
-                            verify_pos, accepted_len, bonus, block_table, verify_hidden,
-                            h_shared, draft_tokens, draft_pos, slot_mapping, row_kind,
-                            hidden_src, qsl_out, seq_lens_out, sample_idx, draft_hidden, err,
-                            stream=None) -> None:
+def _build_args(*, K, block_size, mask_id, pad_id, T_cap, qsl_in, verify_tokens, verify_pos,
+                accepted_len, bonus, block_table, verify_hidden, h_shared, draft_tokens,
+                draft_pos, slot_mapping, row_kind, hidden_src, qsl_out, seq_lens_out,
+                sample_idx, draft_hidden, err):
     a = pspec_build_args()
     a.B = int(qsl_in.numel()) - 1
     a.K = int(K)
@@ -303,9 +314,45 @@ def pspec_build_draft_batch(*, K, block_size, mask_id, pad_id, T_cap, qsl_in, ve
     a.sample_idx = _ptr(sample_idx, torch.int32, "sample_idx")
     a.draft_hidden = _ptr(draft_hidden, None, "draft_hidden")
     a.err = _ptr(err, torch.int32, "err")
+    return a
+
+
+def pspec_build_draft_batch(*, stream=None, **build) -> None:
+    """Keyword arguments as the fields of pspec_build_args (tensors for the arrays)."""
+    a = _build_args(**build)
     st = LIB.pspec_build_draft_batch(ctypes.byref(a), _stream(stream))
     if st != PSPEC_OK:
         raise PspecError("pspec_build_draft_batch", st)
+
+
+def pspec_step_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len, bonus, err,
+                      workspace, build: dict, stream=None) -> None:
+    """Greedy verify followed by the draft-batch build (`build`: the keyword arguments of
+    pspec_build_draft_batch, with accepted_len / bonus None or this call's outputs)."""
+    K = int(target_logits.shape[1]) - 1
+    v = _verify_args(target_logits, None, draft_tokens, None, out_tokens, accepted_len, bonus,
+                     err, None, None, None, None, None, K)
+    b = _build_args(**build)
+    st = LIB.pspec_step_greedy(ctypes.byref(v), ctypes.byref(b),
+                               _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                               _stream(stream))
+    if st != PSPEC_OK:
+        raise PspecError("pspec_step_greedy", st)
+
+
+def pspec_step_rejection(*, target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
+                         accepted_len, bonus, err, workspace, build: dict, residual_mass=None,
+                         stream=None) -> None:
+    """Rejection-rule verify followed by the draft-batch build (see pspec_step_greedy)."""
+    K = int(target_logits.shape[1]) - 1
+    v = _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
+                     accepted_len, bonus, err, None, None, None, None, residual_mass, K)
+    b = _build_args(**build)
+    st = LIB.pspec_step_rejection(ctypes.byref(v), ctypes.byref(b),
+                                  _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                  _stream(stream))
+    if st != PSPEC_OK:
+        raise PspecError("pspec_step_rejection", st)
 
 
 _NOALLOC_SIGNATURE_SET = False

@@ -17,6 +17,7 @@ long long g_seg_override = 0;   // 0 = automatic segment length
 cudaEvent_t g_split_event = nullptr;
 int g_verify_path = 0;          // 0 automatic, 1 full sweep, 2 early exit, 3 work queue
 int g_cluster = 0;              // early-exit cluster size; 0 = automatic
+int g_step_fusion = 0;          // 0 automatic, 1 always, 2 never
 thread_local int t_last_launches = 0;
 thread_local int t_last_path = 0;
 
@@ -46,10 +47,49 @@ pspec_status check_verify(const pspec_verify_args* a, bool rejection) {
   return PSPEC_OK;
 }
 
+// Host checks of a draft-batch construction; fills the launch descriptor on success.
+pspec_status check_build(const pspec_build_args* a, BuildLaunch* L) {
+  if (!a) return PSPEC_ERR_INVALID_ARG;
+  if (a->B < 0 || a->K < 1 || a->H < 1 || a->block_size < 1 || a->max_blocks < 1 ||
+      a->T_in < 0 || a->T_cap < 0)
+    return PSPEC_ERR_INVALID_ARG;
+  if (a->K > PSPEC_MAX_K) return PSPEC_ERR_UNSUPPORTED;
+  if (!dtype_ok(a->hidden_dtype)) return PSPEC_ERR_INVALID_ARG;
+  if ((long long)a->T_cap < (long long)a->T_in + (long long)a->B * (a->K - 1))
+    return PSPEC_ERR_INVALID_ARG;
+  if (!a->qsl_in || !a->err || !a->draft_tokens || !a->draft_pos || !a->slot_mapping ||
+      !a->row_kind || !a->hidden_src || !a->qsl_out)
+    return PSPEC_ERR_INVALID_ARG;
+  if (a->B > 0 && (!a->verify_tokens || !a->verify_pos || !a->accepted_len || !a->bonus ||
+                   !a->block_table || !a->seq_lens_out || !a->sample_idx))
+    return PSPEC_ERR_INVALID_ARG;
+  const bool hidden = a->draft_hidden != nullptr;
+  if (hidden) {
+    if (!a->h_shared || (a->T_in > 0 && !a->verify_hidden)) return PSPEC_ERR_INVALID_ARG;
+    if (((long long)a->H * (long long)elem_bytes(a->hidden_dtype)) % 16 != 0)
+      return PSPEC_ERR_INVALID_ARG;
+    if (!aligned16(a->draft_hidden) || !aligned16(a->h_shared) ||
+        (a->verify_hidden && !aligned16(a->verify_hidden)))
+      return PSPEC_ERR_INVALID_ARG;
+  }
+  const long long meta_threads = (long long)a->T_cap + a->B + 1;
+  const long long hid_rows = (long long)a->T_in + (long long)a->B * (a->K - 1);
+  if ((meta_threads + kThreads - 1) / kThreads + (hid_rows + kWarps - 1) / kWarps >= 0x7fffffffLL)
+    return PSPEC_ERR_UNSUPPORTED;
+  *L = BuildLaunch{};
+  L->a = *a;
+  L->row_vecs = (long long)a->H * (long long)elem_bytes(a->hidden_dtype) / 16;
+  L->meta_blocks = (int)((meta_threads + kThreads - 1) / kThreads);
+  L->hid_rows = (int)hid_rows;
+  return PSPEC_OK;
+}
+
 // The early-exit cluster path, when the arguments allow it and the selection asks for it:
-// returns true and sets *st when it handled the call.
+// returns true and sets *st when it handled the call.  With `fuse` non-null the same launch
+// also builds the draft batch described there (from this call's accepted counts and bonus
+// tokens).
 bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t stream,
-                    pspec_status* st) {
+                    pspec_status* st, const BuildLaunch* fuse = nullptr) {
   const bool diagnostics = a->target_lse || a->draft_lse || a->p_at_draft || a->q_at_draft;
   if (g_verify_path == 1) return false;
   if (g_verify_path == 0 && (a->B < kEarlyExitMinB || diagnostics)) return false;
@@ -76,6 +116,11 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   L.bonus = a->bonus;
   L.residual_mass = rejection ? a->residual_mass : nullptr;
   L.err = a->err;
+  if (fuse) {
+    L.fuse_build = 1;
+    L.b = fuse->a;
+    L.row_vecs = fuse->row_vecs;
+  }
   if (launch_early_exit(L, stream) != cudaSuccess) {
     *st = PSPEC_ERR_CUDA;
     return true;
@@ -160,8 +205,16 @@ size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection) {
   return (sweep > queue ? sweep : queue) + zero_area_bytes(B);
 }
 
-pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
-                                 size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The greedy verify behind both entry points; `fuse` (may be null) is passed to the
+// early-exit path, and *fused tells whether that launch also built the draft batch.
+pspec_status verify_greedy_impl(const pspec_verify_args* a, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream,
+                                const BuildLaunch* fuse, bool* fused) {
+  *fused = false;
   pspec_status st = check_verify(a, false);
   if (st != PSPEC_OK) return st;
   if (a->B == 0) { t_last_launches = 0; return st; }
@@ -170,7 +223,10 @@ pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
   st = check_workspace(workspace, workspace_bytes, p.bytes, a->B, &z);
   if (st != PSPEC_OK) return st;
   if (try_queue(a, false, workspace, workspace_bytes, stream, &st)) return st;
-  if (try_early_exit(a, false, stream, &st)) return st;
+  if (try_early_exit(a, false, stream, &st, fuse)) {
+    *fused = fuse != nullptr && st == PSPEC_OK;
+    return st;
+  }
   GreedyLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.S = p.S; L.seg = p.seg;
@@ -190,8 +246,11 @@ pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
   return PSPEC_OK;
 }
 
-pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
-                                    size_t workspace_bytes, cudaStream_t stream) {
+// The rejection-rule verify behind both entry points (see verify_greedy_impl).
+pspec_status verify_rejection_impl(const pspec_verify_args* a, void* workspace,
+                                   size_t workspace_bytes, cudaStream_t stream,
+                                   const BuildLaunch* fuse, bool* fused) {
+  *fused = false;
   pspec_status st = check_verify(a, true);
   if (st != PSPEC_OK) return st;
   if (a->B == 0) { t_last_launches = 0; return st; }
@@ -200,7 +259,10 @@ pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
   st = check_workspace(workspace, workspace_bytes, p.bytes, a->B, &z);
   if (st != PSPEC_OK) return st;
   if (try_queue(a, true, workspace, workspace_bytes, stream, &st)) return st;
-  if (try_early_exit(a, true, stream, &st)) return st;
+  if (try_early_exit(a, true, stream, &st, fuse)) {
+    *fused = fuse != nullptr && st == PSPEC_OK;
+    return st;
+  }
   RejectionLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.S = p.S; L.seg = p.seg;
@@ -230,39 +292,64 @@ pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
   return PSPEC_OK;
 }
 
+// One step: verify, then the draft batch from the verify's own accepted counts and bonus
+// tokens (b's accepted_len / bonus must be NULL or those same arrays).
+pspec_status step_impl(const pspec_verify_args* v, const pspec_build_args* b, bool rejection,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!v || !b) return PSPEC_ERR_INVALID_ARG;
+  if (b->B != v->B || b->K != v->K) return PSPEC_ERR_INVALID_ARG;
+  if ((b->accepted_len && b->accepted_len != v->accepted_len) || (b->bonus && b->bonus != v->bonus))
+    return PSPEC_ERR_INVALID_ARG;
+  pspec_build_args bb = *b;
+  bb.accepted_len = v->accepted_len;
+  bb.bonus = v->bonus;
+  BuildLaunch BL;
+  pspec_status st = check_build(&bb, &BL);
+  if (st != PSPEC_OK) return st;
+  // one launch for both halves where that measured faster: below kStepFuseMaxB sequences
+  // the saved launch outweighs building each span at the end of its cluster's work
+  const bool want_fuse = g_step_fusion == 1 || (g_step_fusion == 0 && v->B < kStepFuseMaxB);
+  const BuildLaunch* fuse = want_fuse ? &BL : nullptr;
+  bool fused = false;
+  st = rejection ? verify_rejection_impl(v, workspace, workspace_bytes, stream, fuse, &fused)
+                 : verify_greedy_impl(v, workspace, workspace_bytes, stream, fuse, &fused);
+  if (st != PSPEC_OK || fused) return st;
+  const int verify_launches = t_last_launches;
+  if (launch_build(BL, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
+  t_last_launches = verify_launches + 1;
+  return PSPEC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pspec_status pspec_verify_greedy(const pspec_verify_args* a, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  bool fused;
+  return verify_greedy_impl(a, workspace, workspace_bytes, stream, nullptr, &fused);
+}
+
+pspec_status pspec_verify_rejection(const pspec_verify_args* a, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+  bool fused;
+  return verify_rejection_impl(a, workspace, workspace_bytes, stream, nullptr, &fused);
+}
+
+pspec_status pspec_step_greedy(const pspec_verify_args* v, const pspec_build_args* b,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return step_impl(v, b, false, workspace, workspace_bytes, stream);
+}
+
+pspec_status pspec_step_rejection(const pspec_verify_args* v, const pspec_build_args* b,
+                                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return step_impl(v, b, true, workspace, workspace_bytes, stream);
+}
+
 pspec_status pspec_build_draft_batch(const pspec_build_args* a, cudaStream_t stream) {
-  if (!a) return PSPEC_ERR_INVALID_ARG;
-  if (a->B < 0 || a->K < 1 || a->H < 1 || a->block_size < 1 || a->max_blocks < 1 ||
-      a->T_in < 0 || a->T_cap < 0)
-    return PSPEC_ERR_INVALID_ARG;
-  if (a->K > PSPEC_MAX_K) return PSPEC_ERR_UNSUPPORTED;
-  if (!dtype_ok(a->hidden_dtype)) return PSPEC_ERR_INVALID_ARG;
-  if ((long long)a->T_cap < (long long)a->T_in + (long long)a->B * (a->K - 1))
-    return PSPEC_ERR_INVALID_ARG;
-  if (!a->qsl_in || !a->err || !a->draft_tokens || !a->draft_pos || !a->slot_mapping ||
-      !a->row_kind || !a->hidden_src || !a->qsl_out)
-    return PSPEC_ERR_INVALID_ARG;
-  if (a->B > 0 && (!a->verify_tokens || !a->verify_pos || !a->accepted_len || !a->bonus ||
-                   !a->block_table || !a->seq_lens_out || !a->sample_idx))
-    return PSPEC_ERR_INVALID_ARG;
-  const bool hidden = a->draft_hidden != nullptr;
-  if (hidden) {
-    if (!a->h_shared || (a->T_in > 0 && !a->verify_hidden)) return PSPEC_ERR_INVALID_ARG;
-    if (((long long)a->H * (long long)elem_bytes(a->hidden_dtype)) % 16 != 0)
-      return PSPEC_ERR_INVALID_ARG;
-    if (!aligned16(a->draft_hidden) || !aligned16(a->h_shared) ||
-        (a->verify_hidden && !aligned16(a->verify_hidden)))
-      return PSPEC_ERR_INVALID_ARG;
-  }
-  const long long meta_threads = (long long)a->T_cap + a->B + 1;
-  const long long hid_rows = (long long)a->T_in + (long long)a->B * (a->K - 1);
-  if ((meta_threads + kThreads - 1) / kThreads + (hid_rows + kWarps - 1) / kWarps >= 0x7fffffffLL)
-    return PSPEC_ERR_UNSUPPORTED;
-  BuildLaunch L{};
-  L.a = *a;
-  L.row_vecs = (long long)a->H * (long long)elem_bytes(a->hidden_dtype) / 16;
-  L.meta_blocks = (int)((meta_threads + kThreads - 1) / kThreads);
-  L.hid_rows = (int)hid_rows;
+  BuildLaunch L;
+  const pspec_status st = check_build(a, &L);
+  if (st != PSPEC_OK) return st;
   if (launch_build(L, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
   t_last_launches = 1;
   return PSPEC_OK;
@@ -326,6 +413,8 @@ int pspec_last_verify_path(void) { return t_last_path; }
 void pspec_set_verify_path(int path) { g_verify_path = (path >= 1 && path <= 3) ? path : 0; }
 
 void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || G == 16) ? G : 0; }
+
+void pspec_set_step_fusion(int mode) { g_step_fusion = (mode == 1 || mode == 2) ? mode : 0; }
 
 void pspec_set_segment_elems(long long elems) { g_seg_override = elems > 0 ? elems : 0; }
 

@@ -60,7 +60,7 @@ struct EarlyExitLaunch {
   long long ld;
   pspec_dtype dtype;
   int rejection;         // 1: rejection rule, 0: greedy
-  int G;                 // CTAs per cluster (one cluster per sequence): 8 or 16
+  int G;                 // CTAs per cluster (one cluster per sequence): 2, 4, 8 or 16
   long long vs;          // slice of each row per CTA (elements, multiple of 8)
   const void* target;
   const void* draft;
@@ -71,6 +71,9 @@ struct EarlyExitLaunch {
   int32_t* bonus;
   float* residual_mass;  // optional
   int32_t* err;
+  int fuse_build;        // 1: each cluster also builds its sequence's draft span (below)
+  pspec_build_args b;    // draft-batch arguments; accepted_len / bonus = this launch's outputs
+  long long row_vecs;    // 16-byte vectors per hidden row of b
 };
 
 struct SampleLaunch {

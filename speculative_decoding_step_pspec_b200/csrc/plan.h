@@ -19,6 +19,7 @@ constexpr int kResampleTargetCtas = kNumSMs * 8;
 constexpr int kDrawTilesPerCta = 64;     // separate draw launch: at most 8 tiles per warp
 constexpr int kEarlyExitMinB = 64;       // automatic path: early exit from this many sequences
 constexpr int kEarlyExitCluster = 4;     // CTAs per sequence on the early-exit path
+constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this many sequences
 
 // Per-(row, segment) partial of the greedy sweep.
 struct GreedyPart {

@@ -26,6 +26,7 @@
 // shared memory (two CTAs per SM) left HBM idle between positions.
 #include <cooperative_groups.h>
 
+#include "build_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
@@ -144,7 +145,45 @@ __device__ __forceinline__ void slice_values(const DrawRow& D, const SliceRaw<Ta
 #define PSPEC_EE_DRAW_U 1
 #endif
 
-template <typename Tag, int G, bool kRej>
+// Whole-step fusion: the draft span of sequence i (output rows [qsl_out[i], qsl_out[i+1]),
+// clamped into [0, T_cap)), built by the cluster that has just decided a_i and the bonus
+// token.  The CTA holding the token (`meta`) writes the rows' metadata and the sequence's
+// outputs; every CTA of the cluster copies its share of the hidden rows (one warp per
+// row).  The cluster of the last sequence also writes the padding rows and the end offset.
+// The rows are exactly those pspec_build_draft_batch writes for a valid offset array; for
+// an invalid one every write stays in bounds and the layout bit is set, as there.
+__device__ __forceinline__ void ee_build_span(const pspec_build_args& b, long long row_vecs, int i,
+                                           int a, int token, bool meta, int g, int G) {
+  const long long q0 = build_qout(b, i), q1 = build_qout(b, i + 1);
+  const long long lo = q0 < 0 ? 0 : q0;
+  const long long hi = q1 > b.T_cap ? (long long)b.T_cap : q1;
+  int eb = 0;
+  if (meta) {
+    for (long long t = lo + threadIdx.x; t < hi; t += kThreads)
+      build_write_row(b, t, build_classify(b, i, t - q0, a, token), &eb);
+    if (threadIdx.x == 0) build_write_seq(b, i, a, &eb);
+  }
+  if (b.draft_hidden) {
+    const int warp = threadIdx.x >> 5;
+    for (long long t = lo + (long long)g * kWarps + warp; t < hi; t += (long long)G * kWarps)
+      build_copy_hidden(b, row_vecs, t, build_classify(b, i, t - q0, a, token));
+  }
+  if (i == b.B - 1) {                                  // padding rows and the end offset
+    const BuildRow pad{PSPEC_ROW_PAD, -1, b.pad_id, 0, -1};
+    const long long first = build_qout(b, 0);
+    const long long head = first < 0 ? 0 : (first > b.T_cap ? (long long)b.T_cap : first);
+    const long long tail = q1 < 0 ? 0 : q1;
+    const long long step = (long long)G * kThreads;
+    for (long long t = (long long)g * kThreads + threadIdx.x; t < head; t += step)
+      build_write_row(b, t, pad, &eb);
+    for (long long t = tail + (long long)g * kThreads + threadIdx.x; t < b.T_cap; t += step)
+      build_write_row(b, t, pad, &eb);
+    if (g == 0 && threadIdx.x == 0) build_write_seq(b, b.B, 0, &eb);
+  }
+  set_err(b.err, eb);
+}
+
+template <typename Tag, int G, bool kRej, bool kFuse>
 __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyExitLaunch L) {
   using elem = typename Tag::elem;
   constexpr int W = Tag::kVec;
@@ -166,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
   __shared__ double s_tot[16];                               // per-slice draw totals
   __shared__ int s_tile;
   __shared__ double s_base;
+  __shared__ int s_tok;                                      // the emitted token (build)
 
   const long long lo = (long long)g * L.vs;                 // this CTA's slice [lo, lo + n)
   const int n = (int)max(0LL, min((long long)L.V, lo + L.vs) - lo);
@@ -289,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
         if (!match) {
           stop = 1;
           if (g == 0 && lane == 0) { L.bonus[i] = gk; L.out_tokens[(long long)i * (K + 1) + k] = gk; }
+          if (lane == 0) s_tok = gk;
         }
       }
       if (stop && g == 0) {
@@ -309,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
     if (s_stop) break;
   }
 
+  int meta_g = 0;                                            // the CTA that knows the token
   if constexpr (kRej) {
     // ---- the draw at the stop position a = k: r = max(0, p_a - q_a), or p_K after K passes
     const int a = k;
@@ -401,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
     }
     const bool crossing = owner >= 0;
     if (!crossing && Z > 0.0) owner = last_pos;              // rounding: last slice with mass
+    meta_g = owner >= 0 ? owner : 0;
     if (g == owner) {
       if (!own_pass_done) {
         tile_pass();
@@ -456,20 +499,26 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
           L.out_tokens[(long long)i * (K + 1) + a] = token;
           L.bonus[i] = token;
           if (L.residual_mass) L.residual_mass[i] = (float)Z;
+          s_tok = token;
         }
       }
     } else if (owner < 0 && g == 0 && tid == 0) {            // no mass anywhere: token 0
       L.out_tokens[(long long)i * (K + 1) + a] = 0;
       L.bonus[i] = 0;
       if (L.residual_mass) L.residual_mass[i] = 0.f;
+      s_tok = 0;
     }
   }
   cluster.sync();                                            // D: no remote reads after exit
+  if constexpr (kFuse) {                                     // the whole step in this launch
+    __syncthreads();
+    ee_build_span(L.b, L.row_vecs, i, k, g == meta_g ? s_tok : 0, g == meta_g, g, G);
+  }
 }
 
-template <typename Tag, int G, bool kRej>
+template <typename Tag, int G, bool kRej, bool kFuse>
 cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream) {
-  auto kern = ee_kernel<Tag, G, kRej>;
+  auto kern = ee_kernel<Tag, G, kRej, kFuse>;
   cudaError_t e = cudaSuccess;
   if (G > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -490,24 +539,28 @@ cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, L);
 }
 
+template <int G>
+cudaError_t launch_ee_g(const EarlyExitLaunch& L, cudaStream_t s) {
+  const bool bf = L.dtype == PSPEC_BF16;
+  if (L.fuse_build) {
+    if (L.rejection)
+      return bf ? launch_ee<BF16Tag, G, true, true>(L, s) : launch_ee<F32Tag, G, true, true>(L, s);
+    return bf ? launch_ee<BF16Tag, G, false, true>(L, s) : launch_ee<F32Tag, G, false, true>(L, s);
+  }
+  if (L.rejection)
+    return bf ? launch_ee<BF16Tag, G, true, false>(L, s) : launch_ee<F32Tag, G, true, false>(L, s);
+  return bf ? launch_ee<BF16Tag, G, false, false>(L, s) : launch_ee<F32Tag, G, false, false>(L, s);
+}
+
 }  // namespace
 
 cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream) {
-  const bool bf = L.dtype == PSPEC_BF16;
-  if (L.G == 2) {
-    if (L.rejection) return bf ? launch_ee<BF16Tag, 2, true>(L, stream) : launch_ee<F32Tag, 2, true>(L, stream);
-    return bf ? launch_ee<BF16Tag, 2, false>(L, stream) : launch_ee<F32Tag, 2, false>(L, stream);
+  switch (L.G) {
+    case 2: return launch_ee_g<2>(L, stream);
+    case 4: return launch_ee_g<4>(L, stream);
+    case 8: return launch_ee_g<8>(L, stream);
+    default: return launch_ee_g<16>(L, stream);
   }
-  if (L.G == 4) {
-    if (L.rejection) return bf ? launch_ee<BF16Tag, 4, true>(L, stream) : launch_ee<F32Tag, 4, true>(L, stream);
-    return bf ? launch_ee<BF16Tag, 4, false>(L, stream) : launch_ee<F32Tag, 4, false>(L, stream);
-  }
-  if (L.G == 8) {
-    if (L.rejection) return bf ? launch_ee<BF16Tag, 8, true>(L, stream) : launch_ee<F32Tag, 8, true>(L, stream);
-    return bf ? launch_ee<BF16Tag, 8, false>(L, stream) : launch_ee<F32Tag, 8, false>(L, stream);
-  }
-  if (L.rejection) return bf ? launch_ee<BF16Tag, 16, true>(L, stream) : launch_ee<F32Tag, 16, true>(L, stream);
-  return bf ? launch_ee<BF16Tag, 16, false>(L, stream) : launch_ee<F32Tag, 16, false>(L, stream);
 }
 
 }  // namespace pspec

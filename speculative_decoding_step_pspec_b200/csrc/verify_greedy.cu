@@ -73,33 +73,42 @@ greedy_sweep_kernel(const GreedyLaunch L) {
   __syncthreads();
   if (!s_last) return;
 
-  // This CTA finished sequence i last: merge its (K+1) x S partials in segment order.
+  // This CTA finished sequence i last: merge its (K+1) x S partials, warp w taking rows
+  // w, w + 8, ... and lane t segments t, t + 32, ... (argmax: largest value, lowest id).
   __threadfence();
-  if (warp != 0) return;
   const int K = L.K;
   const GreedyPart* part =
       reinterpret_cast<const GreedyPart*>(L.part) + (long long)i * (K + 1) * L.S;
-  int g = 0;          // argmax of row `lane`
-  double lse = 0.0;
-  if (lane <= K) {
+  __shared__ int s_g[PSPEC_MAX_K + 1];
+  __shared__ double s_lse[PSPEC_MAX_K + 1];
+  for (int r = warp; r <= K; r += kWarps) {
     VI b{-INFINITY, kNoIndex};
     float M = -INFINITY;
-    for (int t = 0; t < L.S; ++t) {
-      GreedyPart q = ld_cg(part + (long long)lane * L.S + t);
-      if (q.v > b.v) b = VI{q.v, q.i};
+    for (int t = lane; t < L.S; t += 32) {
+      const GreedyPart q = ld_cg(part + (long long)r * L.S + t);
+      if (vi_better(VI{q.v, q.i}, b)) b = VI{q.v, q.i};
       M = fmaxf(M, q.m);
     }
-    g = b.i == kNoIndex ? 0 : b.i;       // a row of -inf / NaN only: token 0
+    b = warp_argmax(b);
     if (kLse) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
       double S = 0.0;
       if (M != -INFINITY)
-        for (int t = 0; t < L.S; ++t) {
-          GreedyPart q = ld_cg(part + (long long)lane * L.S + t);
+        for (int t = lane; t < L.S; t += 32) {
+          const GreedyPart q = ld_cg(part + (long long)r * L.S + t);
           if (q.m != -INFINITY) S += (double)q.s * exp2((double)q.m - (double)M);
         }
-      lse = M == -INFINITY ? -INFINITY : ((double)M + log2(S)) / (double)kLog2e;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+      if (lane == 0) s_lse[r] = M == -INFINITY ? -INFINITY : ((double)M + log2(S)) / (double)kLog2e;
     }
+    if (lane == 0) s_g[r] = b.i == kNoIndex ? 0 : b.i;   // a row of -inf / NaN only: token 0
   }
+  __syncthreads();
+  if (warp != 0) return;
+  const int g = lane <= K ? s_g[lane] : 0;           // argmax of row `lane`
+  const double lse = (kLse && lane <= K) ? s_lse[lane] : 0.0;
   int d = -1;
   bool bad = false;
   if (lane < K) {

@@ -83,18 +83,26 @@ rej_stats_kernel(const RejectionLaunch L) {
   __shared__ double s_M[2 * PSPEC_MAX_K + 1];
   __shared__ double s_S[2 * PSPEC_MAX_K + 1];
   const RejPart* part = reinterpret_cast<const RejPart*>(L.part) + (long long)i * R * L.S;
-  if (threadIdx.x < R) {
-    const RejPart* pr = part + (long long)threadIdx.x * L.S;
+  // warp w merges rows w, w + 8, ...: lane t takes segments t, t + 32, ... (a fixed tree
+  // order); the loads of all lanes are in flight together
+  for (int r = warp; r < R; r += kWarps) {
+    const RejPart* pr = part + (long long)r * L.S;
     float M = -INFINITY;
-    for (int t = 0; t < L.S; ++t) M = fmaxf(M, ld_cg(&pr[t].m));
+    for (int t = lane; t < L.S; t += 32) M = fmaxf(M, ld_cg(&pr[t].m));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     double S = 0.0;
     if (M != -INFINITY)
-      for (int t = 0; t < L.S; ++t) {
-        RejPart q = ld_cg(pr + t);
+      for (int t = lane; t < L.S; t += 32) {
+        const RejPart q = ld_cg(pr + t);
         if (q.m != -INFINITY) S += (double)q.s * exp2((double)q.m - (double)M);
       }
-    s_M[threadIdx.x] = M;
-    s_S[threadIdx.x] = S;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+    if (lane == 0) {
+      s_M[r] = M;
+      s_S[r] = S;
+    }
   }
   __syncthreads();
   if (warp != 0) return;

@@ -167,3 +167,31 @@ def test_segment_override_changes_workspace():
     finally:
         ps.pspec_set_segment_elems(0)
     assert ps.pspec_verify_workspace_bytes(2, 3, 100000, True) == base
+
+
+@pytest.mark.parametrize("case,vkw,bkw,ws,status", [
+    ("batch_mismatch", {}, {"B": 5}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
+    ("k_mismatch", {}, {"K": 2}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
+    ("foreign_accepted_len", {}, {"accepted_len": FAKE + 256}, (FAKE, 1 << 30),
+     b.PSPEC_ERR_INVALID_ARG),
+    ("foreign_bonus", {}, {"bonus": FAKE + 256}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
+    ("bad_build", {}, {"T_cap": 3}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
+    ("bad_verify", {"ld": 10}, {}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
+    ("short_workspace", {}, {}, (FAKE, 256), b.PSPEC_ERR_WORKSPACE),
+    ("no_workspace", {}, {}, (None, 0), b.PSPEC_ERR_WORKSPACE),
+])
+@pytest.mark.parametrize("fn", ["pspec_step_greedy", "pspec_step_rejection"])
+def test_step_host_checks(fn, case, vkw, bkw, ws, status):
+    """The step calls check both halves before any launch: a build whose accepted counts or
+    bonus tokens are not the verify's outputs, shapes that disagree, or either half's own
+    argument errors return a status and launch nothing."""
+    v = _vargs(**vkw)
+    bb = _bargs(**bkw)
+    ps.pspec_set_verify_path(1)          # full sweep: its workspace check runs before a launch
+    try:
+        st = getattr(b.LIB, fn)(ctypes.byref(v), ctypes.byref(bb), ws[0], ws[1], None)
+    finally:
+        ps.pspec_set_verify_path(0)
+    assert st == status, (case, b.pspec_status_string(st))
+    assert getattr(b.LIB, fn)(None, ctypes.byref(bb), FAKE, 1 << 30, None) == b.PSPEC_ERR_INVALID_ARG
+    assert getattr(b.LIB, fn)(ctypes.byref(v), None, FAKE, 1 << 30, None) == b.PSPEC_ERR_INVALID_ARG

@@ -618,3 +618,158 @@ def test_sampling_workspace_serves_smaller_batches():
     for k in ("draft_tokens", "q_at_draft"):
         assert torch.equal(a[k], ref[k]) and torch.equal(c[k], ref[k]), k
         assert torch.equal(b[k], ref[k][:7]), k
+
+
+# --------------------------------------------------------------------------- whole step
+def _step_check(target, draft, drafts, u, binp, path, expect_fused):
+    """ps.step (verify + build, one launch when the early-exit path takes it) equals the
+    verify call followed by the build call, bit for bit, on every output including the
+    hidden rows it must leave untouched."""
+    rej = u is not None
+    H, dt = binp["verify_hidden"].shape[1], binp["verify_hidden"].dtype
+
+    def bout():
+        o = ps.api.build_outputs(binp["B"], binp["K"], H, binp["T_cap"], dt, DEV)
+        o["draft_hidden"] = U.hidden_sentinel(binp["T_cap"], H, dt, DEV)
+        return o
+    with verify_path(path):
+        if rej:
+            v1 = ps.verify_rejection(target, draft, drafts, u, residual_mass=True)
+        else:
+            v1 = ps.verify_greedy(target, drafts)
+        n_verify = ps.pspec_last_launches()
+        b1 = ps.build_draft_batch(
+            K=binp["K"], block_size=binp["block_size"], mask_id=binp["mask_id"],
+            pad_id=binp["pad_id"], T_cap=binp["T_cap"], qsl_in=binp["qsl_in"],
+            verify_tokens=binp["verify_tokens"], verify_pos=binp["verify_pos"],
+            accepted_len=v1["accepted_len"], bonus=v1["bonus"], block_table=binp["block_table"],
+            verify_hidden=binp["verify_hidden"], h_shared=binp["h_shared"], out=bout())
+        v2, b2 = ps.step(target, drafts, binp, draft_logits=draft if rej else None, uniforms=u,
+                         residual_mass=rej, build_out=bout())
+        n_step = ps.pspec_last_launches()
+    torch.cuda.synchronize()
+    for k in v1:
+        assert torch.equal(v1[k], v2[k]), k
+    for k in b1:
+        assert torch.equal(b1[k], b2[k]), k
+    assert n_step == (1 if expect_fused else n_verify + 1), (n_step, n_verify)
+    return v2, b2
+
+
+@pytest.mark.parametrize("rule", ["greedy", "rejection"])
+def test_step_c64_fused(rule):
+    w = I.C64
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    binp = I.build_inputs(w, DEV, drafts=sampled)
+    rej = rule == "rejection"
+    _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, 0, True)
+
+
+@pytest.mark.parametrize("path,fused", [(0, False), (1, False), (2, True), (3, False)])
+@pytest.mark.parametrize("rule", ["greedy", "rejection"])
+def test_step_tiny_every_path(rule, path, fused):
+    w = I.scaled(I.C64, B=5, V=4096, H=64)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    binp = I.build_inputs(w, DEV, drafts=sampled)
+    rej = rule == "rejection"
+    _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, path, fused)
+
+
+@pytest.mark.parametrize("K,L_extra", [(1, 0), (3, 2), (7, 5)])
+def test_step_random_layouts_fused(K, L_extra):
+    """Spans with more verify rows than K+1 (the drafts are each span's last K rows)."""
+    from tests.oracle_pins import random_build_case
+    rng = np.random.default_rng(500 + K)
+    case = random_build_case(rng, B=37, K=K, H=32, bs=4, L_extra=L_extra)
+    binp = _torchify(case)
+    g = torch.Generator(device=DEV).manual_seed(K)
+    V = 3000
+    target = (torch.randn((37, K + 1, V), generator=g, device=DEV) * 2).to(torch.bfloat16)
+    draft = (target[:, :K].float() + torch.randn((37, K, V), generator=g, device=DEV) * 0.5).to(torch.bfloat16)
+    d = torch.argmax(draft.float(), dim=2).to(torch.int32)
+    u = torch.rand((37, K + 1), generator=g, device=DEV)
+    _step_check(target, draft, d, u, binp, 2, True)
+    _step_check(target, draft, d, None, binp, 2, True)
+
+
+def test_step_fused_invalid_layout_sets_bit():
+    from tests.oracle_pins import random_build_case
+    rng = np.random.default_rng(31)
+    case = random_build_case(rng, B=6, K=3, H=8, bs=4)
+    q = case["qsl_in"].copy()
+    q[3] = q[2] - 1                      # not an offset array: only the error bit is defined
+    binp = _torchify(dict(case, qsl_in=q))
+    target = torch.randn((6, 4, 512), device=DEV).to(torch.bfloat16)
+    d = torch.argmax(target[:, :3].float(), dim=2).to(torch.int32)
+    with verify_path(2):
+        _, bo = ps.step(target, d, binp)
+    torch.cuda.synchronize()
+    assert bo["err"].item() & ps._binding.PSPEC_DEVERR_LAYOUT
+
+
+def test_step_b1024_fused():
+    """Full size with fusion forced on (the automatic choice at 1024 sequences is two
+    launches), then forced off."""
+    w = I.B1024
+    target, draft = I.logits(w, DEV)
+    sampled, _ = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    binp = I.build_inputs(w, DEV, drafts=sampled)
+    try:
+        ps.pspec_set_step_fusion(1)
+        v, _ = _step_check(target, draft, sampled, u, binp, 0, True)
+        ps.pspec_set_step_fusion(2)
+        _step_check(target, draft, sampled, u, binp, 2, False)
+    finally:
+        ps.pspec_set_step_fusion(0)
+    seqs = _sample(w.B, 24, 5)
+    U.compare_rejection(v, U.oracle_rejection(target, draft, sampled, u, seqs), seqs)
+
+
+@pytest.mark.parametrize("path", [0, 1, 3])
+def test_step_cuda_graph_replay(path):
+    """One step captured in a CUDA graph and replayed with new uniforms and drafts copied
+    into the captured buffers gives what the eager calls give for those inputs (the
+    kernels leave their workspace counters at zero, so replays need no reset)."""
+    w = I.scaled(I.C64, B=96, V=20000, H=64)
+    target, draft = I.logits(w, DEV)
+    sampled, _ = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    binp = I.build_inputs(w, DEV, drafts=sampled)
+    ws = ps.Workspace(w.B, w.K, w.V, True)
+    vout = ps.api.verify_outputs(w.B, w.K, DEV, False, True, True)
+    bout = ps.api.build_outputs(w.B, w.K, 64, binp["T_cap"], binp["verify_hidden"].dtype, DEV)
+    d_in, u_in = sampled.clone(), u.clone()
+    with verify_path(path):
+        ps.step(target, d_in, binp, draft_logits=draft, uniforms=u_in, residual_mass=True,
+                workspace=ws, out=vout, build_out=bout)           # warm-up outside capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g):
+                ps.step(target, d_in, binp, draft_logits=draft, uniforms=u_in, residual_mass=True,
+                        workspace=ws, out=vout, build_out=bout)
+        torch.cuda.current_stream().wait_stream(side)
+        gen = torch.Generator(device=DEV).manual_seed(7)
+        for rep in range(3):
+            u_new = torch.rand(u.shape, generator=gen, device=DEV).clamp_(max=I.LAST_BELOW_ONE)
+            d_new = torch.where(torch.rand(sampled.shape, generator=gen, device=DEV) < 0.2,
+                                torch.randint_like(sampled, 0, w.V), sampled)
+            u_in.copy_(u_new)
+            d_in.copy_(d_new)
+            g.replay()
+            ref_v, ref_b = ps.step(target, d_new, binp, draft_logits=draft, uniforms=u_new,
+                                   residual_mass=True)
+            torch.cuda.synchronize()
+            for k in ("out_tokens", "accepted_len", "bonus", "residual_mass"):
+                assert torch.equal(vout[k], ref_v[k]), (rep, k)
+            for k in ("draft_tokens", "draft_pos", "slot_mapping", "row_kind", "hidden_src",
+                      "qsl_out", "seq_lens_out", "sample_idx"):
+                assert torch.equal(bout[k], ref_b[k]), (rep, k)
+    del g
