@@ -52,11 +52,11 @@ def _bind(path: str):
     lib = ctypes.CDLL(path)
     P = ctypes.c_void_p
     i32, i64, f64 = ctypes.c_int, ctypes.c_longlong, ctypes.c_double
-    lib.oracle_verify_greedy.argtypes = [i32, i32, i32, i64, i32, P, P, P, P, P, P, P]
+    lib.oracle_verify_greedy.argtypes = [i32, i32, i32, i64, i32, P, P, P, P, P, P, P, P]
     lib.oracle_verify_greedy.restype = i32
-    lib.oracle_verify_rejection.argtypes = [i32, i32, i32, i64, i32] + [P] * 13 + [f64, P]
+    lib.oracle_verify_rejection.argtypes = [i32, i32, i32, i64, i32] + [P] * 14 + [f64, P]
     lib.oracle_verify_rejection.restype = i32
-    lib.oracle_build_draft_batch.argtypes = [i32] * 10 + [P] * 17
+    lib.oracle_build_draft_batch.argtypes = [i32] * 10 + [P] * 18
     lib.oracle_build_draft_batch.restype = i32
     lib.oracle_sample_rows.argtypes = [i32, i32, i64, i32, P, P, P, P, P, f64]
     lib.oracle_sample_rows.restype = i32
@@ -99,11 +99,13 @@ class OracleLib:
         self.lib = _bind(path)
 
     def verify_greedy(self, target: np.ndarray, draft_tokens: np.ndarray,
-                      want_lse: bool = False, threads: int = 1) -> dict:
-        """Greedy verify of target logits [B, K+1, V] against drafts [B, K] (int32)."""
+                      want_lse: bool = False, threads: int = 1, k_len=None) -> dict:
+        """Greedy verify of target logits [B, K+1, V] against drafts [B, K] (int32);
+        k_len [B] (optional): each sequence's own draft count (R14)."""
         lib = self.lib
         target = np.ascontiguousarray(target)
         draft_tokens = np.ascontiguousarray(draft_tokens, dtype=np.int32)
+        k_len = None if k_len is None else np.ascontiguousarray(k_len, dtype=np.int32)
         B, K1, V = target.shape
         K = K1 - 1
         dt = _logits_dtype(target)
@@ -119,6 +121,7 @@ class OracleLib:
             e = ctypes.c_int(0)
             rc = lib.oracle_verify_greedy(
                 b1 - b0, K, V, V, dt, _ptr(target[b0:b1]), _ptr(draft_tokens[b0:b1]),
+                _ptr(k_len[b0:b1]) if k_len is not None else None,
                 _ptr(out["out_tokens"][b0:b1]), _ptr(out["accepted_len"][b0:b1]),
                 _ptr(out["bonus"][b0:b1]),
                 _ptr(out["target_lse"][b0:b1]) if want_lse else None, ctypes.byref(e))
@@ -132,14 +135,16 @@ class OracleLib:
 
     def verify_rejection(self, target: np.ndarray, draft: np.ndarray, draft_tokens: np.ndarray,
                          uniforms: np.ndarray, tie_eps: float = TIE_EPS,
-                         threads: int = 1) -> dict:
+                         threads: int = 1, k_len=None) -> dict:
         """Rejection-rule verify: target [B, K+1, V], draft [B, K, V], drafts [B, K],
-        uniforms [B, K+1] (float32).  Returns tokens, counts, flags and double diagnostics."""
+        uniforms [B, K+1] (float32), k_len [B] (optional, R14).  Returns tokens, counts,
+        flags and double diagnostics."""
         lib = self.lib
         target = np.ascontiguousarray(target)
         draft = np.ascontiguousarray(draft)
         draft_tokens = np.ascontiguousarray(draft_tokens, dtype=np.int32)
         uniforms = np.ascontiguousarray(uniforms, dtype=np.float32)
+        k_len = None if k_len is None else np.ascontiguousarray(k_len, dtype=np.int32)
         B, K1, V = target.shape
         K = K1 - 1
         assert draft.shape == (B, K, V) and draft.dtype == target.dtype
@@ -164,6 +169,7 @@ class OracleLib:
             rc = lib.oracle_verify_rejection(
                 b1 - b0, K, V, V, dt, _ptr(target[b0:b1]), _ptr(draft[b0:b1]),
                 _ptr(draft_tokens[b0:b1]), _ptr(uniforms[b0:b1]),
+                _ptr(k_len[b0:b1]) if k_len is not None else None,
                 _ptr(o["out_tokens"]), _ptr(o["accepted_len"]), _ptr(o["bonus"]),
                 _ptr(o["p_at_draft"]), _ptr(o["q_at_draft"]), _ptr(o["target_lse"]),
                 _ptr(o["draft_lse"]), _ptr(o["residual_mass"]), _ptr(o["flags"]),
@@ -206,7 +212,7 @@ class OracleLib:
     def build_draft_batch(self, *, K: int, block_size: int, mask_id: int, pad_id: int,
                           T_cap: int, qsl_in, verify_tokens, verify_pos, accepted_len, bonus,
                           block_table, verify_hidden=None, h_shared=None,
-                          draft_hidden_init=None) -> dict:
+                          draft_hidden_init=None, k_len=None) -> dict:
         """P-EAGLE draft-batch construction (single-threaded: offsets are a running sum).
 
         ``verify_hidden`` [T_in, H] and ``h_shared`` [H] may be any dtype of equal element
@@ -219,6 +225,7 @@ class OracleLib:
         accepted_len = np.ascontiguousarray(accepted_len, dtype=np.int32)
         bonus = np.ascontiguousarray(bonus, dtype=np.int32)
         block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+        k_len = None if k_len is None else np.ascontiguousarray(k_len, dtype=np.int32)
         B = qsl_in.shape[0] - 1
         T_in = verify_tokens.shape[0]
         max_blocks = block_table.shape[1] if block_table.ndim == 2 else 1
@@ -248,7 +255,7 @@ class OracleLib:
         rc = lib.oracle_build_draft_batch(
             B, K, H, eb, block_size, max_blocks, mask_id, pad_id, T_in, T_cap,
             _ptr(qsl_in), _ptr(verify_tokens), _ptr(verify_pos), _ptr(accepted_len), _ptr(bonus),
-            _ptr(block_table), _ptr(verify_hidden), _ptr(h_shared),
+            _ptr(k_len) if k_len is not None else None, _ptr(block_table), _ptr(verify_hidden), _ptr(h_shared),
             _ptr(out["draft_tokens"]), _ptr(out["draft_pos"]), _ptr(out["slot_mapping"]),
             _ptr(out["row_kind"]), _ptr(out["hidden_src"]), _ptr(out["qsl_out"]),
             _ptr(out["seq_lens_out"]), _ptr(out["sample_idx"]), _ptr(dh), ctypes.byref(e))

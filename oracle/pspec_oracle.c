@@ -111,8 +111,19 @@ static int row_argmax(const void *base, int dtype, long long off, int V)
     return best;
 }
 
+/* R14: sequence i's own draft count K_i (k_len[i]; K when k_len is NULL), clamped into
+   [0, K] with error bit 0x20 when outside */
+static int draft_count(const int *k_len, int i, int K, int *e)
+{
+    if (!k_len) return K;
+    int k = k_len[i];
+    if (k < 0 || k > K) { *e |= 0x20; k = k < 0 ? 0 : K; }
+    return k;
+}
+
 int oracle_verify_greedy(int B, int K, int V, long long ld, int dtype,
                          const void *target_logits, const int *draft_tokens,
+                         const int *k_len,
                          int *out_tokens, int *accepted_len, int *bonus,
                          double *target_lse, int *err)
 {
@@ -128,15 +139,17 @@ int oracle_verify_greedy(int B, int K, int V, long long ld, int dtype,
             if (target_lse) target_lse[(long long)i * (K + 1) + k] =
                 row_logsumexp(target_logits, dtype, off, V);
         }
-        /* accepted prefix: drafts that equal the greedy choice, in order [P3 Concept] */
+        /* accepted prefix: drafts that equal the greedy choice, in order [P3 Concept];
+           only the sequence's own K_i drafts are tested (R14) */
+        const int Ki = draft_count(k_len, i, K, &e);
         int a = 0;
-        while (a < K) {
+        while (a < Ki) {
             int d = draft_tokens[(long long)i * K + a];
             if (d < 0 || d >= V) { e |= 0x1; break; }
             if (d != amax[a]) break;
             ++a;
         }
-        for (int k = a; k < K; ++k) {     /* R5: range errors past the prefix count too */
+        for (int k = a; k < Ki; ++k) {    /* R5: range errors past the prefix count too */
             int d = draft_tokens[(long long)i * K + k];
             if (d < 0 || d >= V) e |= 0x1;
         }
@@ -155,7 +168,7 @@ int oracle_verify_greedy(int B, int K, int V, long long ld, int dtype,
 int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
                             const void *target_logits, const void *draft_logits,
                             const int *draft_tokens, const float *uniforms,
-                            int *out_tokens, int *accepted_len, int *bonus,
+                            const int *k_len, int *out_tokens, int *accepted_len, int *bonus,
                             double *p_at_draft, double *q_at_draft,
                             double *target_lse, double *draft_lse,
                             double *residual_mass, int *flags, double tie_eps, int *err)
@@ -176,6 +189,7 @@ int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
         const int *d = draft_tokens + (long long)i * K;
         const float *u = uniforms + (long long)i * (K + 1);
         int flag = 0;
+        const int Ki = draft_count(k_len, i, K, &e);       /* R14 */
 
         /* softmax normalisers of the K+1 target rows and the K draft rows */
         for (int k = 0; k <= K; ++k) {
@@ -194,16 +208,16 @@ int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
             if (d[k] >= 0 && d[k] < V) {
                 pk[k] = row_prob(target_logits, dtype, ((long long)i * (K + 1) + k) * ld, d[k], lse_t[k]);
                 qk[k] = row_prob(draft_logits, dtype, ((long long)i * K + k) * ld, d[k], lse_q[k]);
-            } else {
-                e |= 0x1;                 /* R5 */
+            } else if (k < Ki) {
+                e |= 0x1;                 /* R5 (the sequence's own drafts only) */
             }
             if (p_at_draft) p_at_draft[(long long)i * K + k] = pk[k];
             if (q_at_draft) q_at_draft[(long long)i * K + k] = qk[k];
         }
 
         /* accept drafts in order with probability min(1, p/q); stop at the first rejection */
-        int a = K;
-        for (int k = 0; k < K; ++k) {
+        int a = Ki;
+        for (int k = 0; k < Ki; ++k) {
             int accept;
             if (qk[k] > 0.0) {
                 double ratio = pk[k] / qk[k];
@@ -216,10 +230,10 @@ int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
         }
 
         /* the distribution to draw from: norm(max(0, p_a - q_a)) after a rejection,
-           the target's row K when every draft passed */
+           the target's row K_i when every draft passed */
         long long toff = ((long long)i * (K + 1) + a) * ld;
         double Z = 0.0;
-        if (a < K) {
+        if (a < Ki) {
             long long qoff = ((long long)i * K + a) * ld;
             for (int t = 0; t < V; ++t) {
                 double diff = row_prob(target_logits, dtype, toff, t, lse_t[a]) -
@@ -228,7 +242,7 @@ int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
                 Z += r[t];
             }
         }
-        if (a == K || Z == 0.0) {        /* R3: Z = 0 falls back to p itself */
+        if (a == Ki || Z == 0.0) {       /* R3: Z = 0 falls back to p itself */
             Z = 0.0;
             for (int t = 0; t < V; ++t) {
                 r[t] = row_prob(target_logits, dtype, toff, t, lse_t[a]);
@@ -237,8 +251,8 @@ int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
         }
         if (residual_mass) residual_mass[i] = Z;
 
-        /* inverse CDF in token-id order (R3) */
-        double thr = (double)u[K] * Z;
+        /* inverse CDF in token-id order (R3), driven by uniform column K_i (R4, R14) */
+        double thr = (double)u[Ki] * Z;
         double cum = 0.0, prev = 0.0;
         int tok = -1, last_pos = -1;
         for (int t = 0; t < V; ++t) {
@@ -327,7 +341,8 @@ int oracle_build_draft_batch(int B, int K, int H, int hidden_elem_bytes,
                              int block_size, int max_blocks, int mask_id, int pad_id,
                              int T_in, int T_cap,
                              const int *qsl_in, const int *verify_tokens, const int *verify_pos,
-                             const int *accepted_len, const int *bonus, const int *block_table,
+                             const int *accepted_len, const int *bonus, const int *k_len,
+                             const int *block_table,
                              const void *verify_hidden, const void *h_shared,
                              int *draft_tokens, int *draft_pos, long long *slot_mapping,
                              unsigned char *row_kind, int *hidden_src,
@@ -379,15 +394,18 @@ int oracle_build_draft_batch(int B, int K, int H, int hidden_elem_bytes,
         int s = qsl_in[i];
         int L = qsl_in[i + 1] - qsl_in[i];
         int o = qsl_out[i];
-        if (L < K + 1) {                  /* R7: too short to hold K drafts; stays padding */
+        /* R14: the span's last K_i verify rows held this step's drafts; the next step still
+           gets K-1 mask slots */
+        const int Ki = draft_count(k_len, i, K, &e);
+        if (L < Ki + 1) {                 /* R7: too short to hold its drafts; stays padding */
             e |= 0x8;
             seq_lens_out[i] = 0;
             for (int k = 0; k < K; ++k) sample_idx[(long long)i * K + k] = -1;
             continue;
         }
         int a = accepted_len[i];
-        if (a < 0 || a > K) { e |= 0x2; a = a < 0 ? 0 : K; }
-        int c = L - K + a;                /* surviving verify rows; the last one is h_context */
+        if (a < 0 || a > Ki) { e |= 0x2; a = a < 0 ? 0 : Ki; }
+        int c = L - Ki + a;               /* surviving verify rows; the last one is h_context */
         int ntp_pos = verify_pos[s + c - 1];
 
         for (int j = 0; j < L + K - 1; ++j) {

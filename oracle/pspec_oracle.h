@@ -6,7 +6,16 @@
  * is host memory owned by the caller; every function returns 0 on success and 1 on a
  * malformed call (negative sizes, too small a capacity).  Invalid *values* (tokens out of
  * range, accepted counts out of range, block lookups past the table) never stop it: they
- * OR bits into *err (0x1 token range, 0x2 accepted count, 0x4 block lookup, 0x8 layout).
+ * OR bits into *err (0x1 token range, 0x2 accepted count, 0x4 block lookup, 0x8 layout,
+ * 0x20 draft count).
+ *
+ * k_len (every function that takes it; NULL = K for every sequence): sequence i's own draft
+ * count K_i in [0, K] (R14).  Sequence i is then verified exactly as if it were alone with
+ * K = K_i: drafts 0..K_i-1 are tested (with uniforms 0..K_i-1), the bonus after K_i
+ * acceptances comes from target row K_i, the draw uses uniform column K_i, and only those
+ * drafts are range-checked; out_tokens keeps K+1 columns (-1 after the bonus).  In the
+ * draft batch K_i sets how many of the span's verify rows were drafts (c_i = L_i - K_i +
+ * a_i survive); every span still gets K-1 mask rows.
  */
 #ifndef PSPEC_ORACLE_H
 #define PSPEC_ORACLE_H
@@ -24,7 +33,7 @@ enum { ORACLE_ROW_CTX = 0, ORACLE_ROW_NTP = 1, ORACLE_ROW_MASK = 2, ORACLE_ROW_R
    when non-NULL, target_lse [B, K+1] in double. */
 int oracle_verify_greedy(int B, int K, int V, long long ld, int dtype,
                          const void *target_logits, const int *draft_tokens,
-                         int *out_tokens, int *accepted_len, int *bonus,
+                         const int *k_len, int *out_tokens, int *accepted_len, int *bonus,
                          double *target_lse, int *err);
 
 /* Rejection-rule verify.  draft_logits: [B, K, ld]; uniforms: [B, K+1] in [0,1), column K
@@ -35,7 +44,7 @@ int oracle_verify_greedy(int B, int K, int V, long long ld, int dtype,
 int oracle_verify_rejection(int B, int K, int V, long long ld, int dtype,
                             const void *target_logits, const void *draft_logits,
                             const int *draft_tokens, const float *uniforms,
-                            int *out_tokens, int *accepted_len, int *bonus,
+                            const int *k_len, int *out_tokens, int *accepted_len, int *bonus,
                             double *p_at_draft, double *q_at_draft,
                             double *target_lse, double *draft_lse,
                             double *residual_mass, int *flags, double tie_eps, int *err);
@@ -59,7 +68,8 @@ int oracle_build_draft_batch(int B, int K, int H, int hidden_elem_bytes,
                              int block_size, int max_blocks, int mask_id, int pad_id,
                              int T_in, int T_cap,
                              const int *qsl_in, const int *verify_tokens, const int *verify_pos,
-                             const int *accepted_len, const int *bonus, const int *block_table,
+                             const int *accepted_len, const int *bonus, const int *k_len,
+                             const int *block_table,
                              const void *verify_hidden, const void *h_shared,
                              int *draft_tokens, int *draft_pos, long long *slot_mapping,
                              unsigned char *row_kind, int *hidden_src,

@@ -343,16 +343,18 @@ def pin_build_worked_example(o):
     assert r["err"] == 0
 
 
-def random_build_case(rng, B, K, H, bs, V=1000, L_extra=0, permuted=True):
-    """A random valid verify batch with disjoint block tables (a test input, not an oracle)."""
-    L = K + 1 + rng.integers(0, L_extra + 1, size=B)
+def random_build_case(rng, B, K, H, bs, V=1000, L_extra=0, permuted=True, k_len=None):
+    """A random valid verify batch with disjoint block tables (a test input, not an oracle).
+    With k_len [B], sequence i's span ends in its own K_i drafts (L_i >= K_i + 1)."""
+    kn = np.full(B, K) if k_len is None else np.asarray(k_len)
+    L = kn + 1 + rng.integers(0, L_extra + 1, size=B)
     qsl = np.zeros(B + 1, np.int64)
     qsl[1:] = np.cumsum(L)
     T_in = int(qsl[-1])
     ctx = rng.integers(0, 200, size=B)
     pos = np.concatenate([c + np.arange(l) for c, l in zip(ctx, L)])
     tok = rng.integers(0, V, size=T_in)
-    a = rng.integers(0, K + 1, size=B)
+    a = rng.integers(0, kn + 1)
     bonus = rng.integers(0, V, size=B)
     nblk = -(-(ctx + L + K) // bs)
     mb = int(nblk.max())
@@ -365,9 +367,12 @@ def random_build_case(rng, B, K, H, bs, V=1000, L_extra=0, permuted=True):
     hidden = rng.normal(size=(T_in, H)).astype(np.float32)
     hs = rng.normal(size=H).astype(np.float32)
     T_cap = T_in + B * (K - 1) + int(rng.integers(0, 9))
-    return dict(K=K, block_size=bs, mask_id=V, pad_id=V + 1, T_cap=T_cap, qsl_in=qsl,
+    case = dict(K=K, block_size=bs, mask_id=V, pad_id=V + 1, T_cap=T_cap, qsl_in=qsl,
                 verify_tokens=tok, verify_pos=pos, accepted_len=a, bonus=bonus,
                 block_table=table, verify_hidden=hidden, h_shared=hs)
+    if k_len is not None:
+        case["k_len"] = np.asarray(k_len, np.int32)
+    return case
 
 
 def check_build_invariants(case, r):
@@ -384,13 +389,15 @@ def check_build_invariants(case, r):
     vt, vp = np.asarray(case["verify_tokens"]), np.asarray(case["verify_pos"])
     table = np.asarray(case["block_table"])
     valid_slots = []
+    kn = np.asarray(case["k_len"]) if case.get("k_len") is not None else np.full(B, K)
     for i in range(B):
         s, L = int(qsl[i]), int(qsl[i + 1] - qsl[i])
         a = int(case["accepted_len"][i])
-        c = L - K + a
+        Ki = int(kn[i])                                              # R14
+        c = L - Ki + a
         span = slice(qo[i], qo[i + 1])
         ks = kind[span]
-        want = [0] * (c - 1) + [1] + [2] * (K - 1) + [3] * (K - a)
+        want = [0] * (c - 1) + [1] + [2] * (K - 1) + [3] * (Ki - a)
         assert ks.tolist() == want, (i, ks.tolist(), want)
         p = pos[span]
         live = p[: c + K - 1]
@@ -494,9 +501,99 @@ def pin_sampling(o):
             assert abs(thr - Pc[n, t]) < 2e-7, (n, t, thr, Pc[n, t])
 
 
+# ----------------------------------------------------------------------------- K_i (R14)
+def pin_k_len_worked_examples(o):
+    """Hand-derived examples with per-sequence draft counts (the "k_len" entries of
+    tests/golden/verify_worked_examples.json)."""
+    g = _load("verify_worked_examples.json")
+    for c in g["k_len_cases"]:
+        t = np.log(np.array(c["p"], np.float64)).astype(np.float32)[None]
+        q = np.log(np.array(c["q"], np.float64)).astype(np.float32)[None]
+        d = np.array([c["drafts"]], np.int32)
+        u = np.array([c["u"]], np.float32)
+        kl = np.array([c["k_len"]], np.int32)
+        r = o.verify_rejection(t, q, d, u, k_len=kl)
+        e = c["rejection"]
+        assert r["out_tokens"][0].tolist() == e["out_tokens"], (c["name"], r["out_tokens"])
+        assert int(r["accepted_len"][0]) == e["accepted_len"], c["name"]
+        np.testing.assert_allclose(r["residual_mass"][0], e["residual_mass"], rtol=1e-6)
+        assert r["flags"][0] == 0 and r["err"] == 0
+        gr = o.verify_greedy(t, d, k_len=kl)
+        assert gr["out_tokens"][0].tolist() == c["greedy"]["out_tokens"], (c["name"], gr["out_tokens"])
+
+
+def pin_k_len_reduces_to_truncation(o):
+    """A sequence with K_i drafts gives exactly what the fixed-K oracle gives for that
+    sequence alone cut to K = K_i (its first K_i+1 target rows, K_i draft rows and drafts,
+    uniform columns 0..K_i); K_i = 0 draws the bonus from target row 0 with u_0 (the
+    drafter-row sampler) or takes its numpy argmax.  Drafts past K_i are never read: -1
+    there sets no error bit.  A count outside [0, K] sets bit 0x20 and is clamped."""
+    rng = np.random.default_rng(41)
+    B, K, V = 14, 5, 40
+    t = rng.normal(0, 2, size=(B, K + 1, V)).astype(np.float32)
+    q = (t[:, :K] + rng.normal(0, 0.5, size=(B, K, V))).astype(np.float32)
+    d = np.argmax(q, axis=2).astype(np.int32)
+    u = rng.random((B, K + 1), dtype=np.float32)
+    kl = np.array([0, K, 1, 2, 3, 4, 5, 0, 1, 3, 2, 5, 4, 1], np.int32)
+    for i in range(B):
+        d[i, kl[i]:] = -1                                   # unused slots
+    r = o.verify_rejection(t, q, d, u, k_len=kl)
+    gr = o.verify_greedy(t, d, k_len=kl)
+    assert r["err"] == 0 and gr["err"] == 0
+    for i in range(B):
+        Ki = int(kl[i])
+        out, gout = r["out_tokens"][i], gr["out_tokens"][i]
+        if Ki == 0:
+            s = o.sample_rows(t[i, 0][None], u[i, :1])
+            assert out.tolist() == [int(s["tokens"][0])] + [-1] * K
+            assert gout.tolist() == [int(np.argmax(t[i, 0]))] + [-1] * K
+            assert r["accepted_len"][i] == 0 and gr["accepted_len"][i] == 0
+            continue
+        ri = o.verify_rejection(t[i:i + 1, :Ki + 1], q[i:i + 1, :Ki], d[i:i + 1, :Ki],
+                                u[i:i + 1, :Ki + 1])
+        gi = o.verify_greedy(t[i:i + 1, :Ki + 1], d[i:i + 1, :Ki])
+        assert out.tolist() == ri["out_tokens"][0].tolist() + [-1] * (K - Ki), i
+        assert gout.tolist() == gi["out_tokens"][0].tolist() + [-1] * (K - Ki), i
+        assert r["flags"][i] == ri["flags"][0]
+        np.testing.assert_allclose(r["residual_mass"][i], ri["residual_mass"][0], rtol=1e-12)
+        np.testing.assert_allclose(r["p_at_draft"][i, :Ki], ri["p_at_draft"][0], rtol=1e-12)
+    bad = kl.copy()
+    bad[3], bad[4] = -1, K + 2
+    r2 = o.verify_rejection(t, q, np.where(d < 0, 0, d).astype(np.int32), u, k_len=bad)
+    assert r2["err"] & 0x20
+    assert r2["accepted_len"][3] == 0 and r2["accepted_len"][4] <= K
+
+
+def pin_build_k_len(o):
+    """Draft batch with per-sequence K_i: with spans of at least K+1 rows, K_i and accepted
+    count a give the batch that fixed K gives for a + K - K_i (the same surviving rows);
+    spans down to K_i + 1 rows keep the layout invariants (c_i context rows, K-1 masks,
+    K_i - a rejected rows)."""
+    rng = np.random.default_rng(43)
+    K, B = 5, 12
+    kl = rng.integers(0, K + 1, size=B).astype(np.int32)
+    case = random_build_case(rng, B=B, K=K, H=8, bs=4, L_extra=3, k_len=np.full(B, K))
+    case["k_len"] = kl                                      # spans hold >= K+1 rows
+    case["accepted_len"] = rng.integers(0, kl + 1).astype(np.int32)
+    r = o.build_draft_batch(**case)
+    fixed = dict(case, accepted_len=case["accepted_len"] + (K - kl))
+    del fixed["k_len"]
+    rf = o.build_draft_batch(**fixed)
+    assert r["err"] == 0 and rf["err"] == 0
+    for k in ("draft_tokens", "draft_pos", "slot_mapping", "row_kind", "hidden_src", "qsl_out",
+              "seq_lens_out", "sample_idx", "draft_hidden"):
+        assert np.array_equal(r[k], rf[k]), k
+    short = random_build_case(rng, B=B, K=K, H=8, bs=4, L_extra=0, k_len=kl)
+    init = np.full((short["T_cap"], 8), np.nan, np.float32)
+    check_build_invariants(short, o.build_draft_batch(**short, draft_hidden_init=init))
+    over = dict(short, accepted_len=np.where(kl > 0, kl + 1, 0).astype(np.int32))
+    assert o.build_draft_batch(**over)["err"] & 0x2     # a_i > K_i: clamped, bit set
+
+
 ALL_PINS = [
     pin_worked_examples, pin_greedy_matches_numpy_argmax, pin_bf16_decoding,
     pin_probabilities_match_scipy, pin_residual_mass_closed_form, pin_special_cases,
     pin_exact_distribution, pin_build_worked_example, pin_build_invariants,
-    pin_build_invalid_values, pin_sampling,
+    pin_build_invalid_values, pin_sampling, pin_k_len_worked_examples,
+    pin_k_len_reduces_to_truncation, pin_build_k_len,
 ]

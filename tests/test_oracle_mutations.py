@@ -47,6 +47,11 @@ MUTANTS = [
     ("sample_greedy_last_tie", "            tok = row_argmax(logits, dtype, off, V);\n        } else {",
      "            tok = row_argmax(logits, dtype, off, V) + (V > 1);\n        } else {"),
     ("offsets_without_masks", "off += (qsl_in[i + 1] - qsl_in[i]) + K - 1;", "off += (qsl_in[i + 1] - qsl_in[i]) + K;"),
+    ("k_len_draw_column_K", "double thr = (double)u[Ki] * Z;", "double thr = (double)u[K] * Z;"),
+    ("k_len_accept_loop_K", "int a = Ki;\n        for (int k = 0; k < Ki; ++k) {",
+     "int a = K;\n        for (int k = 0; k < K; ++k) {"),
+    ("k_len_greedy_ignored", "while (a < Ki) {", "while (a < K) {"),
+    ("k_len_build_survivors", "int c = L - Ki + a;", "int c = L - K + a;"),
 ]
 
 
