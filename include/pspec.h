@@ -73,6 +73,7 @@ typedef enum { PSPEC_F32 = 0, PSPEC_BF16 = 1 } pspec_dtype;
                                           fewer than K+1 verify rows */
 #define PSPEC_DEVERR_TIMEOUT 0x10      /* a bounded wait for an asynchronous copy ran out
                                           (outputs of that call are not valid) */
+#define PSPEC_DEVERR_KLEN_RANGE 0x20   /* k_len[i] outside [0, K]: clamped into it */
 
 /* Row kinds written to pspec_build_args.row_kind. */
 #define PSPEC_ROW_CTX 0   /* context row: accepted token paired with its target hidden */
@@ -120,6 +121,14 @@ typedef struct {
   float *residual_mass;        /* [B]      Z = sum max(0, p - q) of the resampled row, or
                                            sum p of the bonus row (rejection) */
   int32_t *err;                /* device error word (required); bits are OR-ed in */
+  const int32_t *k_len;        /* [B] per-sequence draft counts K_i in [0, K], or NULL for K
+                                  everywhere ("dynamic draft length", rskf.cn article,
+                                  section 3.2, MTP): sequence i is verified as if it were
+                                  alone with K = K_i -- drafts 0..K_i-1 tested with uniforms
+                                  0..K_i-1, the bonus after K_i acceptances from target row
+                                  K_i, the draw on uniform column K_i, only those drafts
+                                  range-checked; rows past K_i are never needed (the
+                                  early-exit and work-queue paths never read them). */
 } pspec_verify_args;
 
 /*
@@ -254,6 +263,10 @@ typedef struct {
   int32_t *sample_idx;            /* [B, K] out */
   void *draft_hidden;             /* [T_cap, H] out (16-byte aligned rows) */
   int32_t *err;                   /* device error word (required) */
+  const int32_t *k_len;           /* [B] per-sequence draft counts K_i in [0, K], or NULL for
+                                     K everywhere: the last K_i verify rows of span i held
+                                     this step's drafts, so c_i = L_i - K_i + a_i rows survive
+                                     (L_i >= K_i + 1); every span still gets K-1 mask rows */
 } pspec_build_args;
 
 /*

@@ -19,6 +19,7 @@ PSPEC_OK, PSPEC_ERR_INVALID_ARG, PSPEC_ERR_UNSUPPORTED, PSPEC_ERR_CUDA, PSPEC_ER
 PSPEC_F32, PSPEC_BF16 = 0, 1
 PSPEC_DEVERR_TOKEN_RANGE, PSPEC_DEVERR_ACCEPT_RANGE = 0x1, 0x2
 PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT, PSPEC_DEVERR_TIMEOUT = 0x4, 0x8, 0x10
+PSPEC_DEVERR_KLEN_RANGE = 0x20
 PSPEC_ROW_CTX, PSPEC_ROW_NTP, PSPEC_ROW_MASK, PSPEC_ROW_REJ, PSPEC_ROW_PAD = range(5)
 PSPEC_PADDING_SLOT_ID = -1
 PSPEC_MAX_K = 31
@@ -49,7 +50,7 @@ class pspec_verify_args(ctypes.Structure):
         ("target_logits", _P), ("draft_logits", _P), ("draft_tokens", _P), ("uniforms", _P),
         ("out_tokens", _P), ("accepted_len", _P), ("bonus", _P),
         ("target_lse", _P), ("draft_lse", _P), ("p_at_draft", _P), ("q_at_draft", _P),
-        ("residual_mass", _P), ("err", _P),
+        ("residual_mass", _P), ("err", _P), ("k_len", _P),
     ]
 
 
@@ -68,7 +69,7 @@ class pspec_build_args(ctypes.Structure):
         ("bonus", _P), ("block_table", _P), ("verify_hidden", _P), ("h_shared", _P),
         ("draft_tokens", _P), ("draft_pos", _P), ("slot_mapping", _P), ("row_kind", _P),
         ("hidden_src", _P), ("qsl_out", _P), ("seq_lens_out", _P), ("sample_idx", _P),
-        ("draft_hidden", _P), ("err", _P),
+        ("draft_hidden", _P), ("err", _P), ("k_len", _P),
     ]
 
 
@@ -204,7 +205,7 @@ def pspec_verify_workspace_bytes(B: int, K: int, V: int, rejection: bool) -> int
 
 def _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
                  accepted_len, bonus, err, target_lse, draft_lse, p_at_draft, q_at_draft,
-                 residual_mass, K):
+                 residual_mass, K, k_len=None):
     B, V, ld, dt = _logits_layout(target_logits, K + 1, "target_logits")
     a = pspec_verify_args()
     a.B, a.K, a.V, a.ld, a.dtype = B, K, V, ld, dt
@@ -225,14 +226,15 @@ def _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens
     a.q_at_draft = _ptr(q_at_draft, torch.float32, "q_at_draft")
     a.residual_mass = _ptr(residual_mass, torch.float32, "residual_mass")
     a.err = _ptr(err, torch.int32, "err")
+    a.k_len = _ptr(k_len, torch.int32, "k_len")
     return a
 
 
 def pspec_verify_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len, bonus, err,
-                        workspace, target_lse=None, stream=None) -> None:
+                        workspace, target_lse=None, k_len=None, stream=None) -> None:
     K = int(target_logits.shape[1]) - 1
     a = _verify_args(target_logits, None, draft_tokens, None, out_tokens, accepted_len, bonus,
-                     err, target_lse, None, None, None, None, K)
+                     err, target_lse, None, None, None, None, K, k_len)
     st = LIB.pspec_verify_greedy(ctypes.byref(a), _ptr(workspace, torch.uint8, "workspace"),
                                  workspace.numel(), _stream(stream))
     if st != PSPEC_OK:
@@ -242,11 +244,11 @@ def pspec_verify_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len
 def pspec_verify_rejection(*, target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
                            accepted_len, bonus, err, workspace, target_lse=None, draft_lse=None,
                            p_at_draft=None, q_at_draft=None, residual_mass=None,
-                           stream=None) -> None:
+                           k_len=None, stream=None) -> None:
     K = int(target_logits.shape[1]) - 1
     a = _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
                      accepted_len, bonus, err, target_lse, draft_lse, p_at_draft, q_at_draft,
-                     residual_mass, K)
+                     residual_mass, K, k_len)
     st = LIB.pspec_verify_rejection(ctypes.byref(a), _ptr(workspace, torch.uint8, "workspace"),
                                     workspace.numel(), _stream(stream))
     if st != PSPEC_OK:
@@ -277,7 +279,7 @@ def pspec_sample_drafts(*, logits, draft_tokens, err, workspace, uniforms=None, 
 def _build_args(*, K, block_size, mask_id, pad_id, T_cap, qsl_in, verify_tokens, verify_pos,
                 accepted_len, bonus, block_table, verify_hidden, h_shared, draft_tokens,
                 draft_pos, slot_mapping, row_kind, hidden_src, qsl_out, seq_lens_out,
-                sample_idx, draft_hidden, err):
+                sample_idx, draft_hidden, err, k_len=None):
     a = pspec_build_args()
     a.B = int(qsl_in.numel()) - 1
     a.K = int(K)
@@ -314,6 +316,7 @@ def _build_args(*, K, block_size, mask_id, pad_id, T_cap, qsl_in, verify_tokens,
     a.sample_idx = _ptr(sample_idx, torch.int32, "sample_idx")
     a.draft_hidden = _ptr(draft_hidden, None, "draft_hidden")
     a.err = _ptr(err, torch.int32, "err")
+    a.k_len = _ptr(k_len, torch.int32, "k_len")
     return a
 
 
@@ -326,12 +329,12 @@ def pspec_build_draft_batch(*, stream=None, **build) -> None:
 
 
 def pspec_step_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len, bonus, err,
-                      workspace, build: dict, stream=None) -> None:
+                      workspace, build: dict, k_len=None, stream=None) -> None:
     """Greedy verify followed by the draft-batch build (`build`: the keyword arguments of
     pspec_build_draft_batch, with accepted_len / bonus None or this call's outputs)."""
     K = int(target_logits.shape[1]) - 1
     v = _verify_args(target_logits, None, draft_tokens, None, out_tokens, accepted_len, bonus,
-                     err, None, None, None, None, None, K)
+                     err, None, None, None, None, None, K, k_len)
     b = _build_args(**build)
     st = LIB.pspec_step_greedy(ctypes.byref(v), ctypes.byref(b),
                                _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
@@ -342,11 +345,11 @@ def pspec_step_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len, 
 
 def pspec_step_rejection(*, target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
                          accepted_len, bonus, err, workspace, build: dict, residual_mass=None,
-                         stream=None) -> None:
+                         k_len=None, stream=None) -> None:
     """Rejection-rule verify followed by the draft-batch build (see pspec_step_greedy)."""
     K = int(target_logits.shape[1]) - 1
     v = _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
-                     accepted_len, bonus, err, None, None, None, None, residual_mass, K)
+                     accepted_len, bonus, err, None, None, None, None, residual_mass, K, k_len)
     b = _build_args(**build)
     st = LIB.pspec_step_rejection(ctypes.byref(v), ctypes.byref(b),
                                   _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),

@@ -46,8 +46,9 @@ def verify_outputs(Bn: int, K: int, device, diagnostics: bool, rejection: bool,
 
 def verify_greedy(target_logits: torch.Tensor, draft_tokens: torch.Tensor, *,
                   want_lse: bool = False, workspace: Workspace | None = None, out=None,
-                  stream=None) -> dict:
-    """Greedy verify.  Returns out_tokens, accepted_len, bonus, err (+ target_lse)."""
+                  k_len: torch.Tensor | None = None, stream=None) -> dict:
+    """Greedy verify.  Returns out_tokens, accepted_len, bonus, err (+ target_lse).
+    k_len [B] int32 (optional): each sequence's own draft count."""
     Bn, K1, V = target_logits.shape
     K = K1 - 1
     o = out if out is not None else verify_outputs(Bn, K, target_logits.device, want_lse, False)
@@ -55,14 +56,16 @@ def verify_greedy(target_logits: torch.Tensor, draft_tokens: torch.Tensor, *,
     _b.pspec_verify_greedy(target_logits=target_logits, draft_tokens=draft_tokens,
                           out_tokens=o["out_tokens"], accepted_len=o["accepted_len"],
                           bonus=o["bonus"], err=o["err"], workspace=ws.tensor,
-                          target_lse=o.get("target_lse") if want_lse else None, stream=stream)
+                          target_lse=o.get("target_lse") if want_lse else None, k_len=k_len,
+                          stream=stream)
     return o
 
 
 def verify_rejection(target_logits: torch.Tensor, draft_logits: torch.Tensor,
                      draft_tokens: torch.Tensor, uniforms: torch.Tensor, *,
                      diagnostics: bool = False, residual_mass: bool = False,
-                     workspace: Workspace | None = None, out=None, stream=None) -> dict:
+                     workspace: Workspace | None = None, out=None,
+                     k_len: torch.Tensor | None = None, stream=None) -> dict:
     """Rejection-rule verify.  Returns out_tokens, accepted_len, bonus, err (+ fp32
     diagnostics target_lse, draft_lse, p_at_draft, q_at_draft, residual_mass; or only
     residual_mass)."""
@@ -77,7 +80,7 @@ def verify_rejection(target_logits: torch.Tensor, draft_logits: torch.Tensor,
                              bonus=o["bonus"], err=o["err"], workspace=ws.tensor,
                              target_lse=o.get("target_lse"), draft_lse=o.get("draft_lse"),
                              p_at_draft=o.get("p_at_draft"), q_at_draft=o.get("q_at_draft"),
-                             residual_mass=o.get("residual_mass"), stream=stream)
+                             residual_mass=o.get("residual_mass"), k_len=k_len, stream=stream)
     return o
 
 
@@ -120,7 +123,7 @@ def build_outputs(Bn: int, K: int, H: int, T_cap: int, hidden_dtype, device) -> 
 
 def build_draft_batch(*, K: int, block_size: int, mask_id: int, pad_id: int, T_cap: int,
                       qsl_in, verify_tokens, verify_pos, accepted_len, bonus, block_table,
-                      verify_hidden, h_shared, out=None, stream=None) -> dict:
+                      verify_hidden, h_shared, out=None, k_len=None, stream=None) -> dict:
     """P-EAGLE draft-batch construction.  Returns the per-row, per-sequence and hidden
     outputs (see ``include/pspec.h``)."""
     Bn = int(qsl_in.numel()) - 1
@@ -135,14 +138,14 @@ def build_draft_batch(*, K: int, block_size: int, mask_id: int, pad_id: int, T_c
                               row_kind=o["row_kind"], hidden_src=o["hidden_src"],
                               qsl_out=o["qsl_out"], seq_lens_out=o["seq_lens_out"],
                               sample_idx=o["sample_idx"], draft_hidden=o["draft_hidden"],
-                              err=o["err"], stream=stream)
+                              err=o["err"], k_len=k_len, stream=stream)
     return o
 
 
 def step(target_logits: torch.Tensor, draft_tokens: torch.Tensor, build: dict, *,
          draft_logits: torch.Tensor | None = None, uniforms: torch.Tensor | None = None,
          residual_mass: bool = False, workspace: Workspace | None = None, out=None,
-         build_out=None, stream=None) -> tuple:
+         build_out=None, k_len: torch.Tensor | None = None, stream=None) -> tuple:
     """One step: verification (the rejection rule when `uniforms` is given, else greedy)
     and the draft-batch build from its accepted counts and bonus tokens, in one launch when
     the early-exit path takes the verification.  `build` holds the build inputs (K,
@@ -171,10 +174,10 @@ def step(target_logits: torch.Tensor, draft_tokens: torch.Tensor, build: dict, *
                                draft_tokens=draft_tokens, uniforms=uniforms,
                                out_tokens=o["out_tokens"], accepted_len=o["accepted_len"],
                                bonus=o["bonus"], err=o["err"], workspace=ws.tensor, build=bargs,
-                               residual_mass=o.get("residual_mass"), stream=stream)
+                               residual_mass=o.get("residual_mass"), k_len=k_len, stream=stream)
     else:
         _b.pspec_step_greedy(target_logits=target_logits, draft_tokens=draft_tokens,
                              out_tokens=o["out_tokens"], accepted_len=o["accepted_len"],
                              bonus=o["bonus"], err=o["err"], workspace=ws.tensor, build=bargs,
-                             stream=stream)
+                             k_len=k_len, stream=stream)
     return o, bo

@@ -116,6 +116,7 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   L.bonus = a->bonus;
   L.residual_mass = rejection ? a->residual_mass : nullptr;
   L.err = a->err;
+  L.k_len = a->k_len;
   if (fuse) {
     L.fuse_build = 1;
     L.b = fuse->a;
@@ -174,6 +175,7 @@ bool try_queue(const pspec_verify_args* a, bool rejection, void* workspace, size
   L.bonus = a->bonus;
   L.residual_mass = rejection ? a->residual_mass : nullptr;
   L.err = a->err;
+  L.k_len = a->k_len;
   char* ws = static_cast<char*>(workspace);
   L.ctr = z.ctr;
   L.items = z.line0 + kZwItems;
@@ -237,6 +239,7 @@ pspec_status verify_greedy_impl(const pspec_verify_args* a, void* workspace,
   L.bonus = a->bonus;
   L.target_lse = a->target_lse;
   L.err = a->err;
+  L.k_len = a->k_len;
   char* ws = static_cast<char*>(workspace);
   L.cnt = z.line0 + kZwSCnt;
   L.part = ws + p.off_part;
@@ -280,6 +283,7 @@ pspec_status verify_rejection_impl(const pspec_verify_args* a, void* workspace,
   L.q_at_draft = a->q_at_draft;
   L.residual_mass = a->residual_mass;
   L.err = a->err;
+  L.k_len = a->k_len;
   char* ws = static_cast<char*>(workspace);
   L.cnt = z.line0 + kZwSCnt;
   L.cnt2 = z.line0 + kZwSCnt2;
@@ -298,11 +302,13 @@ pspec_status step_impl(const pspec_verify_args* v, const pspec_build_args* b, bo
                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!v || !b) return PSPEC_ERR_INVALID_ARG;
   if (b->B != v->B || b->K != v->K) return PSPEC_ERR_INVALID_ARG;
-  if ((b->accepted_len && b->accepted_len != v->accepted_len) || (b->bonus && b->bonus != v->bonus))
+  if ((b->accepted_len && b->accepted_len != v->accepted_len) || (b->bonus && b->bonus != v->bonus) ||
+      (b->k_len && b->k_len != v->k_len))
     return PSPEC_ERR_INVALID_ARG;
   pspec_build_args bb = *b;
   bb.accepted_len = v->accepted_len;
   bb.bonus = v->bonus;
+  bb.k_len = v->k_len;
   BuildLaunch BL;
   pspec_status st = check_build(&bb, &BL);
   if (st != PSPEC_OK) return st;

@@ -43,7 +43,9 @@ __device__ __forceinline__ int find_seq(const pspec_build_args& a, long long r) 
 __device__ __forceinline__ BuildRow classify(const pspec_build_args& a, long long r) {
   const int i = find_seq(a, r);
   if (i < 0 || i >= a.B) return BuildRow{PSPEC_ROW_PAD, -1, a.pad_id, 0, -1};
-  return build_classify(a, i, r - build_qout(a, i), __ldg(a.accepted_len + i), __ldg(a.bonus + i));
+  int unused = 0;
+  return build_classify(a, i, r - build_qout(a, i), __ldg(a.accepted_len + i),
+                        draft_count(a.k_len, i, a.K, &unused), __ldg(a.bonus + i));
 }
 
 __device__ void meta_role(const pspec_build_args& a, long long t) {
@@ -52,7 +54,8 @@ __device__ void meta_role(const pspec_build_args& a, long long t) {
     build_write_row(a, t, classify(a, t), &eb);
   } else if (t < (long long)a.T_cap + a.B + 1) {  // one sequence (or the end offset)
     const int i = (int)(t - a.T_cap);
-    build_write_seq(a, i, i < a.B ? __ldg(a.accepted_len + i) : 0, &eb);
+    const int Ki = i < a.B ? draft_count(a.k_len, i, a.K, &eb) : a.K;
+    build_write_seq(a, i, i < a.B ? __ldg(a.accepted_len + i) : 0, Ki, &eb);
   }
   set_err(a.err, eb);
 }

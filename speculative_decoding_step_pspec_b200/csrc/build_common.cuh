@@ -8,8 +8,9 @@
 // take PADDING_SLOT_ID = -1 so they cannot write the KV cache.
 //
 // Sequence i's span of the draft batch starts at qsl_out[i] = qsl_in[i] + i(K-1) and holds
-// L_i + K - 1 rows, L_i = qsl_in[i+1] - qsl_in[i] verify rows and c_i = L_i - K + a_i of them
-// surviving:  [c_i - 1 context rows | NTP | K - 1 mask rows | K - a_i rejected rows].
+// L_i + K - 1 rows, L_i = qsl_in[i+1] - qsl_in[i] verify rows of which the last K_i held this
+// step's drafts (K_i = K unless per-sequence counts are given) and c_i = L_i - K_i + a_i
+// survive:  [c_i - 1 context rows | NTP | K - 1 mask rows | K_i - a_i rejected rows].
 // The accepted count and the bonus token are passed as values, so a kernel that has just
 // computed them can build the span without reading them back.
 #pragma once
@@ -31,17 +32,18 @@ __device__ __forceinline__ long long build_qout(const pspec_build_args& a, int i
   return (long long)__ldg(a.qsl_in + i) + (long long)i * (a.K - 1);
 }
 
-// Row j of sequence i's span, for accepted count acc (clamped into [0, K]) and bonus token.
+// Row j of sequence i's span, for the sequence's draft count Ki (its last Ki verify rows
+// held drafts), accepted count acc (clamped into [0, Ki]) and bonus token.
 __device__ __forceinline__ BuildRow build_classify(const pspec_build_args& a, int i, long long j,
-                                                   int acc, int bonus) {
+                                                   int acc, int Ki, int bonus) {
   BuildRow row{PSPEC_ROW_PAD, -1, a.pad_id, 0, -1};
   const int K = a.K;
   const int s = __ldg(a.qsl_in + i);
   const int e = __ldg(a.qsl_in + i + 1);
   const long long L = (long long)e - s;
-  if (s < 0 || e > a.T_in || L < K + 1 || j < 0 || j >= L + K - 1) return row;
-  acc = acc < 0 ? 0 : (acc > K ? K : acc);
-  const int c = (int)L - K + acc;        // surviving verify rows, c >= 1
+  if (s < 0 || e > a.T_in || L < Ki + 1 || j < 0 || j >= L + K - 1) return row;
+  acc = acc < 0 ? 0 : (acc > Ki ? Ki : acc);
+  const int c = (int)L - Ki + acc;       // surviving verify rows, c >= 1
   row.seq = i;
   if (j < c - 1) {                       // context: token j+1 with hidden j
     row.kind = PSPEC_ROW_CTX;
@@ -87,9 +89,10 @@ __device__ __forceinline__ void build_write_row(const pspec_build_args& a, long 
   a.hidden_src[t] = row.src;
 }
 
-// The per-sequence outputs of sequence i < B (acc as given, before clamping: an out-of-range
-// count sets PSPEC_DEVERR_ACCEPT_RANGE), or the end offset and layout check for i == B.
-__device__ __forceinline__ void build_write_seq(const pspec_build_args& a, int i, int acc, int* eb) {
+// The per-sequence outputs of sequence i < B (acc as given, before clamping: a count outside
+// [0, Ki] sets PSPEC_DEVERR_ACCEPT_RANGE), or the end offset and layout check for i == B.
+__device__ __forceinline__ void build_write_seq(const pspec_build_args& a, int i, int acc, int Ki,
+                                                int* eb) {
   const int K = a.K;
   const int s = __ldg(a.qsl_in + i);
   a.qsl_out[i] = (int)build_qout(a, i);
@@ -100,17 +103,17 @@ __device__ __forceinline__ void build_write_seq(const pspec_build_args& a, int i
   const int e = __ldg(a.qsl_in + i + 1);
   const long long L = (long long)e - s;
   if (e < s) *eb |= PSPEC_DEVERR_LAYOUT;
-  if (s < 0 || e > a.T_in || L < K + 1) {
+  if (s < 0 || e > a.T_in || L < Ki + 1) {
     *eb |= PSPEC_DEVERR_LAYOUT;
     a.seq_lens_out[i] = 0;
     for (int k = 0; k < K; ++k) a.sample_idx[(long long)i * K + k] = -1;
     return;
   }
-  if (acc < 0 || acc > K) {
+  if (acc < 0 || acc > Ki) {
     *eb |= PSPEC_DEVERR_ACCEPT_RANGE;
-    acc = acc < 0 ? 0 : K;
+    acc = acc < 0 ? 0 : Ki;
   }
-  const int c = (int)L - K + acc;
+  const int c = (int)L - Ki + acc;
   const int P = __ldg(a.verify_pos + s + c - 1);
   a.seq_lens_out[i] = P + K;
   const int base = (int)build_qout(a, i) + c - 1;

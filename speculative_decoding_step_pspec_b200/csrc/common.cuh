@@ -158,6 +158,18 @@ __device__ __forceinline__ void set_err(int32_t* err, int bits) {
   if (bits) atomicOr(reinterpret_cast<int*>(err), bits);
 }
 
+// Sequence i's own draft count K_i ("dynamic draft length"): k_len[i], or K when k_len is
+// NULL; a value outside [0, K] is clamped into it and sets PSPEC_DEVERR_KLEN_RANGE in *eb.
+__device__ __forceinline__ int draft_count(const int32_t* k_len, int i, int K, int* eb) {
+  if (!k_len) return K;
+  int k = __ldg(k_len + i);
+  if (k < 0 || k > K) {
+    *eb |= PSPEC_DEVERR_KLEN_RANGE;
+    k = k < 0 ? 0 : K;
+  }
+  return k;
+}
+
 // ---------------------------------------------------------------------------------------
 // One segment [lo, hi) of a row, in element order per thread: an unaligned head with
 // scalar loads (up to kVec-1 elements, only when the row does not start on 16 bytes), the

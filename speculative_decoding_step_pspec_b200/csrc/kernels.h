@@ -24,6 +24,7 @@ struct GreedyLaunch {
   int32_t* bonus;
   float* target_lse;     // optional
   int32_t* err;
+  const int32_t* k_len;  // optional per-sequence draft counts
   int* cnt;              // zero area: ticket column (entry i = zcol(cnt, i))
   void* part;            // workspace: GreedyPart [B*(K+1)*S]
 };
@@ -48,6 +49,7 @@ struct RejectionLaunch {
   float* q_at_draft;     // optional
   float* residual_mass;  // optional
   int32_t* err;
+  const int32_t* k_len;  // optional per-sequence draft counts
   int* cnt;              // zero area: sweep ticket column (zcol)
   int* cnt2;             // zero area: resample ticket column (zcol)
   void* part;            // workspace: RejPart [B*(2K+1)*S]
@@ -71,6 +73,7 @@ struct EarlyExitLaunch {
   int32_t* bonus;
   float* residual_mass;  // optional
   int32_t* err;
+  const int32_t* k_len;  // optional per-sequence draft counts
   int fuse_build;        // 1: each cluster also builds its sequence's draft span (below)
   pspec_build_args b;    // draft-batch arguments; accepted_len / bonus = this launch's outputs
   long long row_vecs;    // 16-byte vectors per hidden row of b
@@ -113,6 +116,7 @@ struct QueueLaunch {
   int32_t* bonus;
   float* residual_mass;  // optional
   int32_t* err;
+  const int32_t* k_len;  // optional per-sequence draft counts
   unsigned long long* ctr;  // zero area: queue counters [8]
   int* items;            // zero area: line 0 (item slot s = zitem(items, s)), holding
                          // (i*32 + k) + 1 once published, 0 before

@@ -88,6 +88,7 @@ extern "C" pspec_status pspec_verify_greedy_noalloc(const pspec_verify_args* a,
   L.bonus = a->bonus;
   L.target_lse = a->target_lse;
   L.err = a->err;
+  L.k_len = a->k_len;
   L.cnt = z.line0 + kZwSCnt;
   L.part = ws + p.off_part;
   return launch_greedy(L, stream) == cudaSuccess ? PSPEC_OK : PSPEC_ERR_CUDA;

@@ -40,7 +40,8 @@ struct SeqInfo {
   double mt, st;   // max and sum-exp of target row a_i
   double mq, sq;   // the same for draft row a_i (unused when a_i = K)
   int a;           // accepted drafts a_i
-  int pad[3];
+  int kn;          // the sequence's own draft count K_i
+  int pad[2];
 };
 
 struct VerifyPlan {

@@ -23,17 +23,17 @@ namespace pspec {
 constexpr int kWTile = 256;   // one warp tile: 32 lanes x 8 consecutive elements
 
 // The draw row of sequence i at stop position a: target row a against draft row a (the
-// residual) when a < K, the target row K alone when every draft passed.  Rows are
-// [B, K+1, ld] (target) and [B, K, ld] (draft).
+// residual) when a < K_i, the target row K_i alone when all of the sequence's K_i drafts
+// passed.  Rows are [B, K+1, ld] (target) and [B, K, ld] (draft).
 __device__ __forceinline__ DrawRow make_draw_row(const void* target, const void* draft,
-                                                 long long ld, int K, int elem_bytes, int i,
-                                                 int a, double mt, double st, double mq,
+                                                 long long ld, int K, int Ki, int elem_bytes,
+                                                 int i, int a, double mt, double st, double mq,
                                                  double sq) {
   DrawRow D;
   const char* t = static_cast<const char*>(target);
   const char* q = static_cast<const char*>(draft);
   D.trow = t + ((long long)i * (K + 1) + a) * ld * elem_bytes;
-  D.resid = a < K;
+  D.resid = a < Ki;
   D.qrow = D.resid ? q + ((long long)i * K + a) * ld * elem_bytes : D.trow;
   D.mt = (float)mt;
   D.inv_st = st > 0.0 ? (float)(1.0 / st) : 0.f;

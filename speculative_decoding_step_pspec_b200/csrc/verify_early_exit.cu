@@ -153,20 +153,20 @@ __device__ __forceinline__ void slice_values(const DrawRow& D, const SliceRaw<Ta
 // The rows are exactly those pspec_build_draft_batch writes for a valid offset array; for
 // an invalid one every write stays in bounds and the layout bit is set, as there.
 __device__ __forceinline__ void ee_build_span(const pspec_build_args& b, long long row_vecs, int i,
-                                           int a, int token, bool meta, int g, int G) {
+                                           int a, int Ki, int token, bool meta, int g, int G) {
   const long long q0 = build_qout(b, i), q1 = build_qout(b, i + 1);
   const long long lo = q0 < 0 ? 0 : q0;
   const long long hi = q1 > b.T_cap ? (long long)b.T_cap : q1;
   int eb = 0;
   if (meta) {
     for (long long t = lo + threadIdx.x; t < hi; t += kThreads)
-      build_write_row(b, t, build_classify(b, i, t - q0, a, token), &eb);
-    if (threadIdx.x == 0) build_write_seq(b, i, a, &eb);
+      build_write_row(b, t, build_classify(b, i, t - q0, a, Ki, token), &eb);
+    if (threadIdx.x == 0) build_write_seq(b, i, a, Ki, &eb);
   }
   if (b.draft_hidden) {
     const int warp = threadIdx.x >> 5;
     for (long long t = lo + (long long)g * kWarps + warp; t < hi; t += (long long)G * kWarps)
-      build_copy_hidden(b, row_vecs, t, build_classify(b, i, t - q0, a, token));
+      build_copy_hidden(b, row_vecs, t, build_classify(b, i, t - q0, a, Ki, token));
   }
   if (i == b.B - 1) {                                  // padding rows and the end offset
     const BuildRow pad{PSPEC_ROW_PAD, -1, b.pad_id, 0, -1};
@@ -178,7 +178,7 @@ __device__ __forceinline__ void ee_build_span(const pspec_build_args& b, long lo
       build_write_row(b, t, pad, &eb);
     for (long long t = tail + (long long)g * kThreads + threadIdx.x; t < b.T_cap; t += step)
       build_write_row(b, t, pad, &eb);
-    if (g == 0 && threadIdx.x == 0) build_write_seq(b, b.B, 0, &eb);
+    if (g == 0 && threadIdx.x == 0) build_write_seq(b, b.B, 0, b.K, &eb);
   }
   set_err(b.err, eb);
 }
@@ -193,6 +193,9 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
   const int i = (int)(blockIdx.x / G);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = L.K;
+  int ebk = 0;
+  const int Ki = draft_count(L.k_len, i, K, &ebk);          // the sequence's own drafts
+  if (g == 0 && tid == 0) set_err(L.err, ebk);
 
   __shared__ EEPart part[2];                                 // by position parity
   __shared__ double tot_slice;                               // draw: sum of r over the slice
@@ -212,14 +215,14 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
   const int nvec = n / W;                                   // n is a multiple of 8
 
   int k = 0;
-  for (; k <= K; ++k) {
-    const bool has_q = kRej && k < K;
+  for (; k <= Ki; ++k) {
+    const bool has_q = kRej && k < Ki;
     const elem* trow = static_cast<const elem*>(L.target) + ((long long)i * (K + 1) + k) * L.ld;
     const elem* qrow = has_q ? static_cast<const elem*>(L.draft) + ((long long)i * K + k) * L.ld : trow;
     // the logits at the draft token, needed by every CTA's decision: in flight meanwhile
     float xt_d = 0.f, xq_d = 0.f;
     int d = -1;
-    if (k < K && warp == 0) {
+    if (k < Ki && warp == 0) {
       d = L.draft_tokens[(long long)i * K + k];
       if (kRej && d >= 0 && d < L.V) {
         xt_d = load_scalar(trow, d);
@@ -302,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
         xt_d = __shfl_sync(0xffffffffu, xt_d, 0);
         xq_d = __shfl_sync(0xffffffffu, xq_d, 0);
         bool accept = false;
-        if (k < K && d >= 0 && d < L.V) {
+        if (k < Ki && d >= 0 && d < L.V) {
           const double pp = (Mt != -INFINITY && xt_d != -INFINITY)
                                 ? exp2((double)xt_d * (double)kLog2e - (double)Mt) / st : 0.0;
           const double qq = (Mq != -INFINITY && xq_d != -INFINITY)
@@ -325,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
         b = warp_argmax(b);                 // largest value, lowest index among equals
         const int gk = b.i == kNoIndex ? 0 : b.i;
         d = __shfl_sync(0xffffffffu, d, 0);
-        const bool match = k < K && d >= 0 && d < L.V && d == gk;
+        const bool match = k < Ki && d >= 0 && d < L.V && d == gk;
         if (!match) {
           stop = 1;
           if (g == 0 && lane == 0) { L.bonus[i] = gk; L.out_tokens[(long long)i * (K + 1) + k] = gk; }
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
       if (stop && g == 0) {
         // outputs the two rules share: accepted drafts, the -1 tail, the count, range errors
         int bad = 0;
-        if (lane < K) {
+        if (lane < Ki) {
           const int dj = L.draft_tokens[(long long)i * K + lane];
           bad = dj < 0 || dj >= L.V;
           if (lane < a) L.out_tokens[(long long)i * (K + 1) + lane] = dj;
@@ -356,11 +359,11 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
     const int a = k;
     DrawRow D;
     D.trow = static_cast<const elem*>(L.target) + ((long long)i * (K + 1) + a) * L.ld;
-    D.resid = a < K;
+    D.resid = a < Ki;
     D.qrow = D.resid ? static_cast<const elem*>(L.draft) + ((long long)i * K + a) * L.ld : D.trow;
     D.mt = s_dec[0]; D.inv_st = s_dec[1]; D.mq = s_dec[2]; D.inv_sq = s_dec[3];
     const int ntiles = (n + 255) / 256;
-    const double u = (double)L.uniforms[(long long)i * (K + 1) + K];
+    const double u = (double)L.uniforms[(long long)i * (K + 1) + Ki];
 
     // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8).  Measured on
     // B200 at B=1024: walking the slice last tile first (the part streamed most recently)
@@ -512,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, kEEMinBlocks) ee_kernel(const EarlyE
   cluster.sync();                                            // D: no remote reads after exit
   if constexpr (kFuse) {                                     // the whole step in this launch
     __syncthreads();
-    ee_build_span(L.b, L.row_vecs, i, k, g == meta_g ? s_tok : 0, g == meta_g, g, G);
+    ee_build_span(L.b, L.row_vecs, i, k, Ki, g == meta_g ? s_tok : 0, g == meta_g, g, G);
   }
 }
 

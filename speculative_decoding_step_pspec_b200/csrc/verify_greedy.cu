@@ -109,16 +109,18 @@ greedy_sweep_kernel(const GreedyLaunch L) {
   if (warp != 0) return;
   const int g = lane <= K ? s_g[lane] : 0;           // argmax of row `lane`
   const double lse = (kLse && lane <= K) ? s_lse[lane] : 0.0;
+  int eb = 0;
+  const int Ki = draft_count(L.k_len, i, K, &eb);    // the sequence's own drafts
   int d = -1;
   bool bad = false;
-  if (lane < K) {
+  if (lane < Ki) {
     d = L.draft_tokens[(long long)i * K + lane];
     bad = d < 0 || d >= L.V;
   }
-  unsigned match = __ballot_sync(0xffffffffu, lane < K && !bad && d == g);
+  unsigned match = __ballot_sync(0xffffffffu, lane < Ki && !bad && d == g);
   unsigned anybad = __ballot_sync(0xffffffffu, bad);
   int a = __ffs(~match) - 1;             // first mismatch
-  if (a > K) a = K;
+  if (a > Ki) a = Ki;
   int bonus = __shfl_sync(0xffffffffu, g, a);
   if (lane <= K) {
     L.out_tokens[(long long)i * (K + 1) + lane] = lane < a ? d : (lane == a ? bonus : -1);
@@ -127,7 +129,7 @@ greedy_sweep_kernel(const GreedyLaunch L) {
   if (lane == 0) {
     L.accepted_len[i] = a;
     L.bonus[i] = bonus;
-    if (anybad) set_err(L.err, PSPEC_DEVERR_TOKEN_RANGE);
+    set_err(L.err, eb | (anybad ? PSPEC_DEVERR_TOKEN_RANGE : 0));
     *zcol(L.cnt, i) = 0;                       // ticket back to zero for the next call
   }
 }

@@ -172,12 +172,12 @@ __device__ __forceinline__ void append_item(const QueueLaunch& L, int i, int k) 
 }
 
 // Warp 0, once a sequence stops at a = k: accepted drafts, the -1 tail, the accepted count
-// and the range check of every draft token (as on the other paths).
-__device__ __forceinline__ void write_prefix(const QueueLaunch& L, int i, int a) {
+// and the range check of the sequence's Ki draft tokens (as on the other paths).
+__device__ __forceinline__ void write_prefix(const QueueLaunch& L, int i, int a, int Ki) {
   const int lane = threadIdx.x & 31;
   const int K = L.K;
   int bad = 0;
-  if (lane < K) {
+  if (lane < Ki) {
     const int dj = L.draft_tokens[(long long)i * K + lane];
     bad = dj < 0 || dj >= L.V;
     if (lane < a) L.out_tokens[(long long)i * (K + 1) + lane] = dj;
@@ -190,14 +190,14 @@ __device__ __forceinline__ void write_prefix(const QueueLaunch& L, int i, int a)
 // The end of a draw (all threads): the token from the tile sums ts of row a, then the
 // sequence's outputs; `slot` >= 0 releases the draw slot the units came from.
 template <typename Tag>
-__device__ void finish_draw(const QueueLaunch& L, int i, int a, DrawRow& D, double* ts,
+__device__ void finish_draw(const QueueLaunch& L, int i, int a, int Ki, DrawRow& D, double* ts,
                             QueueShared& sh, int slot) {
   const int K = L.K;
   double Z;
-  const int token = draw_finish<Tag>(D, L.V, L.tiles, (double)L.uniforms[(long long)i * (K + 1) + K],
+  const int token = draw_finish<Tag>(D, L.V, L.tiles, (double)L.uniforms[(long long)i * (K + 1) + Ki],
                                      ts, sh.draw, &Z);
   if ((threadIdx.x >> 5) == 0) {
-    write_prefix(L, i, a);
+    write_prefix(L, i, a, Ki);
     if ((threadIdx.x & 31) == 0) {
       L.out_tokens[(long long)i * (K + 1) + a] = token;
       L.bonus[i] = token;
@@ -217,12 +217,12 @@ template <typename Tag>
 __device__ __noinline__ void draw_whole(const QueueLaunch& L, int i, QueueShared& sh) {
   using elem = typename Tag::elem;
   const SeqInfo si = sh.si;
-  DrawRow D = make_draw_row(L.target, L.draft, L.ld, L.K, (int)sizeof(elem), i, si.a, si.mt, si.st,
-                            si.mq, si.sq);
+  DrawRow D = make_draw_row(L.target, L.draft, L.ld, L.K, si.kn, (int)sizeof(elem), i, si.a, si.mt,
+                            si.st, si.mq, si.sq);
   double* ts = L.tile_sums + (long long)i * L.tiles;
   warp_tile_sums_wide<Tag, PSPEC_QUEUE_DRAW_U>(D, L.V, threadIdx.x >> 5, L.tiles, kWarps, ts);
   __syncthreads();
-  finish_draw<Tag>(L, i, si.a, D, ts, sh, -1);
+  finish_draw<Tag>(L, i, si.a, si.kn, D, ts, sh, -1);
 }
 
 // One draw unit of sequence i (rejection rule): tile sums over its chunk of row a_i; the CTA
@@ -235,8 +235,8 @@ __device__ __noinline__ void draw_unit(const QueueLaunch& L, const Work& w, Queu
   const int c = (int)w.unit;
   const int warp = threadIdx.x >> 5;
   const SeqInfo si = ld_cg(reinterpret_cast<const SeqInfo*>(L.seq) + i);
-  DrawRow D = make_draw_row(L.target, L.draft, L.ld, K, (int)sizeof(elem), i, si.a, si.mt, si.st,
-                            si.mq, si.sq);
+  DrawRow D = make_draw_row(L.target, L.draft, L.ld, K, si.kn, (int)sizeof(elem), i, si.a, si.mt,
+                            si.st, si.mq, si.sq);
   double* ts = L.tile_sums + (long long)i * L.tiles;
   const long long t_lo = (long long)c * L.tiles_per_unit;
   const long long t_hi = min((long long)L.tiles, t_lo + L.tiles_per_unit);
@@ -250,7 +250,7 @@ __device__ __noinline__ void draw_unit(const QueueLaunch& L, const Work& w, Queu
   __syncthreads();
   if (!sh.last) return;
   __threadfence();
-  finish_draw<Tag>(L, i, si.a, D, ts, sh, w.slot);
+  finish_draw<Tag>(L, i, si.a, si.kn, D, ts, sh, w.slot);
 }
 
 // One segment of one row of item (i, k); the CTA completing the item applies the rule.
@@ -264,7 +264,9 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
   const int s = (int)(w.unit % L.S);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int R = kRej ? 2 : 1;
-  const bool live = !(kRej && r == 1 && k == K);      // no draft row at position K
+  int ebk = 0;
+  const int Ki = draft_count(L.k_len, i, K, &ebk);    // the sequence's own drafts
+  const bool live = !(kRej && r == 1 && k == Ki);     // no draft row at position K_i
   const long long lo = (long long)s * L.seg;
   const long long hi = min((long long)L.V, lo + L.seg);
 
@@ -322,7 +324,7 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
   if constexpr (kRej) {
     // warp r merges row r (lane t holds segments t, t+32, ...); warp 2 fetches the draft
     // token, the two logits at it and the uniform meanwhile
-    if (warp < R && (warp == 0 || k < K)) {
+    if (warp < R && (warp == 0 || k < Ki)) {
       const RejPart* pr = part + (long long)warp * L.S;
       RejPart mine = lane < L.S ? ld_cg(pr + lane) : RejPart{-INFINITY, 0.f};
       float m = mine.m;
@@ -343,7 +345,7 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
         sh.M[warp] = m;
         sh.Ssum[warp] = acc;
       }
-    } else if (warp == 2 && lane == 0 && k < K) {
+    } else if (warp == 2 && lane == 0 && k < Ki) {
       const int d = L.draft_tokens[(long long)i * K + k];
       float xt = -INFINITY, xq = -INFINITY;
       if (d >= 0 && d < L.V) {
@@ -357,10 +359,11 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
     }
     __syncthreads();
     if (tid == 0) {
+      if (k == 0) set_err(L.err, ebk);
       const double Mt = sh.M[0], St = sh.Ssum[0];
       bool accept = false;
       double Mq = 0.0, Sq = 1.0;
-      if (k < K) {
+      if (k < Ki) {
         Mq = sh.M[1];
         Sq = sh.Ssum[1];
         const int d = sh.dec_d;
@@ -383,10 +386,11 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
         SeqInfo si;
         si.mt = Mt;
         si.st = St;
-        si.mq = k < K ? Mq : 0.0;
-        si.sq = k < K ? Sq : 1.0;
+        si.mq = k < Ki ? Mq : 0.0;
+        si.sq = k < Ki ? Sq : 1.0;
         si.a = k;
-        si.pad[0] = si.pad[1] = si.pad[2] = 0;
+        si.kn = Ki;
+        si.pad[0] = si.pad[1] = 0;
 #if PSPEC_QUEUE_INLINE_DRAW
         sh.si = si;
 #else
@@ -412,10 +416,11 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
       b = warp_argmax(b);                            // largest value, lowest index among equals
       const int gk = b.i == kNoIndex ? 0 : b.i;      // a row of -inf / NaN only: token 0
       int d = -1;
-      if (lane == 0 && k < K) d = L.draft_tokens[(long long)i * K + k];
+      if (lane == 0 && k < Ki) d = L.draft_tokens[(long long)i * K + k];
       d = __shfl_sync(0xffffffffu, d, 0);
-      const bool match = k < K && d >= 0 && d < L.V && d == gk;
+      const bool match = k < Ki && d >= 0 && d < L.V && d == gk;
       if (lane == 0) {
+        if (k == 0) set_err(L.err, ebk);
         atomicExch(zcol(L.cnt, i), 0);
         if (w.slot >= 0) atomicExch(zitem(L.items, w.slot), 0);
       }
@@ -426,7 +431,7 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
           append_item(L, i, k + 1);
         }
       } else {
-        write_prefix(L, i, k);
+        write_prefix(L, i, k, Ki);
         if (lane == 0) {
           L.out_tokens[(long long)i * (K + 1) + k] = gk;
           L.bonus[i] = gk;

@@ -108,13 +108,15 @@ rej_stats_kernel(const RejectionLaunch L) {
   if (warp != 0) return;
 
   {
+  int eb = 0;
+  const int Ki = draft_count(L.k_len, i, K, &eb);    // the sequence's own drafts
   int d = -1;
   bool bad = false, accept = false;
   double p = 0.0, q = 0.0;
   if (lane < K) {
     d = L.draft_tokens[(long long)i * K + lane];
-    bad = d < 0 || d >= L.V;
-    if (!bad) {
+    bad = lane < Ki && (d < 0 || d >= L.V);
+    if (d >= 0 && d < L.V) {
       const double Mt = s_M[lane], St = s_S[lane];
       const double Mq = s_M[K + 1 + lane], Sq = s_S[K + 1 + lane];
       const float xt = load_scalar(sweep_row<elem>(L, i, lane), d);
@@ -122,13 +124,13 @@ rej_stats_kernel(const RejectionLaunch L) {
       if (Mt != -INFINITY && xt != -INFINITY) p = exp2((double)xt * (double)kLog2e - Mt) / St;
       if (Mq != -INFINITY && xq != -INFINITY) q = exp2((double)xq * (double)kLog2e - Mq) / Sq;
       const double u = (double)L.uniforms[(long long)i * (K + 1) + lane];
-      accept = q > 0.0 ? (u * q < p) : (p > 0.0);
+      accept = lane < Ki && (q > 0.0 ? (u * q < p) : (p > 0.0));
     }
   }
   const unsigned mask = __ballot_sync(0xffffffffu, accept);
   const unsigned anybad = __ballot_sync(0xffffffffu, bad);
   int a = __ffs(~mask) - 1;              // first rejected draft
-  if (a > K) a = K;
+  if (a > Ki) a = Ki;
   if (lane < K) {
     if (L.p_at_draft) L.p_at_draft[(long long)i * K + lane] = (float)p;
     if (L.q_at_draft) L.q_at_draft[(long long)i * K + lane] = (float)q;
@@ -150,13 +152,14 @@ rej_stats_kernel(const RejectionLaunch L) {
     SeqInfo si;
     si.mt = s_M[a];
     si.st = s_S[a];
-    si.mq = a < K ? s_M[K + 1 + a] : 0.0;
-    si.sq = a < K ? s_S[K + 1 + a] : 1.0;
+    si.mq = a < Ki ? s_M[K + 1 + a] : 0.0;
+    si.sq = a < Ki ? s_S[K + 1 + a] : 1.0;
     si.a = a;
-    si.pad[0] = si.pad[1] = si.pad[2] = 0;
+    si.kn = Ki;
+    si.pad[0] = si.pad[1] = 0;
     reinterpret_cast<SeqInfo*>(L.seq)[i] = si;
     L.accepted_len[i] = a;
-    if (anybad) set_err(L.err, PSPEC_DEVERR_TOKEN_RANGE);
+    set_err(L.err, eb | (anybad ? PSPEC_DEVERR_TOKEN_RANGE : 0));
     *zcol(L.cnt, i) = 0;
   }
   }  // warp 0
@@ -175,8 +178,8 @@ rej_draw_kernel(const RejectionLaunch L) {
   __shared__ DrawShared sh;
 
   const SeqInfo si = reinterpret_cast<const SeqInfo*>(L.seq)[i];  // previous launch
-  DrawRow D = make_draw_row(L.target, L.draft, L.ld, K, (int)sizeof(elem), i, si.a, si.mt, si.st,
-                            si.mq, si.sq);
+  DrawRow D = make_draw_row(L.target, L.draft, L.ld, K, si.kn, (int)sizeof(elem), i, si.a, si.mt,
+                            si.st, si.mq, si.sq);
   double* ts = L.tile_sums + (long long)i * L.tiles;
   const long long t_lo = (long long)c * L.tiles_per_chunk;
   const long long t_hi = min((long long)L.tiles, t_lo + L.tiles_per_chunk);
@@ -191,8 +194,8 @@ rej_draw_kernel(const RejectionLaunch L) {
   if (!s_last) return;
   __threadfence();
   double Z;
-  const int token = draw_finish<Tag>(D, L.V, L.tiles, (double)L.uniforms[(long long)i * (K + 1) + K],
-                                     ts, sh, &Z);
+  const int token = draw_finish<Tag>(D, L.V, L.tiles,
+                                     (double)L.uniforms[(long long)i * (K + 1) + si.kn], ts, sh, &Z);
   if (threadIdx.x == 0) {
     L.out_tokens[(long long)i * (K + 1) + si.a] = token;
     L.bonus[i] = token;

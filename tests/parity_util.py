@@ -35,16 +35,18 @@ def np_i32(x: torch.Tensor) -> np.ndarray:
     return x.detach().cpu().numpy().astype(np.int32)
 
 
-def oracle_rejection(target, draft, drafts, u, seqs=None):
+def oracle_rejection(target, draft, drafts, u, seqs=None, k_len=None):
     idx = slice(None) if seqs is None else torch.as_tensor(seqs, device=target.device)
     return oracle.verify_rejection(host_logits(target[idx]), host_logits(draft[idx]),
-                                   np_i32(drafts[idx]), u[idx].cpu().numpy(), threads=THREADS)
+                                   np_i32(drafts[idx]), u[idx].cpu().numpy(), threads=THREADS,
+                                   k_len=None if k_len is None else np_i32(k_len[idx]))
 
 
-def oracle_greedy(target, drafts, seqs=None, want_lse=True):
+def oracle_greedy(target, drafts, seqs=None, want_lse=True, k_len=None):
     idx = slice(None) if seqs is None else torch.as_tensor(seqs, device=target.device)
     return oracle.verify_greedy(host_logits(target[idx]), np_i32(drafts[idx]),
-                                want_lse=want_lse, threads=THREADS)
+                                want_lse=want_lse, threads=THREADS,
+                                k_len=None if k_len is None else np_i32(k_len[idx]))
 
 
 def _rel_ok(a, b, rtol=RTOL, atol=0.0):
@@ -135,7 +137,8 @@ def oracle_build(inp: dict, hidden_init: np.ndarray | None):
         T_cap=inp["T_cap"], qsl_in=np_i32(inp["qsl_in"]), verify_tokens=np_i32(inp["verify_tokens"]),
         verify_pos=np_i32(inp["verify_pos"]), accepted_len=np_i32(inp["accepted_len"]),
         bonus=np_i32(inp["bonus"]), block_table=np_i32(inp["block_table"]),
-        verify_hidden=vh_np, h_shared=hs_np, draft_hidden_init=hidden_init)
+        verify_hidden=vh_np, h_shared=hs_np, draft_hidden_init=hidden_init,
+        k_len=None if inp.get("k_len") is None else np_i32(inp["k_len"]))
 
 
 def hidden_sentinel(T_cap, H, dtype, device):

@@ -127,6 +127,7 @@ def _bargs(**kw):
     a.mask_id, a.pad_id, a.T_in, a.T_cap = 1, 2, 16, 24
     for f, _ in b.pspec_build_args._fields_[10:]:
         setattr(a, f, FAKE)
+    a.k_len = None                       # optional: per-sequence draft counts
     for k, v in kw.items():
         setattr(a, k, v)
     return a
@@ -175,6 +176,7 @@ def test_segment_override_changes_workspace():
     ("foreign_accepted_len", {}, {"accepted_len": FAKE + 256}, (FAKE, 1 << 30),
      b.PSPEC_ERR_INVALID_ARG),
     ("foreign_bonus", {}, {"bonus": FAKE + 256}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
+    ("foreign_k_len", {}, {"k_len": FAKE + 512}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
     ("bad_build", {}, {"T_cap": 3}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
     ("bad_verify", {"ld": 10}, {}, (FAKE, 1 << 30), b.PSPEC_ERR_INVALID_ARG),
     ("short_workspace", {}, {}, (FAKE, 256), b.PSPEC_ERR_WORKSPACE),

@@ -423,7 +423,7 @@ def _build_and_compare(inp, check_hidden=True):
         T_cap=inp["T_cap"], qsl_in=inp["qsl_in"], verify_tokens=inp["verify_tokens"],
         verify_pos=inp["verify_pos"], accepted_len=inp["accepted_len"], bonus=inp["bonus"],
         block_table=inp["block_table"], verify_hidden=inp["verify_hidden"],
-        h_shared=inp["h_shared"], out=out)
+        h_shared=inp["h_shared"], out=out, k_len=inp.get("k_len"))
     torch.cuda.synchronize()
     o = U.oracle_build(inp, init)
     U.compare_build(g, o, check_hidden)
@@ -434,7 +434,8 @@ def _torchify(case, dtype=torch.bfloat16):
     def i32(x):
         return torch.as_tensor(np.asarray(x, np.int32), device=DEV)
     B = len(case["qsl_in"]) - 1
-    return dict(B=B, K=case["K"], H=case["verify_hidden"].shape[1], block_size=case["block_size"],
+    extra = {} if case.get("k_len") is None else {"k_len": i32(case["k_len"])}
+    return dict(**extra, B=B, K=case["K"], H=case["verify_hidden"].shape[1], block_size=case["block_size"],
                 mask_id=case["mask_id"], pad_id=case["pad_id"], T_cap=case["T_cap"],
                 qsl_in=i32(case["qsl_in"]), verify_tokens=i32(case["verify_tokens"]),
                 verify_pos=i32(case["verify_pos"]), accepted_len=i32(case["accepted_len"]),
@@ -773,3 +774,136 @@ def test_step_cuda_graph_replay(path):
                       "qsl_out", "seq_lens_out", "sample_idx"):
                 assert torch.equal(bout[k], ref_b[k]), (rep, k)
     del g
+
+
+# --------------------------------------------------------------------------- per-sequence K_i
+def _k_len_case(B, K, V, seed, with_bad=False):
+    w = I.Workload("t", B, K, V, 64, 16, torch.bfloat16, seed=seed, sigma_t=2.0, sigma_d=0.5)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    g = np.random.default_rng(seed)
+    kl = g.integers(0, K + 1, size=B).astype(np.int32)
+    kl[:4] = [0, K, 1, 0]
+    if with_bad:
+        kl[4], kl[5] = -3, K + 2                 # clamped to 0 and K, error bit set
+    klt = torch.as_tensor(kl, device=DEV)
+    kc = np.clip(kl, 0, K)
+    for t in (sampled, greedy):                  # unused draft slots hold -1
+        m = torch.as_tensor(np.arange(K)[None, :] >= kc[:, None], device=DEV)
+        t.masked_fill_(m, -1)
+    return w, target, draft, sampled, greedy, u, klt
+
+
+@pytest.mark.parametrize("path", [1, 2, 3])
+def test_k_len_verify_every_path(path):
+    """Per-sequence draft counts on every path against the oracle (reading R14): counts
+    0..K, -1 in the unused draft slots (no range error), out-of-range counts clamped with
+    PSPEC_DEVERR_KLEN_RANGE."""
+    w, target, draft, sampled, greedy, u, klt = _k_len_case(96, 7, 20000, 61, with_bad=True)
+    with verify_path(path):
+        g = ps.verify_greedy(target, greedy, k_len=klt)
+        r = ps.verify_rejection(target, draft, sampled, u, k_len=klt, residual_mass=True)
+    torch.cuda.synchronize()
+    assert g["err"].item() == ps._binding.PSPEC_DEVERR_KLEN_RANGE
+    assert r["err"].item() == ps._binding.PSPEC_DEVERR_KLEN_RANGE
+    og = U.oracle_greedy(target, greedy, want_lse=False, k_len=klt)
+    orj = U.oracle_rejection(target, draft, sampled, u, k_len=klt)
+    assert og["err"] == 0x20 and orj["err"] == 0x20
+    g["err"].zero_()
+    r["err"].zero_()
+    U.compare_greedy(g, og)
+    U.compare_rejection(r, orj)
+    kc = klt.clamp(0, 7)
+    assert (g["accepted_len"] <= kc).all() and (r["accepted_len"] <= kc).all()
+
+
+def test_k_len_all_k_equals_fixed_k():
+    """k_len = K for every sequence gives the fixed-K outputs bit for bit."""
+    w = I.scaled(I.C64, B=70, V=30000)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    kl = torch.full((w.B,), w.K, dtype=torch.int32, device=DEV)
+    for path in (1, 2, 3):
+        with verify_path(path):
+            a = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
+            b = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, k_len=kl)
+            c = ps.verify_greedy(target, greedy)
+            d = ps.verify_greedy(target, greedy, k_len=kl)
+        for k in a:
+            assert torch.equal(a[k], b[k]), (path, k)
+        for k in c:
+            assert torch.equal(c[k], d[k]), (path, k)
+
+
+def test_k_len_b1024_sampled():
+    w = I.B1024
+    target, draft = I.logits(w, DEV)
+    sampled, _ = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    kl = torch.as_tensor(np.random.default_rng(3).integers(0, w.K + 1, size=w.B).astype(np.int32),
+                         device=DEV)
+    r = ps.verify_rejection(target, draft, sampled, u, k_len=kl)
+    seqs = _sample(w.B, 32, 13)
+    U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u, seqs, k_len=kl), seqs)
+
+
+@pytest.mark.parametrize("K,L_extra", [(1, 0), (3, 2), (7, 0), (7, 4)])
+def test_k_len_build(K, L_extra):
+    """The draft batch with per-sequence K_i (spans as short as K_i + 1 rows) against the
+    oracle, and the whole step (fused and not) equal to verify + build."""
+    from tests.oracle_pins import random_build_case
+    rng = np.random.default_rng(700 + K)
+    kl = rng.integers(0, K + 1, size=37)
+    case = random_build_case(rng, B=37, K=K, H=32, bs=4, L_extra=L_extra, k_len=kl)
+    binp = _torchify(case)
+    _build_and_compare(binp)
+    g = torch.Generator(device=DEV).manual_seed(K)
+    V = 3000
+    target = (torch.randn((37, K + 1, V), generator=g, device=DEV) * 2).to(torch.bfloat16)
+    draft = (target[:, :K].float() + torch.randn((37, K, V), generator=g, device=DEV) * 0.5).to(torch.bfloat16)
+    d = torch.argmax(draft.float(), dim=2).to(torch.int32)
+    u = torch.rand((37, K + 1), generator=g, device=DEV)
+    klt = binp["k_len"]
+    for path, fused in ((2, True), (1, False), (3, False)):
+        for uu in (u, None):
+            v1, b1 = _step_check_k(target, draft, d, uu, binp, path, fused, klt)
+            assert b1["err"].item() == 0
+
+
+def _step_check_k(target, draft, drafts, u, binp, path, expect_fused, klt):
+    rej = u is not None
+    H, dt = binp["verify_hidden"].shape[1], binp["verify_hidden"].dtype
+
+    def bout():
+        o = ps.api.build_outputs(binp["B"], binp["K"], H, binp["T_cap"], dt, DEV)
+        o["draft_hidden"] = U.hidden_sentinel(binp["T_cap"], H, dt, DEV)
+        return o
+    with verify_path(path):
+        if rej:
+            v1 = ps.verify_rejection(target, draft, drafts, u, residual_mass=True, k_len=klt)
+        else:
+            v1 = ps.verify_greedy(target, drafts, k_len=klt)
+        n_verify = ps.pspec_last_launches()
+        b1 = ps.build_draft_batch(
+            K=binp["K"], block_size=binp["block_size"], mask_id=binp["mask_id"],
+            pad_id=binp["pad_id"], T_cap=binp["T_cap"], qsl_in=binp["qsl_in"],
+            verify_tokens=binp["verify_tokens"], verify_pos=binp["verify_pos"],
+            accepted_len=v1["accepted_len"], bonus=v1["bonus"], block_table=binp["block_table"],
+            verify_hidden=binp["verify_hidden"], h_shared=binp["h_shared"], out=bout(), k_len=klt)
+        v2, b2 = ps.step(target, drafts, binp, draft_logits=draft if rej else None, uniforms=u,
+                         residual_mass=rej, build_out=bout(), k_len=klt)
+        n_step = ps.pspec_last_launches()
+    torch.cuda.synchronize()
+    for k in v1:
+        assert torch.equal(v1[k], v2[k]), k
+    for k in b1:
+        assert torch.equal(b1[k], b2[k]), k
+    assert n_step == (1 if expect_fused else n_verify + 1)
+    # the build against the oracle with the verify's own counts and tokens
+    inp = dict(binp, accepted_len=v1["accepted_len"], bonus=v1["bonus"])
+    dh = U.hidden_sentinel(binp["T_cap"], H, dt, DEV)
+    init = dh.view(torch.int16).cpu().numpy() if dt == torch.bfloat16 else dh.cpu().numpy()
+    U.compare_build(b2, U.oracle_build(inp, init))
+    return v2, b2
