@@ -377,7 +377,10 @@ def run_pspec(args, rank, world, local_rank):
     whole = fused or graph is not None                     # one timed unit: the whole step
     dom_bytes = vbytes + bbytes if whole else vbytes       # a fused launch also builds
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    traffic = profiled_traffic(dom_kernel, args.workload, src_hash)
+    # both rules share the early-exit and work-queue kernels: their profiles are per rule
+    prof_key = dom_kernel + ("_greedy" if not rej and dom_kernel in ("ee_kernel", "queue_kernel") else "")
+    # a whole-step timing (fused launch, graph replay) is not one kernel's: no kernel traffic
+    traffic = None if whole else profiled_traffic(prof_key, args.workload, src_hash)
 
     line = {
         "metric": METRIC, "value": round(aggregate_value(K, world, elapsed_ms), 3), "unit": UNIT,
