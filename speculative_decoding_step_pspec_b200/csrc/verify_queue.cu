@@ -189,12 +189,12 @@ __device__ __forceinline__ void write_prefix(const QueueLaunch& L, int i, int a,
 
 // The end of a draw (all threads): the token from the tile sums ts of row a, then the
 // sequence's outputs; `slot` >= 0 releases the draw slot the units came from.
-template <typename Tag>
+template <typename Tag, typename Bar>
 __device__ void finish_draw(const QueueLaunch& L, int i, int a, int Ki, DrawRow& D, double* ts,
                             QueueShared& sh, int slot) {
   const int K = L.K;
   double Z;
-  const int token = draw_finish<Tag>(D, L.V, L.tiles, (double)L.uniforms[(long long)i * (K + 1) + Ki],
+  const int token = draw_finish<Tag, Bar>(D, L.V, L.tiles, (double)L.uniforms[(long long)i * (K + 1) + Ki],
                                      ts, sh.draw, &Z);
   if ((threadIdx.x >> 5) == 0) {
     write_prefix(L, i, a, Ki);
@@ -213,7 +213,7 @@ __device__ void finish_draw(const QueueLaunch& L, int i, int a, int Ki, DrawRow&
 }
 
 // The whole draw of sequence i by this CTA (the one that just decided it), statistics in sh.si.
-template <typename Tag>
+template <typename Tag, typename Bar>
 __device__ __noinline__ void draw_whole(const QueueLaunch& L, int i, QueueShared& sh) {
   using elem = typename Tag::elem;
   const SeqInfo si = sh.si;
@@ -221,13 +221,13 @@ __device__ __noinline__ void draw_whole(const QueueLaunch& L, int i, QueueShared
                             si.st, si.mq, si.sq);
   double* ts = L.tile_sums + (long long)i * L.tiles;
   warp_tile_sums_wide<Tag, PSPEC_QUEUE_DRAW_U>(D, L.V, threadIdx.x >> 5, L.tiles, kWarps, ts);
-  __syncthreads();
-  finish_draw<Tag>(L, i, si.a, si.kn, D, ts, sh, -1);
+  Bar::sync();
+  finish_draw<Tag, Bar>(L, i, si.a, si.kn, D, ts, sh, -1);
 }
 
 // One draw unit of sequence i (rejection rule): tile sums over its chunk of row a_i; the CTA
 // finishing the last unit draws the token and writes the sequence's outputs.
-template <typename Tag>
+template <typename Tag, typename Bar>
 __device__ __noinline__ void draw_unit(const QueueLaunch& L, const Work& w, QueueShared& sh) {
   using elem = typename Tag::elem;
   const int K = L.K;
@@ -241,20 +241,20 @@ __device__ __noinline__ void draw_unit(const QueueLaunch& L, const Work& w, Queu
   const long long t_lo = (long long)c * L.tiles_per_unit;
   const long long t_hi = min((long long)L.tiles, t_lo + L.tiles_per_unit);
   warp_tile_sums<Tag>(D, L.V, t_lo + warp, t_hi, kWarps, ts);
-  __syncthreads();
+  Bar::sync();
   if (threadIdx.x == 0) {
     __threadfence();
     const int t = atomicAdd(zcol(L.cnt2, i), 1);
     sh.last = (t == L.C - 1);
   }
-  __syncthreads();
+  Bar::sync();
   if (!sh.last) return;
   __threadfence();
-  finish_draw<Tag>(L, i, si.a, si.kn, D, ts, sh, w.slot);
+  finish_draw<Tag, Bar>(L, i, si.a, si.kn, D, ts, sh, w.slot);
 }
 
 // One segment of one row of item (i, k); the CTA completing the item applies the rule.
-template <typename Tag, bool kRej>
+template <typename Tag, bool kRej, typename Bar>
 __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh) {
   using elem = typename Tag::elem;
   const int K = L.K;
@@ -297,7 +297,7 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
     if constexpr (kRej) sh.ms[warp] = ms;
     else sh.vi[warp] = best;
   }
-  __syncthreads();
+  Bar::sync();
   if (warp == 0) {
     if constexpr (kRej) {
       ms = lane < kWarps ? sh.ms[lane] : MS{-INFINITY, 0.f};
@@ -315,7 +315,7 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
       sh.last = (t == R * L.S - 1);
     }
   }
-  __syncthreads();
+  Bar::sync();
   if (!sh.last) return;
   __threadfence();
 
@@ -357,7 +357,7 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
       sh.dec_x[1] = xq;
       sh.dec_u = L.uniforms[(long long)i * (K + 1) + k];
     }
-    __syncthreads();
+    Bar::sync();
     if (tid == 0) {
       if (k == 0) set_err(L.err, ebk);
       const double Mt = sh.M[0], St = sh.Ssum[0];
@@ -403,8 +403,8 @@ __device__ void stream_unit(const QueueLaunch& L, const Work& w, QueueShared& sh
       sh.draw_now = !accept;
     }
 #if PSPEC_QUEUE_INLINE_DRAW
-    __syncthreads();
-    if (sh.draw_now) draw_whole<Tag>(L, i, sh);       // this CTA draws while the rows are fresh
+    Bar::sync();
+    if (sh.draw_now) draw_whole<Tag, Bar>(L, i, sh);       // this CTA draws while the rows are fresh
 #endif
   } else {
     if (warp == 0) {
@@ -460,10 +460,10 @@ __global__ void __launch_bounds__(kThreads, PSPEC_QUEUE_MIN_BLOCKS) queue_kernel
     if (threadIdx.x == 0 && held < 0 && (!kRej || w.kind == kWorkStream))
       held = (long long)atomicAdd(L.ctr + kQHeadS, 1ull);   // claim ahead: overlaps the unit
     if constexpr (kRej) {
-      if (w.kind == kWorkDraw) draw_unit<Tag>(L, w, sh);
-      else stream_unit<Tag, kRej>(L, w, sh);
+      if (w.kind == kWorkDraw) draw_unit<Tag, CtaBarrier>(L, w, sh);
+      else stream_unit<Tag, kRej, CtaBarrier>(L, w, sh);
     } else {
-      stream_unit<Tag, kRej>(L, w, sh);
+      stream_unit<Tag, kRej, CtaBarrier>(L, w, sh);
     }
     __syncthreads();                                 // sh reused by the next unit
   }
@@ -490,6 +490,7 @@ __global__ void __launch_bounds__(kThreads, PSPEC_QUEUE_MIN_BLOCKS) queue_kernel
 template <typename Tag, bool kRej>
 cudaError_t launch_q(const QueueLaunch& L, cudaStream_t stream) {
   auto kern = queue_kernel<Tag, kRej>;
+  const int threads = kThreads;
   static int per_sm[8] = {0};                        // per device
   static int sms[8] = {0};
   int dev = 0;
@@ -497,7 +498,7 @@ cudaError_t launch_q(const QueueLaunch& L, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 8 || per_sm[dev] == 0) {
     int nb = 0, n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, 0);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, threads, 0);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
@@ -509,7 +510,7 @@ cudaError_t launch_q(const QueueLaunch& L, cudaStream_t stream) {
   long long grid = (long long)per_sm[dev] * sms[dev];
   if (grid > units) grid = units;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, kThreads, 0, stream>>>(L);
+  kern<<<(unsigned)grid, threads, 0, stream>>>(L);
   return cudaGetLastError();
 }
 
