@@ -59,6 +59,10 @@ def parse_args():
                    help="time verify and build as two calls even where one fused launch can do both")
     p.add_argument("--build-only", action="store_true",
                    help="time the draft-batch construction alone (profiling aid: no logits)")
+    p.add_argument("--depth-sweep", action="store_true",
+                   help="the depth sweep: B=256, V=128256, K in 1,3,5,7,8, draft noise 0.3,0.7,1.5 "
+                        "(one JSON line with a point per (K, sigma))")
+    p.add_argument("--depth-k", default="", help="comma-separated K values of the depth sweep (default all)")
     p.add_argument("--sample-only", choices=["sample", "argmax"], default=None,
                    help="time draft-token sampling alone over the workload's drafter rows")
     return p.parse_args()
@@ -658,6 +662,66 @@ def run_sample_only(args, local_rank):
         "gpu_launches": args.steps, "clocks": sampler.summary()}), flush=True)
 
 
+def run_depth_sweep(args, local_rank):
+    """Step time, achieved GB/s and the accepted-length histogram per (K, sigma) of the
+    depth-sweep workload (B=256, V=128256, H=4096), rejection rule, automatic path."""
+    import numpy as np
+    import torch
+
+    import speculative_decoding_step_pspec_b200 as ps
+    from speculative_decoding_step_pspec_b200 import inputs as I
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3}[args.path])
+    ps.pspec_set_cluster_size(args.cluster)
+    hbm, _ = peaks()
+    points = []
+    ks = [int(x) for x in args.depth_k.split(",")] if args.depth_k else I.DEPTH_K
+    for K in ks:
+        for sigma in I.DEPTH_SIGMA:
+            w = I.depth(K, sigma)
+            target, draft = I.logits(w, dev)
+            sampled, _ = I.draft_tokens(w, draft)
+            u = I.uniforms(w, dev)
+            bi = I.build_inputs(w, dev, drafts=sampled)
+            ws = ps.Workspace(w.B, w.K, w.V, True, dev)
+            vout = ps.api.verify_outputs(w.B, w.K, dev, False, True)
+            bout = ps.api.build_outputs(w.B, w.K, w.H, bi["T_cap"], bi["verify_hidden"].dtype, dev)
+
+            def step():
+                ps.step(target, sampled, bi, draft_logits=draft, uniforms=u, workspace=ws,
+                        out=vout, build_out=bout)
+            for _ in range(max(3, args.warmup)):
+                step()
+            launches = ps.pspec_last_launches()
+            path = ps.pspec_last_verify_path()
+            torch.cuda.synchronize()
+            n = max(20, args.steps // 5)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(n):
+                step()
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / n
+            assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
+            acc = vout["accepted_len"].cpu().numpy()
+            early = path in (2, 3)
+            vbytes, bbytes = algorithmic_bytes(w, "rejection", acc, early)
+            points.append({"K": K, "sigma": sigma, "ms_per_step": round(ms, 4),
+                           "step_per_s": round(1e3 / ms, 1),
+                           "achieved_gbs": round((vbytes + bbytes) / (ms * 1e-3) / 1e9, 1),
+                           "frac_of_peak": round((vbytes + bbytes) / (ms * 1e-3) / 1e9 / hbm, 4),
+                           "algorithmic_bytes": int(vbytes + bbytes), "launches": launches,
+                           "acceptance_rate": round(float(acc.sum()) / float(np.minimum(acc + 1, K).sum()), 4),
+                           "histogram": np.bincount(acc, minlength=K + 1).tolist()})
+            del target, draft, bi, ws, vout, bout
+            torch.cuda.empty_cache()
+    print(json.dumps({"metric": "depth sweep: step time, GB/s and accepted-length histogram per (K, sigma)",
+                      "workload": "depth: B=256, V=128256, H=4096, bf16, rejection rule, automatic path",
+                      "peak_gbs": hbm, "points": points}), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, rank):
     """The CPU oracle as the reference arm: each step verifies a rotating bounded sample of
@@ -739,6 +803,8 @@ def main():
             run_build_only(args, local_rank)
         elif args.sample_only:
             run_sample_only(args, local_rank)
+        elif args.depth_sweep:
+            run_depth_sweep(args, local_rank)
         else:
             run_pspec(args, rank, world, local_rank)
     finally:

@@ -358,8 +358,8 @@ PSPEC_API int pspec_last_launches(void);
 PSPEC_API void pspec_set_verify_path(int path);
 
 /* Tuning: CTAs per thread-block cluster on the early-exit path (2, 4, 8 or 16; each CTA
-   streams a 1/G slice of a row); 0 restores the automatic choice (4, or 16 when a slice
-   of 4 would exceed 262144 elements).  Process-wide. */
+   streams a 1/G slice of a row); 0 restores the automatic choice (16 below 128 sequences,
+   else 4, or 16 when a slice of 4 would exceed 262144 elements).  Process-wide. */
 PSPEC_API void pspec_set_cluster_size(int G);
 
 /* Tuning: fusion of the two halves of pspec_step_* into one launch (early-exit path only):

@@ -94,7 +94,8 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   if (g_verify_path == 1) return false;
   if (g_verify_path == 0 && (a->B < kEarlyExitMinB || diagnostics)) return false;
   const int eb = (int)elem_bytes(a->dtype);
-  EarlyExitPlan ep = make_early_exit_plan(a->V, g_cluster ? g_cluster : kEarlyExitCluster);
+  const int G_auto = a->B < kEarlyExitSmallB ? 16 : kEarlyExitCluster;
+  EarlyExitPlan ep = make_early_exit_plan(a->V, g_cluster ? g_cluster : G_auto);
   if (!ep.ok && g_cluster == 0) ep = make_early_exit_plan(a->V, 16);
   const bool aligned = aligned16(a->target_logits) && (!rejection || aligned16(a->draft_logits)) &&
                        (a->ld * eb) % 16 == 0;

@@ -12,13 +12,26 @@ namespace pspec {
 
 constexpr int kNumSMs = 148;             // B200
 constexpr int kDrawTile = 256;           // draw tile: one warp, 32 lanes x 8 elements
-constexpr long long kSegMin = 2048;      // one 16-byte vector per thread (bf16)
+// Segments of at least 8192 elements (four 16-byte vectors per thread for bf16): at small
+// batches the sweep then launches a few CTAs per SM instead of many one-vector CTAs
+// (measured on B200, one sequence of V=201088: 2.5 CTAs/SM of 16 KB each beat 10 of 4 KB).
+constexpr long long kSegMin = 8192;
 constexpr long long kSegMax = 65536;     // bounds the tail of the last wave
-constexpr int kTargetCtas = kNumSMs * 32;
-constexpr int kResampleTargetCtas = kNumSMs * 8;
+#ifndef PSPEC_TARGET_CTAS_PER_SM
+#define PSPEC_TARGET_CTAS_PER_SM 32
+#endif
+#ifndef PSPEC_DRAW_CTAS_PER_SM
+#define PSPEC_DRAW_CTAS_PER_SM 1      // separate draw launch: about one CTA per SM, at least
+#endif                                // kDrawTilesPerCta tiles per CTA (batches of one: 6)
+constexpr int kTargetCtas = kNumSMs * PSPEC_TARGET_CTAS_PER_SM;
+constexpr int kResampleTargetCtas = kNumSMs * PSPEC_DRAW_CTAS_PER_SM;
 constexpr int kDrawTilesPerCta = 64;     // separate draw launch: at most 8 tiles per warp
 constexpr int kEarlyExitMinB = 64;       // automatic path: early exit from this many sequences
 constexpr int kEarlyExitCluster = 4;     // CTAs per sequence on the early-exit path
+// Below this many sequences the automatic cluster is 16 CTAs: with 4, a batch of 64 fills
+// only 256 CTA slots of ~900 (measured on B200, c64: 0.100 ms with 16 vs 0.140 ms with 4;
+// at 256 sequences 4 and 8 are within 5 % either way, at 1024 sequences 4 is best).
+constexpr int kEarlyExitSmallB = 128;
 constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this many sequences
 
 // Per-(row, segment) partial of the greedy sweep.

@@ -907,3 +907,29 @@ def _step_check_k(target, draft, drafts, u, binp, path, expect_fused, klt):
     init = dh.view(torch.int16).cpu().numpy() if dt == torch.bfloat16 else dh.cpu().numpy()
     U.compare_build(b2, U.oracle_build(inp, init))
     return v2, b2
+
+
+@pytest.mark.parametrize("G", [2, 4, 8, 16])
+def test_early_exit_every_cluster_size(G):
+    """The early-exit kernel with each cluster size (the automatic choice is 16 below 128
+    sequences, else 4) against the oracle, unfused and with the step fused, K_i included."""
+    w = I.scaled(I.C64, B=40, V=40000, H=64)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    kl = torch.as_tensor(np.random.default_rng(G).integers(0, w.K + 1, size=w.B).astype(np.int32),
+                         device=DEV)
+    binp = I.build_inputs(w, DEV, drafts=sampled)
+    try:
+        ps.pspec_set_cluster_size(G)
+        with verify_path(2):
+            g = ps.verify_greedy(target, greedy)
+            r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
+            rk = ps.verify_rejection(target, draft, sampled, u, k_len=kl)
+        U.compare_greedy(g, U.oracle_greedy(target, greedy, want_lse=False))
+        U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u))
+        U.compare_rejection(rk, U.oracle_rejection(target, draft, sampled, u, k_len=kl))
+        _step_check(target, draft, sampled, u, binp, 2, True)
+        _step_check(target, draft, greedy, None, binp, 2, True)
+    finally:
+        ps.pspec_set_cluster_size(0)
