@@ -45,6 +45,10 @@ def parse_args():
     p.add_argument("--path", choices=["auto", "sweep", "early", "queue"], default="auto",
                    help="verify path: automatic selection, full sweep, early exit, or work queue")
     p.add_argument("--cluster", type=int, default=0, help="early-exit cluster size (0 auto)")
+    p.add_argument("--ee-stream", choices=["auto", "registers", "ring"], default="auto",
+                   help="early-exit row streaming: registers or per-warp shared-memory rings")
+    p.add_argument("--tail", type=int, default=0,
+                   help="early exit: sequences for the 8-CTA tail launch (0 auto, -1 never)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -251,6 +255,8 @@ def run_pspec(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3}[args.path])
     ps.pspec_set_cluster_size(args.cluster)
+    ps.pspec_set_ee_stream({"auto": 0, "registers": 1, "ring": 2}[args.ee_stream])
+    ps.pspec_set_tail_split(args.tail)
     w, d = make_workload(args.workload, dev, rank, args.batch)
     rej = args.mode == "rejection"
     ws = ps.Workspace(w.B, w.K, w.V, rej, dev)
@@ -280,11 +286,14 @@ def run_pspec(args, rank, world, local_rank):
     # one call of the public step API: where a single launch verifies and builds, that is
     # the step that is timed; otherwise the two calls are timed apart
     fused_step()
-    fused = (not args.separate) and ps.pspec_last_launches() == 1
+    n_step = ps.pspec_last_launches()
+    verify()
+    n_verify = ps.pspec_last_launches()
+    fused = (not args.separate) and n_step == n_verify
     for _ in range(max(3, args.warmup)):
         if fused:
             fused_step()
-            lv, lb = 1, 0
+            lv, lb = n_step, 0
         else:
             verify()
             lv = ps.pspec_last_launches()
@@ -346,7 +355,8 @@ def run_pspec(args, rank, world, local_rank):
 
     verify_ms = [e[0].elapsed_time(e[2]) for e in ev]
     build_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    split = rej and not fused and graph is None             # library-recorded split event
+    # library-recorded split event between the sweep's statistics and draw launches
+    split = rej and not fused and graph is None and path == 1
     stats_ms = [e[0].elapsed_time(e[1]) for e in ev] if split else verify_ms
     draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if split else None
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
@@ -407,7 +417,10 @@ def run_pspec(args, rank, world, local_rank):
         "algorithmic_bytes_per_step": {"verify": int(vbytes), "build": int(bbytes),
                                        "verify_full_sweep": int(full_vbytes)},
         "kernels_ms": {
-            dom_kernel + (" (verify + build, one launch)" if fused else "")
+            dom_kernel + (" (verify + build, one launch)" if fused and lv == 1 else "")
+            + (" (verify + build, two launches)" if fused and lv == 2 else "")
+            + (" (two launches: 4-CTA clusters, then 8-CTA clusters for the last sequences)"
+               if early and lv == 2 and not fused else "")
             + (" (CUDA graph replay of the step)" if graph is not None else ""): round(dom_ms, 5),
             **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if draw_ms else {}),
             **({} if whole else {"build_kernel": round(statistics.mean(build_ms), 5)}),
@@ -416,6 +429,7 @@ def run_pspec(args, rank, world, local_rank):
         "roofline": {
             "kernel": dom_kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
             "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic,
+            "launches": lv,
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
             "algorithmic_bytes_per_launch": int(dom_bytes),
         },
@@ -674,6 +688,8 @@ def run_depth_sweep(args, local_rank):
     torch.cuda.set_device(dev)
     ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3}[args.path])
     ps.pspec_set_cluster_size(args.cluster)
+    ps.pspec_set_ee_stream({"auto": 0, "registers": 1, "ring": 2}[args.ee_stream])
+    ps.pspec_set_tail_split(args.tail)
     hbm, _ = peaks()
     points = []
     ks = [int(x) for x in args.depth_k.split(",")] if args.depth_k else I.DEPTH_K

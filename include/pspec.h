@@ -362,6 +362,27 @@ PSPEC_API void pspec_set_verify_path(int path);
    else 4, or 16 when a slice of 4 would exceed 262144 elements).  Process-wide. */
 PSPEC_API void pspec_set_cluster_size(int G);
 
+/* Tuning: how the early-exit path streams logit rows.  0 automatic (= 1), 1 through
+   registers (16-byte loads, six CTAs per SM for the rejection rule), 2 through shared
+   memory: each warp owns a ring of stages filled by bulk asynchronous copies
+   (cp.async.bulk, completion counted on an mbarrier), so the bytes in flight do not depend
+   on the register budget; three CTAs per SM fit, and with fewer sequences in flight the
+   draw's re-read of its rows stays in L2.  On B200 mode 2 measured slower than mode 1 at
+   every batch size tried (fewer warps leave each position latency-bound).  Waits on the
+   stages are bounded: when one runs out, PSPEC_DEVERR_TIMEOUT is set and the outputs are
+   undefined.  Outputs are otherwise the same in both modes.  Process-wide. */
+PSPEC_API void pspec_set_ee_stream(int mode);
+
+/* Tuning: on the early-exit path with 4-CTA clusters, the last n sequences of the batch
+   are verified by a second launch of 8-CTA clusters, queued with programmatic dependent
+   launch so that it starts while the first launch drains (the CTAs of the first launch
+   release it when they are placed; CTA 0 of the second waits for the first grid before it
+   ends, so work queued later on the stream sees all outputs).  0 automatic (rejection
+   rule: min(96, B/2) sequences; greedy rule: one launch), -1 never, n > 0 that many
+   sequences (at most half the batch).  Outputs are the same either way;
+   pspec_last_launches then reports 2.  Process-wide. */
+PSPEC_API void pspec_set_tail_split(int n);
+
 /* Tuning: fusion of the two halves of pspec_step_* into one launch (early-exit path only):
    0 automatic (fewer than 256 sequences), 1 always, 2 never.  Process-wide. */
 PSPEC_API void pspec_set_step_fusion(int mode);

@@ -31,6 +31,7 @@ EXPORTED = (
     "pspec_sample_workspace_bytes", "pspec_sample_drafts",
     "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
     "pspec_step_greedy", "pspec_step_rejection", "pspec_set_step_fusion",
+    "pspec_set_ee_stream", "pspec_set_tail_split",
 )
 
 
@@ -102,6 +103,10 @@ def _load():
     lib.pspec_set_verify_path.restype = None
     lib.pspec_set_step_fusion.argtypes = [_I]
     lib.pspec_set_step_fusion.restype = None
+    lib.pspec_set_ee_stream.argtypes = [_I]
+    lib.pspec_set_ee_stream.restype = None
+    lib.pspec_set_tail_split.argtypes = [_I]
+    lib.pspec_set_tail_split.restype = None
     lib.pspec_set_cluster_size.argtypes = [_I]
     lib.pspec_set_cluster_size.restype = None
     lib.pspec_last_verify_path.argtypes = []
@@ -187,6 +192,16 @@ def pspec_set_verify_path(path: int) -> None:
 def pspec_set_step_fusion(mode: int) -> None:
     """Fusion of pspec_step_*'s two halves into one launch: 0 automatic, 1 always, 2 never."""
     LIB.pspec_set_step_fusion(int(mode))
+
+
+def pspec_set_ee_stream(mode: int) -> None:
+    """Early-exit row streaming: 0 automatic, 1 registers, 2 shared-memory ring (bulk copies)."""
+    LIB.pspec_set_ee_stream(int(mode))
+
+
+def pspec_set_tail_split(n: int) -> None:
+    """Early exit: sequences given to a second launch of 8-CTA clusters (0 auto, -1 never)."""
+    LIB.pspec_set_tail_split(int(n))
 
 
 def pspec_set_segment_elems(elems: int) -> None:

@@ -18,6 +18,8 @@ cudaEvent_t g_split_event = nullptr;
 int g_verify_path = 0;          // 0 automatic, 1 full sweep, 2 early exit, 3 work queue
 int g_cluster = 0;              // early-exit cluster size; 0 = automatic
 int g_step_fusion = 0;          // 0 automatic, 1 always, 2 never
+int g_ee_stream = 0;            // early-exit streaming: 0 automatic, 1 registers, 2 ring
+int g_tail_split = 0;           // early-exit tail launch: 0 automatic, -1 never, n > 0 sequences
 thread_local int t_last_launches = 0;
 thread_local int t_last_path = 0;
 
@@ -108,6 +110,7 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.rejection = rejection;
   L.G = ep.G; L.vs = ep.vs;
+  L.ring = g_ee_stream == 2;
   L.target = a->target_logits;
   L.draft = a->draft_logits;
   L.draft_tokens = a->draft_tokens;
@@ -123,12 +126,39 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
     L.b = fuse->a;
     L.row_vecs = fuse->row_vecs;
   }
-  if (launch_early_exit(L, stream) != cudaSuccess) {
+  L.seq0 = 0;
+  L.nseq = a->B;
+  // The last X sequences go to a second launch of wider clusters that starts as the first
+  // launch's clusters finish (programmatic dependent launch): the sequences that start last
+  // then run their chains of rows twice as wide, which shortens the launch's tail.
+  int X = 0;
+  if (ep.G == kEarlyExitCluster && ep.G != 16 && g_tail_split >= 0)
+    X = g_tail_split > 0 ? g_tail_split : early_exit_tail(a->B, rejection);
+  X = X < a->B / 2 ? X : a->B / 2;
+  const EarlyExitPlan et = make_early_exit_plan(a->V, kEarlyExitTailCluster);
+  int launches = 1;
+  cudaError_t ce;
+  if (X > 0 && et.ok) {
+    EarlyExitLaunch L2 = L;
+    L.nseq = a->B - X;
+    L.pdl = 1;
+    L2.seq0 = a->B - X;
+    L2.nseq = X;
+    L2.G = kEarlyExitTailCluster;
+    L2.vs = et.vs;
+    L2.pdl = 2;
+    ce = launch_early_exit(L, stream);
+    if (ce == cudaSuccess) ce = launch_early_exit(L2, stream);
+    launches = 2;
+  } else {
+    ce = launch_early_exit(L, stream);
+  }
+  if (ce != cudaSuccess) {
     *st = PSPEC_ERR_CUDA;
     return true;
   }
   if (rejection && g_split_event) cudaEventRecord(g_split_event, stream);
-  t_last_launches = 1;
+  t_last_launches = launches;
   t_last_path = 2;
   *st = PSPEC_OK;
   return true;
@@ -422,6 +452,8 @@ void pspec_set_verify_path(int path) { g_verify_path = (path >= 1 && path <= 3) 
 void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || G == 16) ? G : 0; }
 
 void pspec_set_step_fusion(int mode) { g_step_fusion = (mode == 1 || mode == 2) ? mode : 0; }
+void pspec_set_ee_stream(int mode) { g_ee_stream = (mode == 1 || mode == 2) ? mode : 0; }
+void pspec_set_tail_split(int n) { g_tail_split = n < 0 ? -1 : n; }
 
 void pspec_set_segment_elems(long long elems) { g_seg_override = elems > 0 ? elems : 0; }
 

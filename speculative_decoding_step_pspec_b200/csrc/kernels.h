@@ -63,6 +63,10 @@ struct EarlyExitLaunch {
   pspec_dtype dtype;
   int rejection;         // 1: rejection rule, 0: greedy
   int G;                 // CTAs per cluster (one cluster per sequence): 2, 4, 8 or 16
+  int ring;              // 1: rows streamed through per-warp shared-memory stages (bulk copies)
+  int seq0, nseq;        // this launch's sequences [seq0, seq0 + nseq) of the batch's B
+  int pdl;               // split batch: 1 first launch (lets the second start as its CTAs
+                         // are placed), 2 second launch (its CTA 0 ends after the first grid)
   long long vs;          // slice of each row per CTA (elements, multiple of 8)
   const void* target;
   const void* draft;

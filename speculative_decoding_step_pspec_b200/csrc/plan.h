@@ -34,6 +34,28 @@ constexpr int kEarlyExitCluster = 4;     // CTAs per sequence on the early-exit 
 constexpr int kEarlyExitSmallB = 128;
 constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this many sequences
 
+// Early exit, batches of 4-CTA clusters: the last sequences go to a second launch of
+// kEarlyExitTailCluster-CTA clusters that fills the SMs as the first launch drains.
+// Measured on B200 (rejection rule, 8-CTA tail): at 1024 sequences 0.672 ms with 96 in the
+// tail against 0.701 ms with none (64: 0.679, 128: 0.677, 256: 0.695); at 256 sequences
+// 0.243-0.245 ms with 32 to 128 against 0.266 ms; 16-CTA tails gained at most 1.8 %.  The
+// greedy rule was slower with any tail (16 sequences: 0.208 against 0.207 ms), so it keeps
+// one launch.
+#ifndef PSPEC_EE_TAIL_SEQS
+#define PSPEC_EE_TAIL_SEQS 96
+#endif
+#ifndef PSPEC_EE_TAIL_CLUSTER
+#define PSPEC_EE_TAIL_CLUSTER 8
+#endif
+constexpr int kEarlyExitTailCluster = PSPEC_EE_TAIL_CLUSTER;
+inline int early_exit_tail(long long B, bool rejection) {
+  if (!rejection) return 0;
+  return (int)(B / 2 < PSPEC_EE_TAIL_SEQS ? B / 2 : PSPEC_EE_TAIL_SEQS);
+}
+inline int early_exit_tail(long long B) {
+  return B >= 2 * PSPEC_EE_TAIL_SEQS ? PSPEC_EE_TAIL_SEQS : 0;
+}
+
 // Per-(row, segment) partial of the greedy sweep.
 struct GreedyPart {
   float v;   // best value

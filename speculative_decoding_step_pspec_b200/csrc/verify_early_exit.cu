@@ -26,7 +26,10 @@
 // shared memory (two CTAs per SM) left HBM idle between positions.
 #include <cooperative_groups.h>
 
+#include <atomic>
+
 #include "build_common.cuh"
+#include "bulk_ring.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
@@ -54,6 +57,30 @@ namespace {
 #ifndef PSPEC_EE_GREEDY_MIN_BLOCKS
 #define PSPEC_EE_GREEDY_MIN_BLOCKS 4
 #endif
+
+// Streaming through shared memory (kRing): each warp owns kRingStages stages of
+// kRingBytes per row, filled by bulk asynchronous copies; CTAs per SM as the shared memory
+// allows.
+#ifndef PSPEC_EE_RING_BYTES
+#define PSPEC_EE_RING_BYTES 2048
+#endif
+#ifndef PSPEC_EE_RING_STAGES
+#define PSPEC_EE_RING_STAGES 2
+#endif
+#ifndef PSPEC_EE_RING_MIN_BLOCKS
+#define PSPEC_EE_RING_MIN_BLOCKS 3
+#endif
+#ifndef PSPEC_EE_RING_GREEDY_MIN_BLOCKS
+#define PSPEC_EE_RING_GREEDY_MIN_BLOCKS 5
+#endif
+constexpr int kRingBytes = PSPEC_EE_RING_BYTES;          // one row's share of a stage
+constexpr int kRingStages = PSPEC_EE_RING_STAGES;
+constexpr int kRingVecs = kRingBytes / 16;               // 16-byte vectors per row and stage
+constexpr int kRingLaneVecs = kRingVecs / 32;
+static_assert(kRingVecs % 32 == 0 && kRingLaneVecs >= 1, "ring stage: whole vectors per lane");
+
+// Dynamic shared memory of the kRing variants: the warps' stages.
+constexpr int ring_smem_bytes(bool rej) { return kWarps * kRingStages * (rej ? 2 : 1) * kRingBytes; }
 
 constexpr int kEERejUnroll = PSPEC_EE_REJ_UNROLL;   // vectors per row in flight (rejection)
 constexpr int kEEMinBlocks = PSPEC_EE_MIN_BLOCKS;   // CTAs per SM the register budget targets
@@ -194,15 +221,18 @@ __device__ __forceinline__ void ee_build_span(const pspec_build_args& b, long lo
   set_err(b.err, eb);
 }
 
-template <typename Tag, int G, bool kRej, bool kFuse>
-__global__ void __launch_bounds__(kThreads, kRej ? kEEMinBlocks : PSPEC_EE_GREEDY_MIN_BLOCKS)
+template <typename Tag, int G, bool kRej, bool kFuse, bool kRing>
+__global__ void __launch_bounds__(kThreads,
+                                  kRing ? (kRej ? PSPEC_EE_RING_MIN_BLOCKS : PSPEC_EE_RING_GREEDY_MIN_BLOCKS)
+                                        : (kRej ? kEEMinBlocks : PSPEC_EE_GREEDY_MIN_BLOCKS))
 ee_kernel(const EarlyExitLaunch L) {
   using elem = typename Tag::elem;
   constexpr int W = Tag::kVec;
   constexpr int U = kRej ? kEERejUnroll : PSPEC_EE_GREEDY_UNROLL;  // vectors in flight per row
   cg::cluster_group cluster = cg::this_cluster();
   const int g = (int)cluster.block_rank();
-  const int i = (int)(blockIdx.x / G);
+  const int i = L.seq0 + (int)(blockIdx.x / G);
+  if (L.pdl == 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = L.K;
   int ebk = 0;
@@ -226,6 +256,40 @@ ee_kernel(const EarlyExitLaunch L) {
   const int n = (int)max(0LL, min((long long)L.V, lo + L.vs) - lo);
   const int nvec = n / W;                                   // n is a multiple of 8
 
+  // kRing: warp w streams the run [wlo, wlo + wn) of the slice (multiples of 8 elements) in
+  // chunks of SE elements through its own stages; gidx counts the chunks it has consumed,
+  // which fixes each stage's mbarrier phase across positions.
+  constexpr int kRows = kRej ? 2 : 1;
+  constexpr int SE = kRingBytes / (int)sizeof(elem);
+  __shared__ __align__(8) uint64_t s_bar[kRing ? kWarps * kRingStages : 1];
+  extern __shared__ __align__(16) uint4 s_ring[];
+  const int wper = ((n + kWarps - 1) / kWarps + 7) / 8 * 8;
+  const int wlo = min(n, warp * wper);
+  const int wn = min(n, wlo + wper) - wlo;
+  const int nch = (wn + SE - 1) / SE;
+  uint32_t gidx = 0;
+  bool ring_ok = true;
+  uint4* const ring = s_ring + (size_t)warp * kRingStages * kRows * kRingVecs;
+  uint64_t* const bar = s_bar + (kRing ? warp * kRingStages : 0);
+  if constexpr (kRing) {
+    if (lane == 0) {
+      for (int s = 0; s < kRingStages; ++s) mbar_init(&bar[s]);
+      mbar_init_fence();
+    }
+    __syncwarp();
+  }
+  // chunk c of this warp's run of rows (tr, qr) into stage gi mod kRingStages (lane 0 only)
+  auto issue = [&](const elem* tr, const elem* qr, bool hq, int c, uint32_t gi) {
+    const int s = (int)(gi % kRingStages);
+    const int e0 = wlo + c * SE;
+    const unsigned bytes = (unsigned)(min(SE, wn - c * SE) * (int)sizeof(elem));
+    uint4* st = ring + s * kRows * kRingVecs;
+    fence_async_shared();
+    mbar_arrive_expect(&bar[s], hq ? 2 * bytes : bytes);
+    bulk_copy_g2s(st, tr + lo + e0, bytes, &bar[s]);
+    if (hq) bulk_copy_g2s(st + kRingVecs, qr + lo + e0, bytes, &bar[s]);
+  };
+
   int k = 0;
   for (; k <= Ki; ++k) {
     const bool has_q = kRej && k < Ki;
@@ -244,31 +308,77 @@ ee_kernel(const EarlyExitLaunch L) {
     // ---- stream this CTA's slice of the position's rows
     MSAcc at = msacc_init(), aq = msacc_init();
     VI best{-INFINITY, kNoIndex};
-    const uint4* tv = reinterpret_cast<const uint4*>(trow + lo);
-    const uint4* qv = reinterpret_cast<const uint4*>(qrow + lo);
-    int v0 = tid;
-    for (; v0 + (U - 1) * kThreads < nvec; v0 += U * kThreads) {   // full batches
-      uint4 bt[U], bq[U];
+    if constexpr (kRing) {
+      if (lane == 0 && ring_ok)
+        for (int c = 0; c < nch && c < kRingStages; ++c) issue(trow, qrow, has_q, c, gidx + (uint32_t)c);
+      for (int c = 0; c < nch; ++c, ++gidx) {
+        const int s = (int)(gidx % kRingStages);
+        if (ring_ok) {
+          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar[s], (gidx / kRingStages) & 1u));
+          if (!ok) {
+            ring_ok = false;                             // no further copies from this warp
+            if (lane == 0) set_err(L.err, PSPEC_DEVERR_TIMEOUT);
+          }
+        }
+        const uint4* st = ring + s * kRows * kRingVecs;
+        const int mv = min(SE, wn - c * SE) / W;
+        const long long e0 = lo + wlo + (long long)c * SE;   // token id of the chunk's start
+        if (mv == kRingVecs) {
+          uint4 bt[kRingLaneVecs], bq[kRingLaneVecs];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        bt[u] = ld_stream(tv + v0 + u * kThreads);
-        if (has_q) bq[u] = ld_stream(qv + v0 + u * kThreads);
-      }
-      if constexpr (kRej) {
-        consume_ms_batch<Tag, U>(bt, at);
-        if (has_q) consume_ms_batch<Tag, U>(bq, aq);
-      } else {
+          for (int u = 0; u < kRingLaneVecs; ++u) {
+            bt[u] = st[lane + 32 * u];
+            if (has_q) bq[u] = st[kRingVecs + lane + 32 * u];
+          }
+          if constexpr (kRej) {
+            consume_ms_batch<Tag, kRingLaneVecs>(bt, at);
+            if (has_q) consume_ms_batch<Tag, kRingLaneVecs>(bq, aq);
+          } else {
 #pragma unroll
-        for (int u = 0; u < U; ++u) consume_argmax<Tag>(bt[u], lo + (long long)(v0 + u * kThreads) * W, best);
+            for (int u = 0; u < kRingLaneVecs; ++u)
+              consume_argmax<Tag>(bt[u], e0 + (long long)(lane + 32 * u) * W, best);
+          }
+        } else {
+          for (int v = lane; v < mv; v += 32) {
+            if constexpr (kRej) {
+              consume_ms<Tag>(st[v], at);
+              if (has_q) consume_ms<Tag>(st[kRingVecs + v], aq);
+            } else {
+              consume_argmax<Tag>(st[v], e0 + (long long)v * W, best);
+            }
+          }
+        }
+        __syncwarp();                                        // the stage is read: refill it
+        if (lane == 0 && ring_ok && c + kRingStages < nch)
+          issue(trow, qrow, has_q, c + kRingStages, gidx + kRingStages);
       }
-    }
-    for (; v0 < nvec; v0 += kThreads) {                            // the rest, one by one
-      const uint4 x = ld_stream(tv + v0);
-      if constexpr (kRej) {
-        consume_ms<Tag>(x, at);
-        if (has_q) consume_ms<Tag>(ld_stream(qv + v0), aq);
-      } else {
-        consume_argmax<Tag>(x, lo + (long long)v0 * W, best);
+    } else {                                                 // through registers
+      const uint4* tv = reinterpret_cast<const uint4*>(trow + lo);
+      const uint4* qv = reinterpret_cast<const uint4*>(qrow + lo);
+      int v0 = tid;
+      for (; v0 + (U - 1) * kThreads < nvec; v0 += U * kThreads) {   // full batches
+        uint4 bt[U], bq[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          bt[u] = ld_stream(tv + v0 + u * kThreads);
+          if (has_q) bq[u] = ld_stream(qv + v0 + u * kThreads);
+        }
+        if constexpr (kRej) {
+          consume_ms_batch<Tag, U>(bt, at);
+          if (has_q) consume_ms_batch<Tag, U>(bq, aq);
+        } else {
+#pragma unroll
+          for (int u = 0; u < U; ++u) consume_argmax<Tag>(bt[u], lo + (long long)(v0 + u * kThreads) * W, best);
+        }
+      }
+      for (; v0 < nvec; v0 += kThreads) {                            // the rest, one by one
+        const uint4 x = ld_stream(tv + v0);
+        if constexpr (kRej) {
+          consume_ms<Tag>(x, at);
+          if (has_q) consume_ms<Tag>(ld_stream(qv + v0), aq);
+        } else {
+          consume_argmax<Tag>(x, lo + (long long)v0 * W, best);
+        }
       }
     }
     MS mt = msacc_final(at), mq = msacc_final(aq);
@@ -529,42 +639,74 @@ ee_kernel(const EarlyExitLaunch L) {
     __syncthreads();
     ee_build_span(L.b, L.row_vecs, i, k, Ki, g == meta_g ? s_tok : 0, g == meta_g, g, G);
   }
+  // second launch of a split batch: its completion implies the first grid's, so work queued
+  // after it on the stream sees every sequence's outputs
+  if (L.pdl == 2 && blockIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-template <typename Tag, int G, bool kRej, bool kFuse>
+// Shared-memory attributes of a kRing variant, set once per device.
+template <typename Kern>
+cudaError_t ring_attributes(Kern kern, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_relaxed) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_relaxed);
+  return e;
+}
+
+template <typename Tag, int G, bool kRej, bool kFuse, bool kRing>
 cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream) {
-  auto kern = ee_kernel<Tag, G, kRej, kFuse>;
+  auto kern = ee_kernel<Tag, G, kRej, kFuse, kRing>;
   cudaError_t e = cudaSuccess;
   if (G > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
+  const int dyn = kRing ? ring_smem_bytes(kRej) : 0;
+  if constexpr (kRing) {
+    static std::atomic<unsigned long long> done{0};
+    e = ring_attributes(kern, dyn, done);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((long long)L.B * G), 1, 1);
+  cfg.gridDim = dim3((unsigned)((long long)L.nseq * G), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = (size_t)dyn;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = G;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = L.pdl == 2 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, L);
+}
+
+template <int G, bool kRing>
+cudaError_t launch_ee_gr(const EarlyExitLaunch& L, cudaStream_t s) {
+  const bool bf = L.dtype == PSPEC_BF16;
+  if (L.fuse_build) {
+    if (L.rejection)
+      return bf ? launch_ee<BF16Tag, G, true, true, kRing>(L, s) : launch_ee<F32Tag, G, true, true, kRing>(L, s);
+    return bf ? launch_ee<BF16Tag, G, false, true, kRing>(L, s) : launch_ee<F32Tag, G, false, true, kRing>(L, s);
+  }
+  if (L.rejection)
+    return bf ? launch_ee<BF16Tag, G, true, false, kRing>(L, s) : launch_ee<F32Tag, G, true, false, kRing>(L, s);
+  return bf ? launch_ee<BF16Tag, G, false, false, kRing>(L, s) : launch_ee<F32Tag, G, false, false, kRing>(L, s);
 }
 
 template <int G>
 cudaError_t launch_ee_g(const EarlyExitLaunch& L, cudaStream_t s) {
-  const bool bf = L.dtype == PSPEC_BF16;
-  if (L.fuse_build) {
-    if (L.rejection)
-      return bf ? launch_ee<BF16Tag, G, true, true>(L, s) : launch_ee<F32Tag, G, true, true>(L, s);
-    return bf ? launch_ee<BF16Tag, G, false, true>(L, s) : launch_ee<F32Tag, G, false, true>(L, s);
-  }
-  if (L.rejection)
-    return bf ? launch_ee<BF16Tag, G, true, false>(L, s) : launch_ee<F32Tag, G, true, false>(L, s);
-  return bf ? launch_ee<BF16Tag, G, false, false>(L, s) : launch_ee<F32Tag, G, false, false>(L, s);
+  return L.ring ? launch_ee_gr<G, true>(L, s) : launch_ee_gr<G, false>(L, s);
 }
 
 }  // namespace

@@ -39,6 +39,37 @@ class verify_path:
         ps.pspec_set_verify_path(0)
 
 
+class ee_stream:
+    """Early-exit row streaming inside a with-block: 1 registers, 2 per-warp shared-memory
+    rings filled by bulk copies."""
+
+    def __init__(self, mode):
+        self.mode = mode
+
+    def __enter__(self):
+        ps.pspec_set_ee_stream(self.mode)
+
+    def __exit__(self, *a):
+        ps.pspec_set_ee_stream(0)
+
+
+class tail_split:
+    """Inside a with-block, n > 0 hands the last n sequences of an early-exit batch to a
+    second launch (4-CTA clusters forced for the first)."""
+
+    def __init__(self, n):
+        self.n = n
+
+    def __enter__(self):
+        if self.n:
+            ps.pspec_set_cluster_size(4)
+            ps.pspec_set_tail_split(self.n)
+
+    def __exit__(self, *a):
+        ps.pspec_set_cluster_size(0)
+        ps.pspec_set_tail_split(0)
+
+
 def early_exit_allowed(t):
     return t.shape[2] % 8 == 0 and t.data_ptr() % 16 == 0 and (t.stride(1) * t.element_size()) % 16 == 0
 
@@ -58,14 +89,17 @@ def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True)
     U.compare_greedy(gr, og, seqs)
     orj = U.oracle_rejection(target, draft, sampled, u, seqs)
     U.compare_rejection(rj, orj, seqs)
-    for path in (2, 3):                    # early exit where its shape rules allow; queue always
+    # early exit (both ways of streaming rows) where its shape rules allow; queue always
+    for path, stream in ((2, 1), (2, 2), (3, 0)):
         if path == 2 and not early_exit_allowed(target):
             continue
-        with verify_path(path):
+        with verify_path(path), ee_stream(stream):
+            # the early-exit path may hand the batch's last sequences to a second launch
+            ok_launches = (1, 2) if path == 2 else (1,)
             ge = ps.verify_greedy(target, greedy_drafts)
-            assert ps.pspec_last_launches() == 1 and ps.pspec_last_verify_path() == path
+            assert ps.pspec_last_launches() in ok_launches and ps.pspec_last_verify_path() == path
             re = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
-            assert ps.pspec_last_launches() == 1 and ps.pspec_last_verify_path() == path
+            assert ps.pspec_last_launches() in ok_launches and ps.pspec_last_verify_path() == path
         torch.cuda.synchronize()
         assert ge["err"].item() == 0 and re["err"].item() == 0, path
         U.check_verify_invariants(ge, greedy_drafts, V)
@@ -238,10 +272,10 @@ def test_automatic_path_selection(B):
     sampled, _ = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
     a = ps.verify_rejection(target, draft, sampled, u)
-    n_auto = ps.pspec_last_launches()
+    path_auto = ps.pspec_last_verify_path()
     b = ps.verify_rejection(target, draft, sampled, u, diagnostics=True)
-    assert ps.pspec_last_launches() == 2
-    assert n_auto == (1 if B >= 64 else 2)
+    assert ps.pspec_last_launches() == 2 and ps.pspec_last_verify_path() == 1
+    assert path_auto == (2 if B >= 64 else 1)
     o = U.oracle_rejection(target, draft, sampled, u)
     U.compare_rejection(a, o)
     U.compare_rejection(b, o)
@@ -653,7 +687,8 @@ def _step_check(target, draft, drafts, u, binp, path, expect_fused):
         assert torch.equal(v1[k], v2[k]), k
     for k in b1:
         assert torch.equal(b1[k], b2[k]), k
-    assert n_step == (1 if expect_fused else n_verify + 1), (n_step, n_verify)
+    # fused: the verify's own launches (one, or two when the batch is split) also build
+    assert n_step == (n_verify if expect_fused else n_verify + 1), (n_step, n_verify)
     return v2, b2
 
 
@@ -712,30 +747,35 @@ def test_step_fused_invalid_layout_sets_bit():
     assert bo["err"].item() & ps._binding.PSPEC_DEVERR_LAYOUT
 
 
-def test_step_b1024_fused():
+@pytest.mark.parametrize("stream", [1, 2])
+def test_step_b1024_fused(stream):
     """Full size with fusion forced on (the automatic choice at 1024 sequences is two
-    launches), then forced off."""
+    launches), then forced off; rows streamed through registers or shared-memory rings."""
     w = I.B1024
     target, draft = I.logits(w, DEV)
     sampled, _ = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
     binp = I.build_inputs(w, DEV, drafts=sampled)
     try:
+        ps.pspec_set_ee_stream(stream)
         ps.pspec_set_step_fusion(1)
         v, _ = _step_check(target, draft, sampled, u, binp, 0, True)
         ps.pspec_set_step_fusion(2)
         _step_check(target, draft, sampled, u, binp, 2, False)
     finally:
         ps.pspec_set_step_fusion(0)
+        ps.pspec_set_ee_stream(0)
     seqs = _sample(w.B, 24, 5)
     U.compare_rejection(v, U.oracle_rejection(target, draft, sampled, u, seqs), seqs)
 
 
-@pytest.mark.parametrize("path", [0, 1, 3])
-def test_step_cuda_graph_replay(path):
+@pytest.mark.parametrize("path,stream,tail", [(0, 1, 0), (0, 2, 0), (2, 1, 20), (1, 0, 0), (3, 0, 0)])
+def test_step_cuda_graph_replay(path, stream, tail):
     """One step captured in a CUDA graph and replayed with new uniforms and drafts copied
     into the captured buffers gives what the eager calls give for those inputs (the
-    kernels leave their workspace counters at zero, so replays need no reset)."""
+    kernels leave their workspace counters at zero, so replays need no reset); `tail`
+    splits the early-exit launch in two (4-CTA clusters, then 8-CTA clusters queued with
+    programmatic dependent launch)."""
     w = I.scaled(I.C64, B=96, V=20000, H=64)
     target, draft = I.logits(w, DEV)
     sampled, _ = I.draft_tokens(w, draft)
@@ -745,7 +785,7 @@ def test_step_cuda_graph_replay(path):
     vout = ps.api.verify_outputs(w.B, w.K, DEV, False, True, True)
     bout = ps.api.build_outputs(w.B, w.K, 64, binp["T_cap"], binp["verify_hidden"].dtype, DEV)
     d_in, u_in = sampled.clone(), u.clone()
-    with verify_path(path):
+    with verify_path(path), ee_stream(stream), tail_split(tail):
         ps.step(target, d_in, binp, draft_logits=draft, uniforms=u_in, residual_mass=True,
                 workspace=ws, out=vout, build_out=bout)           # warm-up outside capture
         torch.cuda.synchronize()
@@ -900,7 +940,7 @@ def _step_check_k(target, draft, drafts, u, binp, path, expect_fused, klt):
         assert torch.equal(v1[k], v2[k]), k
     for k in b1:
         assert torch.equal(b1[k], b2[k]), k
-    assert n_step == (1 if expect_fused else n_verify + 1)
+    assert n_step == (n_verify if expect_fused else n_verify + 1)
     # the build against the oracle with the verify's own counts and tokens
     inp = dict(binp, accepted_len=v1["accepted_len"], bonus=v1["bonus"])
     dh = U.hidden_sentinel(binp["T_cap"], H, dt, DEV)
@@ -909,10 +949,46 @@ def _step_check_k(target, draft, drafts, u, binp, path, expect_fused, klt):
     return v2, b2
 
 
+@pytest.mark.parametrize("X", [1, 37, 150])
+def test_early_exit_tail_split(X):
+    """The batch split over two early-exit launches (4-CTA clusters, then the last X
+    sequences in 8-CTA clusters queued with programmatic dependent launch) against the
+    oracle, both rules, K_i included, and the step fused and unfused."""
+    w = I.Workload("t", 300, 7, 40000, 64, 16, torch.bfloat16, seed=X, sigma_t=2.0, sigma_d=0.5)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    kl = torch.as_tensor(np.random.default_rng(X).integers(0, w.K + 1, size=w.B).astype(np.int32),
+                         device=DEV)
+    binp = I.build_inputs(w, DEV, drafts=sampled)
+    try:
+        ps.pspec_set_tail_split(X)
+        with verify_path(2):
+            g = ps.verify_greedy(target, greedy)
+            assert ps.pspec_last_launches() == 2
+            r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
+            assert ps.pspec_last_launches() == 2
+            rk = ps.verify_rejection(target, draft, sampled, u, k_len=kl)
+        torch.cuda.synchronize()
+        assert g["err"].item() == 0 and r["err"].item() == 0 and rk["err"].item() == 0
+        U.compare_greedy(g, U.oracle_greedy(target, greedy, want_lse=False))
+        U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u))
+        U.compare_rejection(rk, U.oracle_rejection(target, draft, sampled, u, k_len=kl))
+        for fuse in (1, 2):
+            ps.pspec_set_step_fusion(fuse)
+            _step_check(target, draft, sampled, u, binp, 2, fuse == 1)
+            _step_check(target, draft, greedy, None, binp, 2, fuse == 1)
+    finally:
+        ps.pspec_set_tail_split(0)
+        ps.pspec_set_step_fusion(0)
+
+
+@pytest.mark.parametrize("stream", [1, 2])
 @pytest.mark.parametrize("G", [2, 4, 8, 16])
-def test_early_exit_every_cluster_size(G):
+def test_early_exit_every_cluster_size(G, stream):
     """The early-exit kernel with each cluster size (the automatic choice is 16 below 128
-    sequences, else 4) against the oracle, unfused and with the step fused, K_i included."""
+    sequences, else 4) and both ways of streaming rows against the oracle, unfused and with
+    the step fused, K_i included."""
     w = I.scaled(I.C64, B=40, V=40000, H=64)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
@@ -922,6 +998,7 @@ def test_early_exit_every_cluster_size(G):
     binp = I.build_inputs(w, DEV, drafts=sampled)
     try:
         ps.pspec_set_cluster_size(G)
+        ps.pspec_set_ee_stream(stream)
         with verify_path(2):
             g = ps.verify_greedy(target, greedy)
             r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
@@ -933,3 +1010,4 @@ def test_early_exit_every_cluster_size(G):
         _step_check(target, draft, greedy, None, binp, 2, True)
     finally:
         ps.pspec_set_cluster_size(0)
+        ps.pspec_set_ee_stream(0)
