@@ -300,6 +300,7 @@ def run_pspec(args, rank, world, local_rank):
             build()
             lb = ps.pspec_last_launches()
         path = ps.pspec_last_verify_path()
+        cluster = ps.pspec_last_cluster_size()
     launches_per_step = lv + lb
     torch.cuda.synchronize()
     graph = None
@@ -405,7 +406,7 @@ def run_pspec(args, rank, world, local_rank):
             "workload": f"{args.workload}{'' if not args.batch else ' (B overridden)'}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
                         f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
-            "verify_path": {1: "full sweep", 2: "early exit (cluster per sequence)",
+            "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)",
                             3: "work queue (persistent, position order)"}[path],
             "step": ("one launch (verify + build fused)" if fused else "verify launches + build launch")
                     + (", CUDA graph replay" if graph is not None else ""),

@@ -357,9 +357,12 @@ PSPEC_API int pspec_last_launches(void);
    All paths give the same outputs; they differ in which rows they read. */
 PSPEC_API void pspec_set_verify_path(int path);
 
-/* Tuning: CTAs per thread-block cluster on the early-exit path (2, 4, 8 or 16; each CTA
-   streams a 1/G slice of a row); 0 restores the automatic choice (16 below 128 sequences,
-   else 4, or 16 when a slice of 4 would exceed 262144 elements).  Process-wide. */
+/* Tuning: CTAs per thread-block cluster on the early-exit path (2, 4, 8, 12 or 16; each
+   CTA streams a 1/G slice of a row); 0 restores the automatic choice: 4 from 128 sequences
+   on (16 when a slice of 4 would exceed 262144 elements); below, for the rejection rule
+   the widest of 16, 12 and 8 with which the clusters of all sequences fit on the GPU at
+   once (cudaOccupancyMaxActiveClusters, asked once per device and kernel variant), for the
+   greedy rule 8 (16 below 16 sequences).  Process-wide. */
 PSPEC_API void pspec_set_cluster_size(int G);
 
 /* Tuning: how the early-exit path streams logit rows.  0 automatic (= 1), 1 through
@@ -390,6 +393,10 @@ PSPEC_API void pspec_set_step_fusion(int mode);
 /* The path the most recent successful verify call on this host thread took: 1 full sweep,
    2 early exit, 3 work queue, 0 none yet. */
 PSPEC_API int pspec_last_verify_path(void);
+
+/* CTAs per cluster of the first (or only) launch of the last early-exit verify on this
+   thread (the automatic choice or pspec_set_cluster_size's); 0 before any. */
+PSPEC_API int pspec_last_cluster_size(void);
 
 /* Tuning: force the verify sweeps' segment length (elements of one row handled by one
    CTA; rounded up to a multiple of 8).  0 restores the automatic choice, which aims at

@@ -31,7 +31,7 @@ EXPORTED = (
     "pspec_sample_workspace_bytes", "pspec_sample_drafts",
     "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
     "pspec_step_greedy", "pspec_step_rejection", "pspec_set_step_fusion",
-    "pspec_set_ee_stream", "pspec_set_tail_split",
+    "pspec_set_ee_stream", "pspec_set_tail_split", "pspec_last_cluster_size",
 )
 
 
@@ -111,6 +111,8 @@ def _load():
     lib.pspec_set_cluster_size.restype = None
     lib.pspec_last_verify_path.argtypes = []
     lib.pspec_last_verify_path.restype = _I
+    lib.pspec_last_cluster_size.argtypes = []
+    lib.pspec_last_cluster_size.restype = _I
     lib.pspec_set_segment_elems.argtypes = [ctypes.c_longlong]
     lib.pspec_set_segment_elems.restype = None
     lib.pspec_set_split_event.argtypes = [_P]
@@ -174,7 +176,7 @@ def pspec_last_launches() -> int:
 
 
 def pspec_set_cluster_size(G: int) -> None:
-    """CTAs per cluster on the early-exit path: 4, 8, 16, or 0 for automatic."""
+    """CTAs per cluster on the early-exit path: 2, 4, 8, 12, 16, or 0 for automatic."""
     LIB.pspec_set_cluster_size(int(G))
 
 
@@ -182,6 +184,11 @@ def pspec_last_verify_path() -> int:
     """1 full sweep, 2 early exit, 3 work queue: the path of the most recent verify call on
     this thread."""
     return LIB.pspec_last_verify_path()
+
+
+def pspec_last_cluster_size() -> int:
+    """CTAs per cluster of the last early-exit verify on this thread (0 before any)."""
+    return LIB.pspec_last_cluster_size()
 
 
 def pspec_set_verify_path(path: int) -> None:

@@ -22,6 +22,7 @@ int g_ee_stream = 0;            // early-exit streaming: 0 automatic, 1 register
 int g_tail_split = 0;           // early-exit tail launch: 0 automatic, -1 never, n > 0 sequences
 thread_local int t_last_launches = 0;
 thread_local int t_last_path = 0;
+thread_local int t_last_cluster = 0;   // CTAs per cluster of the last early-exit launch
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -96,12 +97,10 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   if (g_verify_path == 1) return false;
   if (g_verify_path == 0 && (a->B < kEarlyExitMinB || diagnostics)) return false;
   const int eb = (int)elem_bytes(a->dtype);
-  const int G_auto = a->B < kEarlyExitSmallB ? 16 : kEarlyExitCluster;
-  EarlyExitPlan ep = make_early_exit_plan(a->V, g_cluster ? g_cluster : G_auto);
-  if (!ep.ok && g_cluster == 0) ep = make_early_exit_plan(a->V, 16);
   const bool aligned = aligned16(a->target_logits) && (!rejection || aligned16(a->draft_logits)) &&
                        (a->ld * eb) % 16 == 0;
-  if (!ep.ok || !aligned || diagnostics) {
+  const bool v_ok = a->V % 8 == 0 && make_early_exit_plan(a->V, 16).ok;
+  if (!v_ok || !aligned || diagnostics) {
     if (g_verify_path == 0) return false;
     *st = PSPEC_ERR_UNSUPPORTED;            // early exit forced on arguments it cannot take
     return true;
@@ -109,7 +108,6 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   EarlyExitLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.rejection = rejection;
-  L.G = ep.G; L.vs = ep.vs;
   L.ring = g_ee_stream == 2;
   L.target = a->target_logits;
   L.draft = a->draft_logits;
@@ -126,8 +124,40 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
     L.b = fuse->a;
     L.row_vecs = fuse->row_vecs;
   }
+  // Cluster size: 4 from kEarlyExitSmallB sequences on.  Below, the rejection rule takes the
+  // widest cluster (16, 12, 8) with which every sequence's cluster is resident at once (a
+  // batch that needs a second round of clusters costs a second chain of positions); the
+  // greedy rule, with less work per element, 8 (16 below 16 sequences).  Measured on B200
+  // with c64's rows, ms per step for G = 16 / 12 / 8: rejection B = 32: 0.081 / 0.085 /
+  // 0.097, B = 64: 0.099 / 0.095 / 0.103, B = 96: 0.123 / 0.114 / 0.108 (the rule picks 16,
+  // 12, 8); greedy B = 32: 0.043 / 0.047 / 0.041, B = 64: 0.047 / 0.049 / 0.046, B = 96:
+  // 0.054 / 0.053 / 0.046.
   L.seq0 = 0;
   L.nseq = a->B;
+  int G = g_cluster;
+  if (G == 0) {
+    G = kEarlyExitCluster;
+    if (a->B < kEarlyExitSmallB && !rejection) {
+      G = a->B < 16 ? 16 : 8;
+    } else if (a->B < kEarlyExitSmallB) {
+      for (const int cand : {16, 12, 8}) {
+        const EarlyExitPlan pc = make_early_exit_plan(a->V, cand);
+        if (!pc.ok) continue;
+        L.G = cand;
+        L.vs = pc.vs;
+        if (early_exit_max_clusters(L) >= a->B) { G = cand; break; }
+      }
+    }
+  }
+  EarlyExitPlan ep = make_early_exit_plan(a->V, G);
+  if (!ep.ok && g_cluster == 0) ep = make_early_exit_plan(a->V, 16);   // slices of 4 too long
+  if (!ep.ok) {
+    if (g_verify_path == 0) return false;
+    *st = PSPEC_ERR_UNSUPPORTED;
+    return true;
+  }
+  L.G = ep.G;
+  L.vs = ep.vs;
   // The last X sequences go to a second launch of wider clusters that starts as the first
   // launch's clusters finish (programmatic dependent launch): the sequences that start last
   // then run their chains of rows twice as wide, which shortens the launch's tail.
@@ -160,6 +190,7 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   if (rejection && g_split_event) cudaEventRecord(g_split_event, stream);
   t_last_launches = launches;
   t_last_path = 2;
+  t_last_cluster = L.G;
   *st = PSPEC_OK;
   return true;
 }
@@ -446,10 +477,11 @@ const char* pspec_status_string(pspec_status s) {
 int pspec_last_launches(void) { return t_last_launches; }
 
 int pspec_last_verify_path(void) { return t_last_path; }
+int pspec_last_cluster_size(void) { return t_last_cluster; }
 
 void pspec_set_verify_path(int path) { g_verify_path = (path >= 1 && path <= 3) ? path : 0; }
 
-void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || G == 16) ? G : 0; }
+void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || G == 12 || G == 16) ? G : 0; }
 
 void pspec_set_step_fusion(int mode) { g_step_fusion = (mode == 1 || mode == 2) ? mode : 0; }
 void pspec_set_ee_stream(int mode) { g_ee_stream = (mode == 1 || mode == 2) ? mode : 0; }

@@ -62,7 +62,7 @@ struct EarlyExitLaunch {
   long long ld;
   pspec_dtype dtype;
   int rejection;         // 1: rejection rule, 0: greedy
-  int G;                 // CTAs per cluster (one cluster per sequence): 2, 4, 8 or 16
+  int G;                 // CTAs per cluster (one cluster per sequence): 2, 4, 8, 12 or 16
   int ring;              // 1: rows streamed through per-warp shared-memory stages (bulk copies)
   int seq0, nseq;        // this launch's sequences [seq0, seq0 + nseq) of the batch's B
   int pdl;               // split batch: 1 first launch (lets the second start as its CTAs
@@ -145,6 +145,9 @@ cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream, cuda
 cudaError_t launch_queue(const QueueLaunch& L, cudaStream_t stream);
 cudaError_t launch_build(const BuildLaunch& L, cudaStream_t stream);
 cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream);
+// Clusters of the variant L names (G, dtype, rule, fusion, streaming) that fit on the
+// current device at once; 0 when the query fails.  Cached per device and variant.
+int early_exit_max_clusters(const EarlyExitLaunch& L);
 cudaError_t launch_sample(const SampleLaunch& L, cudaStream_t stream);
 
 }  // namespace pspec

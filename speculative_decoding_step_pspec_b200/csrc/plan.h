@@ -28,9 +28,10 @@ constexpr int kResampleTargetCtas = kNumSMs * PSPEC_DRAW_CTAS_PER_SM;
 constexpr int kDrawTilesPerCta = 64;     // separate draw launch: at most 8 tiles per warp
 constexpr int kEarlyExitMinB = 64;       // automatic path: early exit from this many sequences
 constexpr int kEarlyExitCluster = 4;     // CTAs per sequence on the early-exit path
-// Below this many sequences the automatic cluster is 16 CTAs: with 4, a batch of 64 fills
-// only 256 CTA slots of ~900 (measured on B200, c64: 0.100 ms with 16 vs 0.140 ms with 4;
-// at 256 sequences 4 and 8 are within 5 % either way, at 1024 sequences 4 is best).
+// Below this many sequences the automatic cluster is wider than 4 CTAs (16, 12 or 8; see
+// the rule in api.cu): with 4, a batch of 64 fills only 256 CTA
+// slots of ~900 (measured on B200, c64: 0.100 ms with 16 vs 0.140 ms with 4; at 256
+// sequences 4 and 8 are within 5 % either way, at 1024 sequences 4 is best).
 constexpr int kEarlyExitSmallB = 128;
 constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this many sequences
 

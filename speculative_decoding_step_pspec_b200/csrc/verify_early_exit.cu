@@ -7,7 +7,7 @@
 // 60-80 % acceptance is well under half of the full sweep's bytes, and its outputs are
 // the full sweep's outputs.
 //
-// Design (one thread-block cluster of G CTAs per sequence, G = 2, 4, 8 or 16):
+// Design (one thread-block cluster of G CTAs per sequence, G = 2, 4, 8, 12 or 16):
 //   * position k = 0, 1, ...: each CTA streams its 1/G slice of target row k (and of draft
 //     row k for the rejection rule) with 16-byte loads, four vectors per row in flight per
 //     thread, and reduces it to (max, sum exp) or to its argmax;
@@ -660,8 +660,10 @@ cudaError_t ring_attributes(Kern kern, int bytes, std::atomic<unsigned long long
   return e;
 }
 
+// Launches the variant, or with max_clusters set only asks how many of its clusters can be
+// resident at once (cudaOccupancyMaxActiveClusters) and launches nothing.
 template <typename Tag, int G, bool kRej, bool kFuse, bool kRing>
-cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream) {
+cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream, int* max_clusters) {
   auto kern = ee_kernel<Tag, G, kRej, kFuse, kRing>;
   cudaError_t e = cudaSuccess;
   if (G > 8) {
@@ -675,7 +677,7 @@ cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((long long)L.nseq * G), 1, 1);
+  cfg.gridDim = dim3((unsigned)((long long)(L.nseq > 0 ? L.nseq : 1) * G), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = (size_t)dyn;
   cfg.stream = stream;
@@ -688,36 +690,61 @@ cudaError_t launch_ee(const EarlyExitLaunch& L, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = L.pdl == 2 ? 2 : 1;
+  if (max_clusters) return cudaOccupancyMaxActiveClusters(max_clusters, kern, &cfg);
   return cudaLaunchKernelEx(&cfg, kern, L);
 }
 
 template <int G, bool kRing>
-cudaError_t launch_ee_gr(const EarlyExitLaunch& L, cudaStream_t s) {
+cudaError_t launch_ee_gr(const EarlyExitLaunch& L, cudaStream_t s, int* m) {
   const bool bf = L.dtype == PSPEC_BF16;
   if (L.fuse_build) {
     if (L.rejection)
-      return bf ? launch_ee<BF16Tag, G, true, true, kRing>(L, s) : launch_ee<F32Tag, G, true, true, kRing>(L, s);
-    return bf ? launch_ee<BF16Tag, G, false, true, kRing>(L, s) : launch_ee<F32Tag, G, false, true, kRing>(L, s);
+      return bf ? launch_ee<BF16Tag, G, true, true, kRing>(L, s, m) : launch_ee<F32Tag, G, true, true, kRing>(L, s, m);
+    return bf ? launch_ee<BF16Tag, G, false, true, kRing>(L, s, m) : launch_ee<F32Tag, G, false, true, kRing>(L, s, m);
   }
   if (L.rejection)
-    return bf ? launch_ee<BF16Tag, G, true, false, kRing>(L, s) : launch_ee<F32Tag, G, true, false, kRing>(L, s);
-  return bf ? launch_ee<BF16Tag, G, false, false, kRing>(L, s) : launch_ee<F32Tag, G, false, false, kRing>(L, s);
+    return bf ? launch_ee<BF16Tag, G, true, false, kRing>(L, s, m) : launch_ee<F32Tag, G, true, false, kRing>(L, s, m);
+  return bf ? launch_ee<BF16Tag, G, false, false, kRing>(L, s, m) : launch_ee<F32Tag, G, false, false, kRing>(L, s, m);
 }
 
 template <int G>
-cudaError_t launch_ee_g(const EarlyExitLaunch& L, cudaStream_t s) {
-  return L.ring ? launch_ee_gr<G, true>(L, s) : launch_ee_gr<G, false>(L, s);
+cudaError_t launch_ee_g(const EarlyExitLaunch& L, cudaStream_t s, int* m) {
+  return L.ring ? launch_ee_gr<G, true>(L, s, m) : launch_ee_gr<G, false>(L, s, m);
+}
+
+cudaError_t dispatch_ee(const EarlyExitLaunch& L, cudaStream_t stream, int* m) {
+  switch (L.G) {
+    case 2: return launch_ee_g<2>(L, stream, m);
+    case 4: return launch_ee_g<4>(L, stream, m);
+    case 8: return launch_ee_g<8>(L, stream, m);
+    case 12: return launch_ee_g<12>(L, stream, m);
+    default: return launch_ee_g<16>(L, stream, m);
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream) {
-  switch (L.G) {
-    case 2: return launch_ee_g<2>(L, stream);
-    case 4: return launch_ee_g<4>(L, stream);
-    case 8: return launch_ee_g<8>(L, stream);
-    default: return launch_ee_g<16>(L, stream);
+  return dispatch_ee(L, stream, nullptr);
+}
+
+int early_exit_max_clusters(const EarlyExitLaunch& L) {
+  // cached per device and variant: 16 devices x 5 cluster sizes x dtype x rule x fusion x ring
+  static std::atomic<int> cache[16 * 5 * 16];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const int gi = L.G == 2 ? 0 : L.G == 4 ? 1 : L.G == 8 ? 2 : L.G == 12 ? 3 : 4;
+  const int idx = (((((dev & 15) * 5 + gi) * 2 + (L.dtype == PSPEC_BF16)) * 2 + (L.rejection != 0)) * 2 +
+                   (L.fuse_build != 0)) * 2 + (L.ring != 0);
+  const int c = cache[idx].load(std::memory_order_relaxed);
+  if (c > 0) return c - 1;
+  int n = 0;
+  if (dispatch_ee(L, nullptr, &n) != cudaSuccess) {
+    cudaGetLastError();                                       // a failed query is not sticky
+    return 0;
   }
+  cache[idx].store(n + 1, std::memory_order_relaxed);
+  return n;
 }
 
 }  // namespace pspec

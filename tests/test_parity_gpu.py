@@ -984,11 +984,11 @@ def test_early_exit_tail_split(X):
 
 
 @pytest.mark.parametrize("stream", [1, 2])
-@pytest.mark.parametrize("G", [2, 4, 8, 16])
+@pytest.mark.parametrize("G", [2, 4, 8, 12, 16])
 def test_early_exit_every_cluster_size(G, stream):
-    """The early-exit kernel with each cluster size (the automatic choice is 16 below 128
-    sequences, else 4) and both ways of streaming rows against the oracle, unfused and with
-    the step fused, K_i included."""
+    """The early-exit kernel with each cluster size (the automatic choice is 4 from 128
+    sequences on, wider below) and both ways of streaming rows against the oracle, unfused
+    and with the step fused, K_i included."""
     w = I.scaled(I.C64, B=40, V=40000, H=64)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
