@@ -47,6 +47,8 @@ def parse_args():
     p.add_argument("--cluster", type=int, default=0, help="early-exit cluster size (0 auto)")
     p.add_argument("--ee-stream", choices=["auto", "registers", "ring"], default="auto",
                    help="early-exit row streaming: registers or per-warp shared-memory rings")
+    p.add_argument("--fusion", choices=["auto", "always", "never"], default="auto",
+                   help="verify + build in one launch (early-exit path): pspec_set_step_fusion")
     p.add_argument("--tail", type=int, default=0,
                    help="early exit: sequences for the 8-CTA tail launch (0 auto, -1 never)")
     p.add_argument("--e2e-steps", type=int, default=3)
@@ -257,6 +259,7 @@ def run_pspec(args, rank, world, local_rank):
     ps.pspec_set_cluster_size(args.cluster)
     ps.pspec_set_ee_stream({"auto": 0, "registers": 1, "ring": 2}[args.ee_stream])
     ps.pspec_set_tail_split(args.tail)
+    ps.pspec_set_step_fusion({"auto": 0, "always": 1, "never": 2}[args.fusion])
     w, d = make_workload(args.workload, dev, rank, args.batch)
     rej = args.mode == "rejection"
     ws = ps.Workspace(w.B, w.K, w.V, rej, dev)
@@ -691,6 +694,7 @@ def run_depth_sweep(args, local_rank):
     ps.pspec_set_cluster_size(args.cluster)
     ps.pspec_set_ee_stream({"auto": 0, "registers": 1, "ring": 2}[args.ee_stream])
     ps.pspec_set_tail_split(args.tail)
+    ps.pspec_set_step_fusion({"auto": 0, "always": 1, "never": 2}[args.fusion])
     hbm, _ = peaks()
     points = []
     ks = [int(x) for x in args.depth_k.split(",")] if args.depth_k else I.DEPTH_K
