@@ -386,6 +386,15 @@ PSPEC_API void pspec_set_ee_stream(int mode);
    pspec_last_launches then reports 2.  Process-wide. */
 PSPEC_API void pspec_set_tail_split(int n);
 
+/* Tests of the error path: every bounded wait in the kernels (the work queue's waits for
+   published work, the shared-memory ring's stage waits) gives up after `polls` polls
+   instead of its default (about a second of polling); 0 restores the defaults.  With a
+   small value, waits that would have succeeded give up: the call sets PSPEC_DEVERR_TIMEOUT,
+   its outputs are undefined, and the context stays usable (the kernels still end, the
+   work queue resets its state, and copies already requested land before their CTA ends).
+   Process-wide. */
+PSPEC_API void pspec_set_wait_limit(unsigned long long polls);
+
 /* Tuning: fusion of the two halves of pspec_step_* into one launch (early-exit path only):
    0 automatic (fewer than 256 sequences), 1 always, 2 never.  Process-wide. */
 PSPEC_API void pspec_set_step_fusion(int mode);

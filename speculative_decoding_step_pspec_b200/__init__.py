@@ -16,6 +16,7 @@ from ._binding import (  # noqa: F401
 from ._binding import pspec_sample_drafts, pspec_sample_workspace_bytes  # noqa: F401
 from ._binding import pspec_set_step_fusion, pspec_step_greedy, pspec_step_rejection  # noqa: F401
 from ._binding import pspec_last_cluster_size, pspec_set_ee_stream, pspec_set_tail_split  # noqa: F401
+from ._binding import pspec_set_wait_limit  # noqa: F401
 from .api import (  # noqa: F401
     Workspace, build_draft_batch, sample_drafts, step, verify_greedy, verify_rejection,
 )

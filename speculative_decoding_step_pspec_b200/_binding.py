@@ -32,6 +32,7 @@ EXPORTED = (
     "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
     "pspec_step_greedy", "pspec_step_rejection", "pspec_set_step_fusion",
     "pspec_set_ee_stream", "pspec_set_tail_split", "pspec_last_cluster_size",
+    "pspec_set_wait_limit",
 )
 
 
@@ -107,6 +108,8 @@ def _load():
     lib.pspec_set_ee_stream.restype = None
     lib.pspec_set_tail_split.argtypes = [_I]
     lib.pspec_set_tail_split.restype = None
+    lib.pspec_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+    lib.pspec_set_wait_limit.restype = None
     lib.pspec_set_cluster_size.argtypes = [_I]
     lib.pspec_set_cluster_size.restype = None
     lib.pspec_last_verify_path.argtypes = []
@@ -209,6 +212,12 @@ def pspec_set_ee_stream(mode: int) -> None:
 def pspec_set_tail_split(n: int) -> None:
     """Early exit: sequences given to a second launch of 8-CTA clusters (0 auto, -1 never)."""
     LIB.pspec_set_tail_split(int(n))
+
+
+def pspec_set_wait_limit(polls: int) -> None:
+    """Polls before a bounded wait in the kernels gives up (0: the defaults); for tests of
+    the PSPEC_DEVERR_TIMEOUT path."""
+    LIB.pspec_set_wait_limit(int(polls))
 
 
 def pspec_set_segment_elems(elems: int) -> None:

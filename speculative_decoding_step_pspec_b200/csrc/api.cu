@@ -20,6 +20,7 @@ int g_cluster = 0;              // early-exit cluster size; 0 = automatic
 int g_step_fusion = 0;          // 0 automatic, 1 always, 2 never
 int g_ee_stream = 0;            // early-exit streaming: 0 automatic, 1 registers, 2 ring
 int g_tail_split = 0;           // early-exit tail launch: 0 automatic, -1 never, n > 0 sequences
+unsigned long long g_wait_limit = 0;  // polls per bounded wait; 0 = the kernels' defaults
 thread_local int t_last_launches = 0;
 thread_local int t_last_path = 0;
 thread_local int t_last_cluster = 0;   // CTAs per cluster of the last early-exit launch
@@ -109,6 +110,8 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.rejection = rejection;
   L.ring = g_ee_stream == 2;
+  L.spin_limit = g_wait_limit ? (unsigned)(g_wait_limit < (1ull << 21) ? g_wait_limit : (1ull << 21))
+                              : (1u << 21);
   L.target = a->target_logits;
   L.draft = a->draft_logits;
   L.draft_tokens = a->draft_tokens;
@@ -224,6 +227,7 @@ bool try_queue(const pspec_verify_args* a, bool rejection, void* workspace, size
   *st = check_workspace(workspace, bytes, p.bytes, a->B, &z);
   if (*st != PSPEC_OK) return true;
   QueueLaunch L{};
+  L.spin_limit = g_wait_limit ? g_wait_limit : (1ull << 20);
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.rejection = rejection;
   L.S = p.S; L.seg = p.seg;
@@ -486,6 +490,7 @@ void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || 
 void pspec_set_step_fusion(int mode) { g_step_fusion = (mode == 1 || mode == 2) ? mode : 0; }
 void pspec_set_ee_stream(int mode) { g_ee_stream = (mode == 1 || mode == 2) ? mode : 0; }
 void pspec_set_tail_split(int n) { g_tail_split = n < 0 ? -1 : n; }
+void pspec_set_wait_limit(unsigned long long polls) { g_wait_limit = polls; }
 
 void pspec_set_segment_elems(long long elems) { g_seg_override = elems > 0 ? elems : 0; }
 

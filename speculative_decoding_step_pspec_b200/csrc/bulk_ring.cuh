@@ -53,10 +53,11 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, unsign
       : "memory");
 }
 
-// Waits for the phase of parity `parity` to complete; false after kRingSpinLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+// Waits for the phase of parity `parity` to complete; false after `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity,
+                                          unsigned limit = kRingSpinLimit) {
   const uint32_t a = smem_addr(bar);
-  for (unsigned spin = 0; spin < kRingSpinLimit; ++spin) {
+  for (unsigned spin = 0; spin < limit; ++spin) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"

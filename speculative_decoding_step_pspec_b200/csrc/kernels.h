@@ -64,6 +64,7 @@ struct EarlyExitLaunch {
   int rejection;         // 1: rejection rule, 0: greedy
   int G;                 // CTAs per cluster (one cluster per sequence): 2, 4, 8, 12 or 16
   int ring;              // 1: rows streamed through per-warp shared-memory stages (bulk copies)
+  unsigned spin_limit;   // ring streaming: polls before a stage wait gives up
   int seq0, nseq;        // this launch's sequences [seq0, seq0 + nseq) of the batch's B
   int pdl;               // split batch: 1 first launch (lets the second start as its CTAs
                          // are placed), 2 second launch (its CTA 0 ends after the first grid)
@@ -130,6 +131,7 @@ struct QueueLaunch {
   void* part;            // workspace: 8-byte partials [B*R*S]
   void* seq;             // workspace: SeqInfo [B]
   double* tile_sums;     // workspace: [B*tiles]
+  unsigned long long spin_limit;  // polls before a wait gives up (PSPEC_DEVERR_TIMEOUT)
 };
 
 struct BuildLaunch {

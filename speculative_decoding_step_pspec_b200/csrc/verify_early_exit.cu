@@ -267,7 +267,8 @@ ee_kernel(const EarlyExitLaunch L) {
   const int wlo = min(n, warp * wper);
   const int wn = min(n, wlo + wper) - wlo;
   const int nch = (wn + SE - 1) / SE;
-  uint32_t gidx = 0;
+  uint32_t gidx = 0;                                          // chunks consumed
+  uint32_t issued = 0;                                        // chunks requested
   bool ring_ok = true;
   uint4* const ring = s_ring + (size_t)warp * kRingStages * kRows * kRingVecs;
   uint64_t* const bar = s_bar + (kRing ? warp * kRingStages : 0);
@@ -309,12 +310,14 @@ ee_kernel(const EarlyExitLaunch L) {
     MSAcc at = msacc_init(), aq = msacc_init();
     VI best{-INFINITY, kNoIndex};
     if constexpr (kRing) {
-      if (lane == 0 && ring_ok)
-        for (int c = 0; c < nch && c < kRingStages; ++c) issue(trow, qrow, has_q, c, gidx + (uint32_t)c);
+      if (ring_ok)
+        for (int c = 0; c < nch && c < kRingStages; ++c, ++issued)
+          if (lane == 0) issue(trow, qrow, has_q, c, gidx + (uint32_t)c);
       for (int c = 0; c < nch; ++c, ++gidx) {
         const int s = (int)(gidx % kRingStages);
         if (ring_ok) {
-          const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar[s], (gidx / kRingStages) & 1u));
+          const bool ok =
+              __all_sync(0xffffffffu, mbar_wait(&bar[s], (gidx / kRingStages) & 1u, L.spin_limit));
           if (!ok) {
             ring_ok = false;                             // no further copies from this warp
             if (lane == 0) set_err(L.err, PSPEC_DEVERR_TIMEOUT);
@@ -349,8 +352,10 @@ ee_kernel(const EarlyExitLaunch L) {
           }
         }
         __syncwarp();                                        // the stage is read: refill it
-        if (lane == 0 && ring_ok && c + kRingStages < nch)
-          issue(trow, qrow, has_q, c + kRingStages, gidx + kRingStages);
+        if (ring_ok && c + kRingStages < nch) {
+          if (lane == 0) issue(trow, qrow, has_q, c + kRingStages, gidx + kRingStages);
+          ++issued;
+        }
       }
     } else {                                                 // through registers
       const uint4* tv = reinterpret_cast<const uint4*>(trow + lo);
@@ -633,6 +638,14 @@ ee_kernel(const EarlyExitLaunch L) {
       if (L.residual_mass) L.residual_mass[i] = 0.f;
       s_tok = 0;
     }
+  }
+  if constexpr (kRing) {
+    // after a wait gave up, copies this warp requested may still be in flight: let them
+    // land (each stage has at most one outstanding request; full poll budget) before the
+    // CTA's shared memory is released
+    if (!ring_ok)
+      for (uint32_t u = issued > (uint32_t)kRingStages ? issued - kRingStages : 0; u < issued; ++u)
+        mbar_wait(&bar[u % kRingStages], (u / kRingStages) & 1u);
   }
   cluster.sync();                                            // D: no remote reads after exit
   if constexpr (kFuse) {                                     // the whole step in this launch

@@ -37,7 +37,6 @@ namespace pspec {
 namespace {
 
 enum : int { kQHeadS = 0, kQTailS = 1, kQHeadD = 2, kQTailD = 3, kQDone = 4, kQExit = 5 };
-constexpr unsigned long long kSpinLimit = 1ull << 20;   // ~0.1-1 s of polling
 constexpr int kItemShift = 5;                            // item = i << 5 | k (K <= 31)
 
 #ifndef PSPEC_QUEUE_MIN_BLOCKS
@@ -70,10 +69,10 @@ __device__ __forceinline__ int ld_volatile(const int* p) {
   return *reinterpret_cast<const volatile int*>(p);
 }
 
-// Wait (bounded) until a reserved queue slot is published; 0 on timeout.
-__device__ __forceinline__ int wait_published(const int* slot) {
+// Wait (bounded: `limit` polls) until a reserved queue slot is published; 0 on timeout.
+__device__ __forceinline__ int wait_published(const int* slot, unsigned long long limit) {
   int v = ld_volatile(slot);
-  for (unsigned long long w = 0; v == 0 && w < kSpinLimit; ++w) {
+  for (unsigned long long w = 0; v == 0 && w < limit; ++w) {
     __nanosleep(32);
     v = ld_volatile(slot);
   }
@@ -95,7 +94,7 @@ __device__ Work pick_work(const QueueLaunch& L, long long& held, long long& held
         if (held_d < 0) held_d = (long long)atomicAdd(ctr + kQHeadD, 1ull);
         const long long slot = held_d / L.C;
         if ((unsigned long long)slot < ld_volatile(ctr + kQTailD)) {
-          const int v = wait_published(zcol(L.draws, slot));
+          const int v = wait_published(zcol(L.draws, slot), L.spin_limit);
           if (v == 0) {
             set_err(L.err, PSPEC_DEVERR_TIMEOUT);
             return Work{kWorkExit, 0, 0, 0};
@@ -116,7 +115,7 @@ __device__ Work pick_work(const QueueLaunch& L, long long& held, long long& held
     }
     const long long slot = (held - init_units) / units_per_item;
     if ((unsigned long long)slot < ld_volatile(ctr + kQTailS)) {
-      const int v = wait_published(zitem(L.items, slot));
+      const int v = wait_published(zitem(L.items, slot), L.spin_limit);
       if (v == 0) {
         set_err(L.err, PSPEC_DEVERR_TIMEOUT);
         return Work{kWorkExit, 0, 0, 0};
@@ -131,7 +130,7 @@ __device__ Work pick_work(const QueueLaunch& L, long long& held, long long& held
         if (held_d < 0) held_d = (long long)atomicAdd(ctr + kQHeadD, 1ull);
         const long long dslot = held_d / L.C;
         if ((unsigned long long)dslot < ld_volatile(ctr + kQTailD)) {
-          const int v = wait_published(zcol(L.draws, dslot));
+          const int v = wait_published(zcol(L.draws, dslot), L.spin_limit);
           if (v == 0) {
             set_err(L.err, PSPEC_DEVERR_TIMEOUT);
             return Work{kWorkExit, 0, 0, 0};
@@ -144,7 +143,7 @@ __device__ Work pick_work(const QueueLaunch& L, long long& held, long long& held
       }
     }
     if (ld_volatile(ctr + kQDone) >= (unsigned long long)L.B) return Work{kWorkExit, 0, 0, 0};
-    if (spin >= kSpinLimit) {
+    if (spin >= L.spin_limit) {
       set_err(L.err, PSPEC_DEVERR_TIMEOUT);
       return Work{kWorkExit, 0, 0, 0};
     }

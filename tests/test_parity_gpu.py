@@ -949,6 +949,41 @@ def _step_check_k(target, draft, drafts, u, binp, path, expect_fused, klt):
     return v2, b2
 
 
+@pytest.mark.parametrize("path,stream,B", [(3, 0, 64), (2, 2, 64), (2, 2, 8)])
+def test_bounded_waits_give_up_and_context_survives(path, stream, B):
+    """With every bounded wait cut to one poll, the work queue (path 3) and the shared-memory
+    ring (early exit, stream 2) give up waits that would have succeeded: the call reports
+    PSPEC_DEVERR_TIMEOUT (the queue always does here; a ring wait may succeed at its first
+    poll, and then the outputs must be right), the kernels still end, and the next call on
+    the same context and workspace, with the default limits, gives the oracle's outputs."""
+    w = I.Workload("t", B, 5, 40000, 64, 16, torch.bfloat16, seed=B + path, sigma_t=2.0, sigma_d=0.5)
+    target, draft = I.logits(w, DEV)
+    sampled, _ = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    o = U.oracle_rejection(target, draft, sampled, u)
+    ws = ps.Workspace(w.B, w.K, w.V, True)
+    TIMEOUT = ps._binding.PSPEC_DEVERR_TIMEOUT
+    try:
+        ps.pspec_set_wait_limit(1)
+        with verify_path(path), ee_stream(stream):
+            r = ps.verify_rejection(target, draft, sampled, u, workspace=ws)
+            torch.cuda.synchronize()
+    finally:
+        ps.pspec_set_wait_limit(0)
+    err = r["err"].item()
+    assert err & ~TIMEOUT == 0, err
+    if path == 3:
+        assert err & TIMEOUT
+    if not err & TIMEOUT:
+        U.compare_rejection(r, o)
+    with verify_path(path), ee_stream(stream):
+        r2 = ps.verify_rejection(target, draft, sampled, u, workspace=ws)
+    torch.cuda.synchronize()
+    assert r2["err"].item() == 0
+    U.check_verify_invariants(r2, sampled, w.V)
+    U.compare_rejection(r2, o)
+
+
 @pytest.mark.parametrize("X", [1, 37, 150])
 def test_early_exit_tail_split(X):
     """The batch split over two early-exit launches (4-CTA clusters, then the last X
