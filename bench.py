@@ -398,7 +398,8 @@ def run_pspec(args, rank, world, local_rank):
     # both rules share the early-exit and work-queue kernels: their profiles are per rule
     prof_key = dom_kernel + ("_greedy" if not rej and dom_kernel in ("ee_kernel", "queue_kernel") else "")
     # a whole-step timing (fused launch, graph replay) is not one kernel's: no kernel traffic
-    traffic = None if whole else profiled_traffic(prof_key, args.workload, src_hash)
+    # (the profiles hold the named workloads' sizes: none for an overridden batch)
+    traffic = None if (whole or args.batch) else profiled_traffic(prof_key, args.workload, src_hash)
 
     line = {
         "metric": METRIC, "value": round(aggregate_value(K, world, elapsed_ms), 3), "unit": UNIT,
