@@ -42,8 +42,9 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["pspec", "reference"], default="pspec")
     p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
-    p.add_argument("--path", choices=["auto", "sweep", "early", "queue"], default="auto",
-                   help="verify path: automatic selection, full sweep, early exit, or work queue")
+    p.add_argument("--path", choices=["auto", "sweep", "early", "queue", "waves"], default="auto",
+                   help="verify path: automatic selection, full sweep, early exit, work queue, "
+                        "or position waves")
     p.add_argument("--cluster", type=int, default=0, help="early-exit cluster size (0 auto)")
     p.add_argument("--ee-stream", choices=["auto", "registers", "ring"], default="auto",
                    help="early-exit row streaming: registers or per-warp shared-memory rings")
@@ -255,7 +256,7 @@ def run_pspec(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3}[args.path])
+    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3, "waves": 4}[args.path])
     ps.pspec_set_cluster_size(args.cluster)
     ps.pspec_set_ee_stream({"auto": 0, "registers": 1, "ring": 2}[args.ee_stream])
     ps.pspec_set_tail_split(args.tail)
@@ -365,13 +366,18 @@ def run_pspec(args, rank, world, local_rank):
     draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if split else None
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
     acc = vout["accepted_len"].cpu().numpy()
-    early = path in (2, 3)                  # paths that read rows only up to a_i
+    early = path in (2, 3, 4)               # paths that read rows only up to a_i
     vbytes, bbytes = algorithmic_bytes(w, args.mode, acc, early)
     full_vbytes, _ = algorithmic_bytes(w, args.mode, acc, False)
     hbm, peak_src = peaks()
     ms_step = elapsed_ms / K
     step_gbs = (vbytes + bbytes) / (ms_step * 1e-3) / 1e9
-    if path == 3:
+    if path == 4:
+        dom_kernel = "wave_kernel"
+        src = ["speculative_decoding_step_pspec_b200/csrc/verify_waves.cu",
+               "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
+               "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
+    elif path == 3:
         dom_kernel = "queue_kernel"
         src = ["speculative_decoding_step_pspec_b200/csrc/verify_queue.cu",
                "speculative_decoding_step_pspec_b200/csrc/verify_draw.cuh",
@@ -411,7 +417,8 @@ def run_pspec(args, rank, world, local_rank):
                         f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
             "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)",
-                            3: "work queue (persistent, position order)"}[path],
+                            3: "work queue (persistent, position order)",
+                            4: "position waves (one launch per position, then the draw)"}[path],
             "step": ("one launch (verify + build fused)" if fused else "verify launches + build launch")
                     + (", CUDA graph replay" if graph is not None else ""),
             "l2": "inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9),
@@ -425,7 +432,8 @@ def run_pspec(args, rank, world, local_rank):
             dom_kernel + (" (verify + build, one launch)" if fused and lv == 1 else "")
             + (" (verify + build, two launches)" if fused and lv == 2 else "")
             + (" (two launches: 4-CTA clusters, then 8-CTA clusters for the last sequences)"
-               if early and lv == 2 and not fused else "")
+               if path == 2 and lv == 2 and not fused else "")
+            + (f" ({lv - 1} wave launches + the draw launch)" if path == 4 else "")
             + (" (CUDA graph replay of the step)" if graph is not None else ""): round(dom_ms, 5),
             **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if draw_ms else {}),
             **({} if whole else {"build_kernel": round(statistics.mean(build_ms), 5)}),
@@ -691,7 +699,7 @@ def run_depth_sweep(args, local_rank):
     from speculative_decoding_step_pspec_b200 import inputs as I
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3}[args.path])
+    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3, "waves": 4}[args.path])
     ps.pspec_set_cluster_size(args.cluster)
     ps.pspec_set_ee_stream({"auto": 0, "registers": 1, "ring": 2}[args.ee_stream])
     ps.pspec_set_tail_split(args.tail)

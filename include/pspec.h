@@ -354,6 +354,14 @@ PSPEC_API int pspec_last_launches(void);
      pspec_verify_workspace_bytes).  Any V, ld and element alignment.  Every wait in that
      kernel is bounded: when one runs out it sets PSPEC_DEVERR_TIMEOUT, the outputs are
      undefined, and the kernel clears the queue state before it ends.
+   4 always position waves for the rejection rule (the greedy rule then takes path 2): one
+     launch per position k = 0..K over the sequences still undecided at k (the first all
+     of them, the others the list the previous wave appended), each CTA sweeping segments
+     of target row k and draft row k into (max, sum exp) partials and the CTA completing a
+     sequence applying the rule at k, then the full sweep's draw launch; K+2 launches
+     chained with programmatic dependent launch (PSPEC_ERR_UNSUPPORTED with a per-row
+     diagnostic requested, PSPEC_ERR_WORKSPACE when the workspace is smaller than
+     pspec_verify_workspace_bytes).  Any V, ld and element alignment.
    All paths give the same outputs; they differ in which rows they read. */
 PSPEC_API void pspec_set_verify_path(int path);
 

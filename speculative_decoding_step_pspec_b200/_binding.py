@@ -195,7 +195,7 @@ def pspec_last_cluster_size() -> int:
 
 
 def pspec_set_verify_path(path: int) -> None:
-    """0 automatic, 1 full sweep, 2 early exit, 3 work queue (see include/pspec.h)."""
+    """0 automatic, 1 full sweep, 2 early exit, 3 work queue, 4 position waves (see include/pspec.h)."""
     LIB.pspec_set_verify_path(int(path))
 
 

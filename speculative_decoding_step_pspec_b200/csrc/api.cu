@@ -15,7 +15,7 @@ using namespace pspec;
 
 long long g_seg_override = 0;   // 0 = automatic segment length
 cudaEvent_t g_split_event = nullptr;
-int g_verify_path = 0;          // 0 automatic, 1 full sweep, 2 early exit, 3 work queue
+int g_verify_path = 0;          // 0 automatic, 1 sweep, 2 early exit, 3 queue, 4 waves
 int g_cluster = 0;              // early-exit cluster size; 0 = automatic
 int g_step_fusion = 0;          // 0 automatic, 1 always, 2 never
 int g_ee_stream = 0;            // early-exit streaming: 0 automatic, 1 registers, 2 ring
@@ -208,6 +208,62 @@ pspec_status check_workspace(void* ws, size_t bytes, size_t scratch, long long B
   return PSPEC_OK;
 }
 
+// The position-wave path (rejection rule: K+1 wave launches and the draw launch), when
+// forced.  Returns true and sets *st when it handled the call.
+bool try_waves(const pspec_verify_args* a, void* workspace, size_t bytes, cudaStream_t stream,
+               pspec_status* st) {
+  if (g_verify_path != 4) return false;
+  const bool diagnostics = a->target_lse || a->draft_lse || a->p_at_draft || a->q_at_draft;
+  if (diagnostics) {
+    *st = PSPEC_ERR_UNSUPPORTED;              // rows after a_i are never read on this path
+    return true;
+  }
+  const WavePlan p = make_wave_plan(a->B, a->K, a->V);
+  ZeroArea z;
+  *st = check_workspace(workspace, bytes, p.bytes, a->B, &z);
+  if (*st != PSPEC_OK) return true;
+  char* ws = static_cast<char*>(workspace);
+  WaveLaunch W{};
+  W.B = a->B; W.K = a->K; W.V = a->V; W.ld = a->ld; W.dtype = a->dtype;
+  W.target_units = kWaveUnits;
+  W.S_max = p.S_max;
+  W.target = a->target_logits;
+  W.draft = a->draft_logits;
+  W.draft_tokens = a->draft_tokens;
+  W.uniforms = a->uniforms;
+  W.out_tokens = a->out_tokens;
+  W.accepted_len = a->accepted_len;
+  W.err = a->err;
+  W.k_len = a->k_len;
+  W.cnt = z.line0 + kZwSCnt;
+  W.wave_cnt = reinterpret_cast<unsigned*>(z.ctr);
+  W.lists = reinterpret_cast<int*>(ws + p.off_lists);
+  W.part = ws + p.off_part;
+  W.seq = ws + p.off_seq;
+  RejectionLaunch D{};                        // the draw launch over every row a_i
+  D.B = a->B; D.K = a->K; D.V = a->V; D.ld = a->ld; D.dtype = a->dtype;
+  D.tiles = p.draw.tiles; D.tiles_per_chunk = p.draw.tiles_per_chunk; D.C = p.draw.C;
+  D.target = a->target_logits;
+  D.draft = a->draft_logits;
+  D.uniforms = a->uniforms;
+  D.out_tokens = a->out_tokens;
+  D.bonus = a->bonus;
+  D.residual_mass = a->residual_mass;
+  D.err = a->err;
+  D.k_len = a->k_len;
+  D.cnt2 = z.line0 + kZwSCnt2;
+  D.seq = W.seq;
+  D.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
+  if (launch_waves(W, stream) != cudaSuccess || launch_rejection_draw(D, stream) != cudaSuccess) {
+    *st = PSPEC_ERR_CUDA;
+    return true;
+  }
+  t_last_launches = a->K + 2;
+  t_last_path = 4;
+  *st = PSPEC_OK;
+  return true;
+}
+
 // The work-queue path (one persistent launch), when forced.  Returns true and sets *st
 // when it handled the call.
 bool try_queue(const pspec_verify_args* a, bool rejection, void* workspace, size_t bytes,
@@ -262,15 +318,24 @@ bool try_queue(const pspec_verify_args* a, bool rejection, void* workspace, size
   return true;
 }
 
+// Scratch the verify calls need below the zero area: the largest of the paths' plans, so
+// that a workspace of pspec_verify_workspace_bytes serves every path and every call checks
+// against the one size that function reports.
+size_t verify_scratch_bytes(int B, int K, int V, int rejection) {
+  const size_t sweep = align256(make_verify_plan(B, K, V, rejection, g_seg_override).bytes);
+  const size_t queue = align256(make_queue_plan(B, K, V, rejection).bytes);
+  const size_t waves = rejection ? align256(make_wave_plan(B, K, V).bytes) : 0;
+  size_t m = sweep > queue ? sweep : queue;
+  return m > waves ? m : waves;
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection) {
   if (B < 0 || K < 1 || K > PSPEC_MAX_K || V < 1) return 0;
-  const size_t sweep = align256(make_verify_plan(B, K, V, rejection, g_seg_override).bytes);
-  const size_t queue = align256(make_queue_plan(B, K, V, rejection).bytes);
-  return (sweep > queue ? sweep : queue) + zero_area_bytes(B);
+  return verify_scratch_bytes(B, K, V, rejection) + zero_area_bytes(B);
 }
 
 }  // extern "C"
@@ -288,7 +353,7 @@ pspec_status verify_greedy_impl(const pspec_verify_args* a, void* workspace,
   if (a->B == 0) { t_last_launches = 0; return st; }
   const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 0, g_seg_override);
   ZeroArea z;
-  st = check_workspace(workspace, workspace_bytes, p.bytes, a->B, &z);
+  st = check_workspace(workspace, workspace_bytes, verify_scratch_bytes(a->B, a->K, a->V, 0), a->B, &z);
   if (st != PSPEC_OK) return st;
   if (try_queue(a, false, workspace, workspace_bytes, stream, &st)) return st;
   if (try_early_exit(a, false, stream, &st, fuse)) {
@@ -325,9 +390,10 @@ pspec_status verify_rejection_impl(const pspec_verify_args* a, void* workspace,
   if (a->B == 0) { t_last_launches = 0; return st; }
   const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 1, g_seg_override);
   ZeroArea z;
-  st = check_workspace(workspace, workspace_bytes, p.bytes, a->B, &z);
+  st = check_workspace(workspace, workspace_bytes, verify_scratch_bytes(a->B, a->K, a->V, 1), a->B, &z);
   if (st != PSPEC_OK) return st;
   if (try_queue(a, true, workspace, workspace_bytes, stream, &st)) return st;
+  if (try_waves(a, workspace, workspace_bytes, stream, &st)) return st;
   if (try_early_exit(a, true, stream, &st, fuse)) {
     *fused = fuse != nullptr && st == PSPEC_OK;
     return st;
@@ -483,7 +549,7 @@ int pspec_last_launches(void) { return t_last_launches; }
 int pspec_last_verify_path(void) { return t_last_path; }
 int pspec_last_cluster_size(void) { return t_last_cluster; }
 
-void pspec_set_verify_path(int path) { g_verify_path = (path >= 1 && path <= 3) ? path : 0; }
+void pspec_set_verify_path(int path) { g_verify_path = (path >= 1 && path <= 4) ? path : 0; }
 
 void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || G == 12 || G == 16) ? G : 0; }
 

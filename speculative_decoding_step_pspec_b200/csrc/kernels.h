@@ -141,10 +141,36 @@ struct BuildLaunch {
   int hid_rows;          // rows the hidden role inspects: T_in + B*(K-1)
 };
 
+// Position waves (rejection rule): one launch per position k = 0..K over the sequences
+// still undecided, then the sweep's draw launch over every sequence's row a_i.
+struct WaveLaunch {
+  int B, K, V;
+  long long ld;
+  pspec_dtype dtype;
+  long long target_units;  // units (sequence, row, segment) a wave aims for
+  long long S_max;         // segments per row at most (the partials' stride)
+  const void* target;
+  const void* draft;
+  const int32_t* draft_tokens;
+  const float* uniforms;
+  int32_t* out_tokens;
+  int32_t* accepted_len;
+  int32_t* err;
+  const int32_t* k_len;  // optional per-sequence draft counts
+  int* cnt;              // zero area: per-sequence unit ticket column (zcol)
+  unsigned* wave_cnt;    // zero area: K+2 words: sequences appended to wave k, exit ticket
+  int* lists;            // workspace: [(K+1)*B] sequence lists of the waves
+  void* part;            // workspace: RejPart [B*2*S_max]
+  void* seq;             // workspace: SeqInfo [B]
+};
+
 cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream);
 // split_event (may be null) is recorded between the statistics sweep and the draw.
 cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream, cudaEvent_t split_event);
 cudaError_t launch_queue(const QueueLaunch& L, cudaStream_t stream);
+cudaError_t launch_waves(const WaveLaunch& L, cudaStream_t stream);
+// The sweep's draw launch alone (reads SeqInfo, writes the emitted token and bonus).
+cudaError_t launch_rejection_draw(const RejectionLaunch& L, cudaStream_t stream);
 cudaError_t launch_build(const BuildLaunch& L, cudaStream_t stream);
 cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream);
 // Clusters of the variant L names (G, dtype, rule, fusion, streaming) that fit on the

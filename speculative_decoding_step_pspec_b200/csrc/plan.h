@@ -204,6 +204,38 @@ inline EarlyExitPlan make_early_exit_plan(int V, int G) {
   return p;
 }
 
+// Position waves: per wave about kWaveUnits units (two rounds of the resident CTAs), each
+// a segment of at least kWaveSegMin elements of one row.
+#ifndef PSPEC_WAVE_UNITS_PER_SM
+#define PSPEC_WAVE_UNITS_PER_SM 16
+#endif
+constexpr long long kWaveUnits = (long long)kNumSMs * PSPEC_WAVE_UNITS_PER_SM;
+constexpr long long kWaveSegMin = 8192;
+
+struct WavePlan {
+  long long S_max;
+  VerifyPlan draw;        // the sweep's draw launch configuration (tiles, C)
+  size_t off_part, off_seq, off_tiles, off_lists, bytes;
+};
+
+inline WavePlan make_wave_plan(int B, int K, int V) {
+  WavePlan p{};
+  p.S_max = (V + kWaveSegMin - 1) / kWaveSegMin;
+  if (p.S_max < 1) p.S_max = 1;
+  p.draw = make_verify_plan(B, K, V, 1, 0);
+  size_t off = 0;
+  p.off_part = off;
+  off = align256(off + sizeof(RejPart) * (size_t)B * 2 * (size_t)p.S_max);
+  p.off_seq = off;
+  off = align256(off + sizeof(SeqInfo) * (size_t)B);
+  p.off_tiles = off;
+  off = align256(off + sizeof(double) * (size_t)B * p.draw.tiles);
+  p.off_lists = off;
+  off = align256(off + sizeof(int) * (size_t)B * (K + 1));
+  p.bytes = off;
+  return p;
+}
+
 // Work-queue verify: units are segments of about kQueueSeg elements of one row of one
 // (sequence, position) item, draws are cut into units of kQueueDrawTiles warp tiles.
 #ifndef PSPEC_QUEUE_SEG

@@ -26,8 +26,8 @@ def _sample(B, n, seed):
 
 
 class verify_path:
-    """Force the full sweep (1), the early-exit path (2) or the work-queue path (3) inside a
-    with-block."""
+    """Force the full sweep (1), the early-exit path (2), the work-queue path (3) or the
+    position waves (4) inside a with-block."""
 
     def __init__(self, path):
         self.path = path
@@ -89,17 +89,22 @@ def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True)
     U.compare_greedy(gr, og, seqs)
     orj = U.oracle_rejection(target, draft, sampled, u, seqs)
     U.compare_rejection(rj, orj, seqs)
-    # early exit (both ways of streaming rows) where its shape rules allow; queue always
-    for path, stream in ((2, 1), (2, 2), (3, 0)):
-        if path == 2 and not early_exit_allowed(target):
+    # early exit (both ways of streaming rows) where its shape rules allow; the work queue
+    # and the position waves always (the waves are the rejection rule's: the greedy rule
+    # then takes the early exit, where it can)
+    K = target.shape[1] - 1
+    for path, stream in ((2, 1), (2, 2), (3, 0), (4, 0)):
+        if path in (2, 4) and not early_exit_allowed(target):
             continue
         with verify_path(path), ee_stream(stream):
+            gpath = 2 if path == 4 else path
             # the early-exit path may hand the batch's last sequences to a second launch
-            ok_launches = (1, 2) if path == 2 else (1,)
             ge = ps.verify_greedy(target, greedy_drafts)
-            assert ps.pspec_last_launches() in ok_launches and ps.pspec_last_verify_path() == path
+            assert ps.pspec_last_launches() in ((1, 2) if gpath == 2 else (1,))
+            assert ps.pspec_last_verify_path() == gpath
             re = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
-            assert ps.pspec_last_launches() in ok_launches and ps.pspec_last_verify_path() == path
+            assert ps.pspec_last_launches() in {2: (1, 2), 3: (1,), 4: (K + 2,)}[path]
+            assert ps.pspec_last_verify_path() == path
         torch.cuda.synchronize()
         assert ge["err"].item() == 0 and re["err"].item() == 0, path
         U.check_verify_invariants(ge, greedy_drafts, V)
@@ -703,9 +708,11 @@ def test_step_c64_fused(rule):
     _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, 0, True)
 
 
-@pytest.mark.parametrize("path,fused", [(0, False), (1, False), (2, True), (3, False)])
+@pytest.mark.parametrize("path,fused", [(0, False), (1, False), (2, True), (3, False), (4, False)])
 @pytest.mark.parametrize("rule", ["greedy", "rejection"])
 def test_step_tiny_every_path(rule, path, fused):
+    if path == 4 and rule == "greedy":
+        fused = True                         # the greedy rule takes the fused early exit
     w = I.scaled(I.C64, B=5, V=4096, H=64)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
@@ -769,7 +776,8 @@ def test_step_b1024_fused(stream):
     U.compare_rejection(v, U.oracle_rejection(target, draft, sampled, u, seqs), seqs)
 
 
-@pytest.mark.parametrize("path,stream,tail", [(0, 1, 0), (0, 2, 0), (2, 1, 20), (1, 0, 0), (3, 0, 0)])
+@pytest.mark.parametrize("path,stream,tail", [(0, 1, 0), (0, 2, 0), (2, 1, 20), (1, 0, 0), (3, 0, 0),
+                                              (4, 0, 0)])
 def test_step_cuda_graph_replay(path, stream, tail):
     """One step captured in a CUDA graph and replayed with new uniforms and drafts copied
     into the captured buffers gives what the eager calls give for those inputs (the
@@ -835,7 +843,7 @@ def _k_len_case(B, K, V, seed, with_bad=False):
     return w, target, draft, sampled, greedy, u, klt
 
 
-@pytest.mark.parametrize("path", [1, 2, 3])
+@pytest.mark.parametrize("path", [1, 2, 3, 4])
 def test_k_len_verify_every_path(path):
     """Per-sequence draft counts on every path against the oracle (reading R14): counts
     0..K, -1 in the unused draft slots (no range error), out-of-range counts clamped with
