@@ -9,21 +9,27 @@
 //
 // Design (one thread-block cluster of G CTAs per sequence, G = 2, 4, 8, 12 or 16):
 //   * position k = 0, 1, ...: each CTA streams its 1/G slice of target row k (and of draft
-//     row k for the rejection rule) with 16-byte loads, four vectors per row in flight per
-//     thread, and reduces it to (max, sum exp) or to its argmax;
+//     row k for the rejection rule) with 16-byte loads -- two vectors per row in flight per
+//     thread at six CTAs per SM for the rejection rule, eight at four CTAs per SM for the
+//     greedy rule -- and reduces it to (max, sum exp) or to its argmax;
 //   * one cluster barrier; then every CTA reads the G slice partials through distributed
 //     shared memory in rank order and takes the same decision (u q < p, or draft ==
 //     argmax), so no second barrier or broadcast is needed (partials are double-buffered
 //     by position parity, so the next position cannot overwrite what a slower CTA reads);
 //   * rejection rule: at the stop position each CTA sums r = max(0, p - q) over
-//     256-element warp tiles of its slice, re-read right after the statistics pass
-//     (usually from L2); the slice totals are prefix-summed in rank order on every CTA, and
-//     the CTA whose slice holds u_K * Z rescans one tile.  When the draw is from the target
-//     row itself (all drafts passed), the slice totals follow from the statistics already
-//     merged and only the CTA holding u_K * Z goes over its slice.
-// Rows are held in registers, not shared memory, so that six CTAs fit per SM and about a
-// hundred sequences are in flight: measured on B200, caching each 100 KB slice pair in
-// shared memory (two CTAs per SM) left HBM idle between positions.
+//     256-element warp tiles of its slice, re-read right after the statistics pass (from
+//     L2 while the clusters in flight hold less than it, from HBM at large batches); the
+//     slice totals are prefix-summed in rank order on every CTA, and the CTA whose slice
+//     holds u_K * Z rescans one tile.  When the draw is from the target row itself (all
+//     drafts passed), the slice totals follow from the statistics already merged and only
+//     the CTA holding u_K * Z goes over its slice.
+// Rows are held in registers, not shared memory, so that six CTAs fit per SM and about 220
+// sequences are in flight: measured on B200, caching each 100 KB slice pair in shared
+// memory (two CTAs per SM) left HBM idle between positions, and streaming through per-warp
+// rings of bulk copies (kRing, an option) was slower than registers at every batch tried.
+// A large batch may be split over two launches of this kernel (seq0, nseq): the last
+// sequences go to wider clusters queued with programmatic dependent launch, which shortens
+// the end of the launch, where the last sequences' chains of positions run alone.
 #include <cooperative_groups.h>
 
 #include <atomic>
