@@ -47,6 +47,32 @@ def test_status_strings_and_launch_counts():
     ps.pspec_set_verify_path(0)
 
 
+def test_tuning_setters_and_queries():
+    """Every process-wide tuning setter takes its valid values and falls back to the
+    automatic choice on others (setters only: nothing launches); the last-call queries start
+    at zero on a thread that made no call."""
+    assert ps.pspec_last_verify_path() == 0 and ps.pspec_last_cluster_size() == 0
+    try:
+        for path in (1, 2, 3, 4, 9, -1):
+            ps.pspec_set_verify_path(path)
+        for G in (2, 4, 8, 12, 16, 5, 0):
+            ps.pspec_set_cluster_size(G)
+        for n in (96, 1, -1, -7, 0):
+            ps.pspec_set_tail_split(n)
+        for mode in (1, 2, 3, 4, 0):
+            ps.pspec_set_ee_stream(mode)
+            ps.pspec_set_step_fusion(mode)
+        for polls in (1, 1 << 40, 0):
+            ps.pspec_set_wait_limit(polls)
+    finally:
+        ps.pspec_set_verify_path(0)
+        ps.pspec_set_cluster_size(0)
+        ps.pspec_set_tail_split(0)
+        ps.pspec_set_ee_stream(0)
+        ps.pspec_set_step_fusion(0)
+        ps.pspec_set_wait_limit(0)
+
+
 def test_workspace_sizes():
     f = ps.pspec_verify_workspace_bytes
     assert f(0, 7, 1000, True) > 0 or f(0, 7, 1000, True) == 0
@@ -59,6 +85,8 @@ def test_workspace_sizes():
             assert n % 256 == 0 and n >= prev
             prev = n
     assert f(1024, 7, 201088, True) > f(1024, 7, 201088, False)
+    # one size serves every path: the position waves' lists and partials included
+    assert f(1024, 7, 201088, True) >= 1024 * 8 * 4 + 1024 * 2 * 25 * 8
 
 
 def _vargs(**kw):
