@@ -42,18 +42,18 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["pspec", "reference"], default="pspec")
     p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
-    p.add_argument("--path", choices=["auto", "sweep", "early", "queue", "waves"], default="auto",
-                   help="verify path: automatic selection, full sweep, early exit, work queue, "
-                        "or position waves")
+    p.add_argument("--path", choices=["auto", "sweep", "early"], default="auto",
+                   help="verify path: automatic selection, full sweep or early exit")
     p.add_argument("--cluster", type=int, default=0, help="early-exit cluster size (0 auto)")
-    p.add_argument("--ee-stream", choices=["auto", "registers", "ring"], default="auto",
-                   help="early-exit row streaming: registers or per-warp shared-memory rings")
     p.add_argument("--fusion", choices=["auto", "always", "never"], default="auto",
                    help="verify + build in one launch (early-exit path): pspec_set_step_fusion")
     p.add_argument("--tail", type=int, default=0,
                    help="early exit: sequences for the 8-CTA tail launch (0 auto, -1 never)")
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the other workloads (c1, c64, greedy b1024, depth sweep) that a "
+                        "one-GPU run adds to its JSON line")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=512,
                    help="sequences of the workload the CPU oracle baseline verifies")
@@ -201,6 +201,14 @@ def aggregate_value(steps: int, world: int, elapsed_ms: float) -> float:
     return world * steps / (elapsed_ms * 1e-3)
 
 
+def set_tuning(ps, args):
+    """The command line's tuning as the library's process-wide defaults."""
+    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2}[args.path])
+    ps.pspec_set_cluster_size(args.cluster)
+    ps.pspec_set_tail_split(args.tail)
+    ps.pspec_set_step_fusion({"auto": 0, "always": 1, "never": 2}[args.fusion])
+
+
 # ----------------------------------------------------------------------------- workload
 def make_workload(name, device, rank, batch=0):
     import torch
@@ -256,11 +264,7 @@ def run_pspec(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3, "waves": 4}[args.path])
-    ps.pspec_set_cluster_size(args.cluster)
-    ps.pspec_set_ee_stream({"auto": 0, "registers": 1, "ring": 2}[args.ee_stream])
-    ps.pspec_set_tail_split(args.tail)
-    ps.pspec_set_step_fusion({"auto": 0, "always": 1, "never": 2}[args.fusion])
+    set_tuning(ps, args)
     w, d = make_workload(args.workload, dev, rank, args.batch)
     rej = args.mode == "rejection"
     ws = ps.Workspace(w.B, w.K, w.V, rej, dev)
@@ -366,24 +370,13 @@ def run_pspec(args, rank, world, local_rank):
     draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if split else None
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
     acc = vout["accepted_len"].cpu().numpy()
-    early = path in (2, 3, 4)               # paths that read rows only up to a_i
+    early = path == 2                       # the path that reads rows only up to a_i
     vbytes, bbytes = algorithmic_bytes(w, args.mode, acc, early)
     full_vbytes, _ = algorithmic_bytes(w, args.mode, acc, False)
     hbm, peak_src = peaks()
     ms_step = elapsed_ms / K
     step_gbs = (vbytes + bbytes) / (ms_step * 1e-3) / 1e9
-    if path == 4:
-        dom_kernel = "wave_kernel"
-        src = ["speculative_decoding_step_pspec_b200/csrc/verify_waves.cu",
-               "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
-               "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
-    elif path == 3:
-        dom_kernel = "queue_kernel"
-        src = ["speculative_decoding_step_pspec_b200/csrc/verify_queue.cu",
-               "speculative_decoding_step_pspec_b200/csrc/verify_draw.cuh",
-               "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
-               "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
-    elif early:
+    if early:
         dom_kernel = "ee_kernel"
         src = ["speculative_decoding_step_pspec_b200/csrc/verify_early_exit.cu",
                "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
@@ -401,8 +394,8 @@ def run_pspec(args, rank, world, local_rank):
     whole = fused or graph is not None                     # one timed unit: the whole step
     dom_bytes = vbytes + bbytes if whole else vbytes       # a fused launch also builds
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    # both rules share the early-exit and work-queue kernels: their profiles are per rule
-    prof_key = dom_kernel + ("_greedy" if not rej and dom_kernel in ("ee_kernel", "queue_kernel") else "")
+    # both rules share the early-exit kernel: its profiles are per rule
+    prof_key = dom_kernel + ("_greedy" if not rej and dom_kernel == "ee_kernel" else "")
     # a whole-step timing (fused launch, graph replay) is not one kernel's: no kernel traffic
     # (the profiles hold the named workloads' sizes: none for an overridden batch)
     traffic = None if (whole or args.batch) else profiled_traffic(prof_key, args.workload, src_hash)
@@ -416,9 +409,7 @@ def run_pspec(args, rank, world, local_rank):
             "workload": f"{args.workload}{'' if not args.batch else ' (B overridden)'}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
                         f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
-            "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)",
-                            3: "work queue (persistent, position order)",
-                            4: "position waves (one launch per position, then the draw)"}[path],
+            "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)"}[path],
             "step": ("one launch (verify + build fused)" if fused else "verify launches + build launch")
                     + (", CUDA graph replay" if graph is not None else ""),
             "l2": "inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9),
@@ -431,9 +422,8 @@ def run_pspec(args, rank, world, local_rank):
         "kernels_ms": {
             dom_kernel + (" (verify + build, one launch)" if fused and lv == 1 else "")
             + (" (verify + build, two launches)" if fused and lv == 2 else "")
-            + (" (two launches: 4-CTA clusters, then 8-CTA clusters for the last sequences)"
+            + (" (two launches: the large-batch clusters, then wider ones for the last sequences)"
                if path == 2 and lv == 2 and not fused else "")
-            + (f" ({lv - 1} wave launches + the draw launch)" if path == 4 else "")
             + (" (CUDA graph replay of the step)" if graph is not None else ""): round(dom_ms, 5),
             **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if draw_ms else {}),
             **({} if whole else {"build_kernel": round(statistics.mean(build_ms), 5)}),
@@ -461,8 +451,141 @@ def run_pspec(args, rank, world, local_rank):
         line["e2e"] = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args, w, d, acc)
+    if world == 1 and not args.no_extra and not args.batch and args.workload == "b1024":
+        line["other_workloads"] = extra_workloads(args, w, d, dev, hbm)
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- other workloads
+def time_steps(fn, n, flush=None):
+    """Device time of each of n calls of fn (CUDA events on the current stream, one pair per
+    call); with `flush`, a buffer larger than L2 is rewritten before every call, outside the
+    timed pair."""
+    import torch
+    pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(n)]
+    for a, b in pairs:
+        if flush is not None:
+            flush.fill_(1)
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def step_summary(w, mode, ms_list, launches, path, acc, hbm, graph_ms=None):
+    """One workload's numbers: step time, algorithmic GB/s and fraction of the peak, launches
+    per step and the accepted-length histogram."""
+    import numpy as np
+    early = path == 2
+    vbytes, bbytes = algorithmic_bytes(w, mode, acc, early)
+    ms = statistics.median(ms_list)
+    gbs = (vbytes + bbytes) / (ms * 1e-3) / 1e9
+    out = {"workload": f"{w.name}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, bf16, {mode}",
+           "ms_per_step": round(ms, 5), "ms_mean": round(statistics.mean(ms_list), 5),
+           "step_per_s": round(1e3 / ms, 1), "achieved_gbs": round(gbs, 1),
+           "frac_of_peak": round(gbs / hbm, 4), "algorithmic_bytes": int(vbytes + bbytes),
+           "launches_per_step": launches,
+           "verify_path": {1: "full sweep", 2: "early exit"}[path],
+           "acceptance_rate": round(float(acc.sum()) / float(np.minimum(acc + 1, w.K).sum()), 4),
+           "histogram": np.bincount(acc, minlength=w.K + 1).tolist()}
+    if graph_ms is not None:
+        g = statistics.median(graph_ms)
+        out["graph_replay_ms_per_step"] = round(g, 5)
+        out["graph_replay_step_per_s"] = round(1e3 / g, 1)
+    return out
+
+
+def measure_workload(ps, w, inputs, mode, dev, hbm, n, flush, graph=True):
+    """Eager steps through the public step API (and, with `graph`, replays of one step
+    captured in a CUDA graph) on resident inputs, timed per step."""
+    import torch
+    rej = mode == "rejection"
+    bi = inputs["build"]
+    drafts = inputs["sampled"] if rej else inputs["greedy"]
+    ws = ps.Workspace(w.B, w.K, w.V, rej, dev)
+    vout = ps.api.verify_outputs(w.B, w.K, dev, False, rej)
+    bout = ps.api.build_outputs(w.B, w.K, w.H, bi["T_cap"], bi["verify_hidden"].dtype, dev)
+
+    def step():
+        ps.step(inputs["target"], drafts, bi, draft_logits=inputs["draft"] if rej else None,
+                uniforms=inputs["u"] if rej else None, workspace=ws, out=vout, build_out=bout)
+    for _ in range(3):
+        step()
+    launches, path = ps.pspec_last_launches(), ps.pspec_last_verify_path()
+    ms = time_steps(step, n, flush)
+    g_ms = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g):
+                step()
+        torch.cuda.current_stream().wait_stream(side)
+        g.replay()
+        torch.cuda.synchronize()
+        g_ms = time_steps(g.replay, n, flush)
+        del g
+    assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
+    acc = vout["accepted_len"].cpu().numpy()
+    return step_summary(w, mode, ms, launches, path, acc, hbm, g_ms)
+
+
+def extra_workloads(args, w_head, d_head, dev, hbm):
+    """The other configurations, measured after the headline in the same run: the greedy
+    rule on the large batch, the c=1 and c=64 shapes under both rules (eager and as CUDA
+    graph replays, L2 flushed before every step), the c=1 recipe's per-token acceptance
+    over 256 independent sequences, and the depth sweep (B=256, V=128256, K in 1,3,5,7,8,
+    draft noise 0.3, 0.7, 1.5; L2 flushed before every step)."""
+    import numpy as np
+    import torch
+
+    import speculative_decoding_step_pspec_b200 as ps
+    from speculative_decoding_step_pspec_b200 import inputs as I
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out["b1024_greedy"] = measure_workload(ps, w_head, d_head, "greedy", dev, hbm, 20, None,
+                                           graph=False)
+    out["b1024_greedy"]["l2"] = "inputs larger than L2; no flush"
+    for name in ("c1", "c64"):
+        w, d = make_workload(name, dev, 0)
+        for mode in ("rejection", "greedy"):
+            r = measure_workload(ps, w, d, mode, dev, hbm, 50, flush)
+            r["l2"] = "256 MB buffer rewritten before every step (outside the timed events)"
+            out[f"{name}_{mode}"] = r
+        del d
+    # the c=1 recipe's acceptance needs more than one sequence: 256 independent draws
+    wa = I.scaled(I.C1, B=256, seed=I.C1.seed + 77)
+    t, q = I.logits(wa, dev)
+    sampled, _ = I.draft_tokens(wa, q)
+    u = I.uniforms(wa, dev)
+    r = ps.verify_rejection(t, q, sampled, u)
+    acc = r["accepted_len"].cpu().numpy()
+    out["c1_acceptance"] = {
+        "sequences": wa.B, "rule": "rejection",
+        "per_token_rate": round(float(acc.sum()) / float(np.minimum(acc + 1, wa.K).sum()), 4),
+        "mean_accepted": round(float(acc.mean()), 3),
+        "histogram": np.bincount(acc, minlength=wa.K + 1).tolist(),
+        "stated_target": "roughly 0.65-0.75 per-token acceptance"}
+    del t, q, sampled, u, r
+    pts = []
+    for K in I.DEPTH_K:
+        for sigma in I.DEPTH_SIGMA:
+            wd = I.depth(K, sigma)
+            target, draft = I.logits(wd, dev)
+            sampled, greedy = I.draft_tokens(wd, draft)
+            dd = dict(target=target, draft=draft, sampled=sampled, greedy=greedy,
+                      u=I.uniforms(wd, dev), build=I.build_inputs(wd, dev, drafts=sampled))
+            p = measure_workload(ps, wd, dd, "rejection", dev, hbm, 20, flush, graph=False)
+            p.update({"K": K, "sigma": sigma})
+            pts.append(p)
+            del dd, target, draft, sampled, greedy
+            torch.cuda.empty_cache()
+    out["depth_sweep"] = {"l2": "256 MB buffer rewritten before every step", "points": pts}
+    return out
 
 
 def run_e2e(args, w, d, ps, dev, world):
@@ -699,11 +822,7 @@ def run_depth_sweep(args, local_rank):
     from speculative_decoding_step_pspec_b200 import inputs as I
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "queue": 3, "waves": 4}[args.path])
-    ps.pspec_set_cluster_size(args.cluster)
-    ps.pspec_set_ee_stream({"auto": 0, "registers": 1, "ring": 2}[args.ee_stream])
-    ps.pspec_set_tail_split(args.tail)
-    ps.pspec_set_step_fusion({"auto": 0, "always": 1, "never": 2}[args.fusion])
+    set_tuning(ps, args)
     hbm, _ = peaks()
     points = []
     ks = [int(x) for x in args.depth_k.split(",")] if args.depth_k else I.DEPTH_K
@@ -736,7 +855,7 @@ def run_depth_sweep(args, local_rank):
             ms = a.elapsed_time(b) / n
             assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
             acc = vout["accepted_len"].cpu().numpy()
-            early = path in (2, 3)
+            early = path == 2
             vbytes, bbytes = algorithmic_bytes(w, "rejection", acc, early)
             points.append({"K": K, "sigma": sigma, "ms_per_step": round(ms, 4),
                            "step_per_s": round(1e3 / ms, 1),

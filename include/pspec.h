@@ -71,8 +71,6 @@ typedef enum { PSPEC_F32 = 0, PSPEC_BF16 = 1 } pspec_dtype;
                                           negative block id: that row's slot is -1 */
 #define PSPEC_DEVERR_LAYOUT 0x8        /* qsl_in not an offset array, or a sequence with
                                           fewer than K+1 verify rows */
-#define PSPEC_DEVERR_TIMEOUT 0x10      /* a bounded wait for an asynchronous copy ran out
-                                          (outputs of that call are not valid) */
 #define PSPEC_DEVERR_KLEN_RANGE 0x20   /* k_len[i] outside [0, K]: clamped into it */
 
 /* Row kinds written to pspec_build_args.row_kind. */
@@ -84,6 +82,26 @@ typedef enum { PSPEC_F32 = 0, PSPEC_BF16 = 1 } pspec_dtype;
 
 #define PSPEC_PADDING_SLOT_ID (-1)
 #define PSPEC_MAX_K 31    /* the accept decisions of one sequence live in one 32-bit mask */
+
+/*
+ * Tuning of one call (the pages have no counterpart: these choose among equivalent
+ * implementations and never change a result).  A verify or step call whose
+ * pspec_verify_args.options is non-NULL runs with exactly these values; with NULL it runs
+ * with the process-wide defaults that the pspec_set_* functions below change.  The struct
+ * is read before the call returns.  0 in any field means the automatic choice; values
+ * outside the documented range read as 0.
+ */
+typedef struct {
+  int verify_path;           /* 0 automatic, 1 full sweep, 2 early exit (see
+                                pspec_set_verify_path) */
+  int cluster_size;          /* early exit: CTAs per cluster, 2, 4, 8, 12 or 16; 0 automatic */
+  int tail_split;            /* early exit: sequences of the second, wider launch; 0 automatic,
+                                -1 never, n > 0 that many (at most half the batch) */
+  int step_fusion;           /* pspec_step_*: 0 automatic, 1 always one launch, 2 never */
+  long long segment_elems;   /* full sweep: elements of one row per CTA (rounded up to a
+                                multiple of 8); 0 automatic.  Changes the workspace size:
+                                see pspec_verify_workspace_bytes_opt. */
+} pspec_options;
 
 /*
  * Verification arguments.
@@ -128,7 +146,9 @@ typedef struct {
                                   0..K_i-1, the bonus after K_i acceptances from target row
                                   K_i, the draw on uniform column K_i, only those drafts
                                   range-checked; rows past K_i are never needed (the
-                                  early-exit and work-queue paths never read them). */
+                                  early-exit path never reads them). */
+  const pspec_options *options; /* tuning of this call, or NULL for the process-wide
+                                  defaults (pspec_set_*) */
 } pspec_verify_args;
 
 /*
@@ -144,14 +164,20 @@ typedef struct {
  */
 PSPEC_API size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection);
 
+/* The same for calls made with `options` (NULL: the process-wide defaults); only
+   options->segment_elems changes the size. */
+PSPEC_API size_t pspec_verify_workspace_bytes_opt(int B, int K, int V, int rejection,
+                                                  const pspec_options *options);
+
 /*
  * Greedy verification ("any accepted prefix replaces the greedy path").
  * For each sequence i: g_k = argmax over the vocabulary of target row k (the lowest id
  * wins ties); a_i = the number of leading drafts with d_k == g_k; bonus = g_{a_i};
  * out_tokens = [d_0 .. d_{a_i-1}, bonus, -1 ...].  target_lse is written when non-NULL.
- * One kernel launch.  Full sweep: all B*(K+1) target rows, the last CTA of each sequence
- * combining its row partials.  Early exit (see pspec_set_verify_path): one cluster of
- * CTAs per sequence reads rows 0, 1, ... in order and stops at the first mismatch.  Errors: PSPEC_ERR_INVALID_ARG for bad
+ * One kernel launch (two when the early-exit path splits a large batch).  Full sweep: all
+ * B*(K+1) target rows, the last CTA of each sequence combining its row partials.  Early
+ * exit (see pspec_set_verify_path): one cluster of CTAs per sequence reads rows 0, 1, ...
+ * in order and stops at the first mismatch.  Errors: PSPEC_ERR_INVALID_ARG for bad
  * arguments; a draft token outside [0, V) is treated as a mismatch and sets
  * PSPEC_DEVERR_TOKEN_RANGE.
  */
@@ -169,10 +195,10 @@ PSPEC_API pspec_status pspec_verify_greedy(const pspec_verify_args *args, void *
  * residual sums to zero, the draw uses p_{a_i} itself).  Full sweep: two launches, a
  * vocabulary sweep over the 2K+1 rows of every sequence (softmax statistics and the
  * accept mask), then a chunked inverse-CDF draw over each sequence's row a_i.  Early exit
- * (see pspec_set_verify_path): one launch, one cluster of CTAs per sequence reading the
- * target and draft rows of positions 0, 1, ... into shared memory and stopping at the
- * first rejection, where it draws from the rows it holds.  A draft token outside
- * [0, V) has p = q = 0, is rejected, and sets PSPEC_DEVERR_TOKEN_RANGE.
+ * (see pspec_set_verify_path): one launch (two when a large batch is split), one cluster of
+ * CTAs per sequence streaming the target and draft rows of positions 0, 1, ... and stopping
+ * at the first rejection, where it re-reads that position's rows for the draw.  A draft
+ * token outside [0, V) has p = q = 0, is rejected, and sets PSPEC_DEVERR_TOKEN_RANGE.
  */
 PSPEC_API pspec_status pspec_verify_rejection(const pspec_verify_args *args, void *workspace,
                                     size_t workspace_bytes, cudaStream_t stream);
@@ -275,20 +301,25 @@ typedef struct {
  * library a workspace: a serving engine that reserves nearly all HBM for its KV cache at
  * start-up and gives memory out only through its own pool, a program that links only this
  * C library and has no device allocator, or a latency-critical path that cannot afford
- * cudaMalloc's implicit device synchronisation.  This entry point computes exactly what
- * pspec_verify_greedy computes (same kernel, same outputs) but keeps its scratch in a
+ * cudaMalloc's implicit device synchronisation.  This entry point gives the same outputs as
+ * pspec_verify_greedy (and runs the same argument checks), but always runs the full-sweep
+ * greedy kernel -- whatever path pspec_verify_greedy would choose -- with its scratch in a
  * fixed array of PSPEC_NOALLOC_SCRATCH_BYTES inside the library's device image, so neither
  * side calls cudaMalloc, cudaFree or any allocating routine.
  *   - Every GPU that loads the library holds that array until the process exits.
- *   - The first call on a device (with that device current) looks up the array's device
- *     address, once per device; make that first call before any stream capture.
+ *   - Every call looks the array's device address up for the current device and context
+ *     (cudaGetSymbolAddress, which allocates nothing), so the address stays right after
+ *     cudaDeviceReset and in any context the caller makes current.  The first call on a
+ *     device may load the library's device code there; make it before any stream capture.
  *   - All calls on a device share the array, which keeps the last call's contents: each
  *     call clears its tickets first (an asynchronous memset on `stream`), and calls whose
  *     executions overlap on the GPU race on it, so order them (one stream, or events).
- *   - It always uses the automatic segment length (pspec_set_segment_elems does not apply).
- *     A call needs pspec_verify_workspace_bytes(B, K, V, 0) bytes with the automatic
- *     segment length; above PSPEC_NOALLOC_SCRATCH_BYTES it returns PSPEC_ERR_UNSUPPORTED
- *     and launches nothing (B = 1024, K = 7, V = 201088 needs about 0.5 MiB).
+ *   - It always uses the automatic segment length (options and pspec_set_segment_elems do
+ *     not apply).  A call needs pspec_verify_workspace_bytes(B, K, V, 0) bytes with the
+ *     automatic segment length; above PSPEC_NOALLOC_SCRATCH_BYTES it returns
+ *     PSPEC_ERR_UNSUPPORTED and launches nothing (B = 1024, K = 7, V = 201088 needs about
+ *     0.5 MiB).
+ *   - pspec_last_launches() then reports 1 (0 for B = 0) and pspec_last_verify_path() 1.
  * Arguments, layout, outputs and device error bits are those of pspec_verify_greedy.
  */
 #define PSPEC_NOALLOC_SCRATCH_BYTES (4u << 20)
@@ -340,86 +371,60 @@ PSPEC_API const char *pspec_status_string(pspec_status status);
    issued (0 for an empty batch).  Used to count launches per decode step. */
 PSPEC_API int pspec_last_launches(void);
 
-/* Verify path selection (process-wide; not synchronised with calls on other threads):
-   0 (default) automatic -- the early-exit path when B >= 64, no per-row diagnostic is
-     requested (target_lse, draft_lse, p_at_draft, q_at_draft all NULL), V is a multiple
-     of 8 and the logits rows start on 16-byte boundaries; otherwise the full sweep;
+/* The functions below set the PROCESS-WIDE DEFAULTS of the tuning options: they apply to
+   every call whose arguments carry no pspec_options (options == NULL), and they are not
+   synchronised with calls running on other host threads -- a program that tunes calls on
+   several threads or streams passes its own pspec_options with each call instead.
+   pspec_get_options() copies the current defaults. */
+PSPEC_API void pspec_get_options(pspec_options *out);
+
+/* Verify path selection (default of pspec_options.verify_path):
+   0 (default) automatic -- the early-exit path when no per-row diagnostic is requested
+     (target_lse, draft_lse, p_at_draft, q_at_draft all NULL), V is a multiple of 8 and
+     the logits rows start on 16-byte boundaries; for the rejection rule only when B >= 64
+     or B <= 4 (in between, the full sweep measured as fast or faster); otherwise the full
+     sweep;
    1 always the full sweep;
-   2 always the early-exit path (PSPEC_ERR_UNSUPPORTED when the arguments do not allow it);
-   3 always the work-queue path: one persistent launch whose CTAs pull (sequence,
-     position) items cut into row segments from an on-device queue, in position order; the
-     CTA completing an item applies the rule and appends the next position, or the draw,
-     as new units (PSPEC_ERR_UNSUPPORTED with a per-row diagnostic requested,
-     PSPEC_ERR_WORKSPACE when the workspace is smaller than
-     pspec_verify_workspace_bytes).  Any V, ld and element alignment.  Every wait in that
-     kernel is bounded: when one runs out it sets PSPEC_DEVERR_TIMEOUT, the outputs are
-     undefined, and the kernel clears the queue state before it ends.
-   4 always position waves for the rejection rule (the greedy rule then takes path 2): one
-     launch per position k = 0..K over the sequences still undecided at k (the first all
-     of them, the others the list the previous wave appended), each CTA sweeping segments
-     of target row k and draft row k into (max, sum exp) partials and the CTA completing a
-     sequence applying the rule at k, then the full sweep's draw launch; K+2 launches
-     chained with programmatic dependent launch (PSPEC_ERR_UNSUPPORTED with a per-row
-     diagnostic requested, PSPEC_ERR_WORKSPACE when the workspace is smaller than
-     pspec_verify_workspace_bytes).  Any V, ld and element alignment.
-   All paths give the same outputs; they differ in which rows they read. */
+   2 always the early-exit path (PSPEC_ERR_UNSUPPORTED when the arguments do not allow it).
+   Both paths give the same outputs; they differ in which rows they read. */
 PSPEC_API void pspec_set_verify_path(int path);
 
-/* Tuning: CTAs per thread-block cluster on the early-exit path (2, 4, 8, 12 or 16; each
-   CTA streams a 1/G slice of a row); 0 restores the automatic choice: 4 from 128 sequences
-   on (16 when a slice of 4 would exceed 262144 elements); below, for the rejection rule
-   the widest of 16, 12 and 8 with which the clusters of all sequences fit on the GPU at
-   once (cudaOccupancyMaxActiveClusters, asked once per device and kernel variant), for the
-   greedy rule 8 (16 below 16 sequences).  Process-wide. */
+/* Tuning (default of pspec_options.cluster_size): CTAs per thread-block cluster on the
+   early-exit path (2, 4, 8, 12 or 16; each CTA streams a 1/G slice of a row); 0 restores
+   the automatic choice: a fixed width from 128 sequences on (16 when its slices would
+   exceed 262144 elements); below, for the rejection rule the widest of 16, 12 and 8 with
+   which the clusters of all sequences fit on the GPU at once
+   (cudaOccupancyMaxActiveClusters, asked once per device and kernel variant), for the
+   greedy rule 8 (16 below 16 sequences). */
 PSPEC_API void pspec_set_cluster_size(int G);
 
-/* Tuning: how the early-exit path streams logit rows.  0 automatic (= 1), 1 through
-   registers (16-byte loads, six CTAs per SM for the rejection rule), 2 through shared
-   memory: each warp owns a ring of stages filled by bulk asynchronous copies
-   (cp.async.bulk, completion counted on an mbarrier), so the bytes in flight do not depend
-   on the register budget; three CTAs per SM fit, and with fewer sequences in flight the
-   draw's re-read of its rows stays in L2.  On B200 mode 2 measured slower than mode 1 at
-   every batch size tried (fewer warps leave each position latency-bound).  Waits on the
-   stages are bounded: when one runs out, PSPEC_DEVERR_TIMEOUT is set and the outputs are
-   undefined.  Outputs are otherwise the same in both modes.  Process-wide. */
-PSPEC_API void pspec_set_ee_stream(int mode);
-
-/* Tuning: on the early-exit path with 4-CTA clusters, the last n sequences of the batch
-   are verified by a second launch of 8-CTA clusters, queued with programmatic dependent
-   launch so that it starts while the first launch drains (the CTAs of the first launch
-   release it when they are placed; CTA 0 of the second waits for the first grid before it
-   ends, so work queued later on the stream sees all outputs).  0 automatic (rejection
-   rule: min(96, B/2) sequences; greedy rule: one launch), -1 never, n > 0 that many
-   sequences (at most half the batch).  Outputs are the same either way;
-   pspec_last_launches then reports 2.  Process-wide. */
+/* Tuning (default of pspec_options.tail_split): on the early-exit path with the large-batch
+   cluster width, the last n sequences of the batch are verified by a second launch of
+   wider clusters, queued with programmatic dependent launch so that it starts while the
+   first launch drains (the CTAs of the first launch release it when they are placed; CTA 0
+   of the second waits for the first grid before it ends, so work queued later on the
+   stream sees all outputs).  0 automatic, -1 never, n > 0 that many sequences (at most
+   half the batch).  Outputs are the same either way; pspec_last_launches then reports 2. */
 PSPEC_API void pspec_set_tail_split(int n);
 
-/* Tests of the error path: every bounded wait in the kernels (the work queue's waits for
-   published work, the shared-memory ring's stage waits) gives up after `polls` polls
-   instead of its default (about a second of polling); 0 restores the defaults.  With a
-   small value, waits that would have succeeded give up: the call sets PSPEC_DEVERR_TIMEOUT,
-   its outputs are undefined, and the context stays usable (the kernels still end, the
-   work queue resets its state, and copies already requested land before their CTA ends).
-   Process-wide. */
-PSPEC_API void pspec_set_wait_limit(unsigned long long polls);
-
-/* Tuning: fusion of the two halves of pspec_step_* into one launch (early-exit path only):
-   0 automatic (fewer than 256 sequences), 1 always, 2 never.  Process-wide. */
+/* Tuning (default of pspec_options.step_fusion): fusion of the two halves of pspec_step_*
+   into one launch (early-exit path only): 0 automatic (fewer than 256 sequences), 1
+   always, 2 never. */
 PSPEC_API void pspec_set_step_fusion(int mode);
 
 /* The path the most recent successful verify call on this host thread took: 1 full sweep,
-   2 early exit, 3 work queue, 0 none yet. */
+   2 early exit, 0 none yet (or an empty batch). */
 PSPEC_API int pspec_last_verify_path(void);
 
 /* CTAs per cluster of the first (or only) launch of the last early-exit verify on this
    thread (the automatic choice or pspec_set_cluster_size's); 0 before any. */
 PSPEC_API int pspec_last_cluster_size(void);
 
-/* Tuning: force the verify sweeps' segment length (elements of one row handled by one
-   CTA; rounded up to a multiple of 8).  0 restores the automatic choice, which aims at
-   about 32 CTAs per SM and at most 65536 elements per CTA.  The segment length changes
-   pspec_verify_workspace_bytes, so size workspaces after setting it.  Process-wide; not
-   synchronised with calls running on other host threads. */
+/* Tuning (default of pspec_options.segment_elems): force the full sweep's segment length
+   (elements of one row handled by one CTA; rounded up to a multiple of 8).  0 restores the
+   automatic choice, which aims at about 32 CTAs per SM and at most 65536 elements per CTA.
+   The segment length changes pspec_verify_workspace_bytes, so size workspaces after
+   setting it. */
 PSPEC_API void pspec_set_segment_elems(long long elems);
 
 /* Profiling hook: while `event` is non-NULL, every pspec_verify_rejection call records it

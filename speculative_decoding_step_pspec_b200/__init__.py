@@ -3,20 +3,34 @@ with P-EAGLE parallel drafting on one B200 (sm_100a).
 
 libpspec.so (hand-written CUDA, C ABI in ``include/pspec.h``) does all the work; this
 package is its thin ctypes binding (``_binding``, the C names), allocation helpers
-(``api``) and the seeded synthetic input generators (``inputs``).  Importing it fails if
-the library has not been built: there is no CPU fallback.
+(``api``) and the seeded synthetic input generators (``inputs``).
+
+The binding is loaded on first use of any of its names (``ps.verify_greedy``,
+``ps.pspec_set_verify_path``, ``ps._binding`` ...), so that importing only the input
+generators (``from speculative_decoding_step_pspec_b200 import inputs``) does not map the
+library.  That first use raises ImportError when libpspec.so has not been built: there is
+no CPU fallback.
 """
-from ._binding import (  # noqa: F401
-    EXPORTED, LIB, PspecError, library_path, pspec_build_draft_batch,
-    pspec_last_launches, pspec_set_segment_elems, pspec_set_split_event,
-    pspec_set_verify_path, pspec_last_verify_path, pspec_set_cluster_size,
-    pspec_status_string,
-    pspec_verify_greedy, pspec_verify_rejection, pspec_verify_workspace_bytes,
-)
-from ._binding import pspec_sample_drafts, pspec_sample_workspace_bytes  # noqa: F401
-from ._binding import pspec_set_step_fusion, pspec_step_greedy, pspec_step_rejection  # noqa: F401
-from ._binding import pspec_last_cluster_size, pspec_set_ee_stream, pspec_set_tail_split  # noqa: F401
-from ._binding import pspec_set_wait_limit  # noqa: F401
-from .api import (  # noqa: F401
-    Workspace, build_draft_batch, sample_drafts, step, verify_greedy, verify_rejection,
-)
+from __future__ import annotations
+
+import importlib
+
+_API_NAMES = ("Workspace", "build_draft_batch", "sample_drafts", "step", "verify_greedy",
+              "verify_rejection")
+
+
+def __getattr__(name):
+    if name in ("_binding", "api"):
+        return importlib.import_module(f".{name}", __name__)
+    if name in _API_NAMES:
+        return getattr(importlib.import_module(".api", __name__), name)
+    if name in ("EXPORTED", "LIB", "PspecError", "library_path") or name.startswith("pspec_"):
+        b = importlib.import_module("._binding", __name__)
+        if hasattr(b, name):
+            return getattr(b, name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")
+
+
+def load():
+    """Map libpspec.so now (raises ImportError when it has not been built)."""
+    return importlib.import_module("._binding", __name__).LIB

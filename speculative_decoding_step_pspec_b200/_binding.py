@@ -18,7 +18,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpspec.s
 PSPEC_OK, PSPEC_ERR_INVALID_ARG, PSPEC_ERR_UNSUPPORTED, PSPEC_ERR_CUDA, PSPEC_ERR_WORKSPACE = range(5)
 PSPEC_F32, PSPEC_BF16 = 0, 1
 PSPEC_DEVERR_TOKEN_RANGE, PSPEC_DEVERR_ACCEPT_RANGE = 0x1, 0x2
-PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT, PSPEC_DEVERR_TIMEOUT = 0x4, 0x8, 0x10
+PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT = 0x4, 0x8
 PSPEC_DEVERR_KLEN_RANGE = 0x20
 PSPEC_ROW_CTX, PSPEC_ROW_NTP, PSPEC_ROW_MASK, PSPEC_ROW_REJ, PSPEC_ROW_PAD = range(5)
 PSPEC_PADDING_SLOT_ID = -1
@@ -31,8 +31,8 @@ EXPORTED = (
     "pspec_sample_workspace_bytes", "pspec_sample_drafts",
     "pspec_set_segment_elems", "pspec_set_split_event", "pspec_verify_greedy_noalloc",
     "pspec_step_greedy", "pspec_step_rejection", "pspec_set_step_fusion",
-    "pspec_set_ee_stream", "pspec_set_tail_split", "pspec_last_cluster_size",
-    "pspec_set_wait_limit",
+    "pspec_set_tail_split", "pspec_last_cluster_size", "pspec_get_options",
+    "pspec_verify_workspace_bytes_opt",
 )
 
 
@@ -46,6 +46,14 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 
 
+class pspec_options(ctypes.Structure):
+    """Tuning of one call (0 = automatic in every field); see include/pspec.h."""
+    _fields_ = [
+        ("verify_path", _I), ("cluster_size", _I), ("tail_split", _I), ("step_fusion", _I),
+        ("segment_elems", ctypes.c_longlong),
+    ]
+
+
 class pspec_verify_args(ctypes.Structure):
     _fields_ = [
         ("B", _I), ("K", _I), ("V", _I), ("ld", ctypes.c_longlong), ("dtype", _I),
@@ -53,6 +61,7 @@ class pspec_verify_args(ctypes.Structure):
         ("out_tokens", _P), ("accepted_len", _P), ("bonus", _P),
         ("target_lse", _P), ("draft_lse", _P), ("p_at_draft", _P), ("q_at_draft", _P),
         ("residual_mass", _P), ("err", _P), ("k_len", _P),
+        ("options", ctypes.POINTER(pspec_options)),
     ]
 
 
@@ -83,6 +92,10 @@ def _load():
     lib = ctypes.CDLL(_LIB_PATH)
     lib.pspec_verify_workspace_bytes.argtypes = [_I, _I, _I, _I]
     lib.pspec_verify_workspace_bytes.restype = ctypes.c_size_t
+    lib.pspec_verify_workspace_bytes_opt.argtypes = [_I, _I, _I, _I, ctypes.POINTER(pspec_options)]
+    lib.pspec_verify_workspace_bytes_opt.restype = ctypes.c_size_t
+    lib.pspec_get_options.argtypes = [ctypes.POINTER(pspec_options)]
+    lib.pspec_get_options.restype = None
     for fn in ("pspec_verify_greedy", "pspec_verify_rejection"):
         getattr(lib, fn).argtypes = [ctypes.POINTER(pspec_verify_args), _P, ctypes.c_size_t, _P]
         getattr(lib, fn).restype = _I
@@ -104,12 +117,8 @@ def _load():
     lib.pspec_set_verify_path.restype = None
     lib.pspec_set_step_fusion.argtypes = [_I]
     lib.pspec_set_step_fusion.restype = None
-    lib.pspec_set_ee_stream.argtypes = [_I]
-    lib.pspec_set_ee_stream.restype = None
     lib.pspec_set_tail_split.argtypes = [_I]
     lib.pspec_set_tail_split.restype = None
-    lib.pspec_set_wait_limit.argtypes = [ctypes.c_ulonglong]
-    lib.pspec_set_wait_limit.restype = None
     lib.pspec_set_cluster_size.argtypes = [_I]
     lib.pspec_set_cluster_size.restype = None
     lib.pspec_last_verify_path.argtypes = []
@@ -184,8 +193,7 @@ def pspec_set_cluster_size(G: int) -> None:
 
 
 def pspec_last_verify_path() -> int:
-    """1 full sweep, 2 early exit, 3 work queue: the path of the most recent verify call on
-    this thread."""
+    """1 full sweep, 2 early exit: the path of the most recent verify call on this thread."""
     return LIB.pspec_last_verify_path()
 
 
@@ -195,7 +203,7 @@ def pspec_last_cluster_size() -> int:
 
 
 def pspec_set_verify_path(path: int) -> None:
-    """0 automatic, 1 full sweep, 2 early exit, 3 work queue, 4 position waves (see include/pspec.h)."""
+    """Process-wide default: 0 automatic, 1 full sweep, 2 early exit (see include/pspec.h)."""
     LIB.pspec_set_verify_path(int(path))
 
 
@@ -204,20 +212,28 @@ def pspec_set_step_fusion(mode: int) -> None:
     LIB.pspec_set_step_fusion(int(mode))
 
 
-def pspec_set_ee_stream(mode: int) -> None:
-    """Early-exit row streaming: 0 automatic, 1 registers, 2 shared-memory ring (bulk copies)."""
-    LIB.pspec_set_ee_stream(int(mode))
-
-
 def pspec_set_tail_split(n: int) -> None:
-    """Early exit: sequences given to a second launch of 8-CTA clusters (0 auto, -1 never)."""
+    """Early exit: sequences given to a second, wider launch (0 auto, -1 never)."""
     LIB.pspec_set_tail_split(int(n))
 
 
-def pspec_set_wait_limit(polls: int) -> None:
-    """Polls before a bounded wait in the kernels gives up (0: the defaults); for tests of
-    the PSPEC_DEVERR_TIMEOUT path."""
-    LIB.pspec_set_wait_limit(int(polls))
+def pspec_get_options() -> dict:
+    """The process-wide defaults of the tuning options, as a dict."""
+    o = pspec_options()
+    LIB.pspec_get_options(ctypes.byref(o))
+    return {f: getattr(o, f) for f, _ in pspec_options._fields_}
+
+
+def make_options(options) -> "pspec_options | None":
+    """A pspec_options struct from a dict of its fields (missing fields 0), or None."""
+    if options is None or isinstance(options, pspec_options):
+        return options
+    o = pspec_options()
+    for k, v in dict(options).items():
+        if k not in {f for f, _ in pspec_options._fields_}:
+            raise KeyError(f"unknown pspec_options field {k!r}")
+        setattr(o, k, int(v))
+    return o
 
 
 def pspec_set_segment_elems(elems: int) -> None:
@@ -230,15 +246,22 @@ def pspec_set_split_event(event) -> None:
     LIB.pspec_set_split_event(None if event is None else event.cuda_event)
 
 
-def pspec_verify_workspace_bytes(B: int, K: int, V: int, rejection: bool) -> int:
-    return int(LIB.pspec_verify_workspace_bytes(int(B), int(K), int(V), int(bool(rejection))))
+def pspec_verify_workspace_bytes(B: int, K: int, V: int, rejection: bool, options=None) -> int:
+    if options is None:
+        return int(LIB.pspec_verify_workspace_bytes(int(B), int(K), int(V), int(bool(rejection))))
+    o = make_options(options)
+    return int(LIB.pspec_verify_workspace_bytes_opt(int(B), int(K), int(V), int(bool(rejection)),
+                                                    ctypes.byref(o)))
 
 
 def _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
                  accepted_len, bonus, err, target_lse, draft_lse, p_at_draft, q_at_draft,
-                 residual_mass, K, k_len=None):
+                 residual_mass, K, k_len=None, options=None):
     B, V, ld, dt = _logits_layout(target_logits, K + 1, "target_logits")
     a = pspec_verify_args()
+    o = make_options(options)
+    if o is not None:
+        a.options = ctypes.pointer(o)          # kept alive by the struct until the call
     a.B, a.K, a.V, a.ld, a.dtype = B, K, V, ld, dt
     a.target_logits = target_logits.data_ptr()
     if draft_logits is not None:
@@ -262,10 +285,10 @@ def _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens
 
 
 def pspec_verify_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len, bonus, err,
-                        workspace, target_lse=None, k_len=None, stream=None) -> None:
+                        workspace, target_lse=None, k_len=None, options=None, stream=None) -> None:
     K = int(target_logits.shape[1]) - 1
     a = _verify_args(target_logits, None, draft_tokens, None, out_tokens, accepted_len, bonus,
-                     err, target_lse, None, None, None, None, K, k_len)
+                     err, target_lse, None, None, None, None, K, k_len, options)
     st = LIB.pspec_verify_greedy(ctypes.byref(a), _ptr(workspace, torch.uint8, "workspace"),
                                  workspace.numel(), _stream(stream))
     if st != PSPEC_OK:
@@ -275,11 +298,11 @@ def pspec_verify_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len
 def pspec_verify_rejection(*, target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
                            accepted_len, bonus, err, workspace, target_lse=None, draft_lse=None,
                            p_at_draft=None, q_at_draft=None, residual_mass=None,
-                           k_len=None, stream=None) -> None:
+                           k_len=None, options=None, stream=None) -> None:
     K = int(target_logits.shape[1]) - 1
     a = _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
                      accepted_len, bonus, err, target_lse, draft_lse, p_at_draft, q_at_draft,
-                     residual_mass, K, k_len)
+                     residual_mass, K, k_len, options)
     st = LIB.pspec_verify_rejection(ctypes.byref(a), _ptr(workspace, torch.uint8, "workspace"),
                                     workspace.numel(), _stream(stream))
     if st != PSPEC_OK:
@@ -360,12 +383,12 @@ def pspec_build_draft_batch(*, stream=None, **build) -> None:
 
 
 def pspec_step_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len, bonus, err,
-                      workspace, build: dict, k_len=None, stream=None) -> None:
+                      workspace, build: dict, k_len=None, options=None, stream=None) -> None:
     """Greedy verify followed by the draft-batch build (`build`: the keyword arguments of
     pspec_build_draft_batch, with accepted_len / bonus None or this call's outputs)."""
     K = int(target_logits.shape[1]) - 1
     v = _verify_args(target_logits, None, draft_tokens, None, out_tokens, accepted_len, bonus,
-                     err, None, None, None, None, None, K, k_len)
+                     err, None, None, None, None, None, K, k_len, options)
     b = _build_args(**build)
     st = LIB.pspec_step_greedy(ctypes.byref(v), ctypes.byref(b),
                                _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
@@ -376,11 +399,12 @@ def pspec_step_greedy(*, target_logits, draft_tokens, out_tokens, accepted_len, 
 
 def pspec_step_rejection(*, target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
                          accepted_len, bonus, err, workspace, build: dict, residual_mass=None,
-                         k_len=None, stream=None) -> None:
+                         k_len=None, options=None, stream=None) -> None:
     """Rejection-rule verify followed by the draft-batch build (see pspec_step_greedy)."""
     K = int(target_logits.shape[1]) - 1
     v = _verify_args(target_logits, draft_logits, draft_tokens, uniforms, out_tokens,
-                     accepted_len, bonus, err, None, None, None, None, residual_mass, K, k_len)
+                     accepted_len, bonus, err, None, None, None, None, residual_mass, K, k_len,
+                     options)
     b = _build_args(**build)
     st = LIB.pspec_step_rejection(ctypes.byref(v), ctypes.byref(b),
                                   _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),

@@ -11,15 +11,16 @@ from . import _binding as _b
 
 
 class Workspace:
-    """Zero-initialised verify workspace for (B, K, V, mode).  Reusable across calls on one
-    stream: each call leaves its per-sequence counters back at zero."""
+    """Zero-initialised verify workspace for (B, K, V, mode) and the calls' tuning options
+    (None: the process-wide defaults).  Reusable across calls on one stream: each call leaves
+    its per-sequence counters back at zero."""
 
-    def __init__(self, B: int, K: int, V: int, rejection: bool, device="cuda"):
-        n = _b.pspec_verify_workspace_bytes(B, K, V, rejection) if B > 0 else 0
+    def __init__(self, B: int, K: int, V: int, rejection: bool, device="cuda", options=None):
+        n = _b.pspec_verify_workspace_bytes(B, K, V, rejection, options) if B > 0 else 0
         self.tensor = torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
-    def fits(self, B: int, K: int, V: int, rejection: bool) -> bool:
-        return self.tensor.numel() >= _b.pspec_verify_workspace_bytes(B, K, V, rejection)
+    def fits(self, B: int, K: int, V: int, rejection: bool, options=None) -> bool:
+        return self.tensor.numel() >= _b.pspec_verify_workspace_bytes(B, K, V, rejection, options)
 
 
 def verify_outputs(Bn: int, K: int, device, diagnostics: bool, rejection: bool,
@@ -46,18 +47,20 @@ def verify_outputs(Bn: int, K: int, device, diagnostics: bool, rejection: bool,
 
 def verify_greedy(target_logits: torch.Tensor, draft_tokens: torch.Tensor, *,
                   want_lse: bool = False, workspace: Workspace | None = None, out=None,
-                  k_len: torch.Tensor | None = None, stream=None) -> dict:
+                  k_len: torch.Tensor | None = None, options=None, stream=None) -> dict:
     """Greedy verify.  Returns out_tokens, accepted_len, bonus, err (+ target_lse).
-    k_len [B] int32 (optional): each sequence's own draft count."""
+    k_len [B] int32 (optional): each sequence's own draft count.  options (optional): a dict
+    of pspec_options fields for this call alone."""
     Bn, K1, V = target_logits.shape
     K = K1 - 1
     o = out if out is not None else verify_outputs(Bn, K, target_logits.device, want_lse, False)
-    ws = workspace if workspace is not None else Workspace(Bn, K, V, False, target_logits.device)
+    ws = workspace if workspace is not None else Workspace(Bn, K, V, False, target_logits.device,
+                                                           options)
     _b.pspec_verify_greedy(target_logits=target_logits, draft_tokens=draft_tokens,
                           out_tokens=o["out_tokens"], accepted_len=o["accepted_len"],
                           bonus=o["bonus"], err=o["err"], workspace=ws.tensor,
                           target_lse=o.get("target_lse") if want_lse else None, k_len=k_len,
-                          stream=stream)
+                          options=options, stream=stream)
     return o
 
 
@@ -65,22 +68,24 @@ def verify_rejection(target_logits: torch.Tensor, draft_logits: torch.Tensor,
                      draft_tokens: torch.Tensor, uniforms: torch.Tensor, *,
                      diagnostics: bool = False, residual_mass: bool = False,
                      workspace: Workspace | None = None, out=None,
-                     k_len: torch.Tensor | None = None, stream=None) -> dict:
+                     k_len: torch.Tensor | None = None, options=None, stream=None) -> dict:
     """Rejection-rule verify.  Returns out_tokens, accepted_len, bonus, err (+ fp32
     diagnostics target_lse, draft_lse, p_at_draft, q_at_draft, residual_mass; or only
-    residual_mass)."""
+    residual_mass).  options (optional): a dict of pspec_options fields for this call."""
     Bn, K1, V = target_logits.shape
     K = K1 - 1
     o = out if out is not None else verify_outputs(Bn, K, target_logits.device, diagnostics, True,
                                                    residual_mass)
-    ws = workspace if workspace is not None else Workspace(Bn, K, V, True, target_logits.device)
+    ws = workspace if workspace is not None else Workspace(Bn, K, V, True, target_logits.device,
+                                                           options)
     _b.pspec_verify_rejection(target_logits=target_logits, draft_logits=draft_logits,
                              draft_tokens=draft_tokens, uniforms=uniforms,
                              out_tokens=o["out_tokens"], accepted_len=o["accepted_len"],
                              bonus=o["bonus"], err=o["err"], workspace=ws.tensor,
                              target_lse=o.get("target_lse"), draft_lse=o.get("draft_lse"),
                              p_at_draft=o.get("p_at_draft"), q_at_draft=o.get("q_at_draft"),
-                             residual_mass=o.get("residual_mass"), k_len=k_len, stream=stream)
+                             residual_mass=o.get("residual_mass"), k_len=k_len,
+                             options=options, stream=stream)
     return o
 
 
@@ -145,7 +150,7 @@ def build_draft_batch(*, K: int, block_size: int, mask_id: int, pad_id: int, T_c
 def step(target_logits: torch.Tensor, draft_tokens: torch.Tensor, build: dict, *,
          draft_logits: torch.Tensor | None = None, uniforms: torch.Tensor | None = None,
          residual_mass: bool = False, workspace: Workspace | None = None, out=None,
-         build_out=None, k_len: torch.Tensor | None = None, stream=None) -> tuple:
+         build_out=None, k_len: torch.Tensor | None = None, options=None, stream=None) -> tuple:
     """One step: verification (the rejection rule when `uniforms` is given, else greedy)
     and the draft-batch build from its accepted counts and bonus tokens, in one launch when
     the early-exit path takes the verification.  `build` holds the build inputs (K,
@@ -156,7 +161,7 @@ def step(target_logits: torch.Tensor, draft_tokens: torch.Tensor, build: dict, *
     K = K1 - 1
     dev = target_logits.device
     o = out if out is not None else verify_outputs(Bn, K, dev, False, rej, residual_mass)
-    ws = workspace if workspace is not None else Workspace(Bn, K, V, rej, dev)
+    ws = workspace if workspace is not None else Workspace(Bn, K, V, rej, dev, options)
     vh = build["verify_hidden"]
     bo = build_out if build_out is not None else build_outputs(
         Bn, K, int(vh.shape[1]), build["T_cap"], vh.dtype, vh.device)
@@ -174,10 +179,11 @@ def step(target_logits: torch.Tensor, draft_tokens: torch.Tensor, build: dict, *
                                draft_tokens=draft_tokens, uniforms=uniforms,
                                out_tokens=o["out_tokens"], accepted_len=o["accepted_len"],
                                bonus=o["bonus"], err=o["err"], workspace=ws.tensor, build=bargs,
-                               residual_mass=o.get("residual_mass"), k_len=k_len, stream=stream)
+                               residual_mass=o.get("residual_mass"), k_len=k_len,
+                               options=options, stream=stream)
     else:
         _b.pspec_step_greedy(target_logits=target_logits, draft_tokens=draft_tokens,
                              out_tokens=o["out_tokens"], accepted_len=o["accepted_len"],
                              bonus=o["bonus"], err=o["err"], workspace=ws.tensor, build=bargs,
-                             k_len=k_len, stream=stream)
+                             k_len=k_len, options=options, stream=stream)
     return o, bo

@@ -13,17 +13,27 @@ namespace {
 
 using namespace pspec;
 
-long long g_seg_override = 0;   // 0 = automatic segment length
+// Process-wide defaults of the tuning options (pspec_set_*), used by calls whose arguments
+// carry no pspec_options of their own.
+pspec_options g_defaults = {0, 0, 0, 0, 0};
 cudaEvent_t g_split_event = nullptr;
-int g_verify_path = 0;          // 0 automatic, 1 sweep, 2 early exit, 3 queue, 4 waves
-int g_cluster = 0;              // early-exit cluster size; 0 = automatic
-int g_step_fusion = 0;          // 0 automatic, 1 always, 2 never
-int g_ee_stream = 0;            // early-exit streaming: 0 automatic, 1 registers, 2 ring
-int g_tail_split = 0;           // early-exit tail launch: 0 automatic, -1 never, n > 0 sequences
-unsigned long long g_wait_limit = 0;  // polls per bounded wait; 0 = the kernels' defaults
 thread_local int t_last_launches = 0;
 thread_local int t_last_path = 0;
 thread_local int t_last_cluster = 0;   // CTAs per cluster of the last early-exit launch
+
+// The options one call runs with: its own, or the process-wide defaults; out-of-range
+// values read as automatic.
+pspec_options resolve(const pspec_options* o) {
+  pspec_options r = o ? *o : g_defaults;
+  if (r.verify_path < 0 || r.verify_path > 2) r.verify_path = 0;
+  if (!(r.cluster_size == 2 || r.cluster_size == 4 || r.cluster_size == 8 ||
+        r.cluster_size == 12 || r.cluster_size == 16))
+    r.cluster_size = 0;
+  if (r.tail_split < 0) r.tail_split = -1;
+  if (r.step_fusion < 0 || r.step_fusion > 2) r.step_fusion = 0;
+  if (r.segment_elems < 0) r.segment_elems = 0;
+  return r;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -32,7 +42,11 @@ size_t elem_bytes(pspec_dtype d) { return d == PSPEC_BF16 ? 2 : 4; }
 
 bool dtype_ok(pspec_dtype d) { return d == PSPEC_F32 || d == PSPEC_BF16; }
 
-pspec_status check_verify(const pspec_verify_args* a, bool rejection) {
+}  // namespace
+
+namespace pspec {
+
+pspec_status check_verify_host(const pspec_verify_args* a, bool rejection) {
   if (!a) return PSPEC_ERR_INVALID_ARG;
   if (a->B < 0 || a->K < 1 || a->V < 1 || a->ld < a->V) return PSPEC_ERR_INVALID_ARG;
   if (a->K > PSPEC_MAX_K) return PSPEC_ERR_UNSUPPORTED;
@@ -50,6 +64,15 @@ pspec_status check_verify(const pspec_verify_args* a, bool rejection) {
   if (rows * ((a->V + kSegMin - 1) / kSegMin) >= 0x7fffffffLL) return PSPEC_ERR_UNSUPPORTED;
   return PSPEC_OK;
 }
+
+void record_last_call(int launches, int path) {
+  t_last_launches = launches;
+  t_last_path = path;
+}
+
+}  // namespace pspec
+
+namespace {
 
 // Host checks of a draft-batch construction; fills the launch descriptor on success.
 pspec_status check_build(const pspec_build_args* a, BuildLaunch* L) {
@@ -88,30 +111,36 @@ pspec_status check_build(const pspec_build_args* a, BuildLaunch* L) {
   return PSPEC_OK;
 }
 
+// Which rule of the automatic selection takes the early-exit path: every batch size for the
+// greedy rule; for the rejection rule batches of at least kEarlyExitMinB sequences, and
+// batches of at most kEarlyExitRejSmallMax (a handful of sequences, where one launch of a
+// wide cluster per sequence beats the sweep's three launches).
+bool early_exit_wanted(int B, bool rejection) {
+  if (!rejection) return true;
+  return B >= kEarlyExitMinB || B <= kEarlyExitRejSmallMax;
+}
+
 // The early-exit cluster path, when the arguments allow it and the selection asks for it:
 // returns true and sets *st when it handled the call.  With `fuse` non-null the same launch
 // also builds the draft batch described there (from this call's accepted counts and bonus
 // tokens).
-bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t stream,
-                    pspec_status* st, const BuildLaunch* fuse = nullptr) {
+bool try_early_exit(const pspec_verify_args* a, bool rejection, const pspec_options& o,
+                    cudaStream_t stream, pspec_status* st, const BuildLaunch* fuse = nullptr) {
   const bool diagnostics = a->target_lse || a->draft_lse || a->p_at_draft || a->q_at_draft;
-  if (g_verify_path == 1) return false;
-  if (g_verify_path == 0 && (a->B < kEarlyExitMinB || diagnostics)) return false;
+  if (o.verify_path == 1) return false;
+  if (o.verify_path == 0 && (!early_exit_wanted(a->B, rejection) || diagnostics)) return false;
   const int eb = (int)elem_bytes(a->dtype);
   const bool aligned = aligned16(a->target_logits) && (!rejection || aligned16(a->draft_logits)) &&
                        (a->ld * eb) % 16 == 0;
   const bool v_ok = a->V % 8 == 0 && make_early_exit_plan(a->V, 16).ok;
   if (!v_ok || !aligned || diagnostics) {
-    if (g_verify_path == 0) return false;
+    if (o.verify_path == 0) return false;
     *st = PSPEC_ERR_UNSUPPORTED;            // early exit forced on arguments it cannot take
     return true;
   }
   EarlyExitLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.rejection = rejection;
-  L.ring = g_ee_stream == 2;
-  L.spin_limit = g_wait_limit ? (unsigned)(g_wait_limit < (1ull << 21) ? g_wait_limit : (1ull << 21))
-                              : (1u << 21);
   L.target = a->target_logits;
   L.draft = a->draft_logits;
   L.draft_tokens = a->draft_tokens;
@@ -127,17 +156,13 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
     L.b = fuse->a;
     L.row_vecs = fuse->row_vecs;
   }
-  // Cluster size: 4 from kEarlyExitSmallB sequences on.  Below, the rejection rule takes the
-  // widest cluster (16, 12, 8) with which every sequence's cluster is resident at once (a
-  // batch that needs a second round of clusters costs a second chain of positions); the
-  // greedy rule, with less work per element, 8 (16 below 16 sequences).  Measured on B200
-  // with c64's rows, ms per step for G = 16 / 12 / 8: rejection B = 32: 0.081 / 0.085 /
-  // 0.097, B = 64: 0.099 / 0.095 / 0.103, B = 96: 0.123 / 0.114 / 0.108 (the rule picks 16,
-  // 12, 8); greedy B = 32: 0.043 / 0.047 / 0.041, B = 64: 0.047 / 0.049 / 0.046, B = 96:
-  // 0.054 / 0.053 / 0.046.
+  // Cluster size: kEarlyExitCluster from kEarlyExitSmallB sequences on.  Below, the rejection
+  // rule takes the widest cluster (16, 12, 8) with which every sequence's cluster is
+  // resident at once (a batch that needs a second round of clusters costs a second chain of
+  // positions); the greedy rule, with less work per element, 8 (16 below 16 sequences).
   L.seq0 = 0;
   L.nseq = a->B;
-  int G = g_cluster;
+  int G = o.cluster_size;
   if (G == 0) {
     G = kEarlyExitCluster;
     if (a->B < kEarlyExitSmallB && !rejection) {
@@ -153,9 +178,9 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
     }
   }
   EarlyExitPlan ep = make_early_exit_plan(a->V, G);
-  if (!ep.ok && g_cluster == 0) ep = make_early_exit_plan(a->V, 16);   // slices of 4 too long
+  if (!ep.ok && o.cluster_size == 0) ep = make_early_exit_plan(a->V, 16);   // slices too long
   if (!ep.ok) {
-    if (g_verify_path == 0) return false;
+    if (o.verify_path == 0) return false;
     *st = PSPEC_ERR_UNSUPPORTED;
     return true;
   }
@@ -164,9 +189,12 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, cudaStream_t str
   // The last X sequences go to a second launch of wider clusters that starts as the first
   // launch's clusters finish (programmatic dependent launch): the sequences that start last
   // then run their chains of rows twice as wide, which shortens the launch's tail.
+  // Automatic: large batches on the large-batch width; a forced count: any narrower width.
   int X = 0;
-  if (ep.G == kEarlyExitCluster && ep.G != 16 && g_tail_split >= 0)
-    X = g_tail_split > 0 ? g_tail_split : early_exit_tail(a->B, rejection);
+  if (ep.G < kEarlyExitTailCluster && o.tail_split >= 0)
+    X = o.tail_split > 0 ? o.tail_split
+                         : (ep.G == kEarlyExitCluster && a->B >= kEarlyExitSmallB
+                                ? early_exit_tail(a->B, rejection) : 0);
   X = X < a->B / 2 ? X : a->B / 2;
   const EarlyExitPlan et = make_early_exit_plan(a->V, kEarlyExitTailCluster);
   int launches = 1;
@@ -208,134 +236,25 @@ pspec_status check_workspace(void* ws, size_t bytes, size_t scratch, long long B
   return PSPEC_OK;
 }
 
-// The position-wave path (rejection rule: K+1 wave launches and the draw launch), when
-// forced.  Returns true and sets *st when it handled the call.
-bool try_waves(const pspec_verify_args* a, void* workspace, size_t bytes, cudaStream_t stream,
-               pspec_status* st) {
-  if (g_verify_path != 4) return false;
-  const bool diagnostics = a->target_lse || a->draft_lse || a->p_at_draft || a->q_at_draft;
-  if (diagnostics) {
-    *st = PSPEC_ERR_UNSUPPORTED;              // rows after a_i are never read on this path
-    return true;
-  }
-  const WavePlan p = make_wave_plan(a->B, a->K, a->V);
-  ZeroArea z;
-  *st = check_workspace(workspace, bytes, p.bytes, a->B, &z);
-  if (*st != PSPEC_OK) return true;
-  char* ws = static_cast<char*>(workspace);
-  WaveLaunch W{};
-  W.B = a->B; W.K = a->K; W.V = a->V; W.ld = a->ld; W.dtype = a->dtype;
-  W.target_units = kWaveUnits;
-  W.S_max = p.S_max;
-  W.target = a->target_logits;
-  W.draft = a->draft_logits;
-  W.draft_tokens = a->draft_tokens;
-  W.uniforms = a->uniforms;
-  W.out_tokens = a->out_tokens;
-  W.accepted_len = a->accepted_len;
-  W.err = a->err;
-  W.k_len = a->k_len;
-  W.cnt = z.line0 + kZwSCnt;
-  W.wave_cnt = reinterpret_cast<unsigned*>(z.ctr);
-  W.lists = reinterpret_cast<int*>(ws + p.off_lists);
-  W.part = ws + p.off_part;
-  W.seq = ws + p.off_seq;
-  RejectionLaunch D{};                        // the draw launch over every row a_i
-  D.B = a->B; D.K = a->K; D.V = a->V; D.ld = a->ld; D.dtype = a->dtype;
-  D.tiles = p.draw.tiles; D.tiles_per_chunk = p.draw.tiles_per_chunk; D.C = p.draw.C;
-  D.target = a->target_logits;
-  D.draft = a->draft_logits;
-  D.uniforms = a->uniforms;
-  D.out_tokens = a->out_tokens;
-  D.bonus = a->bonus;
-  D.residual_mass = a->residual_mass;
-  D.err = a->err;
-  D.k_len = a->k_len;
-  D.cnt2 = z.line0 + kZwSCnt2;
-  D.seq = W.seq;
-  D.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
-  if (launch_waves(W, stream) != cudaSuccess || launch_rejection_draw(D, stream) != cudaSuccess) {
-    *st = PSPEC_ERR_CUDA;
-    return true;
-  }
-  t_last_launches = a->K + 2;
-  t_last_path = 4;
-  *st = PSPEC_OK;
-  return true;
-}
-
-// The work-queue path (one persistent launch), when forced.  Returns true and sets *st
-// when it handled the call.
-bool try_queue(const pspec_verify_args* a, bool rejection, void* workspace, size_t bytes,
-               cudaStream_t stream, pspec_status* st) {
-  if (g_verify_path != 3) return false;
-  const bool diagnostics = a->target_lse || a->draft_lse || a->p_at_draft || a->q_at_draft;
-  if (diagnostics) {
-    *st = PSPEC_ERR_UNSUPPORTED;              // rows after a_i are never read on this path
-    return true;
-  }
-  if (a->B >= (1 << 26)) {                     // items pack i << 5 | k into an int
-    *st = PSPEC_ERR_UNSUPPORTED;
-    return true;
-  }
-  const QueuePlan p = make_queue_plan(a->B, a->K, a->V, rejection);
-  ZeroArea z;
-  *st = check_workspace(workspace, bytes, p.bytes, a->B, &z);
-  if (*st != PSPEC_OK) return true;
-  QueueLaunch L{};
-  L.spin_limit = g_wait_limit ? g_wait_limit : (1ull << 20);
-  L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
-  L.rejection = rejection;
-  L.S = p.S; L.seg = p.seg;
-  L.tiles = p.tiles; L.tiles_per_unit = p.tiles_per_unit; L.C = p.C;
-  L.target = a->target_logits;
-  L.draft = a->draft_logits;
-  L.draft_tokens = a->draft_tokens;
-  L.uniforms = a->uniforms;
-  L.out_tokens = a->out_tokens;
-  L.accepted_len = a->accepted_len;
-  L.bonus = a->bonus;
-  L.residual_mass = rejection ? a->residual_mass : nullptr;
-  L.err = a->err;
-  L.k_len = a->k_len;
-  char* ws = static_cast<char*>(workspace);
-  L.ctr = z.ctr;
-  L.items = z.line0 + kZwItems;
-  L.draws = z.line0 + kZwDraw;
-  L.cnt = z.line0 + kZwQCnt;
-  L.cnt2 = z.line0 + kZwQCnt2;
-  L.part = ws + p.off_part;
-  L.seq = ws + p.off_seq;
-  L.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
-  if (launch_queue(L, stream) != cudaSuccess) {
-    *st = PSPEC_ERR_CUDA;
-    return true;
-  }
-  if (rejection && g_split_event) cudaEventRecord(g_split_event, stream);
-  t_last_launches = 1;
-  t_last_path = 3;
-  *st = PSPEC_OK;
-  return true;
-}
-
-// Scratch the verify calls need below the zero area: the largest of the paths' plans, so
-// that a workspace of pspec_verify_workspace_bytes serves every path and every call checks
-// against the one size that function reports.
-size_t verify_scratch_bytes(int B, int K, int V, int rejection) {
-  const size_t sweep = align256(make_verify_plan(B, K, V, rejection, g_seg_override).bytes);
-  const size_t queue = align256(make_queue_plan(B, K, V, rejection).bytes);
-  const size_t waves = rejection ? align256(make_wave_plan(B, K, V).bytes) : 0;
-  size_t m = sweep > queue ? sweep : queue;
-  return m > waves ? m : waves;
+// Scratch the verify calls need below the zero area: the full sweep's plan (the early-exit
+// path needs none), so that a workspace of pspec_verify_workspace_bytes serves every path
+// and every call checks against the one size that function reports.
+size_t verify_scratch_bytes(int B, int K, int V, int rejection, const pspec_options& o) {
+  return align256(make_verify_plan(B, K, V, rejection, o.segment_elems).bytes);
 }
 
 }  // namespace
 
 extern "C" {
 
-size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection) {
+size_t pspec_verify_workspace_bytes_opt(int B, int K, int V, int rejection,
+                                        const pspec_options* options) {
   if (B < 0 || K < 1 || K > PSPEC_MAX_K || V < 1) return 0;
-  return verify_scratch_bytes(B, K, V, rejection) + zero_area_bytes(B);
+  return verify_scratch_bytes(B, K, V, rejection, resolve(options)) + zero_area_bytes(B);
+}
+
+size_t pspec_verify_workspace_bytes(int B, int K, int V, int rejection) {
+  return pspec_verify_workspace_bytes_opt(B, K, V, rejection, nullptr);
 }
 
 }  // extern "C"
@@ -348,15 +267,15 @@ pspec_status verify_greedy_impl(const pspec_verify_args* a, void* workspace,
                                 size_t workspace_bytes, cudaStream_t stream,
                                 const BuildLaunch* fuse, bool* fused) {
   *fused = false;
-  pspec_status st = check_verify(a, false);
+  pspec_status st = check_verify_host(a, false);
   if (st != PSPEC_OK) return st;
-  if (a->B == 0) { t_last_launches = 0; return st; }
-  const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 0, g_seg_override);
+  if (a->B == 0) { record_last_call(0, 0); return st; }
+  const pspec_options o = resolve(a->options);
+  const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 0, o.segment_elems);
   ZeroArea z;
-  st = check_workspace(workspace, workspace_bytes, verify_scratch_bytes(a->B, a->K, a->V, 0), a->B, &z);
+  st = check_workspace(workspace, workspace_bytes, verify_scratch_bytes(a->B, a->K, a->V, 0, o), a->B, &z);
   if (st != PSPEC_OK) return st;
-  if (try_queue(a, false, workspace, workspace_bytes, stream, &st)) return st;
-  if (try_early_exit(a, false, stream, &st, fuse)) {
+  if (try_early_exit(a, false, o, stream, &st, fuse)) {
     *fused = fuse != nullptr && st == PSPEC_OK;
     return st;
   }
@@ -375,8 +294,7 @@ pspec_status verify_greedy_impl(const pspec_verify_args* a, void* workspace,
   L.cnt = z.line0 + kZwSCnt;
   L.part = ws + p.off_part;
   if (launch_greedy(L, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
-  t_last_launches = 1;
-  t_last_path = 1;
+  record_last_call(1, 1);
   return PSPEC_OK;
 }
 
@@ -385,16 +303,15 @@ pspec_status verify_rejection_impl(const pspec_verify_args* a, void* workspace,
                                    size_t workspace_bytes, cudaStream_t stream,
                                    const BuildLaunch* fuse, bool* fused) {
   *fused = false;
-  pspec_status st = check_verify(a, true);
+  pspec_status st = check_verify_host(a, true);
   if (st != PSPEC_OK) return st;
-  if (a->B == 0) { t_last_launches = 0; return st; }
-  const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 1, g_seg_override);
+  if (a->B == 0) { record_last_call(0, 0); return st; }
+  const pspec_options o = resolve(a->options);
+  const VerifyPlan p = make_verify_plan(a->B, a->K, a->V, 1, o.segment_elems);
   ZeroArea z;
-  st = check_workspace(workspace, workspace_bytes, verify_scratch_bytes(a->B, a->K, a->V, 1), a->B, &z);
+  st = check_workspace(workspace, workspace_bytes, verify_scratch_bytes(a->B, a->K, a->V, 1, o), a->B, &z);
   if (st != PSPEC_OK) return st;
-  if (try_queue(a, true, workspace, workspace_bytes, stream, &st)) return st;
-  if (try_waves(a, workspace, workspace_bytes, stream, &st)) return st;
-  if (try_early_exit(a, true, stream, &st, fuse)) {
+  if (try_early_exit(a, true, o, stream, &st, fuse)) {
     *fused = fuse != nullptr && st == PSPEC_OK;
     return st;
   }
@@ -423,8 +340,7 @@ pspec_status verify_rejection_impl(const pspec_verify_args* a, void* workspace,
   L.seq = ws + p.off_seq;
   L.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
   if (launch_rejection(L, stream, g_split_event) != cudaSuccess) return PSPEC_ERR_CUDA;
-  t_last_launches = 2;
-  t_last_path = 1;
+  record_last_call(2, 1);
   return PSPEC_OK;
 }
 
@@ -446,7 +362,8 @@ pspec_status step_impl(const pspec_verify_args* v, const pspec_build_args* b, bo
   if (st != PSPEC_OK) return st;
   // one launch for both halves where that measured faster: below kStepFuseMaxB sequences
   // the saved launch outweighs building each span at the end of its cluster's work
-  const bool want_fuse = g_step_fusion == 1 || (g_step_fusion == 0 && v->B < kStepFuseMaxB);
+  const pspec_options o = resolve(v->options);
+  const bool want_fuse = o.step_fusion == 1 || (o.step_fusion == 0 && v->B < kStepFuseMaxB);
   const BuildLaunch* fuse = want_fuse ? &BL : nullptr;
   bool fused = false;
   st = rejection ? verify_rejection_impl(v, workspace, workspace_bytes, stream, fuse, &fused)
@@ -549,16 +466,20 @@ int pspec_last_launches(void) { return t_last_launches; }
 int pspec_last_verify_path(void) { return t_last_path; }
 int pspec_last_cluster_size(void) { return t_last_cluster; }
 
-void pspec_set_verify_path(int path) { g_verify_path = (path >= 1 && path <= 4) ? path : 0; }
+void pspec_set_verify_path(int path) { g_defaults.verify_path = (path == 1 || path == 2) ? path : 0; }
 
-void pspec_set_cluster_size(int G) { g_cluster = (G == 2 || G == 4 || G == 8 || G == 12 || G == 16) ? G : 0; }
+void pspec_set_cluster_size(int G) {
+  g_defaults.cluster_size = (G == 2 || G == 4 || G == 8 || G == 12 || G == 16) ? G : 0;
+}
 
-void pspec_set_step_fusion(int mode) { g_step_fusion = (mode == 1 || mode == 2) ? mode : 0; }
-void pspec_set_ee_stream(int mode) { g_ee_stream = (mode == 1 || mode == 2) ? mode : 0; }
-void pspec_set_tail_split(int n) { g_tail_split = n < 0 ? -1 : n; }
-void pspec_set_wait_limit(unsigned long long polls) { g_wait_limit = polls; }
+void pspec_set_step_fusion(int mode) { g_defaults.step_fusion = (mode == 1 || mode == 2) ? mode : 0; }
+void pspec_set_tail_split(int n) { g_defaults.tail_split = n < 0 ? -1 : n; }
 
-void pspec_set_segment_elems(long long elems) { g_seg_override = elems > 0 ? elems : 0; }
+void pspec_set_segment_elems(long long elems) { g_defaults.segment_elems = elems > 0 ? elems : 0; }
+
+void pspec_get_options(pspec_options* out) {
+  if (out) *out = g_defaults;
+}
 
 void pspec_set_split_event(cudaEvent_t event) { g_split_event = event; }
 

@@ -63,8 +63,6 @@ struct EarlyExitLaunch {
   pspec_dtype dtype;
   int rejection;         // 1: rejection rule, 0: greedy
   int G;                 // CTAs per cluster (one cluster per sequence): 2, 4, 8, 12 or 16
-  int ring;              // 1: rows streamed through per-warp shared-memory stages (bulk copies)
-  unsigned spin_limit;   // ring streaming: polls before a stage wait gives up
   int seq0, nseq;        // this launch's sequences [seq0, seq0 + nseq) of the batch's B
   int pdl;               // split batch: 1 first launch (lets the second start as its CTAs
                          // are placed), 2 second launch (its CTA 0 ends after the first grid)
@@ -102,38 +100,6 @@ struct SampleLaunch {
   void* maxes;           // workspace: (max, index) per chunk [rows*tiles]
 };
 
-struct QueueLaunch {
-  int B, K, V;
-  long long ld;
-  pspec_dtype dtype;
-  int rejection;         // 1: rejection rule, 0: greedy
-  int S;                 // segments per row
-  long long seg;         // elements per segment
-  int tiles;             // 256-element draw tiles per row
-  int tiles_per_unit;    // draw tiles per draw unit
-  int C;                 // draw units per sequence
-  const void* target;
-  const void* draft;
-  const int32_t* draft_tokens;
-  const float* uniforms;
-  int32_t* out_tokens;
-  int32_t* accepted_len;
-  int32_t* bonus;
-  float* residual_mass;  // optional
-  int32_t* err;
-  const int32_t* k_len;  // optional per-sequence draft counts
-  unsigned long long* ctr;  // zero area: queue counters [8]
-  int* items;            // zero area: line 0 (item slot s = zitem(items, s)), holding
-                         // (i*32 + k) + 1 once published, 0 before
-  int* draws;            // zero area: draw slot column (zcol), i + 1 once published
-  int* cnt;              // zero area: stream-unit ticket column (zcol)
-  int* cnt2;             // zero area: draw-unit ticket column (zcol)
-  void* part;            // workspace: 8-byte partials [B*R*S]
-  void* seq;             // workspace: SeqInfo [B]
-  double* tile_sums;     // workspace: [B*tiles]
-  unsigned long long spin_limit;  // polls before a wait gives up (PSPEC_DEVERR_TIMEOUT)
-};
-
 struct BuildLaunch {
   pspec_build_args a;
   long long row_vecs;    // 16-byte vectors per hidden row
@@ -141,41 +107,20 @@ struct BuildLaunch {
   int hid_rows;          // rows the hidden role inspects: T_in + B*(K-1)
 };
 
-// Position waves (rejection rule): one launch per position k = 0..K over the sequences
-// still undecided, then the sweep's draw launch over every sequence's row a_i.
-struct WaveLaunch {
-  int B, K, V;
-  long long ld;
-  pspec_dtype dtype;
-  long long target_units;  // units (sequence, row, segment) a wave aims for
-  long long S_max;         // segments per row at most (the partials' stride)
-  const void* target;
-  const void* draft;
-  const int32_t* draft_tokens;
-  const float* uniforms;
-  int32_t* out_tokens;
-  int32_t* accepted_len;
-  int32_t* err;
-  const int32_t* k_len;  // optional per-sequence draft counts
-  int* cnt;              // zero area: per-sequence unit ticket column (zcol)
-  unsigned* wave_cnt;    // zero area: K+2 words: sequences appended to wave k, exit ticket
-  int* lists;            // workspace: [(K+1)*B] sequence lists of the waves
-  void* part;            // workspace: RejPart [B*2*S_max]
-  void* seq;             // workspace: SeqInfo [B]
-};
-
 cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream);
 // split_event (may be null) is recorded between the statistics sweep and the draw.
 cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream, cudaEvent_t split_event);
-cudaError_t launch_queue(const QueueLaunch& L, cudaStream_t stream);
-cudaError_t launch_waves(const WaveLaunch& L, cudaStream_t stream);
-// The sweep's draw launch alone (reads SeqInfo, writes the emitted token and bonus).
-cudaError_t launch_rejection_draw(const RejectionLaunch& L, cudaStream_t stream);
 cudaError_t launch_build(const BuildLaunch& L, cudaStream_t stream);
 cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream);
-// Clusters of the variant L names (G, dtype, rule, fusion, streaming) that fit on the
+// Clusters of the variant L names (G, dtype, rule, fusion) that fit on the
 // current device at once; 0 when the query fails.  Cached per device and variant.
 int early_exit_max_clusters(const EarlyExitLaunch& L);
 cudaError_t launch_sample(const SampleLaunch& L, cudaStream_t stream);
+
+// Host helpers of the entry points (api.cu), shared by every verify entry point: the
+// argument checks of a verify call, and the per-thread record behind pspec_last_launches()
+// and pspec_last_verify_path().
+pspec_status check_verify_host(const pspec_verify_args* a, bool rejection);
+void record_last_call(int launches, int path);
 
 }  // namespace pspec

@@ -26,22 +26,27 @@ constexpr long long kSegMax = 65536;     // bounds the tail of the last wave
 constexpr int kTargetCtas = kNumSMs * PSPEC_TARGET_CTAS_PER_SM;
 constexpr int kResampleTargetCtas = kNumSMs * PSPEC_DRAW_CTAS_PER_SM;
 constexpr int kDrawTilesPerCta = 64;     // separate draw launch: at most 8 tiles per warp
-constexpr int kEarlyExitMinB = 64;       // automatic path: early exit from this many sequences
-constexpr int kEarlyExitCluster = 4;     // CTAs per sequence on the early-exit path
-// Below this many sequences the automatic cluster is wider than 4 CTAs (16, 12 or 8; see
-// the rule in api.cu): with 4, a batch of 64 fills only 256 CTA
-// slots of ~900 (measured on B200, c64: 0.100 ms with 16 vs 0.140 ms with 4; at 256
-// sequences 4 and 8 are within 5 % either way, at 1024 sequences 4 is best).
+// Automatic path selection: the greedy rule takes the early exit at every batch size; the
+// rejection rule from kEarlyExitMinB sequences on and up to kEarlyExitRejSmallMax sequences
+// (a handful of sequences: one launch of wide clusters beats the sweep's launches), the full
+// sweep in between.
+constexpr int kEarlyExitMinB = 64;
+#ifndef PSPEC_EE_REJ_SMALL_MAX
+#define PSPEC_EE_REJ_SMALL_MAX 4
+#endif
+constexpr int kEarlyExitRejSmallMax = PSPEC_EE_REJ_SMALL_MAX;
+// CTAs per sequence on the early-exit path from kEarlyExitSmallB sequences on.
+#ifndef PSPEC_EE_CLUSTER
+#define PSPEC_EE_CLUSTER 4
+#endif
+constexpr int kEarlyExitCluster = PSPEC_EE_CLUSTER;
+// Below this many sequences the automatic cluster is wider (16, 12 or 8; see the rule in
+// api.cu): with 4, a batch of 64 fills only 256 CTA slots of ~900.
 constexpr int kEarlyExitSmallB = 128;
 constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this many sequences
 
-// Early exit, batches of 4-CTA clusters: the last sequences go to a second launch of
+// Early exit, large batches: the last sequences go to a second launch of
 // kEarlyExitTailCluster-CTA clusters that fills the SMs as the first launch drains.
-// Measured on B200 (rejection rule, 8-CTA tail): at 1024 sequences 0.672 ms with 96 in the
-// tail against 0.701 ms with none (64: 0.679, 128: 0.677, 256: 0.695); at 256 sequences
-// 0.243-0.245 ms with 32 to 128 against 0.266 ms; 16-CTA tails gained at most 1.8 %.  The
-// greedy rule was slower with any tail (16 sequences: 0.208 against 0.207 ms), so it keeps
-// one launch.
 #ifndef PSPEC_EE_TAIL_SEQS
 #define PSPEC_EE_TAIL_SEQS 96
 #endif
@@ -52,9 +57,6 @@ constexpr int kEarlyExitTailCluster = PSPEC_EE_TAIL_CLUSTER;
 inline int early_exit_tail(long long B, bool rejection) {
   if (!rejection) return 0;
   return (int)(B / 2 < PSPEC_EE_TAIL_SEQS ? B / 2 : PSPEC_EE_TAIL_SEQS);
-}
-inline int early_exit_tail(long long B) {
-  return B >= 2 * PSPEC_EE_TAIL_SEQS ? PSPEC_EE_TAIL_SEQS : 0;
 }
 
 // Per-(row, segment) partial of the greedy sweep.
@@ -95,32 +97,25 @@ struct VerifyPlan {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Words that must be zero when a call starts (tickets, queue slots, queue counters) live at
+// Words that must be zero when a call starts (the sweep's per-sequence tickets) live at
 // the END of the caller's workspace, and scratch (partials, statistics, tile sums) grows
-// from its start.  The zero words are laid out backwards from the end, one line of
-// kLineWords words per index, so that their addresses depend on neither B nor K: a call
-// with a smaller batch finds every counter a larger call left at zero, and its scratch
-// never reaches them.  Line j (j = 0, 1, ...) holds queue item slots 32j .. 32j+31 and the
-// per-sequence words of sequence j.
-constexpr int kLineWords = 40;
+// from its start.  The tickets are laid out backwards from the end, one line of
+// kLineWords words per sequence, so that their addresses depend on neither B nor K: a call
+// with a smaller batch finds every ticket a larger call left at zero, and its scratch never
+// reaches them.
+constexpr int kLineWords = 2;
 constexpr size_t kLineBytes = kLineWords * sizeof(int32_t);
-constexpr size_t kCtrBytes = 256;        // queue counters, just below the aligned end
 enum : int {
-  kZwItems = 0,     // 32 queue item slots
-  kZwDraw = 32,     // queue draw slot
-  kZwQCnt = 33,     // queue stream-unit ticket
-  kZwQCnt2 = 34,    // queue draw-unit ticket
-  kZwSCnt = 35,     // sweep ticket
-  kZwSCnt2 = 36,    // sweep draw ticket
+  kZwSCnt = 0,      // sweep ticket
+  kZwSCnt2 = 1,     // sweep draw ticket
 };
 
 // Bytes of zero area for B sequences (with slack for aligning the end down to 256 bytes).
 inline size_t zero_area_bytes(long long B) {
-  return kCtrBytes + ((size_t)B * kLineBytes + 255) / 256 * 256 + 256;
+  return ((size_t)B * kLineBytes + 255) / 256 * 256 + 256;
 }
 
 struct ZeroArea {
-  unsigned long long* ctr;   // 8 queue counters
   int32_t* line0;            // word 0 of line 0; line j starts kLineWords * j words lower
   char* lowest;              // first byte of line B-1 (scratch must end at or below it)
 };
@@ -128,19 +123,14 @@ struct ZeroArea {
 inline ZeroArea zero_area(void* ws, size_t bytes, long long B) {
   const uintptr_t end = (reinterpret_cast<uintptr_t>(ws) + bytes) & ~uintptr_t(255);
   ZeroArea z;
-  z.ctr = reinterpret_cast<unsigned long long*>(end - kCtrBytes);
-  z.line0 = reinterpret_cast<int32_t*>(end - kCtrBytes - kLineBytes);
-  z.lowest = reinterpret_cast<char*>(end - kCtrBytes) - (size_t)(B > 0 ? B : 1) * kLineBytes;
+  z.line0 = reinterpret_cast<int32_t*>(end - kLineBytes);
+  z.lowest = reinterpret_cast<char*>(end) - (size_t)(B > 0 ? B : 1) * kLineBytes;
   return z;
 }
 
 // Entry i of a zero-area column (col = line0 + word): entries run backwards, a line apart.
 __host__ __device__ __forceinline__ int32_t* zcol(int32_t* col, long long i) {
   return col - i * kLineWords;
-}
-// Queue item slot s.
-__host__ __device__ __forceinline__ int32_t* zitem(int32_t* line0, long long s) {
-  return zcol(line0 + (s & 31), s >> 5);
 }
 // Entry r of a plain backward array ending at `end` (the sampling tickets).
 __host__ __device__ __forceinline__ int32_t* zrow(int32_t* end, long long r) { return end - 1 - r; }
@@ -201,87 +191,6 @@ inline EarlyExitPlan make_early_exit_plan(int V, int G) {
   p.vs = ((long long)V + G - 1) / G;
   p.vs = (p.vs + 7) / 8 * 8;
   p.ok = (p.vs + 255) / 256 <= kMaxSliceTiles;
-  return p;
-}
-
-// Position waves: per wave about kWaveUnits units (two rounds of the resident CTAs), each
-// a segment of at least kWaveSegMin elements of one row.
-#ifndef PSPEC_WAVE_UNITS_PER_SM
-#define PSPEC_WAVE_UNITS_PER_SM 16
-#endif
-constexpr long long kWaveUnits = (long long)kNumSMs * PSPEC_WAVE_UNITS_PER_SM;
-constexpr long long kWaveSegMin = 8192;
-
-struct WavePlan {
-  long long S_max;
-  VerifyPlan draw;        // the sweep's draw launch configuration (tiles, C)
-  size_t off_part, off_seq, off_tiles, off_lists, bytes;
-};
-
-inline WavePlan make_wave_plan(int B, int K, int V) {
-  WavePlan p{};
-  p.S_max = (V + kWaveSegMin - 1) / kWaveSegMin;
-  if (p.S_max < 1) p.S_max = 1;
-  p.draw = make_verify_plan(B, K, V, 1, 0);
-  size_t off = 0;
-  p.off_part = off;
-  off = align256(off + sizeof(RejPart) * (size_t)B * 2 * (size_t)p.S_max);
-  p.off_seq = off;
-  off = align256(off + sizeof(SeqInfo) * (size_t)B);
-  p.off_tiles = off;
-  off = align256(off + sizeof(double) * (size_t)B * p.draw.tiles);
-  p.off_lists = off;
-  off = align256(off + sizeof(int) * (size_t)B * (K + 1));
-  p.bytes = off;
-  return p;
-}
-
-// Work-queue verify: units are segments of about kQueueSeg elements of one row of one
-// (sequence, position) item, draws are cut into units of kQueueDrawTiles warp tiles.
-#ifndef PSPEC_QUEUE_SEG
-#define PSPEC_QUEUE_SEG 65536
-#endif
-constexpr long long kQueueSeg = PSPEC_QUEUE_SEG;
-#ifndef PSPEC_QUEUE_DRAW_TILES
-#define PSPEC_QUEUE_DRAW_TILES 256
-#endif
-constexpr int kQueueDrawTiles = PSPEC_QUEUE_DRAW_TILES;
-
-struct QueuePlan {
-  int R;                  // rows per item: 2 (target + draft, rejection) or 1 (greedy)
-  int S;                  // segments per row
-  long long seg;          // elements per segment
-  int tiles;              // 256-element draw tiles per row
-  int tiles_per_unit;     // draw tiles per draw unit
-  int C;                  // draw units per sequence
-  size_t off_part;        // 8-byte partials [B*R*S]
-  size_t off_seq;         // SeqInfo[B]
-  size_t off_tiles;       // double[B*tiles]
-  size_t bytes;
-};
-
-inline QueuePlan make_queue_plan(int B, int K, int V, int rejection) {
-  QueuePlan p{};
-  p.R = rejection ? 2 : 1;
-  long long S = (V + kQueueSeg - 1) / kQueueSeg;
-  if (S < 1) S = 1;
-  long long seg = (V + S - 1) / S;
-  seg = (seg + 7) / 8 * 8;
-  p.seg = seg;
-  p.S = (int)((V + seg - 1) / seg);
-  p.tiles = (V + kDrawTile - 1) / kDrawTile;
-  int C = (p.tiles + kQueueDrawTiles - 1) / kQueueDrawTiles;
-  if (C < 1) C = 1;
-  p.tiles_per_unit = (p.tiles + C - 1) / C;
-  p.C = (p.tiles + p.tiles_per_unit - 1) / p.tiles_per_unit;
-  size_t off = 0;
-  p.off_part = off;
-  off = align256(off + 8 * (size_t)B * p.R * p.S);
-  p.off_seq = off;
-  off = align256(off + (rejection ? sizeof(SeqInfo) * (size_t)B : 0));
-  p.off_tiles = off;
-  off = align256(off + (rejection ? sizeof(double) * (size_t)B * p.tiles : 0));
-  p.bytes = off;
   return p;
 }
 

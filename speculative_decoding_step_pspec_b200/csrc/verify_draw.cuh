@@ -1,5 +1,5 @@
-// verify_draw.cuh -- the rejection rule's draw over one row pair, shared by the two-launch
-// sweep and the work-queue verify.
+// verify_draw.cuh -- the rejection rule's draw over one row pair, used by the full sweep's
+// draw launch.
 //
 // "Accept prefix; resample for rejected suffix" ("Capstone 14: speculative decoding
 // inference server", section "Architecture"): at the first rejection a_i the emitted token
@@ -15,12 +15,6 @@
 #include "verify_common.cuh"
 
 namespace pspec {
-
-// The barrier the draw's block-wide steps use: the whole CTA by default; a kernel whose
-// CTA holds other warps besides the ones drawing passes its own (a named barrier).
-struct CtaBarrier {
-  __device__ __forceinline__ static void sync() { __syncthreads(); }
-};
 
 // ---------------------------------------------------------------------------------------
 // The draw.  r(t) for t in [0, V): max(0, p(t) - q(t)) (resid) or p(t) (target only),
@@ -182,13 +176,12 @@ __device__ void warp_tile_sums_wide(const DrawRow& D, int V, long long t_begin, 
   }
 }
 
-template <typename Bar = CtaBarrier>
 __device__ __forceinline__ double block_sum(double v, double* s_red) {
   v = warp_sum(v);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  Bar::sync();
+  __syncthreads();
   if (lane == 0) s_red[warp] = v;
-  Bar::sync();
+  __syncthreads();
   double t = 0.0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) t += s_red[w];
@@ -196,7 +189,6 @@ __device__ __forceinline__ double block_sum(double v, double* s_red) {
 }
 
 // Exclusive prefix over the CTA of one double per thread; returns the prefix and sets *total.
-template <typename Bar = CtaBarrier>
 __device__ __forceinline__ double block_exclusive_scan(double v, double* s_red, double* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double incl = v;
@@ -205,9 +197,9 @@ __device__ __forceinline__ double block_exclusive_scan(double v, double* s_red, 
     double n = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += n;
   }
-  Bar::sync();
+  __syncthreads();
   if (lane == 31) s_red[warp] = incl;
-  Bar::sync();
+  __syncthreads();
   double base = 0.0, all = 0.0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
@@ -228,22 +220,22 @@ struct DrawShared {
 // first tile whose inclusive prefix exceeds u*Z, and the first token of that tile whose
 // running sum does (the last positive r of the tile if rounding leaves none; token 0 if
 // the row holds no mass at all).  A residual that sums to zero is redrawn from p itself.
-template <typename Tag, typename Bar = CtaBarrier>
+template <typename Tag>
 __device__ int draw_finish(DrawRow& D, int V, int tiles, double u, double* ts, DrawShared& sh,
                            double* Zout) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   double Z = 0.0;
   for (int t0 = 0; t0 < tiles; t0 += kThreads)
-    Z += block_sum<Bar>(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
+    Z += block_sum(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
   if (Z == 0.0 && D.resid) {
     D.resid = false;                       // max(0, p - q) vanished: draw from p
     D.qrow = D.trow;
-    Bar::sync();
+    __syncthreads();
     warp_tile_sums<Tag>(D, V, warp, tiles, kWarps, ts);
-    Bar::sync();
+    __syncthreads();
     Z = 0.0;
     for (int t0 = 0; t0 < tiles; t0 += kThreads)
-      Z += block_sum<Bar>(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
+      Z += block_sum(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
   }
   const double thr = u * Z;
 
@@ -254,15 +246,15 @@ __device__ int draw_finish(DrawRow& D, int V, int tiles, double u, double* ts, D
     const int t = t0 + tid;
     const double v = t < tiles ? ld_cg(ts + t) : 0.0;
     double tot;
-    const double ex = block_exclusive_scan<Bar>(v, sh.red, &tot);
+    const double ex = block_exclusive_scan(v, sh.red, &tot);
     if (tid == 0) sh.found = 0x7fffffff;
-    Bar::sync();
+    __syncthreads();
     if (t < tiles && v > 0.0 && base + ex + v > thr) atomicMin(&sh.found, t);
-    Bar::sync();
+    __syncthreads();
     const int f = sh.found;
     if (f != 0x7fffffff) {
       if (t == f) sh.red[kWarps] = base + ex;
-      Bar::sync();
+      __syncthreads();
       tile = f;
       tile_base = sh.red[kWarps];
       break;                               // f is the same on every thread
@@ -271,12 +263,12 @@ __device__ int draw_finish(DrawRow& D, int V, int tiles, double u, double* ts, D
   }
   if (tile < 0 && Z > 0.0) {
     // rounding kept every prefix at or below u*Z: the last tile holding any mass
-    Bar::sync();                       // every thread has read sh.found
+    __syncthreads();                       // every thread has read sh.found
     if (tid == 0) sh.found = -1;
-    Bar::sync();
+    __syncthreads();
     for (int t = tid; t < tiles; t += kThreads)
       if (ld_cg(ts + t) > 0.0) atomicMax(&sh.found, t);
-    Bar::sync();
+    __syncthreads();
     tile = sh.found;
     tile_base = -INFINITY;                 // no crossing inside: its last positive r
   }
@@ -313,7 +305,7 @@ __device__ int draw_finish(DrawRow& D, int V, int tiles, double u, double* ts, D
     }
     if (lane == 0) sh.token = token;
   }
-  Bar::sync();
+  __syncthreads();
   *Zout = Z;
   return sh.token;
 }

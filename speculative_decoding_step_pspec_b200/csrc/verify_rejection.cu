@@ -206,15 +206,6 @@ rej_draw_kernel(const RejectionLaunch L) {
 
 }  // namespace
 
-cudaError_t launch_rejection_draw(const RejectionLaunch& L, cudaStream_t stream) {
-  const long long grid2 = (long long)L.B * L.C;
-  if (L.dtype == PSPEC_BF16)
-    rej_draw_kernel<BF16Tag><<<(unsigned)grid2, kThreads, 0, stream>>>(L);
-  else
-    rej_draw_kernel<F32Tag><<<(unsigned)grid2, kThreads, 0, stream>>>(L);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream,
                              cudaEvent_t split_event) {
   const long long grid1 = (long long)L.B * (2 * L.K + 1) * L.S;

@@ -2,9 +2,13 @@
 
 Tolerances (floating-point outputs of the fp32 kernels against the double oracle):
   * p_at_draft, q_at_draft, target_lse, draft_lse: 1e-5 relative (the stated bar);
-  * residual_mass Z: 1e-5 relative plus 1e-6 absolute.  Z = sum max(0, p - q) is a
-    difference of two near-equal sums when the draft is good; each fp32 probability carries
-    about 1e-7 relative error, so the sum's absolute error is a few 1e-7 whatever Z is.
+  * residual_mass Z: 1e-5 relative, with an absolute floor of 1e-6 for masses that come
+    out of cancellation.  Z = sum over t of max(0, p(t) - q(t)); where the draft is good,
+    each term is a difference of two near-equal fp32 probabilities that carry about 1e-7
+    relative error each, so the sum's absolute error is a few 1e-7 of sum p(t) over the
+    terms, whatever Z is -- below Z = 0.1 that is more than 1e-5 of Z.  Every comparison
+    prints the largest relative error of Z and how many sequences passed only by the
+    floor (zero in every full-size workload measured).
 Integer outputs (tokens, counts, offsets, slots) must be bit-exact, except for sequences
 the oracle flags as near-ties (an accept decision with |u - p/q| < 1e-6, or a draw within
 1e-6 * Z of a CDF boundary): those are excluded from the integer comparison and counted.
@@ -85,8 +89,15 @@ def compare_rejection(g: dict, o: dict, seqs=None, K=None):
             assert ok.all(), (k, np.argwhere(~ok)[:5], G[k][~ok][:5], o[k][~ok][:5])
     if "residual_mass" in G:
         same_a = G["accepted_len"] == o["accepted_len"]
-        ok = _rel_ok(G["residual_mass"], o["residual_mass"], RTOL, Z_ATOL) | ~same_a
-        assert ok.all(), ("residual_mass", G["residual_mass"][~ok][:5], o["residual_mass"][~ok][:5])
+        gz = np.asarray(G["residual_mass"], np.float64)[same_a]
+        oz = np.asarray(o["residual_mass"], np.float64)[same_a]
+        ok = _rel_ok(gz, oz, RTOL, Z_ATOL)
+        assert ok.all(), ("residual_mass", gz[~ok][:5], oz[~ok][:5])
+        rel_only = _rel_ok(gz, oz, RTOL, 0.0)
+        nz = oz > 0
+        worst = float(np.max(np.abs(gz - oz)[nz] / oz[nz])) if nz.any() else 0.0
+        print(f"[parity] residual mass: {int(same_a.sum())} compared, max relative error "
+              f"{worst:.2e}, {int((~rel_only).sum())} within tolerance only by the absolute floor")
     flagged = int((~clean).sum())
     print(f"[parity] {len(flags)} sequences, {flagged} flagged near-ties, "
           f"{int((~clean & same).sum())} of those identical anyway")

@@ -48,29 +48,58 @@ def test_status_strings_and_launch_counts():
 
 
 def test_tuning_setters_and_queries():
-    """Every process-wide tuning setter takes its valid values and falls back to the
-    automatic choice on others (setters only: nothing launches); the last-call queries start
-    at zero on a thread that made no call."""
+    """Every process-wide tuning setter changes the defaults pspec_get_options reports, takes
+    its valid values and falls back to the automatic choice on others (setters only: nothing
+    launches); the last-call queries start at zero on a thread that made no call."""
     assert ps.pspec_last_verify_path() == 0 and ps.pspec_last_cluster_size() == 0
+    zero = dict(verify_path=0, cluster_size=0, tail_split=0, step_fusion=0, segment_elems=0)
+    assert ps.pspec_get_options() == zero
     try:
-        for path in (1, 2, 3, 4, 9, -1):
+        for path, want in ((1, 1), (2, 2), (3, 0), (4, 0), (9, 0), (-1, 0)):
             ps.pspec_set_verify_path(path)
-        for G in (2, 4, 8, 12, 16, 5, 0):
+            assert ps.pspec_get_options()["verify_path"] == want
+        for G, want in ((2, 2), (4, 4), (8, 8), (12, 12), (16, 16), (5, 0), (0, 0)):
             ps.pspec_set_cluster_size(G)
-        for n in (96, 1, -1, -7, 0):
+            assert ps.pspec_get_options()["cluster_size"] == want
+        for n, want in ((96, 96), (1, 1), (-1, -1), (-7, -1), (0, 0)):
             ps.pspec_set_tail_split(n)
-        for mode in (1, 2, 3, 4, 0):
-            ps.pspec_set_ee_stream(mode)
+            assert ps.pspec_get_options()["tail_split"] == want
+        for mode, want in ((1, 1), (2, 2), (3, 0), (4, 0), (0, 0)):
             ps.pspec_set_step_fusion(mode)
-        for polls in (1, 1 << 40, 0):
-            ps.pspec_set_wait_limit(polls)
+            assert ps.pspec_get_options()["step_fusion"] == want
+        ps.pspec_set_segment_elems(4096)
+        assert ps.pspec_get_options()["segment_elems"] == 4096
     finally:
         ps.pspec_set_verify_path(0)
         ps.pspec_set_cluster_size(0)
         ps.pspec_set_tail_split(0)
-        ps.pspec_set_ee_stream(0)
         ps.pspec_set_step_fusion(0)
-        ps.pspec_set_wait_limit(0)
+        ps.pspec_set_segment_elems(0)
+    assert ps.pspec_get_options() == zero
+
+
+def test_options_struct_layout_and_workspace():
+    """The options struct the binding builds has the header's layout (five fields, the last
+    a 64-bit count at offset 16), the verify argument struct ends with its pointer, and a
+    call's own segment length changes the workspace size as the process-wide one does."""
+    o = b.pspec_options
+    assert [f for f, _ in o._fields_] == ["verify_path", "cluster_size", "tail_split",
+                                          "step_fusion", "segment_elems"]
+    assert o.segment_elems.offset == 16 and ctypes.sizeof(o) == 24
+    assert b.pspec_verify_args._fields_[-1][0] == "options"
+    f = b.pspec_verify_workspace_bytes
+    base = f(64, 7, 151936, True)
+    assert f(64, 7, 151936, True, {}) == base
+    small = f(64, 7, 151936, True, {"segment_elems": 1024})
+    assert small > base
+    ps.pspec_set_segment_elems(1024)
+    try:
+        assert f(64, 7, 151936, True) == small
+        assert f(64, 7, 151936, True, {}) == base     # a call's own options ignore the default
+    finally:
+        ps.pspec_set_segment_elems(0)
+    with pytest.raises(KeyError):
+        b.make_options({"no_such_field": 1})
 
 
 def test_workspace_sizes():
@@ -85,8 +114,9 @@ def test_workspace_sizes():
             assert n % 256 == 0 and n >= prev
             prev = n
     assert f(1024, 7, 201088, True) > f(1024, 7, 201088, False)
-    # one size serves every path: the position waves' lists and partials included
-    assert f(1024, 7, 201088, True) >= 1024 * 8 * 4 + 1024 * 2 * 25 * 8
+    # the sweep's (m, s) partials of all 15 rows per sequence, SeqInfo and the draw's tile
+    # sums, plus the two tickets per sequence at the end
+    assert f(1024, 7, 201088, True) >= 1024 * 15 * 8 + 1024 * 48 + 1024 * 786 * 8 + 1024 * 8
 
 
 def _vargs(**kw):

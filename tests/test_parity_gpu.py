@@ -1,10 +1,11 @@
 """GPU parity: libpspec's kernels (through the C ABI) against the CPU oracle.
 
-Every workload runs at its full size in the launch configuration the benchmark uses; the
-oracle checks all sequences where it finishes in seconds and a seeded sample otherwise,
-and invariants that hold at any size are checked on every sequence.  Smaller cases cover
-several segments and tiles with ragged tails, padded row strides, the edge cases (K = 1,
-K = 31, V < one vector, -inf rows, out-of-range tokens, empty batches) and determinism.
+Every workload runs at its full size in the launch configuration the benchmark uses, and
+the oracle checks every sequence of every workload (the large batch's 1024 sequences on
+both early-exit launches, every point of the depth sweep), besides invariants that hold at
+any size.  Smaller cases cover several segments and tiles with ragged tails, padded row
+strides, the edge cases (K = 1, K = 31, V < one vector, -inf rows, out-of-range tokens,
+empty batches) and determinism.
 """
 import numpy as np
 import pytest
@@ -19,15 +20,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _sample(B, n, seed):
-    if B <= n:
-        return np.arange(B)
-    return np.sort(np.random.default_rng(seed).choice(B, size=n, replace=False))
-
-
 class verify_path:
-    """Force the full sweep (1), the early-exit path (2), the work-queue path (3) or the
-    position waves (4) inside a with-block."""
+    """Force the full sweep (1) or the early-exit path (2) inside a with-block."""
 
     def __init__(self, path):
         self.path = path
@@ -37,20 +31,6 @@ class verify_path:
 
     def __exit__(self, *a):
         ps.pspec_set_verify_path(0)
-
-
-class ee_stream:
-    """Early-exit row streaming inside a with-block: 1 registers, 2 per-warp shared-memory
-    rings filled by bulk copies."""
-
-    def __init__(self, mode):
-        self.mode = mode
-
-    def __enter__(self):
-        ps.pspec_set_ee_stream(self.mode)
-
-    def __exit__(self, *a):
-        ps.pspec_set_ee_stream(0)
 
 
 class tail_split:
@@ -74,10 +54,11 @@ def early_exit_allowed(t):
     return t.shape[2] % 8 == 0 and t.data_ptr() % 16 == 0 and (t.stride(1) * t.element_size()) % 16 == 0
 
 
-def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True):
-    """Both verify rules, on both paths, against the oracle: the full sweep with every
-    diagnostic, then (where its shape rules allow) the early-exit path, which reads rows
-    only up to the first rejection and must give the same tokens."""
+def _verify_both(target, draft, sampled, greedy_drafts, u, diag=True):
+    """Both verify rules, on both paths, against the oracle on every sequence: the full
+    sweep with every diagnostic, then (where its shape rules allow) the early-exit path in
+    its automatic launch configuration, which reads rows only up to the first rejection and
+    must give the same tokens."""
     V = target.shape[2]
     with verify_path(1):
         gr = ps.verify_greedy(target, greedy_drafts, want_lse=diag)
@@ -85,32 +66,25 @@ def _verify_both(target, draft, sampled, greedy_drafts, u, seqs=None, diag=True)
     torch.cuda.synchronize()
     U.check_verify_invariants(gr, greedy_drafts, V)
     U.check_verify_invariants(rj, sampled, V)
-    og = U.oracle_greedy(target, greedy_drafts, seqs)
-    U.compare_greedy(gr, og, seqs)
-    orj = U.oracle_rejection(target, draft, sampled, u, seqs)
-    U.compare_rejection(rj, orj, seqs)
-    # early exit (both ways of streaming rows) where its shape rules allow; the work queue
-    # and the position waves always (the waves are the rejection rule's: the greedy rule
-    # then takes the early exit, where it can)
-    K = target.shape[1] - 1
-    for path, stream in ((2, 1), (2, 2), (3, 0), (4, 0)):
-        if path in (2, 4) and not early_exit_allowed(target):
-            continue
-        with verify_path(path), ee_stream(stream):
-            gpath = 2 if path == 4 else path
+    og = U.oracle_greedy(target, greedy_drafts)
+    U.compare_greedy(gr, og)
+    orj = U.oracle_rejection(target, draft, sampled, u)
+    U.compare_rejection(rj, orj)
+    if early_exit_allowed(target):
+        with verify_path(2):
             # the early-exit path may hand the batch's last sequences to a second launch
             ge = ps.verify_greedy(target, greedy_drafts)
-            assert ps.pspec_last_launches() in ((1, 2) if gpath == 2 else (1,))
-            assert ps.pspec_last_verify_path() == gpath
+            assert ps.pspec_last_launches() in (1, 2)
+            assert ps.pspec_last_verify_path() == 2
             re = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
-            assert ps.pspec_last_launches() in {2: (1, 2), 3: (1,), 4: (K + 2,)}[path]
-            assert ps.pspec_last_verify_path() == path
+            assert ps.pspec_last_launches() in (1, 2)
+            assert ps.pspec_last_verify_path() == 2
         torch.cuda.synchronize()
-        assert ge["err"].item() == 0 and re["err"].item() == 0, path
+        assert ge["err"].item() == 0 and re["err"].item() == 0
         U.check_verify_invariants(ge, greedy_drafts, V)
         U.check_verify_invariants(re, sampled, V)
-        U.compare_greedy(ge, og, seqs)
-        U.compare_rejection(re, orj, seqs)
+        U.compare_greedy(ge, og)
+        U.compare_rejection(re, orj)
     return gr, rj, orj
 
 
@@ -140,13 +114,15 @@ def test_workload_all_sequences(name):
     _build_and_compare(inp)
 
 
-def test_b1024_sampled():
+def test_b1024_all_sequences():
+    """The large batch at full size: all 1024 sequences of both rules against the oracle, on
+    the full sweep and on the early exit's automatic two launches (the batch's last
+    sequences in the second, wider launch)."""
     w = I.B1024
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
-    seqs = _sample(w.B, 48, 7)
-    _, rj, _ = _verify_both(target, draft, sampled, greedy, u, seqs=seqs)
+    _, rj, _ = _verify_both(target, draft, sampled, greedy, u)
     # the step chains: this verify's accepted counts and bonus tokens feed the build
     inp = I.build_inputs(w, DEV, drafts=sampled)
     inp["accepted_len"] = rj["accepted_len"].clone()
@@ -156,12 +132,12 @@ def test_b1024_sampled():
 
 @pytest.mark.parametrize("K", I.DEPTH_K)
 @pytest.mark.parametrize("sigma", I.DEPTH_SIGMA)
-def test_depth_sweep_sampled(K, sigma):
+def test_depth_sweep_all_sequences(K, sigma):
     w = I.depth(K, sigma)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
-    _verify_both(target, draft, sampled, greedy, u, seqs=_sample(w.B, 12, K))
+    _verify_both(target, draft, sampled, greedy, u)
     _build_and_compare(I.build_inputs(w, DEV, drafts=sampled))
 
 
@@ -234,12 +210,11 @@ def test_neg_inf_rows_and_entries():
     o = U.oracle_rejection(target, draft, d, u)
     U.compare_rejection(rj, o)
     assert rj["accepted_len"][3].item() == 0
-    for path in (2, 3):
-        with verify_path(path):
-            ge = ps.verify_greedy(target, d)
-            re = ps.verify_rejection(target, draft, d, u, residual_mass=True)
-        U.compare_greedy(ge, U.oracle_greedy(target, d, want_lse=False))
-        U.compare_rejection(re, o)
+    with verify_path(2):
+        ge = ps.verify_greedy(target, d)
+        re = ps.verify_rejection(target, draft, d, u, residual_mass=True)
+    U.compare_greedy(ge, U.oracle_greedy(target, d, want_lse=False))
+    U.compare_rejection(re, o)
 
 
 def test_out_of_range_draft_tokens():
@@ -268,22 +243,31 @@ def test_out_of_range_draft_tokens():
         U.compare_rejection(re, o)
 
 
-@pytest.mark.parametrize("B", [1, 63, 64, 200])
+@pytest.mark.parametrize("B", [1, 4, 5, 63, 64, 200])
 def test_automatic_path_selection(B):
-    """Automatic selection: the early exit (one launch) from 64 sequences on when no per-row
-    diagnostic is requested; the full sweep (two launches) otherwise; same tokens."""
+    """Automatic selection with no per-row diagnostic requested: the greedy rule takes the
+    early exit at every batch size; the rejection rule from 64 sequences on and up to 4
+    sequences, the full sweep (two launches) in between; a diagnostic always takes the full
+    sweep; same tokens whichever path runs."""
     w = I.Workload("t", B, 5, 4096, 16, 4, torch.bfloat16, seed=B, sigma_t=2.0, sigma_d=0.6)
     target, draft = I.logits(w, DEV)
-    sampled, _ = I.draft_tokens(w, draft)
+    sampled, greedy = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
     a = ps.verify_rejection(target, draft, sampled, u)
     path_auto = ps.pspec_last_verify_path()
     b = ps.verify_rejection(target, draft, sampled, u, diagnostics=True)
     assert ps.pspec_last_launches() == 2 and ps.pspec_last_verify_path() == 1
-    assert path_auto == (2 if B >= 64 else 1)
+    assert path_auto == (2 if (B >= 64 or B <= 4) else 1)
+    g = ps.verify_greedy(target, greedy)
+    assert ps.pspec_last_verify_path() == 2 and ps.pspec_last_launches() == 1
+    gl = ps.verify_greedy(target, greedy, want_lse=True)
+    assert ps.pspec_last_verify_path() == 1
     o = U.oracle_rejection(target, draft, sampled, u)
     U.compare_rejection(a, o)
     U.compare_rejection(b, o)
+    og = U.oracle_greedy(target, greedy)
+    U.compare_greedy(g, og)
+    U.compare_greedy(gl, og)
 
 
 def test_early_exit_refuses_what_it_cannot_take():
@@ -322,52 +306,30 @@ def test_determinism_and_workspace_reuse():
         e2 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
     for k in e1:
         assert torch.equal(e1[k], e2[k]), k
-    # paths take turns on one workspace: queue, sweep, queue, smaller batch on the queue
-    with verify_path(3):
-        q1 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
+    # the paths take turns on one workspace: sweep, early exit, sweep on a smaller batch
     with verify_path(1):
         s1 = ps.verify_rejection(target, draft, sampled, u, diagnostics=True, workspace=ws)
-    with verify_path(3):
-        q2 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
-        q3 = ps.verify_rejection(target[:5], draft[:5], sampled[:5], u[:5], workspace=ws)
-    for k in q1:
-        assert torch.equal(q1[k], q2[k]), k                  # same path: bit-identical
+    with verify_path(2):
+        e3 = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, workspace=ws)
+    with verify_path(1):
+        s2 = ps.verify_rejection(target[:5], draft[:5], sampled[:5], u[:5], workspace=ws)
     for k in ("out_tokens", "accepted_len", "bonus"):
-        assert torch.equal(q1[k], e1[k]), k
+        assert torch.equal(s1[k], e1[k]), k
+        assert torch.equal(e3[k], e1[k]), k
+        assert torch.equal(s2[k], e1[k][:5]), k
     # residual mass is summed in a different order on each path: fp32 within 1e-5
-    assert torch.allclose(q1["residual_mass"], e1["residual_mass"], rtol=1e-5, atol=0)
-    for k in ("out_tokens", "accepted_len", "bonus"):
-        assert torch.equal(s1[k], q1[k]), k
-        assert torch.equal(q3[k], q1[k][:5]), k
+    assert torch.allclose(s1["residual_mass"], e1["residual_mass"], rtol=1e-5, atol=0)
     wsg = ps.Workspace(w.B, w.K, w.V, False)
     g1 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
     g2 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
     for k in g1:
         assert torch.equal(g1[k], g2[k]), k
-    with verify_path(3):
+    with verify_path(2):
         h1 = ps.verify_greedy(target, greedy, workspace=wsg)
         h2 = ps.verify_greedy(target, greedy, workspace=wsg)
     g3 = ps.verify_greedy(target, greedy, want_lse=True, workspace=wsg)
     for k in ("out_tokens", "accepted_len", "bonus"):
         assert torch.equal(h1[k], g1[k]) and torch.equal(h2[k], g1[k]) and torch.equal(g3[k], g1[k]), k
-
-
-def test_queue_refuses_diagnostics_and_short_workspace():
-    w = I.Workload("t", 4, 3, 1001, 16, 4, torch.bfloat16, seed=5, sigma_t=2.0, sigma_d=0.6)
-    target, draft = I.logits(w, DEV)
-    sampled, greedy = I.draft_tokens(w, draft)
-    u = I.uniforms(w, DEV)
-    with verify_path(3):
-        with pytest.raises(ps.PspecError):
-            ps.verify_rejection(target, draft, sampled, u, diagnostics=True)
-        with pytest.raises(ps.PspecError):
-            ps.verify_greedy(target, greedy, want_lse=True)
-        short = ps.Workspace(w.B, w.K, w.V, True)
-        short.tensor = short.tensor[:512]                          # below the queue's need
-        with pytest.raises(ps.PspecError):
-            ps.verify_rejection(target, draft, sampled, u, workspace=short)
-        r = ps.verify_rejection(target, draft, sampled, u)         # odd V is fine here
-    U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u))
 
 
 def test_empty_batch():
@@ -381,14 +343,18 @@ def test_empty_batch():
 
 
 # --------------------------------------------------------------------------- exactness
-def test_threshold_probing_exact_rule():
+@pytest.mark.parametrize("K", [1, 2, 3])
+def test_threshold_probing_exact_rule(K):
     """The kernel's accept decisions flip exactly at tau = min(1, p/q) and its draws follow
     the residual's CDF: u = tau - 2e-6 accepts, tau + 2e-6 rejects, and u at the middle of
-    each CDF interval returns that interval's token (V = 8, K = 2, all 64 draft tuples)."""
+    each CDF interval returns that interval's token (V = 8, all 8^K draft tuples of K = 1,
+    2, 3, with target and draft rows that depend on the drafted prefix): together with the
+    accept probabilities min(1, p/q) and the residual law this fixes, the emitted tokens
+    follow the target's autoregressive law exactly."""
     from tests.oracle_pins import _prefix_logits
     import itertools
     import scipy.special as sps
-    V, K = 8, 2
+    V = 8
     tuples = list(itertools.product(range(V), repeat=K))
     t = np.stack([np.stack([_prefix_logits(tp[:k], V, 1) for k in range(K + 1)]) for tp in tuples])
     q = np.stack([np.stack([_prefix_logits(tp[:k], V, 2) for k in range(K)]) for tp in tuples])
@@ -433,7 +399,8 @@ def test_threshold_probing_exact_rule():
     D = torch.from_numpy(np.stack(rows_d)).to(DEV)
     Uu = torch.from_numpy(np.stack(rows_u)).to(DEV)
     o = oracle.verify_rejection(np.stack(rows_t), np.stack(rows_q), np.stack(rows_d), np.stack(rows_u))
-    for path in (1, 2, 3):
+    print(f"[probing] K={K}: {len(tuples)} tuples, {len(expect_a)} probes")
+    for path in (1, 2):
         with verify_path(path):
             r = ps.verify_rejection(T, Qd, D, Uu)
         a = r["accepted_len"].cpu().numpy()
@@ -588,11 +555,12 @@ def test_sampling_workloads(name):
     _sample_both(logits, u)
 
 
-def test_sampling_b1024_sampled():
+def test_sampling_b1024_all_rows():
+    """All 7168 drafter rows of the large batch against the oracle."""
     w = I.B1024
     _, logits = I.logits(w, DEV)
     u = I.uniforms(w, DEV)[:, :w.K].contiguous()
-    _sample_both(logits, u, seqs=_sample(w.B, 32, 11))
+    _sample_both(logits, u)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -708,11 +676,12 @@ def test_step_c64_fused(rule):
     _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, 0, True)
 
 
-@pytest.mark.parametrize("path,fused", [(0, False), (1, False), (2, True), (3, False), (4, False)])
+@pytest.mark.parametrize("path", [0, 1, 2])
 @pytest.mark.parametrize("rule", ["greedy", "rejection"])
-def test_step_tiny_every_path(rule, path, fused):
-    if path == 4 and rule == "greedy":
-        fused = True                         # the greedy rule takes the fused early exit
+def test_step_tiny_every_path(rule, path):
+    # automatic at 5 sequences: the greedy rule takes the fused early exit, the rejection
+    # rule the full sweep followed by the build launch
+    fused = path == 2 or (path == 0 and rule == "greedy")
     w = I.scaled(I.C64, B=5, V=4096, H=64)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
@@ -754,31 +723,26 @@ def test_step_fused_invalid_layout_sets_bit():
     assert bo["err"].item() & ps._binding.PSPEC_DEVERR_LAYOUT
 
 
-@pytest.mark.parametrize("stream", [1, 2])
-def test_step_b1024_fused(stream):
+def test_step_b1024_fused():
     """Full size with fusion forced on (the automatic choice at 1024 sequences is two
-    launches), then forced off; rows streamed through registers or shared-memory rings."""
+    launches), then forced off; every sequence against the oracle."""
     w = I.B1024
     target, draft = I.logits(w, DEV)
     sampled, _ = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
     binp = I.build_inputs(w, DEV, drafts=sampled)
     try:
-        ps.pspec_set_ee_stream(stream)
         ps.pspec_set_step_fusion(1)
         v, _ = _step_check(target, draft, sampled, u, binp, 0, True)
         ps.pspec_set_step_fusion(2)
         _step_check(target, draft, sampled, u, binp, 2, False)
     finally:
         ps.pspec_set_step_fusion(0)
-        ps.pspec_set_ee_stream(0)
-    seqs = _sample(w.B, 24, 5)
-    U.compare_rejection(v, U.oracle_rejection(target, draft, sampled, u, seqs), seqs)
+    U.compare_rejection(v, U.oracle_rejection(target, draft, sampled, u))
 
 
-@pytest.mark.parametrize("path,stream,tail", [(0, 1, 0), (0, 2, 0), (2, 1, 20), (1, 0, 0), (3, 0, 0),
-                                              (4, 0, 0)])
-def test_step_cuda_graph_replay(path, stream, tail):
+@pytest.mark.parametrize("path,tail", [(0, 0), (2, 20), (1, 0)])
+def test_step_cuda_graph_replay(path, tail):
     """One step captured in a CUDA graph and replayed with new uniforms and drafts copied
     into the captured buffers gives what the eager calls give for those inputs (the
     kernels leave their workspace counters at zero, so replays need no reset); `tail`
@@ -793,7 +757,7 @@ def test_step_cuda_graph_replay(path, stream, tail):
     vout = ps.api.verify_outputs(w.B, w.K, DEV, False, True, True)
     bout = ps.api.build_outputs(w.B, w.K, 64, binp["T_cap"], binp["verify_hidden"].dtype, DEV)
     d_in, u_in = sampled.clone(), u.clone()
-    with verify_path(path), ee_stream(stream), tail_split(tail):
+    with verify_path(path), tail_split(tail):
         ps.step(target, d_in, binp, draft_logits=draft, uniforms=u_in, residual_mass=True,
                 workspace=ws, out=vout, build_out=bout)           # warm-up outside capture
         torch.cuda.synchronize()
@@ -843,7 +807,7 @@ def _k_len_case(B, K, V, seed, with_bad=False):
     return w, target, draft, sampled, greedy, u, klt
 
 
-@pytest.mark.parametrize("path", [1, 2, 3, 4])
+@pytest.mark.parametrize("path", [1, 2])
 def test_k_len_verify_every_path(path):
     """Per-sequence draft counts on every path against the oracle (reading R14): counts
     0..K, -1 in the unused draft slots (no range error), out-of-range counts clamped with
@@ -873,7 +837,7 @@ def test_k_len_all_k_equals_fixed_k():
     sampled, greedy = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
     kl = torch.full((w.B,), w.K, dtype=torch.int32, device=DEV)
-    for path in (1, 2, 3):
+    for path in (1, 2):
         with verify_path(path):
             a = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
             b = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, k_len=kl)
@@ -885,16 +849,17 @@ def test_k_len_all_k_equals_fixed_k():
             assert torch.equal(c[k], d[k]), (path, k)
 
 
-def test_k_len_b1024_sampled():
+def test_k_len_b1024_all_sequences():
     w = I.B1024
     target, draft = I.logits(w, DEV)
-    sampled, _ = I.draft_tokens(w, draft)
+    sampled, greedy = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
     kl = torch.as_tensor(np.random.default_rng(3).integers(0, w.K + 1, size=w.B).astype(np.int32),
                          device=DEV)
     r = ps.verify_rejection(target, draft, sampled, u, k_len=kl)
-    seqs = _sample(w.B, 32, 13)
-    U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u, seqs, k_len=kl), seqs)
+    g = ps.verify_greedy(target, greedy, k_len=kl)
+    U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u, k_len=kl))
+    U.compare_greedy(g, U.oracle_greedy(target, greedy, want_lse=False, k_len=kl))
 
 
 @pytest.mark.parametrize("K,L_extra", [(1, 0), (3, 2), (7, 0), (7, 4)])
@@ -914,7 +879,7 @@ def test_k_len_build(K, L_extra):
     d = torch.argmax(draft.float(), dim=2).to(torch.int32)
     u = torch.rand((37, K + 1), generator=g, device=DEV)
     klt = binp["k_len"]
-    for path, fused in ((2, True), (1, False), (3, False)):
+    for path, fused in ((2, True), (1, False)):
         for uu in (u, None):
             v1, b1 = _step_check_k(target, draft, d, uu, binp, path, fused, klt)
             assert b1["err"].item() == 0
@@ -957,45 +922,10 @@ def _step_check_k(target, draft, drafts, u, binp, path, expect_fused, klt):
     return v2, b2
 
 
-@pytest.mark.parametrize("path,stream,B", [(3, 0, 64), (2, 2, 64), (2, 2, 8)])
-def test_bounded_waits_give_up_and_context_survives(path, stream, B):
-    """With every bounded wait cut to one poll, the work queue (path 3) and the shared-memory
-    ring (early exit, stream 2) give up waits that would have succeeded: the call reports
-    PSPEC_DEVERR_TIMEOUT (the queue always does here; a ring wait may succeed at its first
-    poll, and then the outputs must be right), the kernels still end, and the next call on
-    the same context and workspace, with the default limits, gives the oracle's outputs."""
-    w = I.Workload("t", B, 5, 40000, 64, 16, torch.bfloat16, seed=B + path, sigma_t=2.0, sigma_d=0.5)
-    target, draft = I.logits(w, DEV)
-    sampled, _ = I.draft_tokens(w, draft)
-    u = I.uniforms(w, DEV)
-    o = U.oracle_rejection(target, draft, sampled, u)
-    ws = ps.Workspace(w.B, w.K, w.V, True)
-    TIMEOUT = ps._binding.PSPEC_DEVERR_TIMEOUT
-    try:
-        ps.pspec_set_wait_limit(1)
-        with verify_path(path), ee_stream(stream):
-            r = ps.verify_rejection(target, draft, sampled, u, workspace=ws)
-            torch.cuda.synchronize()
-    finally:
-        ps.pspec_set_wait_limit(0)
-    err = r["err"].item()
-    assert err & ~TIMEOUT == 0, err
-    if path == 3:
-        assert err & TIMEOUT
-    if not err & TIMEOUT:
-        U.compare_rejection(r, o)
-    with verify_path(path), ee_stream(stream):
-        r2 = ps.verify_rejection(target, draft, sampled, u, workspace=ws)
-    torch.cuda.synchronize()
-    assert r2["err"].item() == 0
-    U.check_verify_invariants(r2, sampled, w.V)
-    U.compare_rejection(r2, o)
-
-
 @pytest.mark.parametrize("X", [1, 37, 150])
 def test_early_exit_tail_split(X):
-    """The batch split over two early-exit launches (4-CTA clusters, then the last X
-    sequences in 8-CTA clusters queued with programmatic dependent launch) against the
+    """The batch split over two early-exit launches (the large-batch clusters, then the last
+    X sequences in wider clusters queued with programmatic dependent launch) against the
     oracle, both rules, K_i included, and the step fused and unfused."""
     w = I.Workload("t", 300, 7, 40000, 64, 16, torch.bfloat16, seed=X, sigma_t=2.0, sigma_d=0.5)
     target, draft = I.logits(w, DEV)
@@ -1026,12 +956,11 @@ def test_early_exit_tail_split(X):
         ps.pspec_set_step_fusion(0)
 
 
-@pytest.mark.parametrize("stream", [1, 2])
 @pytest.mark.parametrize("G", [2, 4, 8, 12, 16])
-def test_early_exit_every_cluster_size(G, stream):
-    """The early-exit kernel with each cluster size (the automatic choice is 4 from 128
-    sequences on, wider below) and both ways of streaming rows against the oracle, unfused
-    and with the step fused, K_i included."""
+def test_early_exit_every_cluster_size(G):
+    """The early-exit kernel with each cluster size (the automatic choice is fixed from 128
+    sequences on, wider below) against the oracle, unfused and with the step fused, K_i
+    included."""
     w = I.scaled(I.C64, B=40, V=40000, H=64)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
@@ -1041,7 +970,6 @@ def test_early_exit_every_cluster_size(G, stream):
     binp = I.build_inputs(w, DEV, drafts=sampled)
     try:
         ps.pspec_set_cluster_size(G)
-        ps.pspec_set_ee_stream(stream)
         with verify_path(2):
             g = ps.verify_greedy(target, greedy)
             r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
@@ -1053,4 +981,76 @@ def test_early_exit_every_cluster_size(G, stream):
         _step_check(target, draft, greedy, None, binp, 2, True)
     finally:
         ps.pspec_set_cluster_size(0)
-        ps.pspec_set_ee_stream(0)
+
+
+# --------------------------------------------------------------------------- per-call options
+def test_per_call_options_two_threads_two_streams():
+    """Two host threads, each on a stream of its own, verify the same batch at the same time
+    with different per-call options -- one forces the full sweep with short segments, the
+    other the early exit with 4-CTA clusters and a split batch -- while the process-wide
+    defaults ask for something else again (early exit, 16-CTA clusters).  Each call runs
+    with its own options (the per-thread last-call queries report its path, cluster width
+    and launch count), and every output equals the oracle's; a call without options follows
+    the defaults."""
+    import threading
+    w = I.scaled(I.C64, B=96, V=40000)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    u = I.uniforms(w, DEV)
+    orj = U.oracle_rejection(target, draft, sampled, u)
+    og = U.oracle_greedy(target, greedy, want_lse=False)
+    opts = {"sweep": {"verify_path": 1, "segment_elems": 4096},
+            "early": {"verify_path": 2, "cluster_size": 4, "tail_split": 16}}
+    want = {"sweep": (1, 2, 1), "early": (2, 2, 2)}     # (path, rejection launches, greedy path)
+    results, errors = {}, []
+    start = threading.Barrier(2)
+
+    def worker(name):
+        try:
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                o = opts[name]
+                wsr = ps.Workspace(w.B, w.K, w.V, True, DEV, o)
+                wsg = ps.Workspace(w.B, w.K, w.V, False, DEV, o)
+                start.wait()
+                seen, outs = [], []
+                for _ in range(10):
+                    r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True,
+                                            workspace=wsr, options=o)
+                    seen.append((ps.pspec_last_verify_path(), ps.pspec_last_launches(),
+                                 ps.pspec_last_cluster_size()))
+                    g = ps.verify_greedy(target, greedy, workspace=wsg, options=o)
+                    seen.append((ps.pspec_last_verify_path(),))
+                    outs.append((r, g))
+                s.synchronize()
+            results[name] = (seen, outs)
+        except Exception as e:  # noqa: BLE001
+            errors.append((name, repr(e)))
+
+    ps.pspec_set_verify_path(2)
+    ps.pspec_set_cluster_size(16)
+    try:
+        th = [threading.Thread(target=worker, args=(n,)) for n in opts]
+        for t in th:
+            t.start()
+        for t in th:
+            t.join()
+        assert not errors, errors
+        d = ps.verify_rejection(target, draft, sampled, u)
+        assert ps.pspec_last_verify_path() == 2 and ps.pspec_last_cluster_size() == 16
+    finally:
+        ps.pspec_set_verify_path(0)
+        ps.pspec_set_cluster_size(0)
+    torch.cuda.synchronize()
+    U.compare_rejection(d, orj)
+    for name, (seen, outs) in results.items():
+        path, launches, gpath = want[name]
+        for j in range(0, len(seen), 2):
+            assert seen[j][0] == path and seen[j][1] == launches, (name, seen[j])
+            if name == "early":
+                assert seen[j][2] == 4, (name, seen[j])
+            assert seen[j + 1][0] == gpath, (name, seen[j + 1])
+        for r, g in outs:
+            assert r["err"].item() == 0 and g["err"].item() == 0
+            U.compare_rejection(r, orj)
+            U.compare_greedy(g, og)

@@ -2,10 +2,11 @@
 
 pspec_verify_greedy_noalloc exists for callers that cannot give the library device
 memory (their HBM is reserved up front for the KV cache, or they have no allocator at
-all): it runs the same kernel with scratch that lives inside the library.  Here it must
-produce the same outputs as pspec_verify_greedy, on two calls in a row (the second call
-finds the first call's leftovers in the shared scratch), and refuse requests larger
-than its fixed scratch without launching anything.
+all): it runs the full-sweep greedy kernel with scratch that lives inside the library.
+Here it must produce the same outputs as pspec_verify_greedy, on two calls in a row (the
+second call finds the first call's leftovers in the shared scratch), report its own
+launch count and path to the last-call queries, and refuse requests larger than its fixed
+scratch without launching anything.
 
 This file is collected last, so a run that stops at the first failure has already run
 every other test; it also passes when run alone in a fresh process.
@@ -47,7 +48,11 @@ def test_noalloc_matches_workspace_entry_point(name, B, K, V, dtype):
     torch.cuda.synchronize()
     for call in range(2):
         o = _outputs(B, K)
+        if V % 8 == 0:             # leave the early-exit path in the last-call record first
+            ps.verify_greedy(target, greedy)
+            assert ps.pspec_last_verify_path() == 2
         b.pspec_verify_greedy_noalloc(target_logits=target, draft_tokens=greedy, **o)
+        assert ps.pspec_last_launches() == 1 and ps.pspec_last_verify_path() == 1
         torch.cuda.synchronize()
         for k in ("out_tokens", "accepted_len", "bonus"):
             assert torch.equal(o[k], ref[k]), (name, call, k)
@@ -70,3 +75,7 @@ def test_noalloc_refuses_oversized_requests():
     assert ei.value.status == b.PSPEC_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert (o["accepted_len"] == -7).all()          # nothing was launched
+    # an empty batch launches nothing and says so
+    e = _outputs(0, K)
+    b.pspec_verify_greedy_noalloc(target_logits=target[:0], draft_tokens=drafts[:0], **e)
+    assert ps.pspec_last_launches() == 0 and ps.pspec_last_verify_path() == 0
