@@ -42,8 +42,9 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["pspec", "reference"], default="pspec")
     p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
-    p.add_argument("--path", choices=["auto", "sweep", "early"], default="auto",
-                   help="verify path: automatic selection, full sweep or early exit")
+    p.add_argument("--path", choices=["auto", "sweep", "early", "stream"], default="auto",
+                   help="verify path: automatic selection, full sweep, early exit (clusters), "
+                        "streamed early exit (bulk copies, one SM or two per sequence)")
     p.add_argument("--cluster", type=int, default=0, help="early-exit cluster size (0 auto)")
     p.add_argument("--fusion", choices=["auto", "always", "never"], default="auto",
                    help="verify + build in one launch (early-exit path): pspec_set_step_fusion")
@@ -203,7 +204,7 @@ def aggregate_value(steps: int, world: int, elapsed_ms: float) -> float:
 
 def set_tuning(ps, args):
     """The command line's tuning as the library's process-wide defaults."""
-    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2}[args.path])
+    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "stream": 3}[args.path])
     ps.pspec_set_cluster_size(args.cluster)
     ps.pspec_set_tail_split(args.tail)
     ps.pspec_set_step_fusion({"auto": 0, "always": 1, "never": 2}[args.fusion])
@@ -370,13 +371,21 @@ def run_pspec(args, rank, world, local_rank):
     draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if split else None
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
     acc = vout["accepted_len"].cpu().numpy()
-    early = path == 2                       # the path that reads rows only up to a_i
+    early = path in (2, 3)                  # the paths that read rows only up to a_i
     vbytes, bbytes = algorithmic_bytes(w, args.mode, acc, early)
     full_vbytes, _ = algorithmic_bytes(w, args.mode, acc, False)
     hbm, peak_src = peaks()
     ms_step = elapsed_ms / K
     step_gbs = (vbytes + bbytes) / (ms_step * 1e-3) / 1e9
-    if early:
+    if path == 3:
+        dom_kernel = "stream_kernel"
+        src = ["speculative_decoding_step_pspec_b200/csrc/verify_stream.cu",
+               "speculative_decoding_step_pspec_b200/csrc/mbar.cuh",
+               "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
+               "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
+        if fused:
+            src.append("speculative_decoding_step_pspec_b200/csrc/build_common.cuh")
+    elif early:
         dom_kernel = "ee_kernel"
         src = ["speculative_decoding_step_pspec_b200/csrc/verify_early_exit.cu",
                "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
@@ -395,7 +404,7 @@ def run_pspec(args, rank, world, local_rank):
     dom_bytes = vbytes + bbytes if whole else vbytes       # a fused launch also builds
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     # both rules share the early-exit kernel: its profiles are per rule
-    prof_key = dom_kernel + ("_greedy" if not rej and dom_kernel == "ee_kernel" else "")
+    prof_key = dom_kernel + ("_greedy" if not rej and dom_kernel in ("ee_kernel", "stream_kernel") else "")
     # a whole-step timing (fused launch, graph replay) is not one kernel's: no kernel traffic
     # (the profiles hold the named workloads' sizes: none for an overridden batch)
     traffic = None if (whole or args.batch) else profiled_traffic(prof_key, args.workload, src_hash)
@@ -409,7 +418,9 @@ def run_pspec(args, rank, world, local_rank):
             "workload": f"{args.workload}{'' if not args.batch else ' (B overridden)'}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
                         f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
-            "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)"}[path],
+            "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)",
+                            3: f"streamed early exit ({cluster} CTA(s) of one SM each per sequence, "
+                               "rows by bulk copies)"}[path],
             "step": ("one launch (verify + build fused)" if fused else "verify launches + build launch")
                     + (", CUDA graph replay" if graph is not None else ""),
             "l2": "inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9),
@@ -479,7 +490,7 @@ def step_summary(w, mode, ms_list, launches, path, acc, hbm, graph_ms=None):
     """One workload's numbers: step time, algorithmic GB/s and fraction of the peak, launches
     per step and the accepted-length histogram."""
     import numpy as np
-    early = path == 2
+    early = path in (2, 3)
     vbytes, bbytes = algorithmic_bytes(w, mode, acc, early)
     ms = statistics.median(ms_list)
     gbs = (vbytes + bbytes) / (ms * 1e-3) / 1e9
@@ -488,7 +499,7 @@ def step_summary(w, mode, ms_list, launches, path, acc, hbm, graph_ms=None):
            "step_per_s": round(1e3 / ms, 1), "achieved_gbs": round(gbs, 1),
            "frac_of_peak": round(gbs / hbm, 4), "algorithmic_bytes": int(vbytes + bbytes),
            "launches_per_step": launches,
-           "verify_path": {1: "full sweep", 2: "early exit"}[path],
+           "verify_path": {1: "full sweep", 2: "early exit", 3: "streamed early exit"}[path],
            "acceptance_rate": round(float(acc.sum()) / float(np.minimum(acc + 1, w.K).sum()), 4),
            "histogram": np.bincount(acc, minlength=w.K + 1).tolist()}
     if graph_ms is not None:
@@ -516,6 +527,15 @@ def measure_workload(ps, w, inputs, mode, dev, hbm, n, flush, graph=True):
         step()
     launches, path = ps.pspec_last_launches(), ps.pspec_last_verify_path()
     ms = time_steps(step, n, flush)
+    # the same step with its argument structs filled once (what a C caller or a decode loop
+    # with fixed buffers pays per step: the launches alone)
+    call, _, _ = ps.api.prepare_step(inputs["target"], drafts, bi,
+                                     draft_logits=inputs["draft"] if rej else None,
+                                     uniforms=inputs["u"] if rej else None, workspace=ws,
+                                     out=vout, build_out=bout)
+    stream = torch.cuda.current_stream().cuda_stream
+    call(stream)
+    p_ms = time_steps(lambda: call(stream), n, flush)
     g_ms = None
     if graph:
         g = torch.cuda.CUDAGraph()
@@ -531,7 +551,9 @@ def measure_workload(ps, w, inputs, mode, dev, hbm, n, flush, graph=True):
         del g
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
     acc = vout["accepted_len"].cpu().numpy()
-    return step_summary(w, mode, ms, launches, path, acc, hbm, g_ms)
+    r = step_summary(w, mode, ms, launches, path, acc, hbm, g_ms)
+    r["prepared_call_ms_per_step"] = round(statistics.median(p_ms), 5)
+    return r
 
 
 def extra_workloads(args, w_head, d_head, dev, hbm):
@@ -855,7 +877,7 @@ def run_depth_sweep(args, local_rank):
             ms = a.elapsed_time(b) / n
             assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
             acc = vout["accepted_len"].cpu().numpy()
-            early = path == 2
+            early = path in (2, 3)
             vbytes, bbytes = algorithmic_bytes(w, "rejection", acc, early)
             points.append({"K": K, "sigma": sigma, "ms_per_step": round(ms, 4),
                            "step_per_s": round(1e3 / ms, 1),

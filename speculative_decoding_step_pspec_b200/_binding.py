@@ -18,7 +18,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpspec.s
 PSPEC_OK, PSPEC_ERR_INVALID_ARG, PSPEC_ERR_UNSUPPORTED, PSPEC_ERR_CUDA, PSPEC_ERR_WORKSPACE = range(5)
 PSPEC_F32, PSPEC_BF16 = 0, 1
 PSPEC_DEVERR_TOKEN_RANGE, PSPEC_DEVERR_ACCEPT_RANGE = 0x1, 0x2
-PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT = 0x4, 0x8
+PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT, PSPEC_DEVERR_TIMEOUT = 0x4, 0x8, 0x10
 PSPEC_DEVERR_KLEN_RANGE = 0x20
 PSPEC_ROW_CTX, PSPEC_ROW_NTP, PSPEC_ROW_MASK, PSPEC_ROW_REJ, PSPEC_ROW_PAD = range(5)
 PSPEC_PADDING_SLOT_ID = -1
@@ -50,7 +50,7 @@ class pspec_options(ctypes.Structure):
     """Tuning of one call (0 = automatic in every field); see include/pspec.h."""
     _fields_ = [
         ("verify_path", _I), ("cluster_size", _I), ("tail_split", _I), ("step_fusion", _I),
-        ("segment_elems", ctypes.c_longlong),
+        ("segment_elems", ctypes.c_longlong), ("wait_limit", ctypes.c_ulonglong),
     ]
 
 
@@ -193,7 +193,8 @@ def pspec_set_cluster_size(G: int) -> None:
 
 
 def pspec_last_verify_path() -> int:
-    """1 full sweep, 2 early exit: the path of the most recent verify call on this thread."""
+    """1 full sweep, 2 early exit, 3 streamed early exit: the path of the most recent verify
+    call on this thread."""
     return LIB.pspec_last_verify_path()
 
 
@@ -203,7 +204,8 @@ def pspec_last_cluster_size() -> int:
 
 
 def pspec_set_verify_path(path: int) -> None:
-    """Process-wide default: 0 automatic, 1 full sweep, 2 early exit (see include/pspec.h)."""
+    """Process-wide default: 0 automatic, 1 full sweep, 2 early exit, 3 streamed early exit
+    (see include/pspec.h)."""
     LIB.pspec_set_verify_path(int(path))
 
 
@@ -434,3 +436,40 @@ def pspec_verify_greedy_noalloc(*, target_logits, draft_tokens, out_tokens, acce
     st = LIB.pspec_verify_greedy_noalloc(ctypes.byref(a), _stream(stream))
     if st != PSPEC_OK:
         raise PspecError("pspec_verify_greedy_noalloc", st)
+
+
+class PreparedStep:
+    """A pspec_step_greedy / pspec_step_rejection call whose argument structs were filled
+    once, for a decode loop that reuses the same buffers every step: calling it only issues
+    the C entry point with the saved structs on the given stream (a torch.cuda.Stream, a raw
+    cudaStream_t handle, or None for torch's current stream).  The tensors the structs point
+    at are kept alive by this object and must keep their storage."""
+
+    def __init__(self, rejection: bool, v, b, workspace, keep):
+        self._name = "pspec_step_rejection" if rejection else "pspec_step_greedy"
+        self._fn = getattr(LIB, self._name)
+        self._v, self._b, self._keep = v, b, keep
+        self._vp, self._bp = ctypes.byref(v), ctypes.byref(b)
+        self._ws = _ptr(workspace, torch.uint8, "workspace")
+        self._wsn = workspace.numel()
+
+    def __call__(self, stream=None) -> None:
+        st = self._fn(self._vp, self._bp, self._ws, self._wsn, _stream(stream))
+        if st != PSPEC_OK:
+            raise PspecError(self._name, st)
+
+
+def prepare_step(*, target_logits, draft_tokens, out_tokens, accepted_len, bonus, err,
+                 workspace, build: dict, draft_logits=None, uniforms=None, residual_mass=None,
+                 k_len=None, options=None) -> PreparedStep:
+    """The argument structs of a step call (the rejection rule when `uniforms` is given),
+    filled once; see PreparedStep."""
+    K = int(target_logits.shape[1]) - 1
+    rej = uniforms is not None
+    v = _verify_args(target_logits, draft_logits if rej else None, draft_tokens, uniforms,
+                     out_tokens, accepted_len, bonus, err, None, None, None, None,
+                     residual_mass if rej else None, K, k_len, options)
+    b = _build_args(**build)
+    keep = [target_logits, draft_logits, draft_tokens, uniforms, out_tokens, accepted_len, bonus,
+            err, workspace, residual_mass, k_len, dict(build)]
+    return PreparedStep(rej, v, b, workspace, keep)

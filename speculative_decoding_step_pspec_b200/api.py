@@ -187,3 +187,36 @@ def step(target_logits: torch.Tensor, draft_tokens: torch.Tensor, build: dict, *
                              bonus=o["bonus"], err=o["err"], workspace=ws.tensor, build=bargs,
                              k_len=k_len, options=options, stream=stream)
     return o, bo
+
+
+def prepare_step(target_logits: torch.Tensor, draft_tokens: torch.Tensor, build: dict, *,
+                 draft_logits: torch.Tensor | None = None, uniforms: torch.Tensor | None = None,
+                 residual_mass: bool = False, workspace: Workspace | None = None, out=None,
+                 build_out=None, k_len: torch.Tensor | None = None, options=None) -> tuple:
+    """The arguments of ``step`` marshalled once: returns (call, verify outputs, build
+    outputs), where ``call(stream=None)`` runs the step on the same tensors with no further
+    Python-side marshalling (the buffers' contents may change between calls)."""
+    rej = uniforms is not None
+    Bn, K1, V = target_logits.shape
+    K = K1 - 1
+    dev = target_logits.device
+    o = out if out is not None else verify_outputs(Bn, K, dev, False, rej, residual_mass)
+    ws = workspace if workspace is not None else Workspace(Bn, K, V, rej, dev, options)
+    vh = build["verify_hidden"]
+    bo = build_out if build_out is not None else build_outputs(
+        Bn, K, int(vh.shape[1]), build["T_cap"], vh.dtype, vh.device)
+    bargs = dict(K=build["K"], block_size=build["block_size"], mask_id=build["mask_id"],
+                 pad_id=build["pad_id"], T_cap=build["T_cap"], qsl_in=build["qsl_in"],
+                 verify_tokens=build["verify_tokens"], verify_pos=build["verify_pos"],
+                 accepted_len=None, bonus=None, block_table=build["block_table"],
+                 verify_hidden=vh, h_shared=build["h_shared"], draft_tokens=bo["draft_tokens"],
+                 draft_pos=bo["draft_pos"], slot_mapping=bo["slot_mapping"],
+                 row_kind=bo["row_kind"], hidden_src=bo["hidden_src"], qsl_out=bo["qsl_out"],
+                 seq_lens_out=bo["seq_lens_out"], sample_idx=bo["sample_idx"],
+                 draft_hidden=bo["draft_hidden"], err=bo["err"], k_len=k_len)
+    call = _b.prepare_step(target_logits=target_logits, draft_tokens=draft_tokens,
+                           out_tokens=o["out_tokens"], accepted_len=o["accepted_len"],
+                           bonus=o["bonus"], err=o["err"], workspace=ws.tensor, build=bargs,
+                           draft_logits=draft_logits, uniforms=uniforms,
+                           residual_mass=o.get("residual_mass"), k_len=k_len, options=options)
+    return call, o, bo

@@ -72,6 +72,19 @@ namespace {
 #ifndef PSPEC_EE_GREEDY_PF
 #define PSPEC_EE_GREEDY_PF 0
 #endif
+// 1: the first batch of position k+1 is loaded into registers before the cluster barrier
+// of position k is waited on (wasted when k is the stop position).
+#ifndef PSPEC_EE_SPEC
+#define PSPEC_EE_SPEC 0
+#endif
+// The draw: warp tiles in flight per warp, and (1) an L2 bulk prefetch of the CTA's slice
+// of the draw rows when the draw starts.
+#ifndef PSPEC_EE_DRAW_U
+#define PSPEC_EE_DRAW_U 1
+#endif
+#ifndef PSPEC_EE_DRAW_PF
+#define PSPEC_EE_DRAW_PF 0
+#endif
 
 constexpr int kEERejUnroll = PSPEC_EE_REJ_UNROLL;   // vectors per row in flight (rejection)
 constexpr int kEEMinBlocks = PSPEC_EE_MIN_BLOCKS;   // CTAs per SM the register budget targets
@@ -116,38 +129,16 @@ __device__ __forceinline__ void slice_x8(const DrawRow& D, long long lo, int n, 
 // Whole-step fusion: the draft span of sequence i (output rows [qsl_out[i], qsl_out[i+1]),
 // clamped into [0, T_cap)), built by the cluster that has just decided a_i and the bonus
 // token.  The CTA holding the token (`meta`) writes the rows' metadata and the sequence's
-// outputs; every CTA of the cluster copies its share of the hidden rows (one warp per
-// row).  The cluster of the last sequence also writes the padding rows and the end offset.
-// The rows are exactly those pspec_build_draft_batch writes for a valid offset array; for
-// an invalid one every write stays in bounds and the layout bit is set, as there.
+// outputs; every CTA of the cluster copies its share of the hidden rows (the same
+// per-sequence code as the build launch, with the cluster's G CTAs as the parts).  The
+// cluster of the last sequence also writes the padding rows and the end offset.  The rows
+// are exactly those pspec_build_draft_batch writes for a valid offset array; for an invalid
+// one every write stays in bounds and the layout bit is set, as there.
 __device__ __forceinline__ void ee_build_span(const pspec_build_args& b, long long row_vecs, int i,
                                               int a, int Ki, int token, bool meta, int g, int G) {
-  const long long q0 = build_qout(b, i), q1 = build_qout(b, i + 1);
-  const long long lo = q0 < 0 ? 0 : q0;
-  const long long hi = q1 > b.T_cap ? (long long)b.T_cap : q1;
   int eb = 0;
-  if (meta) {
-    for (long long t = lo + threadIdx.x; t < hi; t += kThreads)
-      build_write_row(b, t, build_classify(b, i, t - q0, a, Ki, token), &eb);
-    if (threadIdx.x == 0) build_write_seq(b, i, a, Ki, &eb);
-  }
-  if (b.draft_hidden) {
-    const int warp = threadIdx.x >> 5;
-    for (long long t = lo + (long long)g * kWarps + warp; t < hi; t += (long long)G * kWarps)
-      build_copy_hidden(b, row_vecs, t, build_classify(b, i, t - q0, a, Ki, token));
-  }
-  if (i == b.B - 1) {                                  // padding rows and the end offset
-    const BuildRow pad{PSPEC_ROW_PAD, -1, b.pad_id, 0, -1};
-    const long long first = build_qout(b, 0);
-    const long long head = first < 0 ? 0 : (first > b.T_cap ? (long long)b.T_cap : first);
-    const long long tail = q1 < 0 ? 0 : q1;
-    const long long step = (long long)G * kThreads;
-    for (long long t = (long long)g * kThreads + threadIdx.x; t < head; t += step)
-      build_write_row(b, t, pad, &eb);
-    for (long long t = tail + (long long)g * kThreads + threadIdx.x; t < b.T_cap; t += step)
-      build_write_row(b, t, pad, &eb);
-    if (g == 0 && threadIdx.x == 0) build_write_seq(b, b.B, 0, b.K, &eb);
-  }
+  build_span(b, row_vecs, i, a, Ki, token, meta, g, G, &eb);
+  if (i == b.B - 1) build_tail_pad(b, g, G, &eb);       // padding rows and the end offset
   set_err(b.err, eb);
 }
 
@@ -207,6 +198,9 @@ ee_kernel(const EarlyExitLaunch L) {
   float dMt = -INFINITY, dMq = -INFINITY;
   double dSt = 0.0, dSq = 0.0;
   int gk = 0;                                                // greedy: argmax of the stop row
+  constexpr bool kSpec = PSPEC_EE_SPEC != 0;
+  uint4 nt[kSpec ? U : 1], nq[kSpec ? U : 1];                // next position's first batch
+  bool pre = false;                                          // ... already in nt / nq
   int k = 0;
   for (;; ++k) {
     const bool has_q = kRej && k < Ki;
@@ -233,10 +227,15 @@ ee_kernel(const EarlyExitLaunch L) {
           if (has_q) prefetch_batch(qrow, b + PF, BV, nvec);
         }
         uint4 bt[U], bq[U];
+        if (kSpec && pre && b == 0) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          bt[u] = ld_stream(tv + v0 + u * kThreads);
-          if (has_q) bq[u] = ld_stream(qv + v0 + u * kThreads);
+          for (int u = 0; u < U; ++u) { bt[u] = nt[kSpec ? u : 0]; bq[u] = nq[kSpec ? u : 0]; }
+        } else {
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            bt[u] = ld_stream(tv + v0 + u * kThreads);
+            if (has_q) bq[u] = ld_stream(qv + v0 + u * kThreads);
+          }
         }
         if constexpr (kRej) {
           consume_ms_batch<Tag, U>(bt, at);
@@ -272,6 +271,17 @@ ee_kernel(const EarlyExitLaunch L) {
       if (lane == 0) s_part[k & 1][warp] = make_float4(best.v, __int_as_float(best.i), 0.f, 0.f);
     }
     cluster_arrive();
+    pre = false;
+    if (kSpec && k + 1 <= Ki && tid + (U - 1) * kThreads < nvec) {
+      const uint4* tv = reinterpret_cast<const uint4*>(trow + L.ld);
+      const uint4* qv = reinterpret_cast<const uint4*>(qrow + L.ld);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        nt[kSpec ? u : 0] = ld_stream(tv + tid + u * kThreads);
+        if (kRej && k + 1 < Ki) nq[kSpec ? u : 0] = ld_stream(qv + tid + u * kThreads);
+      }
+      pre = true;
+    }
     cluster_wait();
 
     // ---- every warp takes the same decision from the same partials, merged in one fixed
@@ -358,17 +368,31 @@ ee_kernel(const EarlyExitLaunch L) {
     D.mq = dMq; D.inv_sq = dSq > 0.0 ? (float)(1.0 / dSq) : 0.f;
     const int ntiles = (n + 255) / 256;
     const double u = (double)L.uniforms[(long long)i * (K + 1) + Ki];
-    // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8).
+    // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8), DU tiles
+    // per warp in flight.
     auto tile_pass = [&]() {
-      for (int t = warp; t < ntiles; t += kWarps) {
-        float xt[8], xq[8], r[8];
-        slice_x8<Tag>(D, lo, n, t * 256 + lane * 8, xt, xq);
-        draw_r8(D, xt, xq, r);
-        float sum = 0.f;
+      constexpr int DU = PSPEC_EE_DRAW_U;
+      if (PSPEC_EE_DRAW_PF && tid == 0) {
+        prefetch_l2(static_cast<const elem*>(D.trow) + lo, (unsigned)(n * sizeof(elem)));
+        if (D.resid) prefetch_l2(static_cast<const elem*>(D.qrow) + lo, (unsigned)(n * sizeof(elem)));
+      }
+      for (int t0 = warp; t0 < ntiles; t0 += kWarps * DU) {
+        float xt[DU][8], xq[DU][8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sum += r[j];
-        const double ts = warp_sum_d((double)sum);
-        if (lane == 0) tsum[t] = ts;
+        for (int u = 0; u < DU; ++u)
+          slice_x8<Tag>(D, lo, n, (t0 + u * kWarps) * 256 + lane * 8, xt[u], xq[u]);
+#pragma unroll
+        for (int u = 0; u < DU; ++u) {
+          const int t = t0 + u * kWarps;
+          if (t >= ntiles) break;                            // the same on every lane
+          float r[8];
+          draw_r8(D, xt[u], xq[u], r);
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sum += r[j];
+          const double ts = warp_sum_d((double)sum);
+          if (lane == 0) tsum[t] = ts;
+        }
       }
     };
     bool own_pass_done = false;

@@ -21,7 +21,8 @@ DEV = "cuda"
 
 
 class verify_path:
-    """Force the full sweep (1) or the early-exit path (2) inside a with-block."""
+    """Force the full sweep (1), the early-exit path (2) or the streamed early exit (3)
+    inside a with-block."""
 
     def __init__(self, path):
         self.path = path
@@ -54,6 +55,18 @@ def early_exit_allowed(t):
     return t.shape[2] % 8 == 0 and t.data_ptr() % 16 == 0 and (t.stride(1) * t.element_size()) % 16 == 0
 
 
+def stream_allowed(t, G=2):
+    """The streamed early exit's shape rule: every CTA's slice holds at least 16 chunks of
+    4 KB of each row (so V >= 32768 * G for bf16, 16384 * G for fp32) and at most 512."""
+    if not early_exit_allowed(t):
+        return False
+    V, eb = t.shape[2], t.element_size()
+    vs = -(-V // G)
+    vs = -(-vs // 8) * 8
+    n_min = min(vs, V - (G - 1) * vs)
+    return n_min > 0 and -(-n_min * eb // 4096) >= 16 and -(-vs * eb // 4096) <= 512
+
+
 def _verify_both(target, draft, sampled, greedy_drafts, u, diag=True):
     """Both verify rules, on both paths, against the oracle on every sequence: the full
     sweep with every diagnostic, then (where its shape rules allow) the early-exit path in
@@ -70,17 +83,19 @@ def _verify_both(target, draft, sampled, greedy_drafts, u, diag=True):
     U.compare_greedy(gr, og)
     orj = U.oracle_rejection(target, draft, sampled, u)
     U.compare_rejection(rj, orj)
-    if early_exit_allowed(target):
-        with verify_path(2):
+    for path in (2, 3):
+        if not (early_exit_allowed(target) if path == 2 else stream_allowed(target)):
+            continue
+        with verify_path(path):
             # the early-exit path may hand the batch's last sequences to a second launch
             ge = ps.verify_greedy(target, greedy_drafts)
             assert ps.pspec_last_launches() in (1, 2)
-            assert ps.pspec_last_verify_path() == 2
+            assert ps.pspec_last_verify_path() == path
             re = ps.verify_rejection(target, draft, sampled, u, residual_mass=True)
             assert ps.pspec_last_launches() in (1, 2)
-            assert ps.pspec_last_verify_path() == 2
+            assert ps.pspec_last_verify_path() == path
         torch.cuda.synchronize()
-        assert ge["err"].item() == 0 and re["err"].item() == 0
+        assert ge["err"].item() == 0 and re["err"].item() == 0, path
         U.check_verify_invariants(ge, greedy_drafts, V)
         U.check_verify_invariants(re, sampled, V)
         U.compare_greedy(ge, og)
@@ -233,7 +248,7 @@ def test_out_of_range_draft_tokens():
     o = U.oracle_rejection(target, draft, bad, u)
     U.compare_rejection(rj, o)
     assert gr["accepted_len"][0].item() == 0 and rj["accepted_len"][0].item() == 0
-    for path in (2, 3):
+    for path in (2,):
         with verify_path(path):
             ge = ps.verify_greedy(target, bad)
             re = ps.verify_rejection(target, draft, bad, u)
@@ -984,10 +999,11 @@ def test_early_exit_every_cluster_size(G):
 
 
 # --------------------------------------------------------------------------- per-call options
-def test_per_call_options_two_threads_two_streams():
-    """Two host threads, each on a stream of its own, verify the same batch at the same time
-    with different per-call options -- one forces the full sweep with short segments, the
-    other the early exit with 4-CTA clusters and a split batch -- while the process-wide
+def test_per_call_options_threads_and_streams():
+    """Three host threads, each on a stream of its own, verify the same batch at the same time
+    with different per-call options -- one forces the full sweep with short segments, one
+    the early exit with 4-CTA clusters and a split batch, one the streamed early exit with
+    one CTA per sequence -- while the process-wide
     defaults ask for something else again (early exit, 16-CTA clusters).  Each call runs
     with its own options (the per-thread last-call queries report its path, cluster width
     and launch count), and every output equals the oracle's; a call without options follows
@@ -1000,10 +1016,12 @@ def test_per_call_options_two_threads_two_streams():
     orj = U.oracle_rejection(target, draft, sampled, u)
     og = U.oracle_greedy(target, greedy, want_lse=False)
     opts = {"sweep": {"verify_path": 1, "segment_elems": 4096},
-            "early": {"verify_path": 2, "cluster_size": 4, "tail_split": 16}}
-    want = {"sweep": (1, 2, 1), "early": (2, 2, 2)}     # (path, rejection launches, greedy path)
+            "early": {"verify_path": 2, "cluster_size": 4, "tail_split": 16},
+            "stream": {"verify_path": 3, "cluster_size": 1}}
+    # (path, rejection launches, greedy path)
+    want = {"sweep": (1, 2, 1), "early": (2, 2, 2), "stream": (3, 1, 3)}
     results, errors = {}, []
-    start = threading.Barrier(2)
+    start = threading.Barrier(len(opts))
 
     def worker(name):
         try:
@@ -1047,10 +1065,148 @@ def test_per_call_options_two_threads_two_streams():
         path, launches, gpath = want[name]
         for j in range(0, len(seen), 2):
             assert seen[j][0] == path and seen[j][1] == launches, (name, seen[j])
-            if name == "early":
-                assert seen[j][2] == 4, (name, seen[j])
+            if name != "sweep":
+                assert seen[j][2] == opts[name]["cluster_size"], (name, seen[j])
             assert seen[j + 1][0] == gpath, (name, seen[j + 1])
         for r, g in outs:
             assert r["err"].item() == 0 and g["err"].item() == 0
             U.compare_rejection(r, orj)
             U.compare_greedy(g, og)
+
+
+
+# --------------------------------------------------------------------------- streamed early exit
+def _stream_case(B, K, V, seed, sigma_d=0.6, dtype=torch.bfloat16, H=64):
+    w = I.Workload("t", B, K, V, H, 16, dtype, seed=seed, sigma_t=3.0, sigma_d=sigma_d)
+    target, draft = I.logits(w, DEV)
+    sampled, greedy = I.draft_tokens(w, draft)
+    return w, target, draft, sampled, greedy, I.uniforms(w, DEV)
+
+
+@pytest.mark.parametrize("G", [1, 2])
+@pytest.mark.parametrize("dtype,V", [(torch.bfloat16, 131072), (torch.float32, 40000),
+                                     (torch.bfloat16, 200000)])
+def test_stream_cluster_sizes_and_dtypes(G, dtype, V):
+    """The streamed early exit with one CTA and with a cluster of two per sequence, both
+    dtypes, a ragged last chunk, against the oracle; K_i included; the step fused and not."""
+    w, target, draft, sampled, greedy, u = _stream_case(40, 7, V, seed=V + G, dtype=dtype)
+    if not stream_allowed(target, G):
+        pytest.skip("shape outside the streamed path")
+    kl = torch.as_tensor(np.random.default_rng(G).integers(0, w.K + 1, size=w.B).astype(np.int32),
+                         device=DEV)
+    opts = {"verify_path": 3, "cluster_size": G}
+    g = ps.verify_greedy(target, greedy, options=opts)
+    assert ps.pspec_last_verify_path() == 3 and ps.pspec_last_cluster_size() == G
+    r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, options=opts)
+    rk = ps.verify_rejection(target, draft, sampled, u, k_len=kl, options=opts)
+    gk = ps.verify_greedy(target, greedy, k_len=kl, options=opts)
+    torch.cuda.synchronize()
+    for o in (g, r, rk, gk):
+        assert o["err"].item() == 0
+    U.compare_greedy(g, U.oracle_greedy(target, greedy, want_lse=False))
+    U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u))
+    U.compare_rejection(rk, U.oracle_rejection(target, draft, sampled, u, k_len=kl))
+    U.compare_greedy(gk, U.oracle_greedy(target, greedy, want_lse=False, k_len=kl))
+    binp = I.build_inputs(w, DEV, drafts=sampled)
+    try:
+        ps.pspec_set_cluster_size(G)
+        _step_check(target, draft, sampled, u, binp, 3, True)
+        _step_check(target, draft, greedy, None, binp, 3, True)
+        ps.pspec_set_step_fusion(2)
+        _step_check(target, draft, sampled, u, binp, 3, False)
+    finally:
+        ps.pspec_set_cluster_size(0)
+        ps.pspec_set_step_fusion(0)
+
+
+def test_stream_edge_decisions():
+    """Sequences that accept every draft (draft rows equal to the target's), that reject at
+    position 0 (a draft token with p = 0), with no drafts at all (K_i = 0), and with an
+    out-of-range draft token, on the streamed path against the oracle."""
+    w, target, draft, sampled, greedy, u = _stream_case(12, 5, 131072, seed=77)
+    draft[0] = target[0, :5]                              # identical rows: all accepted
+    target[1, 0, 17] = -float("inf")
+    sampled[1, 0] = 17                                    # p(d) = 0: rejected at once
+    sampled[2, 3] = -5                                    # out of range
+    greedy[2, 1] = w.V + 3
+    kl = torch.full((w.B,), w.K, dtype=torch.int32, device=DEV)
+    kl[3] = 0
+    kl[4] = 1
+    for k_len in (None, kl):
+        r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, k_len=k_len,
+                                options={"verify_path": 3})
+        g = ps.verify_greedy(target, greedy, k_len=k_len, options={"verify_path": 3})
+        torch.cuda.synchronize()
+        assert r["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
+        assert g["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
+        r["err"].zero_()
+        g["err"].zero_()
+        U.compare_rejection(r, U.oracle_rejection(target, draft, sampled, u, k_len=k_len))
+        U.compare_greedy(g, U.oracle_greedy(target, greedy, want_lse=False, k_len=k_len))
+        if k_len is None:
+            assert r["accepted_len"][0].item() == w.K and r["accepted_len"][1].item() == 0
+
+
+def test_stream_graph_replay():
+    """The streamed step captured in a CUDA graph and replayed with new uniforms and drafts
+    gives, bit for bit, what the eager calls on the same path give, and those match the
+    oracle (two paths may differ only on draws the oracle flags as near a CDF boundary,
+    because they round their prefix sums in different orders)."""
+    w, target, draft, sampled, greedy, u = _stream_case(160, 7, 131072, seed=5)
+    binp = I.build_inputs(w, DEV, drafts=sampled)
+    ws = ps.Workspace(w.B, w.K, w.V, True)
+    vout = ps.api.verify_outputs(w.B, w.K, DEV, False, True, True)
+    bout = ps.api.build_outputs(w.B, w.K, w.H, binp["T_cap"], binp["verify_hidden"].dtype, DEV)
+    d_in, u_in = sampled.clone(), u.clone()
+    opts = {"verify_path": 3}
+    ps.step(target, d_in, binp, draft_logits=draft, uniforms=u_in, residual_mass=True,
+            workspace=ws, out=vout, build_out=bout, options=opts)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g):
+            ps.step(target, d_in, binp, draft_logits=draft, uniforms=u_in, residual_mass=True,
+                    workspace=ws, out=vout, build_out=bout, options=opts)
+    torch.cuda.current_stream().wait_stream(side)
+    gen = torch.Generator(device=DEV).manual_seed(11)
+    for rep in range(3):
+        u_new = torch.rand(u.shape, generator=gen, device=DEV).clamp_(max=I.LAST_BELOW_ONE)
+        d_new = torch.where(torch.rand(sampled.shape, generator=gen, device=DEV) < 0.2,
+                            torch.randint_like(sampled, 0, w.V), sampled)
+        u_in.copy_(u_new)
+        d_in.copy_(d_new)
+        g.replay()
+        ref_v, ref_b = ps.step(target, d_new, binp, draft_logits=draft, uniforms=u_new,
+                               residual_mass=True, options=opts)
+        torch.cuda.synchronize()
+        for k in ("out_tokens", "accepted_len", "bonus", "residual_mass"):
+            assert torch.equal(vout[k], ref_v[k]), (rep, k)
+        U.compare_rejection(ref_v, U.oracle_rejection(target, draft, d_new, u_new))
+        for k in ("draft_tokens", "draft_pos", "slot_mapping", "row_kind", "hidden_src",
+                  "qsl_out", "seq_lens_out", "sample_idx"):
+            assert torch.equal(bout[k], ref_b[k]), (rep, k)
+    del g
+
+
+@pytest.mark.parametrize("B", [8, 150])
+def test_stream_bounded_waits_give_up_and_context_survives(B):
+    """With every bounded wait of the streamed path cut to one poll, waits that would have
+    succeeded give up: the call reports PSPEC_DEVERR_TIMEOUT (or, where every wait happened
+    to succeed at its first poll, right outputs), the kernel still ends, and the next call
+    on the same context with the default limit gives the oracle's outputs."""
+    w, target, draft, sampled, greedy, u = _stream_case(B, 5, 131072, seed=B)
+    o = U.oracle_rejection(target, draft, sampled, u)
+    TIMEOUT = ps._binding.PSPEC_DEVERR_TIMEOUT
+    r = ps.verify_rejection(target, draft, sampled, u, options={"verify_path": 3, "wait_limit": 1})
+    torch.cuda.synchronize()
+    err = r["err"].item()
+    assert err & ~TIMEOUT == 0, err
+    print(f"[timeout] B={B}: error word {err:#x}")
+    if not err & TIMEOUT:
+        U.compare_rejection(r, o)
+    r2 = ps.verify_rejection(target, draft, sampled, u, options={"verify_path": 3})
+    torch.cuda.synchronize()
+    assert r2["err"].item() == 0
+    U.compare_rejection(r2, o)
