@@ -42,9 +42,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["pspec", "reference"], default="pspec")
     p.add_argument("--mode", choices=["rejection", "greedy"], default="rejection")
-    p.add_argument("--path", choices=["auto", "sweep", "early", "stream"], default="auto",
-                   help="verify path: automatic selection, full sweep, early exit (clusters), "
-                        "streamed early exit (bulk copies, one SM or two per sequence)")
+    p.add_argument("--path", choices=["auto", "sweep", "early"], default="auto",
+                   help="verify path: automatic selection, full sweep or early exit")
     p.add_argument("--cluster", type=int, default=0, help="early-exit cluster size (0 auto)")
     p.add_argument("--fusion", choices=["auto", "always", "never"], default="auto",
                    help="verify + build in one launch (early-exit path): pspec_set_step_fusion")
@@ -204,7 +203,7 @@ def aggregate_value(steps: int, world: int, elapsed_ms: float) -> float:
 
 def set_tuning(ps, args):
     """The command line's tuning as the library's process-wide defaults."""
-    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2, "stream": 3}[args.path])
+    ps.pspec_set_verify_path({"auto": 0, "sweep": 1, "early": 2}[args.path])
     ps.pspec_set_cluster_size(args.cluster)
     ps.pspec_set_tail_split(args.tail)
     ps.pspec_set_step_fusion({"auto": 0, "always": 1, "never": 2}[args.fusion])
@@ -371,21 +370,13 @@ def run_pspec(args, rank, world, local_rank):
     draw_ms = [e[1].elapsed_time(e[2]) for e in ev] if split else None
     assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
     acc = vout["accepted_len"].cpu().numpy()
-    early = path in (2, 3)                  # the paths that read rows only up to a_i
+    early = path == 2                       # the path that reads rows only up to a_i
     vbytes, bbytes = algorithmic_bytes(w, args.mode, acc, early)
     full_vbytes, _ = algorithmic_bytes(w, args.mode, acc, False)
     hbm, peak_src = peaks()
     ms_step = elapsed_ms / K
     step_gbs = (vbytes + bbytes) / (ms_step * 1e-3) / 1e9
-    if path == 3:
-        dom_kernel = "stream_kernel"
-        src = ["speculative_decoding_step_pspec_b200/csrc/verify_stream.cu",
-               "speculative_decoding_step_pspec_b200/csrc/mbar.cuh",
-               "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
-               "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
-        if fused:
-            src.append("speculative_decoding_step_pspec_b200/csrc/build_common.cuh")
-    elif early:
+    if early:
         dom_kernel = "ee_kernel"
         src = ["speculative_decoding_step_pspec_b200/csrc/verify_early_exit.cu",
                "speculative_decoding_step_pspec_b200/csrc/verify_common.cuh",
@@ -404,7 +395,7 @@ def run_pspec(args, rank, world, local_rank):
     dom_bytes = vbytes + bbytes if whole else vbytes       # a fused launch also builds
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     # both rules share the early-exit kernel: its profiles are per rule
-    prof_key = dom_kernel + ("_greedy" if not rej and dom_kernel in ("ee_kernel", "stream_kernel") else "")
+    prof_key = dom_kernel + ("_greedy" if not rej and dom_kernel == "ee_kernel" else "")
     # a whole-step timing (fused launch, graph replay) is not one kernel's: no kernel traffic
     # (the profiles hold the named workloads' sizes: none for an overridden batch)
     traffic = None if (whole or args.batch) else profiled_traffic(prof_key, args.workload, src_hash)
@@ -418,9 +409,7 @@ def run_pspec(args, rank, world, local_rank):
             "workload": f"{args.workload}{'' if not args.batch else ' (B overridden)'}: B={w.B}, K={w.K}, V={w.V}, H={w.H}, block_size="
                         f"{w.block_size}, bf16 logits, {args.mode} verify + P-EAGLE draft-batch build",
             "B": w.B, "K": w.K, "V": w.V, "H": w.H, "mode": args.mode,
-            "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)",
-                            3: f"streamed early exit ({cluster} CTA(s) of one SM each per sequence, "
-                               "rows by bulk copies)"}[path],
+            "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)"}[path],
             "step": ("one launch (verify + build fused)" if fused else "verify launches + build launch")
                     + (", CUDA graph replay" if graph is not None else ""),
             "l2": "inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9),
@@ -490,7 +479,7 @@ def step_summary(w, mode, ms_list, launches, path, acc, hbm, graph_ms=None):
     """One workload's numbers: step time, algorithmic GB/s and fraction of the peak, launches
     per step and the accepted-length histogram."""
     import numpy as np
-    early = path in (2, 3)
+    early = path == 2
     vbytes, bbytes = algorithmic_bytes(w, mode, acc, early)
     ms = statistics.median(ms_list)
     gbs = (vbytes + bbytes) / (ms * 1e-3) / 1e9
@@ -499,7 +488,7 @@ def step_summary(w, mode, ms_list, launches, path, acc, hbm, graph_ms=None):
            "step_per_s": round(1e3 / ms, 1), "achieved_gbs": round(gbs, 1),
            "frac_of_peak": round(gbs / hbm, 4), "algorithmic_bytes": int(vbytes + bbytes),
            "launches_per_step": launches,
-           "verify_path": {1: "full sweep", 2: "early exit", 3: "streamed early exit"}[path],
+           "verify_path": {1: "full sweep", 2: "early exit"}[path],
            "acceptance_rate": round(float(acc.sum()) / float(np.minimum(acc + 1, w.K).sum()), 4),
            "histogram": np.bincount(acc, minlength=w.K + 1).tolist()}
     if graph_ms is not None:
@@ -877,7 +866,7 @@ def run_depth_sweep(args, local_rank):
             ms = a.elapsed_time(b) / n
             assert int(vout["err"].item()) == 0 and int(bout["err"].item()) == 0
             acc = vout["accepted_len"].cpu().numpy()
-            early = path in (2, 3)
+            early = path == 2
             vbytes, bbytes = algorithmic_bytes(w, "rejection", acc, early)
             points.append({"K": K, "sigma": sigma, "ms_per_step": round(ms, 4),
                            "step_per_s": round(1e3 / ms, 1),

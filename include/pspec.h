@@ -71,9 +71,6 @@ typedef enum { PSPEC_F32 = 0, PSPEC_BF16 = 1 } pspec_dtype;
                                           negative block id: that row's slot is -1 */
 #define PSPEC_DEVERR_LAYOUT 0x8        /* qsl_in not an offset array, or a sequence with
                                           fewer than K+1 verify rows */
-#define PSPEC_DEVERR_TIMEOUT 0x10      /* a bounded wait inside the streamed early exit ran
-                                          out: that call's outputs are not valid (the
-                                          kernel still ends; see pspec_options.wait_limit) */
 #define PSPEC_DEVERR_KLEN_RANGE 0x20   /* k_len[i] outside [0, K]: clamped into it */
 
 /* Row kinds written to pspec_build_args.row_kind. */
@@ -95,20 +92,15 @@ typedef enum { PSPEC_F32 = 0, PSPEC_BF16 = 1 } pspec_dtype;
  * outside the documented range read as 0.
  */
 typedef struct {
-  int verify_path;           /* 0 automatic, 1 full sweep, 2 early exit, 3 streamed early
-                                exit (see pspec_set_verify_path) */
-  int cluster_size;          /* early exit: CTAs per cluster, 2, 4, 8, 12 or 16; streamed
-                                early exit: 1 or 2; 0 automatic */
+  int verify_path;           /* 0 automatic, 1 full sweep, 2 early exit (see
+                                pspec_set_verify_path) */
+  int cluster_size;          /* early exit: CTAs per cluster, 2, 4, 8, 12 or 16; 0 automatic */
   int tail_split;            /* early exit: sequences of the second, wider launch; 0 automatic,
                                 -1 never, n > 0 that many (at most half the batch) */
   int step_fusion;           /* pspec_step_*: 0 automatic, 1 always one launch, 2 never */
   long long segment_elems;   /* full sweep: elements of one row per CTA (rounded up to a
                                 multiple of 8); 0 automatic.  Changes the workspace size:
                                 see pspec_verify_workspace_bytes_opt. */
-  unsigned long long wait_limit; /* streamed early exit: polls before each bounded wait gives
-                                up (0: the default, about a second); a small value makes
-                                waits that would have succeeded give up, for tests of the
-                                PSPEC_DEVERR_TIMEOUT path */
 } pspec_options;
 
 /*

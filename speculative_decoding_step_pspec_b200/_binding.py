@@ -18,7 +18,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpspec.s
 PSPEC_OK, PSPEC_ERR_INVALID_ARG, PSPEC_ERR_UNSUPPORTED, PSPEC_ERR_CUDA, PSPEC_ERR_WORKSPACE = range(5)
 PSPEC_F32, PSPEC_BF16 = 0, 1
 PSPEC_DEVERR_TOKEN_RANGE, PSPEC_DEVERR_ACCEPT_RANGE = 0x1, 0x2
-PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT, PSPEC_DEVERR_TIMEOUT = 0x4, 0x8, 0x10
+PSPEC_DEVERR_BLOCK_RANGE, PSPEC_DEVERR_LAYOUT = 0x4, 0x8
 PSPEC_DEVERR_KLEN_RANGE = 0x20
 PSPEC_ROW_CTX, PSPEC_ROW_NTP, PSPEC_ROW_MASK, PSPEC_ROW_REJ, PSPEC_ROW_PAD = range(5)
 PSPEC_PADDING_SLOT_ID = -1
@@ -50,7 +50,7 @@ class pspec_options(ctypes.Structure):
     """Tuning of one call (0 = automatic in every field); see include/pspec.h."""
     _fields_ = [
         ("verify_path", _I), ("cluster_size", _I), ("tail_split", _I), ("step_fusion", _I),
-        ("segment_elems", ctypes.c_longlong), ("wait_limit", ctypes.c_ulonglong),
+        ("segment_elems", ctypes.c_longlong),
     ]
 
 
@@ -193,8 +193,7 @@ def pspec_set_cluster_size(G: int) -> None:
 
 
 def pspec_last_verify_path() -> int:
-    """1 full sweep, 2 early exit, 3 streamed early exit: the path of the most recent verify
-    call on this thread."""
+    """1 full sweep, 2 early exit: the path of the most recent verify call on this thread."""
     return LIB.pspec_last_verify_path()
 
 
@@ -204,8 +203,7 @@ def pspec_last_cluster_size() -> int:
 
 
 def pspec_set_verify_path(path: int) -> None:
-    """Process-wide default: 0 automatic, 1 full sweep, 2 early exit, 3 streamed early exit
-    (see include/pspec.h)."""
+    """Process-wide default: 0 automatic, 1 full sweep, 2 early exit (see include/pspec.h)."""
     LIB.pspec_set_verify_path(int(path))
 
 

@@ -26,8 +26,8 @@ thread_local int t_last_cluster = 0;   // CTAs per cluster of the last early-exi
 // values read as automatic.
 pspec_options resolve(const pspec_options* o) {
   pspec_options r = o ? *o : g_defaults;
-  if (r.verify_path < 0 || r.verify_path > 3) r.verify_path = 0;
-  if (!(r.cluster_size == 1 || r.cluster_size == 2 || r.cluster_size == 4 || r.cluster_size == 8 ||
+  if (r.verify_path < 0 || r.verify_path > 2) r.verify_path = 0;
+  if (!(r.cluster_size == 2 || r.cluster_size == 4 || r.cluster_size == 8 ||
         r.cluster_size == 12 || r.cluster_size == 16))
     r.cluster_size = 0;
   if (r.tail_split < 0) r.tail_split = -1;
@@ -100,19 +100,15 @@ pspec_status check_build(const pspec_build_args* a, BuildLaunch* L) {
         (a->verify_hidden && !aligned16(a->verify_hidden)))
       return PSPEC_ERR_INVALID_ARG;
   }
+  const long long meta_threads = (long long)a->T_cap + a->B + 1;
+  const long long hid_rows = (long long)a->T_in + (long long)a->B * (a->K - 1);
+  if ((meta_threads + kThreads - 1) / kThreads + (hid_rows + kWarps - 1) / kWarps >= 0x7fffffffLL)
+    return PSPEC_ERR_UNSUPPORTED;
   *L = BuildLaunch{};
   L->a = *a;
   L->row_vecs = (long long)a->H * (long long)elem_bytes(a->hidden_dtype) / 16;
-  // CTAs per sequence: kBuildRowsPerPart rows each of a uniform span (2K rows)
-  const long long parts = (2LL * a->K + kBuildRowsPerPart - 1) / kBuildRowsPerPart;
-  const long long pad_rows = (long long)a->T_cap - a->T_in - (long long)a->B * (a->K - 1) + 1;
-  long long pad_blocks = (pad_rows + kBuildThreads - 1) / kBuildThreads;
-  if (pad_blocks < 1) pad_blocks = 1;
-  if (pad_blocks > 1024) pad_blocks = 1024;
-  if ((long long)a->B * parts + pad_blocks >= 0x7fffffffLL) return PSPEC_ERR_UNSUPPORTED;
-  L->parts = (int)parts;
-  L->rows_per_part = kBuildRowsPerPart;
-  L->pad_blocks = (int)pad_blocks;
+  L->meta_blocks = (int)((meta_threads + kThreads - 1) / kThreads);
+  L->hid_rows = (int)hid_rows;
   return PSPEC_OK;
 }
 
@@ -146,7 +142,6 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, const pspec_opti
   EarlyExitLaunch L{};
   L.B = a->B; L.K = a->K; L.V = a->V; L.ld = a->ld; L.dtype = a->dtype;
   L.rejection = rejection;
-  L.spin_limit = (unsigned)(o.wait_limit < 0xffffffffull ? o.wait_limit : 0xffffffffull);
   L.target = a->target_logits;
   L.draft = a->draft_logits;
   L.draft_tokens = a->draft_tokens;
@@ -162,37 +157,13 @@ bool try_early_exit(const pspec_verify_args* a, bool rejection, const pspec_opti
     L.b = fuse->a;
     L.row_vecs = fuse->row_vecs;
   }
-  // The streamed early exit (one SM, or a cluster of two, per sequence; rows fed by bulk
-  // copies): forced by path 3, automatic from kStreamMinB sequences on where V allows it.
-  const int Gs = (o.cluster_size == 1 || o.cluster_size == 2) ? o.cluster_size : kStreamCluster;
-  const bool stream_ok = stream_shape_ok(a->V, Gs, a->dtype);
-  if (o.verify_path == 3 || (o.verify_path == 0 && a->B >= kStreamMinB && stream_ok)) {
-    if (!stream_ok) {
-      *st = PSPEC_ERR_UNSUPPORTED;
-      return true;
-    }
-    L.G = Gs;
-    L.vs = stream_slice(a->V, Gs);
-    L.seq0 = 0;
-    L.nseq = a->B;
-    if (launch_stream(L, stream) != cudaSuccess) {
-      *st = PSPEC_ERR_CUDA;
-      return true;
-    }
-    if (rejection && g_split_event) cudaEventRecord(g_split_event, stream);
-    t_last_launches = 1;
-    t_last_path = 3;
-    t_last_cluster = Gs;
-    *st = PSPEC_OK;
-    return true;
-  }
   // Cluster size: kEarlyExitCluster from kEarlyExitSmallB sequences on.  Below, the rejection
   // rule takes the widest cluster (16, 12, 8) with which every sequence's cluster is
   // resident at once (a batch that needs a second round of clusters costs a second chain of
   // positions); the greedy rule, with less work per element, 8 (16 below 16 sequences).
   L.seq0 = 0;
   L.nseq = a->B;
-  int G = o.cluster_size == 1 ? 0 : o.cluster_size;
+  int G = o.cluster_size;
   if (G == 0) {
     G = kEarlyExitCluster;
     if (a->B < kEarlyExitSmallB && !rejection) {
@@ -496,10 +467,10 @@ int pspec_last_launches(void) { return t_last_launches; }
 int pspec_last_verify_path(void) { return t_last_path; }
 int pspec_last_cluster_size(void) { return t_last_cluster; }
 
-void pspec_set_verify_path(int path) { g_defaults.verify_path = (path >= 1 && path <= 3) ? path : 0; }
+void pspec_set_verify_path(int path) { g_defaults.verify_path = (path == 1 || path == 2) ? path : 0; }
 
 void pspec_set_cluster_size(int G) {
-  g_defaults.cluster_size = (G == 1 || G == 2 || G == 4 || G == 8 || G == 12 || G == 16) ? G : 0;
+  g_defaults.cluster_size = (G == 2 || G == 4 || G == 8 || G == 12 || G == 16) ? G : 0;
 }
 
 void pspec_set_step_fusion(int mode) { g_defaults.step_fusion = (mode == 1 || mode == 2) ? mode : 0; }

@@ -120,6 +120,35 @@ __device__ __forceinline__ void build_write_seq(const pspec_build_args& a, int i
   for (int k = 0; k < K; ++k) a.sample_idx[(long long)i * K + k] = base + k;
 }
 
+// One warp: the hidden state of output row r (a verify row for CTX / NTP, h_shared for
+// MASK; rejected and padding rows keep their contents), 16-byte vectors, four in flight.
+__device__ __forceinline__ void build_copy_hidden(const pspec_build_args& a, long long row_vecs,
+                                                  long long r, const BuildRow& row) {
+  const uint4* src;
+  if (row.kind == PSPEC_ROW_CTX || row.kind == PSPEC_ROW_NTP)
+    src = static_cast<const uint4*>(a.verify_hidden) + (long long)row.src * row_vecs;
+  else if (row.kind == PSPEC_ROW_MASK)
+    src = static_cast<const uint4*>(a.h_shared);
+  else
+    return;
+  uint4* dst = static_cast<uint4*>(a.draft_hidden) + r * row_vecs;
+  const int lane = threadIdx.x & 31;
+  constexpr int U = 4;
+  for (long long v0 = lane; v0 < row_vecs; v0 += 32 * U) {
+    uint4 buf[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long v = v0 + 32LL * u;
+      if (v < row_vecs) buf[u] = __ldg(src + v);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long v = v0 + 32LL * u;
+      if (v < row_vecs) dst[v] = buf[u];
+    }
+  }
+}
+
 // The hidden rows of sequence i's span, as flat 16-byte vectors: the span's first c rows
 // (CTX and NTP) copy the c consecutive verify rows s .. s+c-1, the next K-1 rows (MASK)
 // repeat h_shared, and rejected rows are not written.  This call copies the vectors

@@ -48,12 +48,6 @@ __device__ __forceinline__ T ld_cg(const T* p) {
   return out;
 }
 
-// Asks the copy engine to bring [p, p + bytes) into L2 (p 16-byte aligned, bytes a
-// multiple of 16); nothing waits for it and no register holds the data.
-__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // The thread-block cluster barrier in two halves: arrive (release: this thread's earlier
 // shared-memory writes become visible to the cluster) and wait (acquire), so that a thread
 // can issue independent work between them.  Every thread of every CTA of the cluster

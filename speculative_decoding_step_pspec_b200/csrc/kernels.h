@@ -63,8 +63,6 @@ struct EarlyExitLaunch {
   pspec_dtype dtype;
   int rejection;         // 1: rejection rule, 0: greedy
   int G;                 // CTAs per cluster (one cluster per sequence): 2, 4, 8, 12 or 16
-                         // (streamed path: 1 or 2)
-  unsigned spin_limit;   // streamed path: polls per bounded wait (0: the default)
   int seq0, nseq;        // this launch's sequences [seq0, seq0 + nseq) of the batch's B
   int pdl;               // split batch: 1 first launch (lets the second start as its CTAs
                          // are placed), 2 second launch (its CTA 0 ends after the first grid)
@@ -102,24 +100,11 @@ struct SampleLaunch {
   void* maxes;           // workspace: (max, index) per chunk [rows*tiles]
 };
 
-// Draft-batch construction: `parts` CTAs of kBuildThreads threads per sequence, each owning
-// `rows_per_part` rows of its output span (the first also writes the per-sequence outputs),
-// then `pad_blocks` CTAs for the padding rows.
-#ifndef PSPEC_BUILD_THREADS
-#define PSPEC_BUILD_THREADS 128
-#endif
-#ifndef PSPEC_BUILD_ROWS
-#define PSPEC_BUILD_ROWS 2
-#endif
-constexpr int kBuildThreads = PSPEC_BUILD_THREADS;
-constexpr int kBuildRowsPerPart = PSPEC_BUILD_ROWS;
-
 struct BuildLaunch {
   pspec_build_args a;
   long long row_vecs;    // 16-byte vectors per hidden row
-  int parts;             // CTAs per sequence
-  int rows_per_part;     // span rows per CTA and step
-  int pad_blocks;        // CTAs writing the padding rows
+  int meta_blocks;       // CTAs of the metadata role (the rest copy hidden rows)
+  int hid_rows;          // rows the hidden role inspects: T_in + B*(K-1)
 };
 
 cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream);
@@ -131,13 +116,6 @@ cudaError_t launch_early_exit(const EarlyExitLaunch& L, cudaStream_t stream);
 // current device at once; 0 when the query fails.  Cached per device and variant.
 int early_exit_max_clusters(const EarlyExitLaunch& L);
 cudaError_t launch_sample(const SampleLaunch& L, cudaStream_t stream);
-// The streamed early exit (bulk copies into a shared-memory ring, one CTA or a cluster of
-// two per sequence, a whole SM each): whether V, the cluster size and the dtype allow it,
-// its slice length, and the launch.
-bool stream_shape_ok(int V, int G, pspec_dtype dtype);
-long long stream_slice(int V, int G);
-cudaError_t launch_stream(const EarlyExitLaunch& L, cudaStream_t stream);
-
 // Host helpers of the entry points (api.cu), shared by every verify entry point: the
 // argument checks of a verify call, and the per-thread record behind pspec_last_launches()
 // and pspec_last_verify_path().

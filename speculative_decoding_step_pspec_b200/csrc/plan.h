@@ -44,16 +44,6 @@ constexpr int kEarlyExitCluster = PSPEC_EE_CLUSTER;
 // api.cu): with 4, a batch of 64 fills only 256 CTA slots of ~900.
 constexpr int kEarlyExitSmallB = 128;
 constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this many sequences
-// The streamed early exit: automatic from this many sequences on, with clusters of this
-// many CTAs (1 or 2) per sequence.
-#ifndef PSPEC_STREAM_MIN_B
-#define PSPEC_STREAM_MIN_B (1 << 30)
-#endif
-#ifndef PSPEC_STREAM_CLUSTER
-#define PSPEC_STREAM_CLUSTER 2
-#endif
-constexpr int kStreamMinB = PSPEC_STREAM_MIN_B;
-constexpr int kStreamCluster = PSPEC_STREAM_CLUSTER;
 
 // Early exit, large batches: the last sequences go to a second launch of
 // kEarlyExitTailCluster-CTA clusters that fills the SMs as the first launch drains.

@@ -22,11 +22,6 @@
 //   * the draft tokens sit in lane registers from the start (lane k holds d_k) and the
 //     logits at d_k are requested when position k starts, so nothing in the decision waits
 //     on a dependent load;
-//   * optionally (PSPEC_EE_PF batches ahead) one thread of each CTA asks the copy engine to
-//     bring the slice's next batches into L2 (cp.async.bulk.prefetch.L2), continuing into
-//     the next position's first batches; the register loads then wait for L2 rather than
-//     for DRAM.  What is prefetched for a position that is never read is counted in the
-//     DRAM traffic;
 //   * rejection rule: at the stop position each CTA sums r = max(0, p - q) over
 //     256-element warp tiles of its slice, re-read right after the statistics pass (from
 //     L2 while the clusters in flight hold less than it); the slice totals are prefix-summed
@@ -64,26 +59,6 @@ namespace {
 #endif
 #ifndef PSPEC_EE_GREEDY_MIN_BLOCKS
 #define PSPEC_EE_GREEDY_MIN_BLOCKS 4
-#endif
-// L2 prefetch distance in batches (one batch = U vectors per thread of each row); 0 = off.
-#ifndef PSPEC_EE_PF
-#define PSPEC_EE_PF 0
-#endif
-#ifndef PSPEC_EE_GREEDY_PF
-#define PSPEC_EE_GREEDY_PF 0
-#endif
-// 1: the first batch of position k+1 is loaded into registers before the cluster barrier
-// of position k is waited on (wasted when k is the stop position).
-#ifndef PSPEC_EE_SPEC
-#define PSPEC_EE_SPEC 0
-#endif
-// The draw: warp tiles in flight per warp, and (1) an L2 bulk prefetch of the CTA's slice
-// of the draw rows when the draw starts.
-#ifndef PSPEC_EE_DRAW_U
-#define PSPEC_EE_DRAW_U 1
-#endif
-#ifndef PSPEC_EE_DRAW_PF
-#define PSPEC_EE_DRAW_PF 0
 #endif
 
 constexpr int kEERejUnroll = PSPEC_EE_REJ_UNROLL;   // vectors per row in flight (rejection)
@@ -142,22 +117,12 @@ __device__ __forceinline__ void ee_build_span(const pspec_build_args& b, long lo
   set_err(b.err, eb);
 }
 
-// The copy engine brings batch `pb` of this CTA's slice of a row into L2 (vectors
-// [pb * BV, (pb + 1) * BV) of the slice's nvec, BV = U * kThreads); nothing when past the end.
-__device__ __forceinline__ void prefetch_batch(const void* row_lo, int pb, int BV, int nvec) {
-  const long long v0 = (long long)pb * BV;
-  if (v0 >= nvec) return;
-  const long long v1 = v0 + BV < nvec ? v0 + BV : nvec;
-  prefetch_l2(static_cast<const uint4*>(row_lo) + v0, (unsigned)((v1 - v0) * 16));
-}
-
 template <typename Tag, int G, bool kRej, bool kFuse>
 __global__ void __launch_bounds__(kThreads, kRej ? kEEMinBlocks : PSPEC_EE_GREEDY_MIN_BLOCKS)
 ee_kernel(const EarlyExitLaunch L) {
   using elem = typename Tag::elem;
   constexpr int W = Tag::kVec;
   constexpr int U = kRej ? kEERejUnroll : PSPEC_EE_GREEDY_UNROLL;  // vectors in flight per row
-  constexpr int PF = kRej ? PSPEC_EE_PF : PSPEC_EE_GREEDY_PF;       // L2 prefetch distance
   constexpr int BV = U * kThreads;                                  // vectors per row and batch
   constexpr int NP = G * kWarps;                                    // warp partials per position
   constexpr int PL = (NP + 31) / 32;                                // of them per lane
@@ -188,19 +153,11 @@ ee_kernel(const EarlyExitLaunch L) {
 
   // lane k of every warp holds draft k of the sequence (-1 past K_i)
   const int dreg = lane < Ki ? __ldg(L.draft_tokens + (long long)i * K + lane) : -1;
-  if (PF > 0 && tid == 0)
-    for (int pb = 0; pb < PF; ++pb) {
-      prefetch_batch(tbase, pb, BV, nvec);
-      if (kRej && Ki > 0) prefetch_batch(qbase, pb, BV, nvec);
-    }
 
   // decision state of the stop position (every warp holds the same values)
   float dMt = -INFINITY, dMq = -INFINITY;
   double dSt = 0.0, dSq = 0.0;
   int gk = 0;                                                // greedy: argmax of the stop row
-  constexpr bool kSpec = PSPEC_EE_SPEC != 0;
-  uint4 nt[kSpec ? U : 1], nq[kSpec ? U : 1];                // next position's first batch
-  bool pre = false;                                          // ... already in nt / nq
   int k = 0;
   for (;; ++k) {
     const bool has_q = kRej && k < Ki;
@@ -220,22 +177,13 @@ ee_kernel(const EarlyExitLaunch L) {
     {
       const uint4* tv = reinterpret_cast<const uint4*>(trow);
       const uint4* qv = reinterpret_cast<const uint4*>(qrow);
-      int v0 = tid, b = 0;
-      for (; v0 + (U - 1) * kThreads < nvec; v0 += BV, ++b) {       // full batches
-        if (PF > 0 && tid == 0) {
-          prefetch_batch(trow, b + PF, BV, nvec);
-          if (has_q) prefetch_batch(qrow, b + PF, BV, nvec);
-        }
+      int v0 = tid;
+      for (; v0 + (U - 1) * kThreads < nvec; v0 += BV) {            // full batches
         uint4 bt[U], bq[U];
-        if (kSpec && pre && b == 0) {
 #pragma unroll
-          for (int u = 0; u < U; ++u) { bt[u] = nt[kSpec ? u : 0]; bq[u] = nq[kSpec ? u : 0]; }
-        } else {
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            bt[u] = ld_stream(tv + v0 + u * kThreads);
-            if (has_q) bq[u] = ld_stream(qv + v0 + u * kThreads);
-          }
+        for (int u = 0; u < U; ++u) {
+          bt[u] = ld_stream(tv + v0 + u * kThreads);
+          if (has_q) bq[u] = ld_stream(qv + v0 + u * kThreads);
         }
         if constexpr (kRej) {
           consume_ms_batch<Tag, U>(bt, at);
@@ -255,12 +203,6 @@ ee_kernel(const EarlyExitLaunch L) {
         }
       }
     }
-    // the next position's first batches, in case it is needed (k + 1 <= K_i)
-    if (PF > 0 && tid == 0 && k + 1 <= Ki)
-      for (int pb = 0; pb < PF; ++pb) {
-        prefetch_batch(trow + L.ld, pb, BV, nvec);
-        if (kRej && k + 1 < Ki) prefetch_batch(qrow + L.ld, pb, BV, nvec);
-      }
     // ---- this warp's partial, then the cluster barrier in two halves
     if constexpr (kRej) {
       const MS mt = warp_merge_ms(msacc_final(at));
@@ -270,18 +212,8 @@ ee_kernel(const EarlyExitLaunch L) {
       best = warp_argmax(best);
       if (lane == 0) s_part[k & 1][warp] = make_float4(best.v, __int_as_float(best.i), 0.f, 0.f);
     }
+    __syncwarp();
     cluster_arrive();
-    pre = false;
-    if (kSpec && k + 1 <= Ki && tid + (U - 1) * kThreads < nvec) {
-      const uint4* tv = reinterpret_cast<const uint4*>(trow + L.ld);
-      const uint4* qv = reinterpret_cast<const uint4*>(qrow + L.ld);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        nt[kSpec ? u : 0] = ld_stream(tv + tid + u * kThreads);
-        if (kRej && k + 1 < Ki) nq[kSpec ? u : 0] = ld_stream(qv + tid + u * kThreads);
-      }
-      pre = true;
-    }
     cluster_wait();
 
     // ---- every warp takes the same decision from the same partials, merged in one fixed
@@ -368,31 +300,17 @@ ee_kernel(const EarlyExitLaunch L) {
     D.mq = dMq; D.inv_sq = dSq > 0.0 ? (float)(1.0 / dSq) : 0.f;
     const int ntiles = (n + 255) / 256;
     const double u = (double)L.uniforms[(long long)i * (K + 1) + Ki];
-    // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8), DU tiles
-    // per warp in flight.
+    // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8).
     auto tile_pass = [&]() {
-      constexpr int DU = PSPEC_EE_DRAW_U;
-      if (PSPEC_EE_DRAW_PF && tid == 0) {
-        prefetch_l2(static_cast<const elem*>(D.trow) + lo, (unsigned)(n * sizeof(elem)));
-        if (D.resid) prefetch_l2(static_cast<const elem*>(D.qrow) + lo, (unsigned)(n * sizeof(elem)));
-      }
-      for (int t0 = warp; t0 < ntiles; t0 += kWarps * DU) {
-        float xt[DU][8], xq[DU][8];
+      for (int t = warp; t < ntiles; t += kWarps) {
+        float xt[8], xq[8], r[8];
+        slice_x8<Tag>(D, lo, n, t * 256 + lane * 8, xt, xq);
+        draw_r8(D, xt, xq, r);
+        float sum = 0.f;
 #pragma unroll
-        for (int u = 0; u < DU; ++u)
-          slice_x8<Tag>(D, lo, n, (t0 + u * kWarps) * 256 + lane * 8, xt[u], xq[u]);
-#pragma unroll
-        for (int u = 0; u < DU; ++u) {
-          const int t = t0 + u * kWarps;
-          if (t >= ntiles) break;                            // the same on every lane
-          float r[8];
-          draw_r8(D, xt[u], xq[u], r);
-          float sum = 0.f;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) sum += r[j];
-          const double ts = warp_sum_d((double)sum);
-          if (lane == 0) tsum[t] = ts;
-        }
+        for (int j = 0; j < 8; ++j) sum += r[j];
+        const double ts = warp_sum_d((double)sum);
+        if (lane == 0) tsum[t] = ts;
       }
     };
     bool own_pass_done = false;

@@ -52,14 +52,13 @@ def test_tuning_setters_and_queries():
     its valid values and falls back to the automatic choice on others (setters only: nothing
     launches); the last-call queries start at zero on a thread that made no call."""
     assert ps.pspec_last_verify_path() == 0 and ps.pspec_last_cluster_size() == 0
-    zero = dict(verify_path=0, cluster_size=0, tail_split=0, step_fusion=0, segment_elems=0,
-                wait_limit=0)
+    zero = dict(verify_path=0, cluster_size=0, tail_split=0, step_fusion=0, segment_elems=0)
     assert ps.pspec_get_options() == zero
     try:
-        for path, want in ((1, 1), (2, 2), (3, 3), (4, 0), (9, 0), (-1, 0)):
+        for path, want in ((1, 1), (2, 2), (3, 0), (4, 0), (9, 0), (-1, 0)):
             ps.pspec_set_verify_path(path)
             assert ps.pspec_get_options()["verify_path"] == want
-        for G, want in ((1, 1), (2, 2), (4, 4), (8, 8), (12, 12), (16, 16), (5, 0), (0, 0)):
+        for G, want in ((1, 0), (2, 2), (4, 4), (8, 8), (12, 12), (16, 16), (5, 0), (0, 0)):
             ps.pspec_set_cluster_size(G)
             assert ps.pspec_get_options()["cluster_size"] == want
         for n, want in ((96, 96), (1, 1), (-1, -1), (-7, -1), (0, 0)):
@@ -80,14 +79,13 @@ def test_tuning_setters_and_queries():
 
 
 def test_options_struct_layout_and_workspace():
-    """The options struct the binding builds has the header's layout (four ints, then two
-    64-bit counts at offsets 16 and 24), the verify argument struct ends with its pointer,
-    and a call's own segment length changes the workspace size as the process-wide one
-    does."""
+    """The options struct the binding builds has the header's layout (four ints, then a
+    64-bit count at offset 16), the verify argument struct ends with its pointer, and a
+    call's own segment length changes the workspace size as the process-wide one does."""
     o = b.pspec_options
     assert [f for f, _ in o._fields_] == ["verify_path", "cluster_size", "tail_split",
-                                          "step_fusion", "segment_elems", "wait_limit"]
-    assert o.segment_elems.offset == 16 and o.wait_limit.offset == 24 and ctypes.sizeof(o) == 32
+                                          "step_fusion", "segment_elems"]
+    assert o.segment_elems.offset == 16 and ctypes.sizeof(o) == 24
     assert b.pspec_verify_args._fields_[-1][0] == "options"
     f = b.pspec_verify_workspace_bytes
     base = f(64, 7, 151936, True)

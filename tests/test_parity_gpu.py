@@ -21,8 +21,7 @@ DEV = "cuda"
 
 
 class verify_path:
-    """Force the full sweep (1), the early-exit path (2) or the streamed early exit (3)
-    inside a with-block."""
+    """Force the full sweep (1) or the early-exit path (2) inside a with-block."""
 
     def __init__(self, path):
         self.path = path
@@ -55,18 +54,6 @@ def early_exit_allowed(t):
     return t.shape[2] % 8 == 0 and t.data_ptr() % 16 == 0 and (t.stride(1) * t.element_size()) % 16 == 0
 
 
-def stream_allowed(t, G=2):
-    """The streamed early exit's shape rule: every CTA's slice holds at least 16 chunks of
-    4 KB of each row (so V >= 32768 * G for bf16, 16384 * G for fp32) and at most 512."""
-    if not early_exit_allowed(t):
-        return False
-    V, eb = t.shape[2], t.element_size()
-    vs = -(-V // G)
-    vs = -(-vs // 8) * 8
-    n_min = min(vs, V - (G - 1) * vs)
-    return n_min > 0 and -(-n_min * eb // 4096) >= 16 and -(-vs * eb // 4096) <= 512
-
-
 def _verify_both(target, draft, sampled, greedy_drafts, u, diag=True):
     """Both verify rules, on both paths, against the oracle on every sequence: the full
     sweep with every diagnostic, then (where its shape rules allow) the early-exit path in
@@ -83,8 +70,8 @@ def _verify_both(target, draft, sampled, greedy_drafts, u, diag=True):
     U.compare_greedy(gr, og)
     orj = U.oracle_rejection(target, draft, sampled, u)
     U.compare_rejection(rj, orj)
-    for path in (2, 3):
-        if not (early_exit_allowed(target) if path == 2 else stream_allowed(target)):
+    for path in (2,):
+        if not early_exit_allowed(target):
             continue
         with verify_path(path):
             # the early-exit path may hand the batch's last sequences to a second launch
@@ -1002,8 +989,8 @@ def test_early_exit_every_cluster_size(G):
 def test_per_call_options_threads_and_streams():
     """Three host threads, each on a stream of its own, verify the same batch at the same time
     with different per-call options -- one forces the full sweep with short segments, one
-    the early exit with 4-CTA clusters and a split batch, one the streamed early exit with
-    one CTA per sequence -- while the process-wide
+    the early exit with 4-CTA clusters and a split batch, one the early exit with 8-CTA
+    clusters in one launch -- while the process-wide
     defaults ask for something else again (early exit, 16-CTA clusters).  Each call runs
     with its own options (the per-thread last-call queries report its path, cluster width
     and launch count), and every output equals the oracle's; a call without options follows
@@ -1017,9 +1004,9 @@ def test_per_call_options_threads_and_streams():
     og = U.oracle_greedy(target, greedy, want_lse=False)
     opts = {"sweep": {"verify_path": 1, "segment_elems": 4096},
             "early": {"verify_path": 2, "cluster_size": 4, "tail_split": 16},
-            "stream": {"verify_path": 3, "cluster_size": 1}}
+            "early8": {"verify_path": 2, "cluster_size": 8, "step_fusion": 2}}
     # (path, rejection launches, greedy path)
-    want = {"sweep": (1, 2, 1), "early": (2, 2, 2), "stream": (3, 1, 3)}
+    want = {"sweep": (1, 2, 1), "early": (2, 2, 2), "early8": (2, 1, 2)}
     results, errors = {}, []
     start = threading.Barrier(len(opts))
 
@@ -1075,28 +1062,26 @@ def test_per_call_options_threads_and_streams():
 
 
 
-# --------------------------------------------------------------------------- streamed early exit
-def _stream_case(B, K, V, seed, sigma_d=0.6, dtype=torch.bfloat16, H=64):
+# --------------------------------------------------------------------------- early exit, more shapes
+def _ee_case(B, K, V, seed, sigma_d=0.6, dtype=torch.bfloat16, H=64):
     w = I.Workload("t", B, K, V, H, 16, dtype, seed=seed, sigma_t=3.0, sigma_d=sigma_d)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
     return w, target, draft, sampled, greedy, I.uniforms(w, DEV)
 
 
-@pytest.mark.parametrize("G", [1, 2])
+@pytest.mark.parametrize("G", [4, 16])
 @pytest.mark.parametrize("dtype,V", [(torch.bfloat16, 131072), (torch.float32, 40000),
-                                     (torch.bfloat16, 200000)])
-def test_stream_cluster_sizes_and_dtypes(G, dtype, V):
-    """The streamed early exit with one CTA and with a cluster of two per sequence, both
-    dtypes, a ragged last chunk, against the oracle; K_i included; the step fused and not."""
-    w, target, draft, sampled, greedy, u = _stream_case(40, 7, V, seed=V + G, dtype=dtype)
-    if not stream_allowed(target, G):
-        pytest.skip("shape outside the streamed path")
+                                     (torch.bfloat16, 200008)])
+def test_early_exit_dtypes_and_ragged_slices(G, dtype, V):
+    """The early exit with both dtypes and a last slice shorter than the others, against the
+    oracle; K_i included; the step fused and not."""
+    w, target, draft, sampled, greedy, u = _ee_case(40, 7, V, seed=V + G, dtype=dtype)
     kl = torch.as_tensor(np.random.default_rng(G).integers(0, w.K + 1, size=w.B).astype(np.int32),
                          device=DEV)
-    opts = {"verify_path": 3, "cluster_size": G}
+    opts = {"verify_path": 2, "cluster_size": G}
     g = ps.verify_greedy(target, greedy, options=opts)
-    assert ps.pspec_last_verify_path() == 3 and ps.pspec_last_cluster_size() == G
+    assert ps.pspec_last_verify_path() == 2 and ps.pspec_last_cluster_size() == G
     r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, options=opts)
     rk = ps.verify_rejection(target, draft, sampled, u, k_len=kl, options=opts)
     gk = ps.verify_greedy(target, greedy, k_len=kl, options=opts)
@@ -1110,20 +1095,20 @@ def test_stream_cluster_sizes_and_dtypes(G, dtype, V):
     binp = I.build_inputs(w, DEV, drafts=sampled)
     try:
         ps.pspec_set_cluster_size(G)
-        _step_check(target, draft, sampled, u, binp, 3, True)
-        _step_check(target, draft, greedy, None, binp, 3, True)
+        _step_check(target, draft, sampled, u, binp, 2, True)
+        _step_check(target, draft, greedy, None, binp, 2, True)
         ps.pspec_set_step_fusion(2)
-        _step_check(target, draft, sampled, u, binp, 3, False)
+        _step_check(target, draft, sampled, u, binp, 2, False)
     finally:
         ps.pspec_set_cluster_size(0)
         ps.pspec_set_step_fusion(0)
 
 
-def test_stream_edge_decisions():
+def test_early_exit_edge_decisions():
     """Sequences that accept every draft (draft rows equal to the target's), that reject at
-    position 0 (a draft token with p = 0), with no drafts at all (K_i = 0), and with an
-    out-of-range draft token, on the streamed path against the oracle."""
-    w, target, draft, sampled, greedy, u = _stream_case(12, 5, 131072, seed=77)
+    position 0 (a draft token with p = 0), with no drafts at all (K_i = 0) or one, and with
+    out-of-range draft tokens, on the early exit against the oracle."""
+    w, target, draft, sampled, greedy, u = _ee_case(12, 5, 131072, seed=77)
     draft[0] = target[0, :5]                              # identical rows: all accepted
     target[1, 0, 17] = -float("inf")
     sampled[1, 0] = 17                                    # p(d) = 0: rejected at once
@@ -1134,8 +1119,8 @@ def test_stream_edge_decisions():
     kl[4] = 1
     for k_len in (None, kl):
         r = ps.verify_rejection(target, draft, sampled, u, residual_mass=True, k_len=k_len,
-                                options={"verify_path": 3})
-        g = ps.verify_greedy(target, greedy, k_len=k_len, options={"verify_path": 3})
+                                options={"verify_path": 2})
+        g = ps.verify_greedy(target, greedy, k_len=k_len, options={"verify_path": 2})
         torch.cuda.synchronize()
         assert r["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
         assert g["err"].item() == ps._binding.PSPEC_DEVERR_TOKEN_RANGE
@@ -1145,68 +1130,3 @@ def test_stream_edge_decisions():
         U.compare_greedy(g, U.oracle_greedy(target, greedy, want_lse=False, k_len=k_len))
         if k_len is None:
             assert r["accepted_len"][0].item() == w.K and r["accepted_len"][1].item() == 0
-
-
-def test_stream_graph_replay():
-    """The streamed step captured in a CUDA graph and replayed with new uniforms and drafts
-    gives, bit for bit, what the eager calls on the same path give, and those match the
-    oracle (two paths may differ only on draws the oracle flags as near a CDF boundary,
-    because they round their prefix sums in different orders)."""
-    w, target, draft, sampled, greedy, u = _stream_case(160, 7, 131072, seed=5)
-    binp = I.build_inputs(w, DEV, drafts=sampled)
-    ws = ps.Workspace(w.B, w.K, w.V, True)
-    vout = ps.api.verify_outputs(w.B, w.K, DEV, False, True, True)
-    bout = ps.api.build_outputs(w.B, w.K, w.H, binp["T_cap"], binp["verify_hidden"].dtype, DEV)
-    d_in, u_in = sampled.clone(), u.clone()
-    opts = {"verify_path": 3}
-    ps.step(target, d_in, binp, draft_logits=draft, uniforms=u_in, residual_mass=True,
-            workspace=ws, out=vout, build_out=bout, options=opts)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        with torch.cuda.graph(g):
-            ps.step(target, d_in, binp, draft_logits=draft, uniforms=u_in, residual_mass=True,
-                    workspace=ws, out=vout, build_out=bout, options=opts)
-    torch.cuda.current_stream().wait_stream(side)
-    gen = torch.Generator(device=DEV).manual_seed(11)
-    for rep in range(3):
-        u_new = torch.rand(u.shape, generator=gen, device=DEV).clamp_(max=I.LAST_BELOW_ONE)
-        d_new = torch.where(torch.rand(sampled.shape, generator=gen, device=DEV) < 0.2,
-                            torch.randint_like(sampled, 0, w.V), sampled)
-        u_in.copy_(u_new)
-        d_in.copy_(d_new)
-        g.replay()
-        ref_v, ref_b = ps.step(target, d_new, binp, draft_logits=draft, uniforms=u_new,
-                               residual_mass=True, options=opts)
-        torch.cuda.synchronize()
-        for k in ("out_tokens", "accepted_len", "bonus", "residual_mass"):
-            assert torch.equal(vout[k], ref_v[k]), (rep, k)
-        U.compare_rejection(ref_v, U.oracle_rejection(target, draft, d_new, u_new))
-        for k in ("draft_tokens", "draft_pos", "slot_mapping", "row_kind", "hidden_src",
-                  "qsl_out", "seq_lens_out", "sample_idx"):
-            assert torch.equal(bout[k], ref_b[k]), (rep, k)
-    del g
-
-
-@pytest.mark.parametrize("B", [8, 150])
-def test_stream_bounded_waits_give_up_and_context_survives(B):
-    """With every bounded wait of the streamed path cut to one poll, waits that would have
-    succeeded give up: the call reports PSPEC_DEVERR_TIMEOUT (or, where every wait happened
-    to succeed at its first poll, right outputs), the kernel still ends, and the next call
-    on the same context with the default limit gives the oracle's outputs."""
-    w, target, draft, sampled, greedy, u = _stream_case(B, 5, 131072, seed=B)
-    o = U.oracle_rejection(target, draft, sampled, u)
-    TIMEOUT = ps._binding.PSPEC_DEVERR_TIMEOUT
-    r = ps.verify_rejection(target, draft, sampled, u, options={"verify_path": 3, "wait_limit": 1})
-    torch.cuda.synchronize()
-    err = r["err"].item()
-    assert err & ~TIMEOUT == 0, err
-    print(f"[timeout] B={B}: error word {err:#x}")
-    if not err & TIMEOUT:
-        U.compare_rejection(r, o)
-    r2 = ps.verify_rejection(target, draft, sampled, u, options={"verify_path": 3})
-    torch.cuda.synchronize()
-    assert r2["err"].item() == 0
-    U.compare_rejection(r2, o)
