@@ -20,6 +20,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import re
 import statistics
@@ -135,7 +136,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x2: "applications_clocks_setting", 0x10: "sync_boost"}
 
-    def __init__(self, torch_device: int, period_s: float = 0.01):
+    def __init__(self, torch_device: int, period_s: float = 0.002):
         import subprocess
         import torch
         self.samples, self.max_sm, self.err = [], None, None
@@ -159,29 +160,45 @@ class ClockSampler:
 
     def __enter__(self):
         self.t_start = time.time()
+        self.t_timed_end = None
         return self
+
+    def mark_timed_end(self):
+        """End of the timed region; samples after it (up to the context's exit) come from
+        the same steps run on, untimed, so that a timed region shorter than NVML's update
+        interval still has clock readings beside it."""
+        self.t_timed_end = time.time()
 
     def __exit__(self, *a):
         self.t_end = time.time()
+        if self.t_timed_end is None:
+            self.t_timed_end = self.t_end
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=30)
         for ln in out.splitlines():
             f = ln.split()
             if len(f) == 4 and self.t_start <= float(f[0]) <= self.t_end:
-                self.samples.append((int(f[1]), float(f[2]), int(f[3])))
+                self.samples.append((float(f[0]), int(f[1]), float(f[2]), int(f[3])))
 
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_sm, "reasons": [], "source": "nvml",
                     "note": self.err or "no samples inside the timed region"}
-        sms = [s[0] for s in self.samples]
+        timed = [s for s in self.samples if s[0] <= self.t_timed_end]
+        use = timed or self.samples
+        sms = [s[1] for s in use]
         bits = 0
         for s in self.samples:
-            bits |= s[2]
+            bits |= s[3]
         reasons = sorted(v for k, v in self.REASONS.items() if bits & k)
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": self.max_sm,
-                "sm_mhz_min": min(sms), "power_w_max": round(max(s[1] for s in self.samples), 1),
-                "reasons": reasons, "samples": len(sms), "source": "nvml, 10 ms period"}
+                "sm_mhz_min": min(s[1] for s in self.samples),
+                "power_w_max": round(max(s[2] for s in self.samples), 1),
+                "reasons": reasons, "samples_timed_region": len(timed),
+                "samples": len(self.samples),
+                "source": "nvml, polled every ~2 ms" + (
+                    "" if timed else "; sm_mhz from the same steps run on for 0.25 s right "
+                    "after the timed region (none of its samples fell inside it)")}
 
 
 def max_over_ranks(ms: float, world: int, device) -> float:
@@ -336,6 +353,16 @@ def run_pspec(args, rank, world, local_rank):
     for e in ev:          # torch only times events it has seen recorded; the library
         e[1].record()     # re-records the split event between the two verify launches
     torch.cuda.synchronize()
+
+    def one_step():
+        if graph is not None:
+            graph.replay()
+        elif fused:
+            fused_step()
+        else:
+            verify()
+            build()
+
     with sampler:
         t0.record()
         for s in range(K):
@@ -357,7 +384,12 @@ def run_pspec(args, rank, world, local_rank):
                 ev[s][3].record()
         t1.record()
         torch.cuda.synchronize()
-    ps.pspec_set_split_event(None)
+        sampler.mark_timed_end()
+        ps.pspec_set_split_event(None)
+        # clock readings beside a short timed region: the same steps for 0.25 s more
+        for _ in range(min(4000, int(math.ceil(250.0 / max(t0.elapsed_time(t1) / K, 1e-3))))):
+            one_step()
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
@@ -458,16 +490,24 @@ def run_pspec(args, rank, world, local_rank):
 
 
 # ----------------------------------------------------------------------------- other workloads
+def flush_l2(buf):
+    """Evicts the step's data from L2: a buffer larger than L2 is written, then read back, so
+    that L2 ends up holding clean lines of it and the timed launch does not pay for writing
+    back the flush's own dirty lines."""
+    buf.fill_(1)
+    buf.max()
+
+
 def time_steps(fn, n, flush=None):
     """Device time of each of n calls of fn (CUDA events on the current stream, one pair per
-    call); with `flush`, a buffer larger than L2 is rewritten before every call, outside the
-    timed pair."""
+    call); with `flush`, a buffer larger than L2 is written and read before every call,
+    outside the timed pair."""
     import torch
     pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
              for _ in range(n)]
     for a, b in pairs:
         if flush is not None:
-            flush.fill_(1)
+            flush_l2(flush)
         a.record()
         fn()
         b.record()
@@ -565,7 +605,7 @@ def extra_workloads(args, w_head, d_head, dev, hbm):
         w, d = make_workload(name, dev, 0)
         for mode in ("rejection", "greedy"):
             r = measure_workload(ps, w, d, mode, dev, hbm, 50, flush)
-            r["l2"] = "256 MB buffer rewritten before every step (outside the timed events)"
+            r["l2"] = "256 MB buffer written then read before every step (outside the timed events)"
             out[f"{name}_{mode}"] = r
         del d
     # the c=1 recipe's acceptance needs more than one sequence: 256 independent draws
@@ -595,7 +635,7 @@ def extra_workloads(args, w_head, d_head, dev, hbm):
             pts.append(p)
             del dd, target, draft, sampled, greedy
             torch.cuda.empty_cache()
-    out["depth_sweep"] = {"l2": "256 MB buffer rewritten before every step", "points": pts}
+    out["depth_sweep"] = {"l2": "256 MB buffer written then read before every step", "points": pts}
     return out
 
 
@@ -743,7 +783,7 @@ def run_build_only(args, local_rank):
     torch.cuda.synchronize()
     times = []
     for _ in range(args.steps):
-        flush.fill_(1)
+        flush_l2(flush)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         build()
@@ -795,7 +835,7 @@ def run_sample_only(args, local_rank):
     with sampler:
         for a, b in ev:
             if flush is not None:
-                flush.fill_(1)
+                flush_l2(flush)
             a.record()
             ps.sample_drafts(draft, u, workspace=ws, out=out)
             b.record()
@@ -814,7 +854,7 @@ def run_sample_only(args, local_rank):
         "mode": args.sample_only, "rows": w.B * w.K, "steps": args.steps,
         "ms_mean": round(ms, 5), "ms_median": round(statistics.median(times), 5),
         "rows_per_s": round(w.B * w.K / (ms * 1e-3), 1),
-        "l2": "rows larger than L2; no flush" if flush is None else "256 MB flush between launches",
+        "l2": "rows larger than L2; no flush" if flush is None else "256 MB buffer written then read between launches",
         "roofline": {"kernel": "sample_kernel", "bound": "hbm", "achieved": round(gbs, 1),
                      "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
                      "traffic": profiled_traffic("sample_kernel", args.workload,

@@ -83,6 +83,11 @@ __device__ void meta_role(const pspec_build_args& a, long long t) {
 }
 
 __global__ void __launch_bounds__(kThreads) build_kernel(const BuildLaunch L) {
+  // Launched as a programmatic dependent of the stream's previous kernel: the CTAs may be
+  // placed while that kernel's last CTAs still run (the verify launches allow it once all
+  // their CTAs have started), and wait here until it has finished and its writes are
+  // visible.  After any other kernel this returns at once.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if ((int)blockIdx.x < L.meta_blocks) {
     meta_role(L.a, (long long)blockIdx.x * kThreads + threadIdx.x);
   } else {
@@ -97,8 +102,17 @@ __global__ void __launch_bounds__(kThreads) build_kernel(const BuildLaunch L) {
 cudaError_t launch_build(const BuildLaunch& L, cudaStream_t stream) {
   long long hid_blocks = L.a.draft_hidden ? (L.hid_rows + kWarps - 1) / kWarps : 0;
   long long grid = L.meta_blocks + hid_blocks;
-  build_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(L);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, build_kernel, L);
 }
 
 }  // namespace pspec

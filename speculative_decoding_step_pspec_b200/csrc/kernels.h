@@ -64,8 +64,8 @@ struct EarlyExitLaunch {
   int rejection;         // 1: rejection rule, 0: greedy
   int G;                 // CTAs per cluster (one cluster per sequence): 2, 4, 8, 12 or 16
   int seq0, nseq;        // this launch's sequences [seq0, seq0 + nseq) of the batch's B
-  int pdl;               // split batch: 1 first launch (lets the second start as its CTAs
-                         // are placed), 2 second launch (its CTA 0 ends after the first grid)
+  int pdl;               // split batch: 1 first launch, 2 second launch (a programmatic
+                         // dependent of the first; its CTA 0 ends after the first grid)
   long long vs;          // slice of each row per CTA (elements, multiple of 8)
   const void* target;
   const void* draft;

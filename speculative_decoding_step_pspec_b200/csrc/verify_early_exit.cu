@@ -23,9 +23,10 @@
 //     logits at d_k are requested when position k starts, so nothing in the decision waits
 //     on a dependent load;
 //   * rejection rule: at the stop position each CTA sums r = max(0, p - q) over
-//     256-element warp tiles of its slice, re-read right after the statistics pass (from
-//     L2 while the clusters in flight hold less than it); the slice totals are prefix-summed
-//     in rank order on every CTA, and the CTA whose slice holds u_K * Z rescans one tile.
+//     256-element warp tiles of its slice, re-read right after the statistics pass and
+//     backwards (the most recently streamed lines first, while L2 still holds them); the
+//     slice totals are prefix-summed in rank order on every CTA, and the CTA whose slice
+//     holds u_K * Z rescans one tile.
 //     When the draw is from the target row itself (all drafts passed), the slice totals
 //     follow from the statistics already merged and only the CTA holding u_K * Z goes over
 //     its slice.
@@ -129,7 +130,12 @@ ee_kernel(const EarlyExitLaunch L) {
   cg::cluster_group cluster = cg::this_cluster();
   const int g = (int)cluster.block_rank();
   const int i = L.seq0 + (int)(blockIdx.x / G);
-  if (L.pdl == 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Every CTA lets the stream's next programmatic launch begin once it has started: the
+  // second launch of a split batch, or the draft-batch build, whose CTAs are then placed
+  // as this grid's finish and wait (griddepcontrol.wait) for its completion.  A dependent
+  // grid launches only after all of this grid's CTAs have started, so none of them can be
+  // kept from a slot by the waiting CTAs.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = L.K;
   int ebk = 0;
@@ -300,9 +306,12 @@ ee_kernel(const EarlyExitLaunch L) {
     D.mq = dMq; D.inv_sq = dSq > 0.0 ? (float)(1.0 / dSq) : 0.f;
     const int ntiles = (n + 255) / 256;
     const double u = (double)L.uniforms[(long long)i * (K + 1) + Ki];
-    // Sums of r over this CTA's tiles (all warps; tile t goes to warp t mod 8).
+    // Sums of r over this CTA's tiles, the warps taking every 8th tile from the last one
+    // down: the statistics pass streamed the slice from its start, so its end is the part
+    // most likely still in L2, and going backwards the re-read meets the freshest lines
+    // before the other clusters' streams evict them.
     auto tile_pass = [&]() {
-      for (int t = warp; t < ntiles; t += kWarps) {
+      for (int t = ntiles - 1 - warp; t >= 0; t -= kWarps) {
         float xt[8], xq[8], r[8];
         slice_x8<Tag>(D, lo, n, t * 256 + lane * 8, xt, xq);
         draw_r8(D, xt, xq, r);
