@@ -336,7 +336,10 @@ PSPEC_API pspec_status pspec_verify_greedy_noalloc(const pspec_verify_args *args
  * (PSPEC_DEVERR_BLOCK_RANGE); a sequence with L_i < K+1 keeps its span as PAD rows with
  * seq_lens_out 0 and sample_idx -1 (PSPEC_DEVERR_LAYOUT); a qsl_in that is not an offset
  * array (qsl_in[0] != 0, decreasing, or qsl_in[B] > T_in) sets PSPEC_DEVERR_LAYOUT and
- * leaves the outputs unspecified but every access in bounds.
+ * leaves the outputs unspecified but every access in bounds.  The launch is a programmatic
+ * dependent of the stream's previous kernel (its CTAs may be placed while that kernel's
+ * last CTAs run, and wait for its completion before reading anything), which ordinary
+ * stream order already implies; after a non-kernel operation it is an ordinary launch.
  */
 PSPEC_API pspec_status pspec_build_draft_batch(const pspec_build_args *args, cudaStream_t stream);
 
@@ -403,8 +406,12 @@ PSPEC_API void pspec_set_cluster_size(int G);
    wider clusters, queued with programmatic dependent launch so that it starts while the
    first launch drains (the CTAs of the first launch release it when they are placed; CTA 0
    of the second waits for the first grid before it ends, so work queued later on the
-   stream sees all outputs).  0 automatic, -1 never, n > 0 that many sequences (at most
-   half the batch).  Outputs are the same either way; pspec_last_launches then reports 2. */
+   stream sees all outputs).  0 automatic (from 128 sequences on: the last 96 for the
+   rejection rule, the last 64 for the greedy rule), -1 never, n > 0 that many sequences (at
+   most half the batch).  Outputs are the same either way; pspec_last_launches then reports
+   2.  Every early-exit CTA also releases the stream's next programmatic launch when it is
+   placed: the draft-batch build of pspec_step_* and pspec_build_draft_batch is launched
+   that way and waits for the verify grid's completion before it reads anything. */
 PSPEC_API void pspec_set_tail_split(int n);
 
 /* Tuning (default of pspec_options.step_fusion): fusion of the two halves of pspec_step_*

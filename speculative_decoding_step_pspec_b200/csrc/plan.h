@@ -46,17 +46,21 @@ constexpr int kEarlyExitSmallB = 128;
 constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this many sequences
 
 // Early exit, large batches: the last sequences go to a second launch of
-// kEarlyExitTailCluster-CTA clusters that fills the SMs as the first launch drains.
+// kEarlyExitTailCluster-CTA clusters that fills the SMs as the first launch drains
+// (96 sequences for the rejection rule, 64 for the greedy rule's shorter chains).
 #ifndef PSPEC_EE_TAIL_SEQS
 #define PSPEC_EE_TAIL_SEQS 96
+#endif
+#ifndef PSPEC_EE_GREEDY_TAIL_SEQS
+#define PSPEC_EE_GREEDY_TAIL_SEQS 64
 #endif
 #ifndef PSPEC_EE_TAIL_CLUSTER
 #define PSPEC_EE_TAIL_CLUSTER 8
 #endif
 constexpr int kEarlyExitTailCluster = PSPEC_EE_TAIL_CLUSTER;
 inline int early_exit_tail(long long B, bool rejection) {
-  if (!rejection) return 0;
-  return (int)(B / 2 < PSPEC_EE_TAIL_SEQS ? B / 2 : PSPEC_EE_TAIL_SEQS);
+  const long long X = rejection ? PSPEC_EE_TAIL_SEQS : PSPEC_EE_GREEDY_TAIL_SEQS;
+  return (int)(B / 2 < X ? B / 2 : X);
 }
 
 // Per-(row, segment) partial of the greedy sweep.

@@ -154,21 +154,29 @@ ee_kernel(const EarlyExitLaunch L) {
   const long long lo = (long long)g * L.vs;                 // this CTA's slice [lo, lo + n)
   const int n = (int)max(0LL, min((long long)L.V, lo + L.vs) - lo);
   const int nvec = n / W;                                   // n is a multiple of 8
-  const elem* const tbase = static_cast<const elem*>(L.target) + (long long)i * (K + 1) * L.ld + lo;
-  const elem* const qbase = kRej ? static_cast<const elem*>(L.draft) + (long long)i * K * L.ld + lo : tbase;
+  // this CTA's slice of target row k / draft row k (recomputed where needed rather than
+  // kept in registers through the stream)
+  auto trow_of = [&](int kk) {
+    return static_cast<const elem*>(L.target) + ((long long)i * (K + 1) + kk) * L.ld + lo;
+  };
+  auto qrow_of = [&](int kk) {
+    return static_cast<const elem*>(L.draft) + ((long long)i * K + kk) * L.ld + lo;
+  };
 
   // lane k of every warp holds draft k of the sequence (-1 past K_i)
   const int dreg = lane < Ki ? __ldg(L.draft_tokens + (long long)i * K + lane) : -1;
 
-  // decision state of the stop position (every warp holds the same values)
-  float dMt = -INFINITY, dMq = -INFINITY;
-  double dSt = 0.0, dSq = 0.0;
+  // decision state of the stop position: every warp computes the same values and warp 0
+  // leaves them in shared memory for the draw, so none of them occupies registers while
+  // the rows stream
+  __shared__ float s_dM[2];                                  // (Mt, Mq)
+  __shared__ double s_dS[2];                                 // (St, Sq)
   int gk = 0;                                                // greedy: argmax of the stop row
   int k = 0;
   for (;; ++k) {
     const bool has_q = kRej && k < Ki;
-    const elem* trow = tbase + (long long)k * L.ld;
-    const elem* qrow = has_q ? qbase + (long long)k * L.ld : trow;
+    const elem* trow = trow_of(k);
+    const elem* qrow = has_q ? qrow_of(k) : trow;
     // the draft token of this position and (rejection) the logits there, wanted at the
     // decision: requested now, so the stream below hides their latency
     const int d = k < Ki ? __shfl_sync(0xffffffffu, dreg, k & 31) : -1;
@@ -265,7 +273,10 @@ ee_kernel(const EarlyExitLaunch L) {
         accept = qq > 0.0 ? (u * qq < pp) : (pp > 0.0);
       }
       stop = !accept;
-      if (stop) { dMt = Mt; dMq = Mq; dSt = st; dSq = sq; }
+      if (stop && warp == 0 && lane == 0) {
+        s_dM[0] = Mt; s_dM[1] = Mq;
+        s_dS[0] = st; s_dS[1] = sq;
+      }
     } else {
       VI b{pr[0].x, __float_as_int(pr[0].y)};
 #pragma unroll
@@ -298,10 +309,13 @@ ee_kernel(const EarlyExitLaunch L) {
   if constexpr (kRej) {
     // ---- the draw at the stop position a = k: r = max(0, p_a - q_a), or p_K after K passes
     const int a = k;
+    __syncthreads();                                         // the stop position's state
+    const float dMt = s_dM[0], dMq = s_dM[1];
+    const double dSt = s_dS[0], dSq = s_dS[1];
     DrawRow D;
-    D.trow = tbase + (long long)a * L.ld - lo;
+    D.trow = trow_of(a) - lo;
     D.resid = a < Ki;
-    D.qrow = D.resid ? qbase + (long long)a * L.ld - lo : D.trow;
+    D.qrow = D.resid ? qrow_of(a) - lo : D.trow;
     D.mt = dMt; D.inv_st = dSt > 0.0 ? (float)(1.0 / dSt) : 0.f;
     D.mq = dMq; D.inv_sq = dSq > 0.0 ? (float)(1.0 / dSq) : 0.f;
     const int ntiles = (n + 255) / 256;
