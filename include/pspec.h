@@ -406,8 +406,8 @@ PSPEC_API void pspec_set_cluster_size(int G);
    wider clusters, queued with programmatic dependent launch so that it starts while the
    first launch drains (the CTAs of the first launch release it when they are placed; CTA 0
    of the second waits for the first grid before it ends, so work queued later on the
-   stream sees all outputs).  0 automatic (from 128 sequences on: the last 96 for the
-   rejection rule, the last 64 for the greedy rule), -1 never, n > 0 that many sequences (at
+   stream sees all outputs).  0 automatic (from 128 sequences on: the last B/8, at most 96
+   for the rejection rule and 64 for the greedy rule), -1 never, n > 0 that many sequences (at
    most half the batch).  Outputs are the same either way; pspec_last_launches then reports
    2.  Every early-exit CTA also releases the stream's next programmatic launch when it is
    placed: the draft-batch build of pspec_step_* and pspec_build_draft_batch is launched

@@ -45,9 +45,11 @@ constexpr int kEarlyExitCluster = PSPEC_EE_CLUSTER;
 constexpr int kEarlyExitSmallB = 128;
 constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this many sequences
 
-// Early exit, large batches: the last sequences go to a second launch of
-// kEarlyExitTailCluster-CTA clusters that fills the SMs as the first launch drains
-// (96 sequences for the rejection rule, 64 for the greedy rule's shorter chains).
+// Early exit, large batches: the last B/8 sequences, at most 96 for the rejection rule and
+// 64 for the greedy rule's shorter chains, go to a second launch of
+// kEarlyExitTailCluster-CTA clusters that fills the SMs as the first launch drains.
+// (Measured: at 1024 sequences 96 against 64 or 160; at 256, where the first launch's
+// clusters nearly all fit at once, 32 against 64 or 96.)
 #ifndef PSPEC_EE_TAIL_SEQS
 #define PSPEC_EE_TAIL_SEQS 96
 #endif
@@ -60,7 +62,7 @@ constexpr int kStepFuseMaxB = 256;       // automatic step fusion below this man
 constexpr int kEarlyExitTailCluster = PSPEC_EE_TAIL_CLUSTER;
 inline int early_exit_tail(long long B, bool rejection) {
   const long long X = rejection ? PSPEC_EE_TAIL_SEQS : PSPEC_EE_GREEDY_TAIL_SEQS;
-  return (int)(B / 2 < X ? B / 2 : X);
+  return (int)(B / 8 < X ? B / 8 : X);
 }
 
 // Per-(row, segment) partial of the greedy sweep.
