@@ -384,9 +384,10 @@ PSPEC_API void pspec_get_options(pspec_options *out);
 /* Verify path selection (default of pspec_options.verify_path):
    0 (default) automatic -- the early-exit path when no per-row diagnostic is requested
      (target_lse, draft_lse, p_at_draft, q_at_draft all NULL), V is a multiple of 8 and
-     the logits rows start on 16-byte boundaries; for the rejection rule only when B >= 64
-     or B <= 4 (in between, the full sweep measured as fast or faster); otherwise the full
-     sweep;
+     the logits rows start on 16-byte boundaries, and the batch is large enough for the
+     early exit to pay: B >= 160 for the rejection rule, B >= 64 for the greedy rule (below,
+     the full sweep measured faster: it reads every row at once, while the early exit walks
+     each sequence's positions one after another); otherwise the full sweep;
    1 always the full sweep;
    2 always the early-exit path (PSPEC_ERR_UNSUPPORTED when the arguments do not allow it).
    Both paths give the same outputs; they differ in which rows they read. */

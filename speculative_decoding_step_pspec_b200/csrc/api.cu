@@ -112,13 +112,11 @@ pspec_status check_build(const pspec_build_args* a, BuildLaunch* L) {
   return PSPEC_OK;
 }
 
-// Which rule of the automatic selection takes the early-exit path: every batch size for the
-// greedy rule; for the rejection rule batches of at least kEarlyExitMinB sequences, and
-// batches of at most kEarlyExitRejSmallMax (a handful of sequences, where one launch of a
-// wide cluster per sequence beats the sweep's three launches).
+// Whether the automatic selection takes the early-exit path: from kEarlyExitMinB sequences on
+// for the rejection rule, from kEarlyExitGreedyMinB on for the greedy rule (plan.h gives the
+// measurements behind both).
 bool early_exit_wanted(int B, bool rejection) {
-  if (!rejection) return true;
-  return B >= kEarlyExitMinB || B <= kEarlyExitRejSmallMax;
+  return B >= (rejection ? kEarlyExitMinB : kEarlyExitGreedyMinB);
 }
 
 // The early-exit cluster path, when the arguments allow it and the selection asks for it:

@@ -26,15 +26,17 @@ constexpr long long kSegMax = 65536;     // bounds the tail of the last wave
 constexpr int kTargetCtas = kNumSMs * PSPEC_TARGET_CTAS_PER_SM;
 constexpr int kResampleTargetCtas = kNumSMs * PSPEC_DRAW_CTAS_PER_SM;
 constexpr int kDrawTilesPerCta = 64;     // separate draw launch: at most 8 tiles per warp
-// Automatic path selection: the greedy rule takes the early exit at every batch size; the
-// rejection rule from kEarlyExitMinB sequences on and up to kEarlyExitRejSmallMax sequences
-// (a handful of sequences: one launch of wide clusters beats the sweep's launches), the full
-// sweep in between.
-constexpr int kEarlyExitMinB = 64;
-#ifndef PSPEC_EE_REJ_SMALL_MAX
-#define PSPEC_EE_REJ_SMALL_MAX 4
-#endif
-constexpr int kEarlyExitRejSmallMax = PSPEC_EE_REJ_SMALL_MAX;
+// Automatic path selection: the early exit from kEarlyExitMinB sequences on for the
+// rejection rule and from kEarlyExitGreedyMinB on for the greedy rule, the full sweep below.
+// A small batch reads few bytes either way; there the early exit's chain of positions (one
+// round of loads, a cluster barrier and a decision per position, ~9 us each on a 16-CTA
+// cluster) costs more than the sweep, which reads every row at once on all SMs.  Measured
+// crossovers (prepared step calls, L2 flushed): rejection between 128 and 192 sequences
+// (V = 201088) and between 128 and 160 (V = 151936); greedy at 64-96 and 48-64.  At one
+// sequence the sweep's 0.032 ms is constant while the early exit's runs from 0.029 ms (a
+// rejection at position 0) to 0.070 ms (five acceptances): 0.044 ms averaged over 16 seeds.
+constexpr int kEarlyExitMinB = 160;
+constexpr int kEarlyExitGreedyMinB = 64;
 // CTAs per sequence on the early-exit path from kEarlyExitSmallB sequences on.
 #ifndef PSPEC_EE_CLUSTER
 #define PSPEC_EE_CLUSTER 4

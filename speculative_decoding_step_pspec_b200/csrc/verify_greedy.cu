@@ -26,6 +26,9 @@ template <typename Tag, bool kLse>
 __global__ void __launch_bounds__(kThreads)
 greedy_sweep_kernel(const GreedyLaunch L) {
   using elem = typename Tag::elem;
+  // the stream's next programmatic launch (the step's build) may be placed once every CTA
+  // of this grid has started; it waits for this grid's completion before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long item = blockIdx.x;
   const int s = (int)(item % L.S);
   const long long rowg = item / L.S;                 // i*(K+1) + k

@@ -39,6 +39,9 @@ template <typename Tag>
 __global__ void __launch_bounds__(kThreads)
 rej_stats_kernel(const RejectionLaunch L) {
   using elem = typename Tag::elem;
+  // the draw launch is a programmatic dependent of this one: its CTAs may be placed once
+  // every CTA of this grid has started, and wait for this grid's completion
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int K = L.K;
   const int R = 2 * K + 1;
   const long long item = blockIdx.x;
@@ -170,6 +173,10 @@ template <typename Tag>
 __global__ void __launch_bounds__(kThreads)
 rej_draw_kernel(const RejectionLaunch L) {
   using elem = typename Tag::elem;
+  // the statistics launch's outputs (SeqInfo, tile plans) are read only after it completed;
+  // then the stream's next programmatic launch (the step's build) may be placed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int K = L.K;
   const int i = blockIdx.x / L.C;
   const int c = blockIdx.x % L.C;
@@ -220,11 +227,18 @@ cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream,
     e = cudaEventRecord(split_event, stream);
     if (e != cudaSuccess) return e;
   }
-  if (L.dtype == PSPEC_BF16)
-    rej_draw_kernel<BF16Tag><<<(unsigned)grid2, kThreads, 0, stream>>>(L);
-  else
-    rej_draw_kernel<F32Tag><<<(unsigned)grid2, kThreads, 0, stream>>>(L);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (L.dtype == PSPEC_BF16) return cudaLaunchKernelEx(&cfg, rej_draw_kernel<BF16Tag>, L);
+  return cudaLaunchKernelEx(&cfg, rej_draw_kernel<F32Tag>, L);
 }
 
 }  // namespace pspec

@@ -245,12 +245,13 @@ def test_out_of_range_draft_tokens():
         U.compare_rejection(re, o)
 
 
-@pytest.mark.parametrize("B", [1, 4, 5, 63, 64, 200])
+@pytest.mark.parametrize("B", [1, 4, 63, 64, 159, 160, 200])
 def test_automatic_path_selection(B):
-    """Automatic selection with no per-row diagnostic requested: the greedy rule takes the
-    early exit at every batch size (two launches from 128 sequences on); the rejection rule from 64 sequences on and up to 4
-    sequences, the full sweep (two launches) in between; a diagnostic always takes the full
-    sweep; same tokens whichever path runs."""
+    """Automatic selection with no per-row diagnostic requested: the early exit from 160
+    sequences on for the rejection rule and from 64 on for the greedy rule (two launches
+    from 128 sequences on), the full sweep below (two launches for the rejection rule, one
+    for the greedy rule); a diagnostic always takes the full sweep; same tokens whichever
+    path runs."""
     w = I.Workload("t", B, 5, 4096, 16, 4, torch.bfloat16, seed=B, sigma_t=2.0, sigma_d=0.6)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
@@ -259,10 +260,13 @@ def test_automatic_path_selection(B):
     path_auto = ps.pspec_last_verify_path()
     b = ps.verify_rejection(target, draft, sampled, u, diagnostics=True)
     assert ps.pspec_last_launches() == 2 and ps.pspec_last_verify_path() == 1
-    assert path_auto == (2 if (B >= 64 or B <= 4) else 1)
+    assert path_auto == (2 if B >= 160 else 1)
     g = ps.verify_greedy(target, greedy)
-    # from 128 sequences on the last sequences go to a second launch (tail split)
-    assert ps.pspec_last_verify_path() == 2 and ps.pspec_last_launches() == (2 if B >= 128 else 1)
+    if B >= 64:
+        # from 128 sequences on the last sequences go to a second launch (tail split)
+        assert ps.pspec_last_verify_path() == 2 and ps.pspec_last_launches() == (2 if B >= 128 else 1)
+    else:
+        assert ps.pspec_last_verify_path() == 1 and ps.pspec_last_launches() == 1
     gl = ps.verify_greedy(target, greedy, want_lse=True)
     assert ps.pspec_last_verify_path() == 1
     o = U.oracle_rejection(target, draft, sampled, u)
@@ -669,22 +673,25 @@ def _step_check(target, draft, drafts, u, binp, path, expect_fused):
 
 
 @pytest.mark.parametrize("rule", ["greedy", "rejection"])
-def test_step_c64_fused(rule):
+@pytest.mark.parametrize("path", [0, 2])
+def test_step_c64_fused(rule, path):
+    # automatic at 64 sequences: the greedy rule takes the fused early exit, the rejection
+    # rule the full sweep followed by the build launch; forced early exit fuses both
     w = I.C64
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
     binp = I.build_inputs(w, DEV, drafts=sampled)
     rej = rule == "rejection"
-    _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, 0, True)
+    fused = path == 2 or not rej
+    _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, path, fused)
 
 
 @pytest.mark.parametrize("path", [0, 1, 2])
 @pytest.mark.parametrize("rule", ["greedy", "rejection"])
 def test_step_tiny_every_path(rule, path):
-    # automatic at 5 sequences: the greedy rule takes the fused early exit, the rejection
-    # rule the full sweep followed by the build launch
-    fused = path == 2 or (path == 0 and rule == "greedy")
+    # automatic at 5 sequences: both rules take the full sweep followed by the build launch
+    fused = path == 2
     w = I.scaled(I.C64, B=5, V=4096, H=64)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
