@@ -351,12 +351,13 @@ PSPEC_API pspec_status pspec_build_draft_batch(const pspec_build_args *args, cud
  * pspec_verify_greedy / pspec_verify_rejection(v, ...) followed by
  * pspec_build_draft_batch(b) with b's accepted_len and bonus taken from v's outputs
  * (b->accepted_len and b->bonus must be NULL or v->accepted_len and v->bonus; b->B and b->K
- * must equal v->B and v->K).  When the early-exit path takes the verification and fusion
- * is on (pspec_set_step_fusion; automatic: fewer than 256 sequences, where the saved launch
- * measured faster than building each span at the end of its cluster's work), ONE launch
- * does both: the cluster that decides sequence i writes sequence i's span of the draft
- * batch (its metadata and its hidden rows), and the cluster of the last sequence writes
- * the padding rows; otherwise the verify launches are followed by the build launch.
+ * must equal v->B and v->K).  When fusion is on (pspec_set_step_fusion; automatic: fewer
+ * than 256 sequences, where the saved launch measured faster than building each span at the
+ * end of the work that decides it), the verify's own last launch also builds: on the
+ * early-exit path the cluster that decides sequence i, on the full sweep the CTA that
+ * decides it (greedy) or draws its token (rejection), writes sequence i's span of the draft
+ * batch (its metadata and its hidden rows), and the one of the last sequence writes the
+ * padding rows; otherwise the verify launches are followed by the build launch.
  * pspec_last_launches() reports which.  Errors: those of the two calls it stands for; the
  * build's device-side error bits go to b->err, the verify's to v->err.
  */
@@ -415,8 +416,8 @@ PSPEC_API void pspec_set_cluster_size(int G);
    that way and waits for the verify grid's completion before it reads anything. */
 PSPEC_API void pspec_set_tail_split(int n);
 
-/* Tuning (default of pspec_options.step_fusion): fusion of the two halves of pspec_step_*
-   into one launch (early-exit path only): 0 automatic (fewer than 256 sequences), 1
+/* Tuning (default of pspec_options.step_fusion): fusion of the build of pspec_step_* into
+   the verify's last launch (either path): 0 automatic (fewer than 256 sequences), 1
    always, 2 never. */
 PSPEC_API void pspec_set_step_fusion(int mode);
 

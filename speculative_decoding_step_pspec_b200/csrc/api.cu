@@ -292,7 +292,13 @@ pspec_status verify_greedy_impl(const pspec_verify_args* a, void* workspace,
   char* ws = static_cast<char*>(workspace);
   L.cnt = z.line0 + kZwSCnt;
   L.part = ws + p.off_part;
+  if (fuse) {                                 // the deciding CTA of each sequence builds too
+    L.fuse_build = 1;
+    L.b = fuse->a;
+    L.row_vecs = fuse->row_vecs;
+  }
   if (launch_greedy(L, stream) != cudaSuccess) return PSPEC_ERR_CUDA;
+  *fused = fuse != nullptr;
   record_last_call(1, 1);
   return PSPEC_OK;
 }
@@ -338,7 +344,13 @@ pspec_status verify_rejection_impl(const pspec_verify_args* a, void* workspace,
   L.part = ws + p.off_part;
   L.seq = ws + p.off_seq;
   L.tile_sums = reinterpret_cast<double*>(ws + p.off_tiles);
+  if (fuse) {                                 // the draw's deciding CTA builds too
+    L.fuse_build = 1;
+    L.b = fuse->a;
+    L.row_vecs = fuse->row_vecs;
+  }
   if (launch_rejection(L, stream, g_split_event) != cudaSuccess) return PSPEC_ERR_CUDA;
+  *fused = fuse != nullptr;
   record_last_call(2, 1);
   return PSPEC_OK;
 }

@@ -27,6 +27,9 @@ struct GreedyLaunch {
   const int32_t* k_len;  // optional per-sequence draft counts
   int* cnt;              // zero area: ticket column (entry i = zcol(cnt, i))
   void* part;            // workspace: GreedyPart [B*(K+1)*S]
+  int fuse_build;        // 1: the CTA that decides a sequence also builds its draft span
+  pspec_build_args b;    // draft-batch arguments (accepted_len / bonus = this launch's outputs)
+  long long row_vecs;    // 16-byte vectors per hidden row of b
 };
 
 struct RejectionLaunch {
@@ -55,6 +58,9 @@ struct RejectionLaunch {
   void* part;            // workspace: RejPart [B*(2K+1)*S]
   void* seq;             // workspace: SeqInfo [B]
   double* tile_sums;     // workspace: [B*tiles] sums of r over 256-element tiles
+  int fuse_build;        // 1: the draw's last CTA of a sequence also builds its draft span
+  pspec_build_args b;    // draft-batch arguments (accepted_len / bonus = this launch's outputs)
+  long long row_vecs;    // 16-byte vectors per hidden row of b
 };
 
 struct EarlyExitLaunch {

@@ -13,6 +13,7 @@
 // an atomic ticket per sequence elects the CTA that finishes the sequence last, and that
 // CTA merges the partials in segment order (deterministic, lowest id wins ties) and
 // writes the accepted length, the bonus token and the output tokens.  No CTA waits.
+#include "build_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
@@ -22,7 +23,7 @@ namespace pspec {
 
 namespace {
 
-template <typename Tag, bool kLse>
+template <typename Tag, bool kLse, bool kFuse>
 __global__ void __launch_bounds__(kThreads)
 greedy_sweep_kernel(const GreedyLaunch L) {
   using elem = typename Tag::elem;
@@ -109,7 +110,8 @@ greedy_sweep_kernel(const GreedyLaunch L) {
     if (lane == 0) s_g[r] = b.i == kNoIndex ? 0 : b.i;   // a row of -inf / NaN only: token 0
   }
   __syncthreads();
-  if (warp != 0) return;
+  __shared__ int s_fin[3];                           // (a, K_i, bonus) for the fused build
+  if (warp == 0) {
   const int g = lane <= K ? s_g[lane] : 0;           // argmax of row `lane`
   const double lse = (kLse && lane <= K) ? s_lse[lane] : 0.0;
   int eb = 0;
@@ -134,6 +136,18 @@ greedy_sweep_kernel(const GreedyLaunch L) {
     L.bonus[i] = bonus;
     set_err(L.err, eb | (anybad ? PSPEC_DEVERR_TOKEN_RANGE : 0));
     *zcol(L.cnt, i) = 0;                       // ticket back to zero for the next call
+    s_fin[0] = a;
+    s_fin[1] = Ki;
+    s_fin[2] = bonus;
+  }
+  }  // warp 0
+  if constexpr (kFuse) {
+    // the whole step in this launch: the sequence's draft span, built by this CTA
+    __syncthreads();
+    int ebb = 0;
+    build_span(L.b, L.row_vecs, i, s_fin[0], s_fin[1], s_fin[2], true, 0, 1, &ebb);
+    if (i == L.b.B - 1) build_tail_pad(L.b, 0, 1, &ebb);
+    set_err(L.b.err, ebb);
   }
 }
 
@@ -142,12 +156,23 @@ greedy_sweep_kernel(const GreedyLaunch L) {
 cudaError_t launch_greedy(const GreedyLaunch& L, cudaStream_t stream) {
   const long long grid = (long long)L.B * (L.K + 1) * L.S;
   const bool lse = L.target_lse != nullptr;
+  const bool f = L.fuse_build != 0;
   if (L.dtype == PSPEC_BF16) {
-    if (lse) greedy_sweep_kernel<BF16Tag, true><<<(unsigned)grid, kThreads, 0, stream>>>(L);
-    else greedy_sweep_kernel<BF16Tag, false><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+    if (lse) {
+      if (f) greedy_sweep_kernel<BF16Tag, true, true><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+      else greedy_sweep_kernel<BF16Tag, true, false><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+    } else {
+      if (f) greedy_sweep_kernel<BF16Tag, false, true><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+      else greedy_sweep_kernel<BF16Tag, false, false><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+    }
   } else {
-    if (lse) greedy_sweep_kernel<F32Tag, true><<<(unsigned)grid, kThreads, 0, stream>>>(L);
-    else greedy_sweep_kernel<F32Tag, false><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+    if (lse) {
+      if (f) greedy_sweep_kernel<F32Tag, true, true><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+      else greedy_sweep_kernel<F32Tag, true, false><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+    } else {
+      if (f) greedy_sweep_kernel<F32Tag, false, true><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+      else greedy_sweep_kernel<F32Tag, false, false><<<(unsigned)grid, kThreads, 0, stream>>>(L);
+    }
   }
   return cudaGetLastError();
 }

@@ -17,6 +17,7 @@
 // Each warp sums r = max(0, p - q) (or p) over its own tiles, with no block barrier per
 // tile, and stores one double per tile; the CTA that finishes a sequence last prefix-sums
 // the tile sums, picks the tile holding u_K * Z and rescans that tile with one warp.
+#include "build_common.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "plan.h"
@@ -168,8 +169,9 @@ rej_stats_kernel(const RejectionLaunch L) {
   }  // warp 0
 }
 
-// The draw launch: B x C CTAs over the warp tiles of each sequence's row a_i.
-template <typename Tag>
+// The draw launch: B x C CTAs over the warp tiles of each sequence's row a_i.  With kFuse
+// the CTA that draws a sequence's token also builds its draft span (the whole step).
+template <typename Tag, bool kFuse>
 __global__ void __launch_bounds__(kThreads)
 rej_draw_kernel(const RejectionLaunch L) {
   using elem = typename Tag::elem;
@@ -203,11 +205,20 @@ rej_draw_kernel(const RejectionLaunch L) {
   double Z;
   const int token = draw_finish<Tag>(D, L.V, L.tiles,
                                      (double)L.uniforms[(long long)i * (K + 1) + si.kn], ts, sh, &Z);
+  __shared__ int s_tok;
   if (threadIdx.x == 0) {
     L.out_tokens[(long long)i * (K + 1) + si.a] = token;
     L.bonus[i] = token;
     if (L.residual_mass) L.residual_mass[i] = (float)Z;
     *zcol(L.cnt2, i) = 0;
+    s_tok = token;
+  }
+  if constexpr (kFuse) {
+    __syncthreads();
+    int eb = 0;
+    build_span(L.b, L.row_vecs, i, si.a, si.kn, s_tok, true, 0, 1, &eb);
+    if (i == L.b.B - 1) build_tail_pad(L.b, 0, 1, &eb);
+    set_err(L.b.err, eb);
   }
 }
 
@@ -237,8 +248,12 @@ cudaError_t launch_rejection(const RejectionLaunch& L, cudaStream_t stream,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (L.dtype == PSPEC_BF16) return cudaLaunchKernelEx(&cfg, rej_draw_kernel<BF16Tag>, L);
-  return cudaLaunchKernelEx(&cfg, rej_draw_kernel<F32Tag>, L);
+  if (L.fuse_build) {
+    if (L.dtype == PSPEC_BF16) return cudaLaunchKernelEx(&cfg, rej_draw_kernel<BF16Tag, true>, L);
+    return cudaLaunchKernelEx(&cfg, rej_draw_kernel<F32Tag, true>, L);
+  }
+  if (L.dtype == PSPEC_BF16) return cudaLaunchKernelEx(&cfg, rej_draw_kernel<BF16Tag, false>, L);
+  return cudaLaunchKernelEx(&cfg, rej_draw_kernel<F32Tag, false>, L);
 }
 
 }  // namespace pspec

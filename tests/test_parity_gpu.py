@@ -675,23 +675,24 @@ def _step_check(target, draft, drafts, u, binp, path, expect_fused):
 @pytest.mark.parametrize("rule", ["greedy", "rejection"])
 @pytest.mark.parametrize("path", [0, 2])
 def test_step_c64_fused(rule, path):
-    # automatic at 64 sequences: the greedy rule takes the fused early exit, the rejection
-    # rule the full sweep followed by the build launch; forced early exit fuses both
+    # automatic at 64 sequences: the greedy rule takes the early exit, the rejection rule the
+    # full sweep; either way the build runs inside the verify's last launch
     w = I.C64
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
     u = I.uniforms(w, DEV)
     binp = I.build_inputs(w, DEV, drafts=sampled)
     rej = rule == "rejection"
-    fused = path == 2 or not rej
-    _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, path, fused)
+    # below 256 sequences the build runs inside the verify's last launch on either path
+    _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, path, True)
 
 
 @pytest.mark.parametrize("path", [0, 1, 2])
 @pytest.mark.parametrize("rule", ["greedy", "rejection"])
 def test_step_tiny_every_path(rule, path):
-    # automatic at 5 sequences: both rules take the full sweep followed by the build launch
-    fused = path == 2
+    # automatic at 5 sequences: both rules take the full sweep; on every path the build runs
+    # inside the verify's last launch (fewer than 256 sequences)
+    fused = True
     w = I.scaled(I.C64, B=5, V=4096, H=64)
     target, draft = I.logits(w, DEV)
     sampled, greedy = I.draft_tokens(w, draft)
@@ -701,9 +702,11 @@ def test_step_tiny_every_path(rule, path):
     _step_check(target, draft, sampled if rej else greedy, u if rej else None, binp, path, fused)
 
 
+@pytest.mark.parametrize("path", [1, 2])
 @pytest.mark.parametrize("K,L_extra", [(1, 0), (3, 2), (7, 5)])
-def test_step_random_layouts_fused(K, L_extra):
-    """Spans with more verify rows than K+1 (the drafts are each span's last K rows)."""
+def test_step_random_layouts_fused(K, L_extra, path):
+    """Spans with more verify rows than K+1 (the drafts are each span's last K rows), the
+    build fused into the full sweep's deciding CTAs (path 1) or the early exit's clusters."""
     from tests.oracle_pins import random_build_case
     rng = np.random.default_rng(500 + K)
     case = random_build_case(rng, B=37, K=K, H=32, bs=4, L_extra=L_extra)
@@ -714,11 +717,12 @@ def test_step_random_layouts_fused(K, L_extra):
     draft = (target[:, :K].float() + torch.randn((37, K, V), generator=g, device=DEV) * 0.5).to(torch.bfloat16)
     d = torch.argmax(draft.float(), dim=2).to(torch.int32)
     u = torch.rand((37, K + 1), generator=g, device=DEV)
-    _step_check(target, draft, d, u, binp, 2, True)
-    _step_check(target, draft, d, None, binp, 2, True)
+    _step_check(target, draft, d, u, binp, path, True)
+    _step_check(target, draft, d, None, binp, path, True)
 
 
-def test_step_fused_invalid_layout_sets_bit():
+@pytest.mark.parametrize("path", [1, 2])
+def test_step_fused_invalid_layout_sets_bit(path):
     from tests.oracle_pins import random_build_case
     rng = np.random.default_rng(31)
     case = random_build_case(rng, B=6, K=3, H=8, bs=4)
@@ -727,8 +731,9 @@ def test_step_fused_invalid_layout_sets_bit():
     binp = _torchify(dict(case, qsl_in=q))
     target = torch.randn((6, 4, 512), device=DEV).to(torch.bfloat16)
     d = torch.argmax(target[:, :3].float(), dim=2).to(torch.int32)
-    with verify_path(2):
+    with verify_path(path):
         _, bo = ps.step(target, d, binp)
+        assert ps.pspec_last_launches() == 1
     torch.cuda.synchronize()
     assert bo["err"].item() & ps._binding.PSPEC_DEVERR_LAYOUT
 
@@ -889,10 +894,17 @@ def test_k_len_build(K, L_extra):
     d = torch.argmax(draft.float(), dim=2).to(torch.int32)
     u = torch.rand((37, K + 1), generator=g, device=DEV)
     klt = binp["k_len"]
-    for path, fused in ((2, True), (1, False)):
-        for uu in (u, None):
-            v1, b1 = _step_check_k(target, draft, d, uu, binp, path, fused, klt)
-            assert b1["err"].item() == 0
+    # 37 sequences: the build runs inside the verify's last launch on either path (automatic
+    # fusion), and after it when fusion is switched off
+    try:
+        for fusion, fused in ((0, True), (2, False)):
+            ps.pspec_set_step_fusion(fusion)
+            for path in (2, 1):
+                for uu in (u, None):
+                    v1, b1 = _step_check_k(target, draft, d, uu, binp, path, fused, klt)
+                    assert b1["err"].item() == 0
+    finally:
+        ps.pspec_set_step_fusion(0)
 
 
 def _step_check_k(target, draft, drafts, u, binp, path, expect_fused, klt):
