@@ -176,18 +176,6 @@ __device__ void warp_tile_sums_wide(const DrawRow& D, int V, long long t_begin, 
   }
 }
 
-__device__ __forceinline__ double block_sum(double v, double* s_red) {
-  v = warp_sum(v);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) s_red[warp] = v;
-  __syncthreads();
-  double t = 0.0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) t += s_red[w];
-  return t;
-}
-
 // Exclusive prefix over the CTA of one double per thread; returns the prefix and sets *total.
 __device__ __forceinline__ double block_exclusive_scan(double v, double* s_red, double* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -224,42 +212,47 @@ template <typename Tag>
 __device__ int draw_finish(DrawRow& D, int V, int tiles, double u, double* ts, DrawShared& sh,
                            double* Zout) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  double Z = 0.0;
-  for (int t0 = 0; t0 < tiles; t0 += kThreads)
-    Z += block_sum(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
+  // Each thread owns a run of consecutive tiles: one pass of loads and one block-wide scan
+  // give Z and every run's starting prefix, and the run holding u*Z finds its tile alone.
+  const int per = (tiles + kThreads - 1) / kThreads;
+  const int t_begin = tid * per;
+  const int t_end = t_begin + per < tiles ? t_begin + per : tiles;
+  double loc = 0.0;
+  for (int t = t_begin; t < t_end; ++t) loc += ld_cg(ts + t);
+  double Z;
+  double base = block_exclusive_scan(loc, sh.red, &Z);
   if (Z == 0.0 && D.resid) {
     D.resid = false;                       // max(0, p - q) vanished: draw from p
     D.qrow = D.trow;
     __syncthreads();
     warp_tile_sums<Tag>(D, V, warp, tiles, kWarps, ts);
     __syncthreads();
-    Z = 0.0;
-    for (int t0 = 0; t0 < tiles; t0 += kThreads)
-      Z += block_sum(t0 + tid < tiles ? ld_cg(ts + t0 + tid) : 0.0, sh.red);
+    loc = 0.0;
+    for (int t = t_begin; t < t_end; ++t) loc += ld_cg(ts + t);
+    base = block_exclusive_scan(loc, sh.red, &Z);
   }
   const double thr = u * Z;
 
-  int tile = -1;
+  // the first tile with mass whose inclusive prefix exceeds u*Z
+  if (tid == 0) sh.found = 0x7fffffff;
+  __syncthreads();
+  int mine = 0x7fffffff;
+  double mine_base = 0.0, run = base;
+  for (int t = t_begin; t < t_end; ++t) {
+    const double v = ld_cg(ts + t);
+    if (v > 0.0 && run + v > thr) { mine = t; mine_base = run; break; }
+    run += v;
+  }
+  if (mine != 0x7fffffff) atomicMin(&sh.found, mine);
+  __syncthreads();
+  int tile = sh.found;
   double tile_base = 0.0;
-  double base = 0.0;
-  for (int t0 = 0; t0 < tiles; t0 += kThreads) {
-    const int t = t0 + tid;
-    const double v = t < tiles ? ld_cg(ts + t) : 0.0;
-    double tot;
-    const double ex = block_exclusive_scan(v, sh.red, &tot);
-    if (tid == 0) sh.found = 0x7fffffff;
+  if (tile != 0x7fffffff) {
+    if (mine == tile) sh.red[kWarps] = mine_base;
     __syncthreads();
-    if (t < tiles && v > 0.0 && base + ex + v > thr) atomicMin(&sh.found, t);
-    __syncthreads();
-    const int f = sh.found;
-    if (f != 0x7fffffff) {
-      if (t == f) sh.red[kWarps] = base + ex;
-      __syncthreads();
-      tile = f;
-      tile_base = sh.red[kWarps];
-      break;                               // f is the same on every thread
-    }
-    base += tot;
+    tile_base = sh.red[kWarps];
+  } else {
+    tile = -1;
   }
   if (tile < 0 && Z > 0.0) {
     // rounding kept every prefix at or below u*Z: the last tile holding any mass
