@@ -55,11 +55,22 @@ namespace {
 #ifndef PSPEC_EE_MIN_BLOCKS
 #define PSPEC_EE_MIN_BLOCKS 6
 #endif
+// Greedy rule: six vectors per row at five CTAs per SM on the large-batch width, where the
+// clusters fill the GPU many times over (b1024: 0.185 ms against 0.191-0.208 for 4-8
+// vectors at 4-6 CTAs per SM); eight vectors at four CTAs per SM on the wider clusters of
+// small batches and of the tail launch, whose chains of positions are latency-bound (c64:
+// 0.033 ms against 0.039 with six vectors).
 #ifndef PSPEC_EE_GREEDY_UNROLL
-#define PSPEC_EE_GREEDY_UNROLL 8
+#define PSPEC_EE_GREEDY_UNROLL 6
 #endif
 #ifndef PSPEC_EE_GREEDY_MIN_BLOCKS
-#define PSPEC_EE_GREEDY_MIN_BLOCKS 4
+#define PSPEC_EE_GREEDY_MIN_BLOCKS 5
+#endif
+#ifndef PSPEC_EE_GREEDY_WIDE_UNROLL
+#define PSPEC_EE_GREEDY_WIDE_UNROLL 8
+#endif
+#ifndef PSPEC_EE_GREEDY_WIDE_MIN_BLOCKS
+#define PSPEC_EE_GREEDY_WIDE_MIN_BLOCKS 4
 #endif
 
 constexpr int kEERejUnroll = PSPEC_EE_REJ_UNROLL;   // vectors per row in flight (rejection)
@@ -119,11 +130,14 @@ __device__ __forceinline__ void ee_build_span(const pspec_build_args& b, long lo
 }
 
 template <typename Tag, int G, bool kRej, bool kFuse>
-__global__ void __launch_bounds__(kThreads, kRej ? kEEMinBlocks : PSPEC_EE_GREEDY_MIN_BLOCKS)
+__global__ void __launch_bounds__(kThreads, kRej ? kEEMinBlocks
+                                                 : (G <= 4 ? PSPEC_EE_GREEDY_MIN_BLOCKS
+                                                           : PSPEC_EE_GREEDY_WIDE_MIN_BLOCKS))
 ee_kernel(const EarlyExitLaunch L) {
   using elem = typename Tag::elem;
   constexpr int W = Tag::kVec;
-  constexpr int U = kRej ? kEERejUnroll : PSPEC_EE_GREEDY_UNROLL;  // vectors in flight per row
+  constexpr int U = kRej ? kEERejUnroll                              // vectors in flight per row
+                         : (G <= 4 ? PSPEC_EE_GREEDY_UNROLL : PSPEC_EE_GREEDY_WIDE_UNROLL);
   constexpr int BV = U * kThreads;                                  // vectors per row and batch
   constexpr int NP = G * kWarps;                                    // warp partials per position
   constexpr int PL = (NP + 31) / 32;                                // of them per lane
