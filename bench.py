@@ -50,7 +50,7 @@ def parse_args():
                    help="verify + build in one launch (early-exit path): pspec_set_step_fusion")
     p.add_argument("--tail", type=int, default=0,
                    help="early exit: sequences for the 8-CTA tail launch (0 auto, -1 never)")
-    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--e2e-steps", type=int, default=8)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-extra", action="store_true",
                    help="skip the other workloads (c1, c64, greedy b1024, depth sweep) that a "
