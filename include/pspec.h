@@ -431,7 +431,7 @@ PSPEC_API int pspec_last_cluster_size(void);
 
 /* Tuning (default of pspec_options.segment_elems): force the full sweep's segment length
    (elements of one row handled by one CTA; rounded up to a multiple of 8).  0 restores the
-   automatic choice, which aims at about 32 CTAs per SM and at most 65536 elements per CTA.
+   automatic choice, which aims at about 4 CTAs per SM with 8192 to 65536 elements per CTA.
    The segment length changes pspec_verify_workspace_bytes, so size workspaces after
    setting it. */
 PSPEC_API void pspec_set_segment_elems(long long elems);

@@ -18,12 +18,21 @@ constexpr int kDrawTile = 256;           // draw tile: one warp, 32 lanes x 8 el
 constexpr long long kSegMin = 8192;
 constexpr long long kSegMax = 65536;     // bounds the tail of the last wave
 #ifndef PSPEC_TARGET_CTAS_PER_SM
-#define PSPEC_TARGET_CTAS_PER_SM 32
+#define PSPEC_TARGET_CTAS_PER_SM 32         // draft sampling: segments per row
+#endif
+// The verify sweep aims at about four CTAs per SM: fewer, longer segments cost fewer CTA
+// starts and fewer partials for each sequence's last CTA to merge.  Measured on B200 (step
+// time, L2 flushed): 4 sequences 0.038 -> 0.034 ms, 16 sequences 0.058 -> 0.052 ms, 64
+// sequences 0.093 -> 0.087 ms against 32 CTAs per SM; one sequence unchanged (the 8192-
+// element minimum decides there) and 1024 sequences unchanged (the 65536-element maximum).
+#ifndef PSPEC_SWEEP_CTAS_PER_SM
+#define PSPEC_SWEEP_CTAS_PER_SM 4
 #endif
 #ifndef PSPEC_DRAW_CTAS_PER_SM
 #define PSPEC_DRAW_CTAS_PER_SM 1      // separate draw launch: about one CTA per SM, at least
 #endif                                // kDrawTilesPerCta tiles per CTA (batches of one: 6)
 constexpr int kTargetCtas = kNumSMs * PSPEC_TARGET_CTAS_PER_SM;
+constexpr int kSweepTargetCtas = kNumSMs * PSPEC_SWEEP_CTAS_PER_SM;
 constexpr int kResampleTargetCtas = kNumSMs * PSPEC_DRAW_CTAS_PER_SM;
 constexpr int kDrawTilesPerCta = 64;     // separate draw launch: at most 8 tiles per warp
 // Automatic path selection: the early exit from kEarlyExitMinB sequences on for the
@@ -151,7 +160,7 @@ inline VerifyPlan make_verify_plan(int B, int K, int V, int rejection, long long
   long long s_lo = (V + kSegMax - 1) / kSegMax;
   long long s_hi = (V + kSegMin - 1) / kSegMin;
   if (s_hi < 1) s_hi = 1;
-  long long S = rows_total > 0 ? (kTargetCtas + rows_total - 1) / rows_total : 1;
+  long long S = rows_total > 0 ? (kSweepTargetCtas + rows_total - 1) / rows_total : 1;
   if (S < s_lo) S = s_lo;
   if (S > s_hi) S = s_hi;
   if (S < 1) S = 1;
