@@ -2,13 +2,11 @@
 
 Tolerances (floating-point outputs of the fp32 kernels against the double oracle):
   * p_at_draft, q_at_draft, target_lse, draft_lse: 1e-5 relative (the stated bar);
-  * residual_mass Z: 1e-5 relative, with an absolute floor of 1e-6 for masses that come
-    out of cancellation.  Z = sum over t of max(0, p(t) - q(t)); where the draft is good,
-    each term is a difference of two near-equal fp32 probabilities that carry about 1e-7
-    relative error each, so the sum's absolute error is a few 1e-7 of sum p(t) over the
-    terms, whatever Z is -- below Z = 0.1 that is more than 1e-5 of Z.  Every comparison
-    prints the largest relative error of Z and how many sequences passed only by the
-    floor (zero in every full-size workload measured).
+  * residual_mass Z: 1e-5 relative, no absolute floor.  Z = sum over t of
+    max(0, p(t) - q(t)); the kernels form each term from fp32 probabilities, add a lane's few
+    terms in fp32 and everything above that in double, so the error is about that of the
+    terms (1e-7 of each p(t)), which stays below 1e-5 of Z on every workload measured.  Every comparison prints the largest
+    relative error of Z.
 Integer outputs (tokens, counts, offsets, slots) must be bit-exact, except for sequences
 the oracle flags as near-ties (an accept decision with |u - p/q| < 1e-6, or a draw within
 1e-6 * Z of a CDF boundary): those are excluded from the integer comparison and counted.
@@ -24,7 +22,6 @@ import oracle
 
 THREADS = max(1, os.cpu_count() or 1)
 RTOL = 1e-5
-Z_ATOL = 1e-6
 
 
 def host_logits(x: torch.Tensor) -> np.ndarray:
@@ -91,13 +88,12 @@ def compare_rejection(g: dict, o: dict, seqs=None, K=None):
         same_a = G["accepted_len"] == o["accepted_len"]
         gz = np.asarray(G["residual_mass"], np.float64)[same_a]
         oz = np.asarray(o["residual_mass"], np.float64)[same_a]
-        ok = _rel_ok(gz, oz, RTOL, Z_ATOL)
-        assert ok.all(), ("residual_mass", gz[~ok][:5], oz[~ok][:5])
-        rel_only = _rel_ok(gz, oz, RTOL, 0.0)
         nz = oz > 0
         worst = float(np.max(np.abs(gz - oz)[nz] / oz[nz])) if nz.any() else 0.0
         print(f"[parity] residual mass: {int(same_a.sum())} compared, max relative error "
-              f"{worst:.2e}, {int((~rel_only).sum())} within tolerance only by the absolute floor")
+              f"{worst:.2e}")
+        ok = _rel_ok(gz, oz)
+        assert ok.all(), ("residual_mass", gz[~ok][:5], oz[~ok][:5])
     flagged = int((~clean).sum())
     print(f"[parity] {len(flags)} sequences, {flagged} flagged near-ties, "
           f"{int((~clean & same).sum())} of those identical anyway")
