@@ -368,34 +368,53 @@ def run_pspec(args, rank, world, local_rank):
     in_bytes = sum(x.numel() * x.element_size() for x in (d["target"], d["draft"]) if x is not None)
     flush_buf = (torch.empty(256 << 20, dtype=torch.uint8, device=dev)
                  if in_bytes < (256 << 20) else None)
+    def instrumented_step(e):
+        """One step with events at its start, between the verify and the build and at its
+        end (the library records e[1] between the sweep's two verify launches)."""
+        e[0].record()
+        if graph is not None:
+            graph.replay()
+            e[2].record()
+            e[3].record()
+        elif fused:
+            fused_step()
+            e[2].record()
+            e[3].record()
+        else:
+            if rej:
+                ps.pspec_set_split_event(e[1])
+            verify()
+            e[2].record()
+            build()
+            e[3].record()
+            ps.pspec_set_split_event(None)
+
+    # With inputs larger than L2 the K steps are timed as a whole with nothing between their
+    # launches: an event recorded between the verify and the build holds the build back
+    # until the verify has drained (it is a programmatic dependent that would otherwise be
+    # placed while the verify's last clusters run), which costs a few microseconds a step.
+    # The per-kernel times then come from K more steps with events between the launches.
+    # With an L2 flush before every step, the steps carry their own events.
+    instrument_timed = flush_buf is not None
     with sampler:
         t0.record()
         for s in range(K):
             if flush_buf is not None:
                 flush_l2(flush_buf)
-            ev[s][0].record()
-            if graph is not None:
-                graph.replay()
-                ev[s][2].record()
-                ev[s][3].record()
-            elif fused:
-                fused_step()
-                ev[s][2].record()
-                ev[s][3].record()
+            if instrument_timed:
+                instrumented_step(ev[s])
             else:
-                if rej:
-                    ps.pspec_set_split_event(ev[s][1])
-                verify()
-                ev[s][2].record()
-                build()
-                ev[s][3].record()
+                one_step()
         t1.record()
         torch.cuda.synchronize()
         sampler.mark_timed_end()
-        ps.pspec_set_split_event(None)
         # clock readings beside a short timed region: the same steps for 0.25 s more
         for _ in range(min(4000, int(math.ceil(250.0 / max(t0.elapsed_time(t1) / K, 1e-3))))):
             one_step()
+        torch.cuda.synchronize()
+    if not instrument_timed:
+        for s in range(K):
+            instrumented_step(ev[s])
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -453,7 +472,9 @@ def run_pspec(args, rank, world, local_rank):
             "verify_path": {1: "full sweep", 2: f"early exit ({cluster}-CTA cluster per sequence)"}[path],
             "step": ("one launch (verify + build fused)" if fused else "verify launches + build launch")
                     + (", CUDA graph replay" if graph is not None else ""),
-            "l2": ("inputs larger than L2 (%.2f GB of logits per step); no flush" % (vbytes / 1e9)
+            "l2": ("inputs larger than L2 (%.2f GB of logits per step); no flush; the K steps "
+                   "timed as a whole, per-kernel times from K more steps with events between "
+                   "the launches" % (vbytes / 1e9)
                    if flush_buf is None else
                    "256 MB buffer written then read before every step, outside the step's events; "
                    "elapsed time = sum of the per-step event times"),
@@ -513,8 +534,17 @@ def flush_l2(buf):
 def time_steps(fn, n, flush=None):
     """Device time of each of n calls of fn (CUDA events on the current stream, one pair per
     call); with `flush`, a buffer larger than L2 is written and read before every call,
-    outside the timed pair."""
+    outside the timed pair.  Without it (inputs larger than L2) the n calls are timed as a
+    whole, nothing recorded between them, and each gets the mean."""
     import torch
+    if flush is None:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) / n] * n
     pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
              for _ in range(n)]
     for a, b in pairs:
