@@ -393,9 +393,10 @@ def run_pspec(args, rank, world, local_rank):
     # launches: an event recorded between the verify and the build holds the build back
     # until the verify has drained (it is a programmatic dependent that would otherwise be
     # placed while the verify's last clusters run), which costs a few microseconds a step.
-    # The per-kernel times then come from K more steps with events between the launches.
+    # The per-kernel times then come from up to 50 more steps with events between the launches.
     # With an L2 flush before every step, the steps carry their own events.
     instrument_timed = flush_buf is not None
+    n_inst = K if instrument_timed else min(K, 50)
     with sampler:
         # two more untimed steps once the sampler runs, and no synchronisation before t0:
         # the GPU is still busy with them when t0 is reached, so the host has queued the
@@ -416,15 +417,18 @@ def run_pspec(args, rank, world, local_rank):
         t1.record()
         torch.cuda.synchronize()
         sampler.mark_timed_end()
+        if not instrument_timed:
+            # right after the timed steps, at most 50 of them (a long run heats the part
+            # towards its power cap, and later steps would not be the ones timed)
+            one_step()                     # untimed: the GPU is busy when the first is queued
+            for s in range(n_inst):
+                instrumented_step(ev[s])
         # clock readings beside a short timed region: the same steps for 0.25 s more
         for _ in range(min(4000, int(math.ceil(250.0 / max(t0.elapsed_time(t1) / K, 1e-3))))):
             one_step()
         torch.cuda.synchronize()
     if not instrument_timed:
-        one_step()                         # untimed: the GPU is busy when the first is queued
-        for s in range(K):
-            instrumented_step(ev[s])
-        torch.cuda.synchronize()
+        ev = ev[:n_inst]
     if world > 1:
         dist.barrier()
     own_ms = (t0.elapsed_time(t1) if flush_buf is None
@@ -482,8 +486,8 @@ def run_pspec(args, rank, world, local_rank):
             "step": ("one launch (verify + build fused)" if fused else "verify launches + build launch")
                     + (", CUDA graph replay" if graph is not None else ""),
             "l2": ("inputs larger than L2 (%.2f GB of logits per step); no flush; the K steps "
-                   "timed as a whole, per-kernel times from K more steps with events between "
-                   "the launches" % (vbytes / 1e9)
+                   "timed as a whole, per-kernel times from min(K, 50) more steps with events "
+                   "between the launches" % (vbytes / 1e9)
                    if flush_buf is None else
                    "256 MB buffer written then read before every step, outside the step's events; "
                    "elapsed time = sum of the per-step event times"),

@@ -24,7 +24,8 @@
 //     on a dependent load;
 //   * rejection rule: at the stop position each CTA sums r = max(0, p - q) over
 //     256-element warp tiles of its slice, re-read right after the statistics pass and
-//     backwards (the most recently streamed lines first, while L2 still holds them); the
+//     backwards (the most recently streamed lines first, while L2 still holds them), two
+//     tiles' loads in flight per warp and kept packed as loaded until they are summed; the
 //     slice totals are prefix-summed in rank order on every CTA, and the CTA whose slice
 //     holds u_K * Z rescans one tile.
 //     When the draw is from the target row itself (all drafts passed), the slice totals
@@ -339,15 +340,41 @@ ee_kernel(const EarlyExitLaunch L) {
     // most likely still in L2, and going backwards the re-read meets the freshest lines
     // before the other clusters' streams evict them.
     auto tile_pass = [&]() {
-      for (int t = ntiles - 1 - warp; t >= 0; t -= kWarps) {
-        float xt[8], xq[8], r[8];
-        slice_x8<Tag>(D, lo, n, t * 256 + lane * 8, xt, xq);
-        draw_r8(D, xt, xq, r);
-        float sum = 0.f;
+      if constexpr (Tag::kVec == 8) {
+        // two tiles' loads in flight per warp, kept packed until they are summed
+        const uint16_t* tp = static_cast<const uint16_t*>(D.trow) + lo;
+        const uint16_t* qp = static_cast<const uint16_t*>(D.qrow) + lo;
+        for (int t = ntiles - 1 - warp; t >= 0; t -= 2 * kWarps) {
+          const int t2 = t - kWarps;
+          const int e0 = t * 256 + lane * 8, e1 = t2 * 256 + lane * 8;
+          const bool in0 = e0 < n, in1 = t2 >= 0 && e1 < n;
+          uint4 a = make_uint4(0, 0, 0, 0), aq = a, b = a, bq = a;
+          if (in0) {
+            a = ld_stream(tp + e0);
+            if (D.resid) aq = ld_stream(qp + e0);
+          }
+          if (in1) {
+            b = ld_stream(tp + e1);
+            if (D.resid) bq = ld_stream(qp + e1);
+          }
+          const double ts0 = warp_sum_d((double)(in0 ? draw_sum8_bf16(D, a, aq) : 0.f));
+          if (lane == 0) tsum[t] = ts0;
+          if (t2 >= 0) {
+            const double ts1 = warp_sum_d((double)(in1 ? draw_sum8_bf16(D, b, bq) : 0.f));
+            if (lane == 0) tsum[t2] = ts1;
+          }
+        }
+      } else {
+        for (int t = ntiles - 1 - warp; t >= 0; t -= kWarps) {
+          float xt[8], xq[8], r[8];
+          slice_x8<Tag>(D, lo, n, t * 256 + lane * 8, xt, xq);
+          draw_r8(D, xt, xq, r);
+          float sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sum += r[j];
-        const double ts = warp_sum_d((double)sum);
-        if (lane == 0) tsum[t] = ts;
+          for (int j = 0; j < 8; ++j) sum += r[j];
+          const double ts = warp_sum_d((double)sum);
+          if (lane == 0) tsum[t] = ts;
+        }
       }
     };
     bool own_pass_done = false;
