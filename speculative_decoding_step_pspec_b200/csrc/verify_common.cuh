@@ -105,8 +105,8 @@ struct DrawRow {
 
 
 // r of eight consecutive elements, computed on packed fp32 pairs.  Every pass over the
-// same elements (tile sums, rescans) goes through this function or draw_sum8_bf16, which
-// repeats its arithmetic in the same order, so all of them see bit-identical values.
+// same elements (tile sums, rescans) goes through this function, so all of them see
+// bit-identical values.
 __device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b) {
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
       "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
@@ -139,35 +139,6 @@ __device__ __forceinline__ void draw_r8(const DrawRow& D, const float (&xt)[8], 
       r[j + 1] = p1;
     }
   }
-}
-
-// Lane sum of r over eight consecutive bf16 logits still packed as loaded: the arithmetic
-// of draw_r8 followed by a sequential sum, in the same order, so that the tile sums agree
-// bit for bit with the rescans that go through draw_r8.
-__device__ __forceinline__ float draw_sum8_bf16(const DrawRow& D, const uint4& wt, const uint4& wq) {
-  if (D.mt == -INFINITY) return 0.f;
-  const uint32_t tw[4] = {wt.x, wt.y, wt.z, wt.w};
-  const uint32_t qw[4] = {wq.x, wq.y, wq.z, wq.w};
-  const bool use_q = D.resid && D.mq != -INFINITY;
-  float s = 0.f;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float a0, a1;
-    ffma2(a0, a1, bf16_lo(tw[k]), bf16_hi(tw[k]), kLog2e, -D.mt);
-    float p0, p1;
-    fmul2(p0, p1, ex2(a0), ex2(a1), D.inv_st);
-    float r0 = p0, r1 = p1;
-    if (use_q) {
-      float b0, b1, q0, q1;
-      ffma2(b0, b1, bf16_lo(qw[k]), bf16_hi(qw[k]), kLog2e, -D.mq);
-      fmul2(q0, q1, ex2(b0), ex2(b1), D.inv_sq);
-      r0 = fmaxf(p0 - q0, 0.f);
-      r1 = fmaxf(p1 - q1, 0.f);
-    }
-    s += r0;
-    s += r1;
-  }
-  return s;
 }
 
 // ---- argmax over 16-byte vectors: the vector's max on packed pairs, and only a vector

@@ -114,6 +114,35 @@ __device__ __forceinline__ void slice_x8(const DrawRow& D, long long lo, int n, 
   }
 }
 
+// Lane sum of r over eight consecutive bf16 logits still packed as loaded: the arithmetic
+// of draw_r8 followed by a sequential sum, in the same order, so that the tile sums agree
+// bit for bit with the rescans that go through draw_r8.
+__device__ __forceinline__ float draw_sum8_bf16(const DrawRow& D, const uint4& wt, const uint4& wq) {
+  if (D.mt == -INFINITY) return 0.f;
+  const uint32_t tw[4] = {wt.x, wt.y, wt.z, wt.w};
+  const uint32_t qw[4] = {wq.x, wq.y, wq.z, wq.w};
+  const bool use_q = D.resid && D.mq != -INFINITY;
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float a0, a1;
+    ffma2(a0, a1, bf16_lo(tw[k]), bf16_hi(tw[k]), kLog2e, -D.mt);
+    float p0, p1;
+    fmul2(p0, p1, ex2(a0), ex2(a1), D.inv_st);
+    float r0 = p0, r1 = p1;
+    if (use_q) {
+      float b0, b1, q0, q1;
+      ffma2(b0, b1, bf16_lo(qw[k]), bf16_hi(qw[k]), kLog2e, -D.mq);
+      fmul2(q0, q1, ex2(b0), ex2(b1), D.inv_sq);
+      r0 = fmaxf(p0 - q0, 0.f);
+      r1 = fmaxf(p1 - q1, 0.f);
+    }
+    s += r0;
+    s += r1;
+  }
+  return s;
+}
+
 // Whole-step fusion: the draft span of sequence i (output rows [qsl_out[i], qsl_out[i+1]),
 // clamped into [0, T_cap)), built by the cluster that has just decided a_i and the bonus
 // token.  The CTA holding the token (`meta`) writes the rows' metadata and the sequence's
@@ -335,17 +364,19 @@ ee_kernel(const EarlyExitLaunch L) {
     D.mq = dMq; D.inv_sq = dSq > 0.0 ? (float)(1.0 / dSq) : 0.f;
     const int ntiles = (n + 255) / 256;
     const double u = (double)L.uniforms[(long long)i * (K + 1) + Ki];
-    // Sums of r over this CTA's tiles, the warps taking every 8th tile from the last one
-    // down: the statistics pass streamed the slice from its start, so its end is the part
+    // Sums of r over this CTA's tiles, from the last one down (bf16: the warps take
+    // adjacent pairs, every 8th pair; fp32: every 8th tile): the statistics pass streamed
+    // the slice from its start, so its end is the part
     // most likely still in L2, and going backwards the re-read meets the freshest lines
     // before the other clusters' streams evict them.
     auto tile_pass = [&]() {
       if constexpr (Tag::kVec == 8) {
-        // two tiles' loads in flight per warp, kept packed until they are summed
+        // two adjacent tiles' loads in flight per warp, kept packed until they are summed,
+        // and the two tile sums reduced across the warp together
         const uint16_t* tp = static_cast<const uint16_t*>(D.trow) + lo;
         const uint16_t* qp = static_cast<const uint16_t*>(D.qrow) + lo;
-        for (int t = ntiles - 1 - warp; t >= 0; t -= 2 * kWarps) {
-          const int t2 = t - kWarps;
+        for (int t = ntiles - 1 - 2 * warp; t >= 0; t -= 2 * kWarps) {
+          const int t2 = t - 1;
           const int e0 = t * 256 + lane * 8, e1 = t2 * 256 + lane * 8;
           const bool in0 = e0 < n, in1 = t2 >= 0 && e1 < n;
           uint4 a = make_uint4(0, 0, 0, 0), aq = a, b = a, bq = a;
@@ -357,11 +388,16 @@ ee_kernel(const EarlyExitLaunch L) {
             b = ld_stream(tp + e1);
             if (D.resid) bq = ld_stream(qp + e1);
           }
-          const double ts0 = warp_sum_d((double)(in0 ? draw_sum8_bf16(D, a, aq) : 0.f));
-          if (lane == 0) tsum[t] = ts0;
-          if (t2 >= 0) {
-            const double ts1 = warp_sum_d((double)(in1 ? draw_sum8_bf16(D, b, bq) : 0.f));
-            if (lane == 0) tsum[t2] = ts1;
+          double d0 = (double)(in0 ? draw_sum8_bf16(D, a, aq) : 0.f);
+          double d1 = (double)(in1 ? draw_sum8_bf16(D, b, bq) : 0.f);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            d0 += __shfl_xor_sync(0xffffffffu, d0, o);
+            d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+          }
+          if (lane == 0) {
+            tsum[t] = d0;
+            if (t2 >= 0) tsum[t2] = d1;
           }
         }
       } else {
