@@ -19,9 +19,12 @@
 //     draft == argmax), so no broadcast follows.  Partials are double-buffered by position
 //     parity: a warp writing position k+1 has passed the barrier of position k, which every
 //     reader of position k-1 had reached first;
-//   * the draft tokens sit in lane registers from the start (lane k holds d_k) and the
-//     logits at d_k are requested when position k starts, so nothing in the decision waits
-//     on a dependent load;
+//   * the draft tokens sit in lane registers from the start (lane k holds d_k), the
+//     uniforms u_0..u_K in shared memory, and the logits at d_k are requested when position
+//     k starts, so nothing in the decision waits on a global load.  The decision u q < p is
+//     taken in fp32 when the two sides differ by more than 1e-4 (the fp32 error is a few
+//     1e-6), else in double as before: the same decisions, without two double exponentials
+//     and divisions at every position;
 //   * rejection rule: at the stop position each CTA sums r = max(0, p - q) over
 //     256-element warp tiles of its slice, re-read right after the statistics pass and
 //     backwards (the most recently streamed lines first, while L2 still holds them), two
@@ -209,6 +212,10 @@ ee_kernel(const EarlyExitLaunch L) {
 
   // lane k of every warp holds draft k of the sequence (-1 past K_i)
   const int dreg = lane < Ki ? __ldg(L.draft_tokens + (long long)i * K + lane) : -1;
+  // the uniforms of positions 0..K, read from shared memory at each decision
+  __shared__ float s_u[32];
+  if (kRej && tid <= K) s_u[tid] = __ldg(L.uniforms + (long long)i * (K + 1) + tid);
+  __syncthreads();
 
   // decision state of the stop position: every warp computes the same values and warp 0
   // leaves them in shared memory for the draw, so none of them occupies registers while
@@ -311,12 +318,23 @@ ee_kernel(const EarlyExitLaunch L) {
       xq_d = __shfl_sync(0xffffffffu, xq_d, 0);
       bool accept = false;
       if (k < Ki && d >= 0 && d < L.V) {
-        const double pp = (Mt != -INFINITY && xt_d != -INFINITY)
-                              ? exp2((double)xt_d * (double)kLog2e - (double)Mt) / st : 0.0;
-        const double qq = (Mq != -INFINITY && xq_d != -INFINITY)
-                              ? exp2((double)xq_d * (double)kLog2e - (double)Mq) / sq : 0.0;
-        const double u = (double)L.uniforms[(long long)i * (K + 1) + k];
-        accept = qq > 0.0 ? (u * qq < pp) : (pp > 0.0);
+        const float uf = s_u[k];
+        // fp32 first; the double form decides whenever the two sides are within 1e-4
+        const float p32 = (Mt != -INFINITY && xt_d != -INFINITY)
+                              ? ex2(fmaf(xt_d, kLog2e, -Mt)) / (float)st : 0.f;
+        const float q32 = (Mq != -INFINITY && xq_d != -INFINITY)
+                              ? ex2(fmaf(xq_d, kLog2e, -Mq)) / (float)sq : 0.f;
+        const float lhs = uf * q32;
+        if (p32 > 1e-30f && q32 > 1e-30f && fabsf(lhs - p32) > 1e-4f * fmaxf(lhs, p32)) {
+          accept = lhs < p32;
+        } else {
+          const double pp = (Mt != -INFINITY && xt_d != -INFINITY)
+                                ? exp2((double)xt_d * (double)kLog2e - (double)Mt) / st : 0.0;
+          const double qq = (Mq != -INFINITY && xq_d != -INFINITY)
+                                ? exp2((double)xq_d * (double)kLog2e - (double)Mq) / sq : 0.0;
+          const double u = (double)uf;
+          accept = qq > 0.0 ? (u * qq < pp) : (pp > 0.0);
+        }
       }
       stop = !accept;
       if (stop && warp == 0 && lane == 0) {
