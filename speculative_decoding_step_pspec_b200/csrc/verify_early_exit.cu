@@ -146,6 +146,18 @@ __device__ __forceinline__ float draw_sum8_bf16(const DrawRow& D, const uint4& w
   return s;
 }
 
+// A warp's (m, s) partials merged max first: one exponential per lane instead of one per
+// shuffle step.
+__device__ __forceinline__ MS warp_merge_ms_maxfirst(MS v) {
+  float M = v.m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float s = (v.m == -INFINITY) ? 0.f : v.s * ex2(v.m - M);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return MS{M, M == -INFINITY ? 0.f : s};
+}
+
 // Whole-step fusion: the draft span of sequence i (output rows [qsl_out[i], qsl_out[i+1]),
 // clamped into [0, T_cap)), built by the cluster that has just decided a_i and the bonus
 // token.  The CTA holding the token (`meta`) writes the rows' metadata and the sequence's
@@ -270,8 +282,8 @@ ee_kernel(const EarlyExitLaunch L) {
     }
     // ---- this warp's partial, then the cluster barrier in two halves
     if constexpr (kRej) {
-      const MS mt = warp_merge_ms(msacc_final(at));
-      const MS mq = warp_merge_ms(msacc_final(aq));
+      const MS mt = warp_merge_ms_maxfirst(msacc_final(at));
+      const MS mq = warp_merge_ms_maxfirst(msacc_final(aq));
       if (lane == 0) s_part[k & 1][warp] = make_float4(mt.m, mt.s, mq.m, mq.s);
     } else {
       best = warp_argmax(best);
