@@ -208,6 +208,8 @@ ee_kernel(const EarlyExitLaunch L) {
   __shared__ double s_tot[16];                               // per-slice draw totals
   __shared__ int s_tile;
   __shared__ double s_base;
+  __shared__ double s_wt[kWarps];                            // draw: per-warp sums of tile sums
+  __shared__ int s_found, s_last;
   __shared__ int s_tok;                                      // the emitted token (build)
 
   const long long lo = (long long)g * L.vs;                 // this CTA's slice [lo, lo + n)
@@ -407,6 +409,7 @@ ee_kernel(const EarlyExitLaunch L) {
         // and the two tile sums reduced across the warp together
         const uint16_t* tp = static_cast<const uint16_t*>(D.trow) + lo;
         const uint16_t* qp = static_cast<const uint16_t*>(D.qrow) + lo;
+        double wsum = 0.0;
         for (int t = ntiles - 1 - 2 * warp; t >= 0; t -= 2 * kWarps) {
           const int t2 = t - 1;
           const int e0 = t * 256 + lane * 8, e1 = t2 * 256 + lane * 8;
@@ -431,8 +434,12 @@ ee_kernel(const EarlyExitLaunch L) {
             tsum[t] = d0;
             if (t2 >= 0) tsum[t2] = d1;
           }
+          wsum += d0;
+          if (t2 >= 0) wsum += d1;
         }
+        if (lane == 0) s_wt[warp] = wsum;
       } else {
+        double wsum = 0.0;
         for (int t = ntiles - 1 - warp; t >= 0; t -= kWarps) {
           float xt[8], xq[8], r[8];
           slice_x8<Tag>(D, lo, n, t * 256 + lane * 8, xt, xq);
@@ -442,7 +449,9 @@ ee_kernel(const EarlyExitLaunch L) {
           for (int j = 0; j < 8; ++j) sum += r[j];
           const double ts = warp_sum_d((double)sum);
           if (lane == 0) tsum[t] = ts;
+          wsum += ts;
         }
+        if (lane == 0) s_wt[warp] = wsum;
       }
     };
     bool own_pass_done = false;
@@ -451,7 +460,7 @@ ee_kernel(const EarlyExitLaunch L) {
       __syncthreads();
       if (tid == 0) {
         double tt = 0.0;
-        for (int t = 0; t < ntiles; ++t) tt += tsum[t];
+        for (int w = 0; w < kWarps; ++w) tt += s_wt[w];
         tot_slice = tt;
       }
       cluster.sync();                                        // slice totals in place
@@ -500,17 +509,42 @@ ee_kernel(const EarlyExitLaunch L) {
         tile_pass();
         __syncthreads();
       }
-      if (tid == 0) {
-        int tile = -1, last_tile = -1;
-        double b2 = base, tb = base;
-        for (int t = 0; t < ntiles; ++t) {
-          if (tsum[t] > 0.0) last_tile = t;
-          if (tile < 0 && crossing && tsum[t] > 0.0 && b2 + tsum[t] > thr) { tile = t; tb = b2; }
-          b2 += tsum[t];
+      {
+        // the tile holding u*Z: every thread takes a run of consecutive tile sums, one
+        // block-wide exclusive scan gives each run its base, the run holding the crossing
+        // (or the last positive tile, when rounding leaves none) reports it
+        if (tid == 0) { s_found = 0x7fffffff; s_last = -1; }
+        const int per = (ntiles + kThreads - 1) / kThreads;
+        const int t0 = min(tid * per, ntiles), t1 = min(t0 + per, ntiles);
+        double loc = 0.0;
+        for (int t = t0; t < t1; ++t) loc += tsum[t];
+        double incl = loc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const double v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
         }
-        if (tile < 0) { tile = last_tile; tb = -INFINITY; } // no crossing: its last positive r
-        s_tile = tile;
-        s_base = tb;
+        if (lane == 31) s_wt[warp] = incl;
+        __syncthreads();
+        double b2 = base + incl - loc;
+        for (int w = 0; w < warp; ++w) b2 += s_wt[w];
+        int mine = 0x7fffffff, lastp = -1;
+        double mb = 0.0;
+        for (int t = t0; t < t1; ++t) {
+          const double ts = tsum[t];
+          if (ts > 0.0) lastp = t;
+          if (mine == 0x7fffffff && crossing && ts > 0.0 && b2 + ts > thr) { mine = t; mb = b2; }
+          b2 += ts;
+        }
+        if (mine != 0x7fffffff) atomicMin(&s_found, mine);
+        if (lastp >= 0) atomicMax(&s_last, lastp);
+        __syncthreads();
+        if (s_found != 0x7fffffff) {
+          if (mine == s_found) { s_tile = mine; s_base = mb; }
+        } else if (tid == 0) {
+          s_tile = s_last;                                   // no crossing: its last positive r
+          s_base = -INFINITY;
+        }
       }
       __syncthreads();
       if (warp == 0) {
