@@ -423,6 +423,16 @@ def run_pspec(args, rank, world, local_rank):
             one_step()                     # untimed: the GPU is busy when the first is queued
             for s in range(n_inst):
                 instrumented_step(ev[s])
+        b2b = None
+        if not instrument_timed and graph is None and not fused and path == 2:
+            # the early-exit verify alone, n_inst calls back to back with nothing recorded
+            # between them: the dominant kernel's own duration, without the gap that an event
+            # between two launches opens (the front end drains, then starts the next launch)
+            b2b = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            b2b[0].record()
+            for _ in range(n_inst):
+                verify()
+            b2b[1].record()
         # clock readings beside a short timed region: the same steps for 0.25 s more
         for _ in range(min(4000, int(math.ceil(250.0 / max(t0.elapsed_time(t1) / K, 1e-3))))):
             one_step()
@@ -464,6 +474,9 @@ def run_pspec(args, rank, world, local_rank):
                "speculative_decoding_step_pspec_b200/csrc/common.cuh"]
     src_hash = kernel_source_hash(src)
     dom_ms = statistics.mean(stats_ms)
+    dom_ms_events = dom_ms
+    if b2b is not None:
+        dom_ms = b2b[0].elapsed_time(b2b[1]) / n_inst
     whole = fused or graph is not None                     # one timed unit: the whole step
     dom_bytes = vbytes + bbytes if whole else vbytes       # a fused launch also builds
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -503,9 +516,14 @@ def run_pspec(args, rank, world, local_rank):
             + (" (two launches: the large-batch clusters, then wider ones for the last sequences)"
                if path == 2 and lv == 2 and not fused else "")
             + (" (CUDA graph replay of the step)" if graph is not None else ""): round(dom_ms, 5),
+            **({"ee_kernel with events between the step's launches": round(dom_ms_events, 5)}
+               if b2b is not None else {}),
             **({"rej_draw_kernel": round(statistics.mean(draw_ms), 5)} if draw_ms else {}),
             **({} if whole else {"build_kernel": round(statistics.mean(build_ms), 5)}),
         },
+        **({"kernels_ms_timing": "ee_kernel: min(K, 50) verify calls back to back, nothing "
+                                 "recorded between them; build_kernel: min(K, 50) steps with "
+                                 "events between the launches"} if b2b is not None else {}),
         **({} if whole else {"build_gbs": round(bbytes / (statistics.mean(build_ms) * 1e-3) / 1e9, 1)}),
         "roofline": {
             "kernel": dom_kernel, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
