@@ -146,12 +146,28 @@ __device__ __forceinline__ float draw_sum8_bf16(const DrawRow& D, const uint4& w
   return s;
 }
 
+// Warp-wide float max in one redux instruction: the float's bits mapped to an unsigned key
+// that orders like the value (negatives inverted, positives with the sign bit set).
+__device__ __forceinline__ unsigned float_key(float f) {
+  const unsigned u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float warp_max_redux(float v) {
+  const unsigned k = __reduce_max_sync(0xffffffffu, float_key(v));
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+// (value, index) argmax over the warp: the largest value, then the lowest index among the
+// lanes equal to it (-0 and +0 count as equal, as in vi_better).
+__device__ __forceinline__ VI warp_argmax_redux(VI a) {
+  const float M = warp_max_redux(a.v);
+  const unsigned i = __reduce_min_sync(0xffffffffu, a.v == M ? (unsigned)a.i : 0xffffffffu);
+  return VI{M, i == 0xffffffffu ? kNoIndex : (int)i};
+}
+
 // A warp's (m, s) partials merged max first: one exponential per lane instead of one per
 // shuffle step.
 __device__ __forceinline__ MS warp_merge_ms_maxfirst(MS v) {
-  float M = v.m;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float M = warp_max_redux(v.m);
   float s = (v.m == -INFINITY) ? 0.f : v.s * ex2(v.m - M);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -288,7 +304,7 @@ ee_kernel(const EarlyExitLaunch L) {
       const MS mq = warp_merge_ms_maxfirst(msacc_final(aq));
       if (lane == 0) s_part[k & 1][warp] = make_float4(mt.m, mt.s, mq.m, mq.s);
     } else {
-      best = warp_argmax(best);
+      best = warp_argmax_redux(best);
       if (lane == 0) s_part[k & 1][warp] = make_float4(best.v, __int_as_float(best.i), 0.f, 0.f);
     }
     __syncwarp();
@@ -313,11 +329,8 @@ ee_kernel(const EarlyExitLaunch L) {
       float Mt = pr[0].x, Mq = pr[0].z;
 #pragma unroll
       for (int j = 1; j < PL; ++j) { Mt = fmaxf(Mt, pr[j].x); Mq = fmaxf(Mq, pr[j].z); }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        Mt = fmaxf(Mt, __shfl_xor_sync(0xffffffffu, Mt, o));
-        Mq = fmaxf(Mq, __shfl_xor_sync(0xffffffffu, Mq, o));
-      }
+      Mt = warp_max_redux(Mt);
+      Mq = warp_max_redux(Mq);
       // each warp partial s * 2^(m - M) scaled in fp32 (the SFU exponential: a double exp2
       // per partial cost ~2 % of the verify), the terms summed in double
       double st = 0.0, sq = 0.0;
@@ -362,7 +375,7 @@ ee_kernel(const EarlyExitLaunch L) {
         const VI c{pr[j].x, __float_as_int(pr[j].y)};
         if (vi_better(c, b)) b = c;
       }
-      b = warp_argmax(b);                 // largest value, lowest index among equals
+      b = warp_argmax_redux(b);           // largest value, lowest index among equals
       gk = b.i == kNoIndex ? 0 : b.i;
       stop = !(k < Ki && d >= 0 && d < L.V && d == gk);
     }
